@@ -1,0 +1,230 @@
+"""Host oracle for W4A16 weight-only RTN quantization — TEST INFRASTRUCTURE ONLY.
+
+Only ``tests/``, ``__graft_entry__.smoke()`` and the CPU-baseline leg of
+``bench.py`` may import this package.  The CUDA library never calls it, and it
+shares no code with the CUDA library.
+
+The arithmetic lives in ``oracle.c`` (plain scalar C, binary32 quantizer,
+binary64 matmul); this module compiles it with gcc and exposes it through
+ctypes on numpy arrays.  bf16 tensors are passed as ``uint16`` bit patterns.
+
+Parity status of each function (what pins it is in ``tests/test_oracle_pins.py``):
+  bf16_from_f32 / bf16_from_f64 / f32_from_bf16 — pinned (torch conversion,
+      exact rational brute force)
+  quantize (asym, sym), pack/unpack, dequantize — pinned (hand-computed groups,
+      nearest-grid-point brute force, error bounds, invariants)
+  gemm_f64 / gemm_sampled — pinned (exact rational brute force, one-hot and
+      all-ones special cases)
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import subprocess
+import threading
+
+import numpy as np
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+_SRC = os.path.join(_HERE, "oracle.c")
+_LIB = os.path.join(_HERE, "liboracle.so")
+_lock = threading.Lock()
+_lib = None
+
+CFLAGS = ["-O2", "-ffp-contract=off", "-fno-fast-math", "-fopenmp", "-fPIC", "-shared",
+          "-std=c11", "-Wall"]
+
+
+def build(force: bool = False) -> str:
+    """Compile oracle.c into liboracle.so next to it (gcc, no fast-math).
+
+    ``W4A16_ORACLE_LIB`` names an already-built library to load instead; the
+    mutation tests use it to run the pins against deliberately broken copies.
+    """
+    override = os.environ.get("W4A16_ORACLE_LIB")
+    if override:
+        return override
+    if force or not os.path.exists(_LIB) or os.path.getmtime(_LIB) < os.path.getmtime(_SRC):
+        tmp = _LIB + f".tmp{os.getpid()}"
+        subprocess.check_call(["gcc", *CFLAGS, "-o", tmp, _SRC, "-lm"])
+        os.replace(tmp, _LIB)
+    return _LIB
+
+
+def _load():
+    global _lib
+    with _lock:
+        if _lib is None:
+            lib = ctypes.CDLL(build())
+            i64, i32, vp = ctypes.c_int64, ctypes.c_int32, ctypes.c_void_p
+            lib.oracle_bf16_to_f32.argtypes = [ctypes.c_uint16]
+            lib.oracle_bf16_to_f32.restype = ctypes.c_float
+            lib.oracle_f32_to_bf16_rn.argtypes = [ctypes.c_float]
+            lib.oracle_f32_to_bf16_rn.restype = ctypes.c_uint16
+            lib.oracle_f64_to_bf16_rn.argtypes = [ctypes.c_double]
+            lib.oracle_f64_to_bf16_rn.restype = ctypes.c_uint16
+            lib.oracle_group_asym.argtypes = [vp, i64, vp, vp, vp]
+            lib.oracle_group_sym.argtypes = [vp, i64, vp, vp]
+            lib.oracle_pack_codes.argtypes = [vp, i64, vp]
+            lib.oracle_unpack_codes.argtypes = [vp, i64, i32, vp]
+            lib.oracle_quantize.argtypes = [vp, i64, i64, i64, i32, vp, vp, vp]
+            lib.oracle_quantize.restype = ctypes.c_int
+            lib.oracle_dequantize.argtypes = [vp, vp, vp, i64, i64, i64, i32, vp]
+            lib.oracle_dequantize.restype = ctypes.c_int
+            lib.oracle_gemm_f64.argtypes = [vp, i64, i64, vp, i64, vp]
+            lib.oracle_gemm_w4a16_sampled.argtypes = [vp, i64, i64, vp, vp, vp, i64, i64, i32,
+                                                      vp, vp, i64, vp]
+            lib.oracle_gemm_w4a16_sampled.restype = ctypes.c_int
+            lib.oracle_round_to_bf16.argtypes = [vp, i64, vp]
+            lib.oracle_f32_array_to_bf16.argtypes = [vp, i64, vp]
+            lib.oracle_num_threads.restype = ctypes.c_int
+            _lib = lib
+    return _lib
+
+
+def _ptr(a: np.ndarray | None):
+    if a is None:
+        return None
+    assert a.flags["C_CONTIGUOUS"], "oracle arrays must be C-contiguous"
+    return a.ctypes.data_as(ctypes.c_void_p)
+
+
+def _u16(a) -> np.ndarray:
+    a = np.ascontiguousarray(a)
+    assert a.dtype == np.uint16, f"expected uint16 bf16 bit patterns, got {a.dtype}"
+    return a
+
+
+# ---------------------------------------------------------------- conversions
+def f32_from_bf16(bits) -> np.ndarray:
+    """bf16 bit patterns -> float32 values (exact)."""
+    b = np.ascontiguousarray(bits, dtype=np.uint16)
+    return (b.astype(np.uint32) << 16).view(np.float32)
+
+
+def bf16_from_f32(x) -> np.ndarray:
+    """float32 -> bf16 bits, round to nearest even (elementwise oracle call)."""
+    lib = _load()
+    x = np.ascontiguousarray(x, dtype=np.float32)
+    out = np.empty(x.shape, dtype=np.uint16)
+    lib.oracle_f32_array_to_bf16(_ptr(x), x.size, _ptr(out))
+    return out
+
+
+def bf16_from_f64(y) -> np.ndarray:
+    """float64 -> bf16 bits with a single round-to-nearest-even."""
+    lib = _load()
+    y = np.ascontiguousarray(y, dtype=np.float64)
+    out = np.empty(y.shape, dtype=np.uint16)
+    lib.oracle_round_to_bf16(_ptr(y), y.size, _ptr(out))
+    return out
+
+
+# ---------------------------------------------------------------- groups
+def group_asym(x) -> tuple[int, int, np.ndarray]:
+    """One asymmetric group -> (scale bf16 bits, zero point, codes)."""
+    lib = _load()
+    x = np.ascontiguousarray(x, dtype=np.float32)
+    s = np.zeros(1, dtype=np.uint16)
+    z = np.zeros(1, dtype=np.int32)
+    q = np.zeros(x.size, dtype=np.int32)
+    lib.oracle_group_asym(_ptr(x), x.size, _ptr(s), _ptr(z), _ptr(q))
+    return int(s[0]), int(z[0]), q
+
+
+def group_sym(x) -> tuple[int, np.ndarray]:
+    """One symmetric group -> (scale bf16 bits, codes)."""
+    lib = _load()
+    x = np.ascontiguousarray(x, dtype=np.float32)
+    s = np.zeros(1, dtype=np.uint16)
+    q = np.zeros(x.size, dtype=np.int32)
+    lib.oracle_group_sym(_ptr(x), x.size, _ptr(s), _ptr(q))
+    return int(s[0]), q
+
+
+def pack_codes(q) -> np.ndarray:
+    lib = _load()
+    q = np.ascontiguousarray(q, dtype=np.int32)
+    out = np.zeros(q.size // 2, dtype=np.uint8)
+    lib.oracle_pack_codes(_ptr(q), q.size, _ptr(out))
+    return out
+
+
+def unpack_codes(packed, n: int, sym: bool) -> np.ndarray:
+    lib = _load()
+    p = np.ascontiguousarray(packed, dtype=np.uint8)
+    q = np.zeros(n, dtype=np.int32)
+    lib.oracle_unpack_codes(_ptr(p), n, int(bool(sym)), _ptr(q))
+    return q
+
+
+# ---------------------------------------------------------------- matrices
+def quantize(W_bits, g: int, sym: bool):
+    """W[N, K] bf16 bits -> (packed u8[N, K/2], scales bf16[N, K/g], zeros bf16[N, K/g])."""
+    lib = _load()
+    W = _u16(W_bits)
+    N, K = W.shape
+    G = K // g
+    packed = np.zeros((N, K // 2), dtype=np.uint8)
+    scales = np.zeros((N, G), dtype=np.uint16)
+    zeros = np.zeros((N, G), dtype=np.uint16)
+    rc = lib.oracle_quantize(_ptr(W), N, K, g, int(bool(sym)), _ptr(packed), _ptr(scales),
+                             _ptr(zeros))
+    if rc != 0:
+        raise ValueError(f"oracle_quantize rejected N={N} K={K} g={g}")
+    return packed, scales, zeros
+
+
+def dequantize(packed, scales, zeros, K: int, g: int, sym: bool) -> np.ndarray:
+    lib = _load()
+    p = np.ascontiguousarray(packed, dtype=np.uint8)
+    s = _u16(scales)
+    z = _u16(zeros) if zeros is not None else np.zeros_like(s)
+    N = p.shape[0]
+    out = np.zeros((N, K), dtype=np.uint16)
+    rc = lib.oracle_dequantize(_ptr(p), _ptr(s), _ptr(z), N, K, g, int(bool(sym)), _ptr(out))
+    if rc != 0:
+        raise ValueError("oracle_dequantize rejected its arguments")
+    return out
+
+
+def gemm_f64(X_bits, W_hat_bits) -> np.ndarray:
+    """Y64[M, N] = X[M, K] · W_hat[N, K]^T in binary64."""
+    lib = _load()
+    X, W = _u16(X_bits), _u16(W_hat_bits)
+    M, K = X.shape
+    N, K2 = W.shape
+    assert K == K2
+    Y = np.zeros((M, N), dtype=np.float64)
+    lib.oracle_gemm_f64(_ptr(X), M, K, _ptr(W), N, _ptr(Y))
+    return Y
+
+
+def gemm_w4a16(X_bits, packed, scales, zeros, g: int, sym: bool) -> np.ndarray:
+    """Full reference: dequantize, then binary64 matmul."""
+    X = _u16(X_bits)
+    W_hat = dequantize(packed, scales, zeros, X.shape[1], g, sym)
+    return gemm_f64(X, W_hat)
+
+
+def gemm_sampled(X_bits, packed, scales, zeros, g: int, sym: bool, ms, ns) -> np.ndarray:
+    """Y64 at the listed (m, n) positions, dequantizing row n on the fly."""
+    lib = _load()
+    X = _u16(X_bits)
+    M, K = X.shape
+    p = np.ascontiguousarray(packed, dtype=np.uint8)
+    s = _u16(scales)
+    z = _u16(zeros) if zeros is not None else np.zeros_like(s)
+    N = p.shape[0]
+    ms = np.ascontiguousarray(ms, dtype=np.int64)
+    ns = np.ascontiguousarray(ns, dtype=np.int64)
+    out = np.zeros(ms.size, dtype=np.float64)
+    rc = lib.oracle_gemm_w4a16_sampled(_ptr(X), M, K, _ptr(p), _ptr(s), _ptr(z), N, g,
+                                       int(bool(sym)), _ptr(ms), _ptr(ns), ms.size, _ptr(out))
+    if rc != 0:
+        raise ValueError("oracle_gemm_w4a16_sampled rejected its arguments")
+    return out
+
+
+def num_threads() -> int:
+    return int(_load().oracle_num_threads())

@@ -1,0 +1,367 @@
+"""Pins for the host oracle: checks against what the pages and mathematics fix.
+
+No expectation here is computed by re-typing the oracle's formulas.  The pins
+are: hand-computed groups (tests/golden/hand_groups.json), a library routine
+(torch's float32 -> bf16 conversion), exact rational brute force (fractions),
+nearest-grid-point brute force over all 16 codes, closed-form constructions
+(on-grid groups, exactly representable products, one-hot and all-ones
+activations) and invariants (ranges, z = 0 in symmetric mode, power-of-two
+scale invariance, error bounds).
+"""
+import json
+import os
+from fractions import Fraction
+
+import numpy as np
+import pytest
+import torch
+
+import oracle
+import workloads
+
+GOLDEN = os.path.join(os.path.dirname(__file__), "golden", "hand_groups.json")
+CASES = json.load(open(GOLDEN))["cases"]
+
+
+def _f32(vals):
+    return np.array([float(v) for v in vals], dtype=np.float32)
+
+
+# ------------------------------------------------------------------ golden groups
+@pytest.mark.parametrize("case", CASES, ids=[c["name"] for c in CASES])
+def test_hand_computed_group(case):
+    x = _f32(case["x"])
+    sym = case["mode"] == "sym"
+    if sym:
+        s_bits, q = oracle.group_sym(x)
+        z = 0
+    else:
+        s_bits, z, q = oracle.group_asym(x)
+    assert s_bits == int(case["s_bits"], 16)
+    assert float(oracle.f32_from_bf16(np.array([s_bits], np.uint16))[0]) == float(case["s"])
+    assert z == case["z"]
+    assert list(q) == case["q"]
+    packed = oracle.pack_codes(q)
+    assert list(packed) == [int(b, 16) for b in case["packed"]]
+
+
+@pytest.mark.parametrize("case", CASES, ids=[c["name"] for c in CASES])
+def test_hand_computed_group_through_matrix_path(case):
+    """Same groups through quantize/dequantize on a [3, 8] matrix (two groups per
+    row, rows and groups permuted) to pin row/group/nibble indexing."""
+    x = _f32(case["x"])
+    sym = case["mode"] == "sym"
+    other = _f32(CASES[0]["x"])                 # a different group beside it
+    rows = [np.concatenate([x, other]), np.concatenate([other, x]), np.concatenate([x, x])]
+    W = oracle.bf16_from_f32(np.stack(rows))
+    P, S, Z = oracle.quantize(W, 4, sym)
+    exp_bytes = [int(b, 16) for b in case["packed"]]
+    for r, slot in ((0, 0), (1, 1), (2, 0), (2, 1)):
+        assert list(P[r, 2 * slot:2 * slot + 2]) == exp_bytes
+        assert S[r, slot] == int(case["s_bits"], 16)
+        assert float(oracle.f32_from_bf16(Z[r, slot:slot + 1])[0]) == (0.0 if sym else case["z"])
+    Wh = oracle.dequantize(P, S, Z, 8, 4, sym)
+    xh = oracle.f32_from_bf16(Wh)
+    exp = [float(v) for v in case["x_hat"]]
+    assert list(xh[0, :4]) == exp and list(xh[1, 4:]) == exp and list(xh[2, 4:]) == exp
+
+
+# ------------------------------------------------------------------ bf16 conversions
+def _interesting_floats(n=20000, seed=0):
+    rng = np.random.default_rng(seed)
+    a = rng.standard_normal(n).astype(np.float32) * np.float32(3.0)
+    b = (rng.integers(0, 2**32, n, dtype=np.uint64).astype(np.uint32)).view(np.float32)
+    b = b[np.isfinite(b)]
+    # exact ties: upper 16 bits arbitrary, lower 16 bits = 0x8000
+    t = ((rng.integers(0, 2**16, 4000, dtype=np.uint64).astype(np.uint32) << 16) | 0x8000)
+    t = t.view(np.float32)
+    t = t[np.isfinite(t)]
+    special = np.array([0.0, -0.0, 1e-45, -1e-45, 1e-39, 3.3895313e38, 3.4e38, -3.4e38,
+                        np.inf, -np.inf], dtype=np.float32)
+    return np.concatenate([a, b, t, special]).astype(np.float32)
+
+
+def test_f32_to_bf16_matches_torch():
+    x = _interesting_floats()
+    ours = oracle.bf16_from_f32(x)
+    ref = workloads.bits(torch.from_numpy(x).to(torch.bfloat16))
+    assert np.array_equal(ours, ref)
+
+
+def test_bf16_to_f32_is_exact_upper_half():
+    b = np.arange(0, 2**16, dtype=np.uint32).astype(np.uint16)
+    f = oracle.f32_from_bf16(b)
+    t = workloads.from_bits(b).to(torch.float32).numpy()
+    fin = np.isfinite(t)
+    assert np.array_equal(f[fin], t[fin])
+
+
+def _bf16_value(bits16):
+    f = oracle.f32_from_bf16(np.array([bits16], np.uint16))[0]
+    return Fraction(float(f))
+
+
+def _bf16_rne_bruteforce(d: float) -> int:
+    """Nearest bf16 to the exact value of d, ties to even mantissa (pure Python)."""
+    exact = Fraction(d)
+    if d == 0:
+        return 0x8000 if np.signbit(d) else 0
+    c = int(np.array([np.float32(d)]).view(np.uint32)[0] >> 16)
+    best = None
+    for cand in range(max(c - 2, 0), min(c + 3, 0xFFFF) + 1):
+        if (cand & 0x7F80) == 0x7F80:
+            continue
+        if (cand >> 15) != (1 if d < 0 else 0):
+            continue
+        dist = abs(_bf16_value(cand) - exact)
+        key = (dist, cand & 1)
+        if best is None or key < best[0]:
+            best = (key, cand)
+    return best[1]
+
+
+def test_f64_to_bf16_single_rounding_bruteforce():
+    rng = np.random.default_rng(1)
+    vals = list(rng.standard_normal(3000) * 10.0)
+    # doubles just beside bf16 ties: a binary32-then-bf16 double rounding would break these
+    for _ in range(500):
+        hi = int(rng.integers(0x3C00, 0x4400))
+        base = float(Fraction(float(oracle.f32_from_bf16(np.array([hi], np.uint16))[0])))
+        ulp = float(_bf16_value(hi + 1) - _bf16_value(hi))
+        mid = base + ulp / 2
+        vals += [mid, np.nextafter(mid, np.inf), np.nextafter(mid, -np.inf),
+                 mid + ulp * 2.0**-20, mid - ulp * 2.0**-20]
+    vals = np.array(vals, dtype=np.float64)
+    ours = oracle.bf16_from_f64(vals)
+    for v, o in zip(vals, ours):
+        assert int(o) == _bf16_rne_bruteforce(float(v)), (v, hex(o))
+
+
+# ------------------------------------------------------------------ packing
+@pytest.mark.parametrize("sym", [False, True])
+def test_unpack_pack_all_256_bytes(sym):
+    allb = np.arange(256, dtype=np.uint8)
+    q = oracle.unpack_codes(allb, 512, sym)
+    assert np.array_equal(oracle.pack_codes(q), allb)
+    lo, hi = q[0::2], q[1::2]
+    if sym:
+        assert lo.min() == -8 and lo.max() == 7
+        assert np.array_equal(lo, ((allb & 0xF).astype(np.int32) ^ 8) - 8)
+    else:
+        assert np.array_equal(lo, allb & 0xF) and np.array_equal(hi, allb >> 4)
+
+
+@pytest.mark.parametrize("sym", [False, True])
+def test_pack_unpack_all_code_pairs(sym):
+    r = np.arange(-8, 8) if sym else np.arange(16)
+    a, b = np.meshgrid(r, r, indexing="ij")
+    q = np.stack([a.ravel(), b.ravel()], 1).ravel().astype(np.int32)
+    assert np.array_equal(oracle.unpack_codes(oracle.pack_codes(q), q.size, sym), q)
+
+
+# ------------------------------------------------------------------ quantizer properties
+def _groups(seed, g, n):
+    """Random groups of assorted shapes: Gaussian, outlier-laden, one-sided, tiny, huge."""
+    rng = np.random.default_rng(seed)
+    out = []
+    for i in range(n):
+        kind = i % 6
+        x = rng.standard_normal(g)
+        if kind == 1:
+            x[rng.integers(0, g)] *= 50.0
+        elif kind == 2:
+            x = np.abs(x) + 0.1
+        elif kind == 3:
+            x = -np.abs(x) - 0.1
+        elif kind == 4:
+            x *= 2.0**-60
+        elif kind == 5:
+            x *= 2.0**40
+        out.append(oracle.f32_from_bf16(oracle.bf16_from_f32(x.astype(np.float32))))
+    return out
+
+
+@pytest.mark.parametrize("g", [4, 32, 64, 128])
+def test_asym_codes_are_nearest_grid_points(g):
+    """Brute force over all 16 codes: the chosen code minimises |x − (c − z)s|,
+    up to the rounding of the binary32 quotient x/s next to a tie."""
+    for x in _groups(10 + g, g, 240):
+        s_bits, z, q = oracle.group_asym(x)
+        s = float(oracle.f32_from_bf16(np.array([s_bits], np.uint16))[0])
+        assert 0 <= z <= 15 and np.all((q >= 0) & (q <= 15))
+        if s == 0.0:
+            assert np.all(q == 0) and z == 0
+            continue
+        xs = x.astype(np.float64)
+        grid = (np.arange(16)[None, :] - z) * s               # exact in binary64
+        dist = np.abs(xs[:, None] - grid)
+        chosen = dist[np.arange(g), q]
+        slack = np.abs(xs) * 2.0**-22 + s * 2.0**-20
+        assert np.all(chosen <= dist.min(1) + slack)
+
+
+@pytest.mark.parametrize("g", [4, 32, 128])
+def test_sym_codes_are_nearest_grid_points(g):
+    for x in _groups(20 + g, g, 240):
+        s_bits, q = oracle.group_sym(x)
+        s = float(oracle.f32_from_bf16(np.array([s_bits], np.uint16))[0])
+        assert np.all((q >= -7) & (q <= 7)), "absmax/7 never reaches -8"
+        if s == 0.0:
+            assert np.all(q == 0)
+            continue
+        xs = x.astype(np.float64)
+        grid = np.arange(-8, 8)[None, :] * s
+        dist = np.abs(xs[:, None] - grid)
+        chosen = dist[np.arange(g), q + 8]
+        slack = np.abs(xs) * 2.0**-22 + s * 2.0**-20
+        assert np.all(chosen <= dist.min(1) + slack)
+
+
+@pytest.mark.parametrize("g", [32, 128])
+def test_error_bound_half_step(g):
+    """|x − (q − z)s| ≤ s/2 for unclamped codes; clamped codes can exceed it only
+    by the bf16 rounding of s: ≤ s/2 + 15·2^-8·s."""
+    for x in _groups(30 + g, g, 240):
+        s_bits, z, q = oracle.group_asym(x)
+        s = float(oracle.f32_from_bf16(np.array([s_bits], np.uint16))[0])
+        if s == 0.0:
+            continue
+        err = np.abs(x.astype(np.float64) - (q - z) * s)
+        inner = (q > 0) & (q < 15)
+        assert np.all(err[inner] <= s / 2 * (1 + 2.0**-20))
+        assert np.all(err <= s / 2 + 15 * 2.0**-8 * s)
+        # the group minimum maps to code 0 (rint is odd-symmetric); the maximum to 14 or 15
+        lo, hi = np.argmin(x), np.argmax(x)
+        if x[lo] < 0:
+            assert q[lo] == 0
+        if x[hi] > 0:
+            assert q[hi] >= 14
+
+
+def test_sym_zero_points_are_zero_and_error_bound():
+    W = workloads.bits(workloads.make_weight(37, 256, 0.02, seed=5, outlier_frac=0.05,
+                                             outlier_scale=20.0))
+    P, S, Z = oracle.quantize(W, 64, sym=True)
+    assert np.all(Z == 0)
+    q = oracle.unpack_codes(P.reshape(-1), P.size * 2, True).reshape(37, 256)
+    s = np.repeat(oracle.f32_from_bf16(S).astype(np.float64), 64, axis=1)
+    x = oracle.f32_from_bf16(W).astype(np.float64)
+    assert np.all(np.abs(x - q * s) <= s / 2 * (1 + 2.0**-20) + 0.0)
+
+
+@pytest.mark.parametrize("sym", [False, True])
+@pytest.mark.parametrize("e", [-7, 5])
+def test_power_of_two_scale_invariance(sym, e):
+    W = workloads.make_weight(16, 256, 0.02, seed=7, outlier_frac=0.02, outlier_scale=20.0)
+    W2 = (W.to(torch.float32) * 2.0**e).to(torch.bfloat16)     # exact scaling
+    P1, S1, Z1 = oracle.quantize(workloads.bits(W), 32, sym)
+    P2, S2, Z2 = oracle.quantize(workloads.bits(W2), 32, sym)
+    assert np.array_equal(P1, P2) and np.array_equal(Z1, Z2)
+    assert np.array_equal(oracle.f32_from_bf16(S1) * np.float32(2.0**e), oracle.f32_from_bf16(S2))
+
+
+@pytest.mark.parametrize("g", [32, 64, 128])
+def test_on_grid_matrix_is_recovered_exactly(g):
+    """Closed form: W = (q − z)·s with s of ≤ 4 significant bits and each group
+    using codes 0 and 15 re-quantizes to exactly (s, z, q), and dequantizes to W."""
+    rng = np.random.default_rng(g)
+    N, K = 6, 4 * g
+    G = K // g
+    q = rng.integers(0, 16, size=(N, K))
+    q[:, ::g] = 0
+    q[:, 1::g] = 15
+    z = rng.integers(0, 16, size=(N, G))
+    mant = rng.choice([8, 9, 10, 11, 12, 13, 14, 15], size=(N, G))   # 4 significant bits
+    s = mant * 2.0 ** rng.integers(-14, -6, size=(N, G)).astype(np.float64)
+    x = (q - np.repeat(z, g, 1)) * np.repeat(s, g, 1)
+    Wb = oracle.bf16_from_f32(x.astype(np.float32))
+    assert np.array_equal(oracle.f32_from_bf16(Wb).astype(np.float64), x)
+    P, S, Z = oracle.quantize(Wb, g, sym=False)
+    assert np.array_equal(oracle.f32_from_bf16(S).astype(np.float64), s)
+    assert np.array_equal(oracle.f32_from_bf16(Z).astype(np.int64), z)
+    qq = oracle.unpack_codes(P.reshape(-1), N * K, False).reshape(N, K)
+    assert np.array_equal(qq, q)
+    Wh = oracle.dequantize(P, S, Z, K, g, False)
+    assert np.array_equal(Wh, Wb)
+
+
+@pytest.mark.parametrize("sym", [False, True])
+def test_dequantize_closed_form_indexing(sym):
+    """Hand-built packed/scales/zeros whose products (q − z)·s are exact in bf16:
+    dequantize must place each value at its (row, k)."""
+    rng = np.random.default_rng(3 + sym)
+    N, K, g = 5, 192, 64
+    G = K // g
+    q = rng.integers(-8, 8, size=(N, K)) if sym else rng.integers(0, 16, size=(N, K))
+    z = np.zeros((N, G), np.int64) if sym else rng.integers(0, 16, size=(N, G))
+    s = rng.choice([8, 10, 12, 14], size=(N, G)) * 2.0 ** rng.integers(-12, 0, size=(N, G))
+    packed = oracle.pack_codes(q.reshape(-1)).reshape(N, K // 2)
+    # scales and zeros are exact in bf16 by construction (≤ 4 significant bits, small ints)
+    S = oracle.bf16_from_f32(s.astype(np.float32))
+    Z = oracle.bf16_from_f32(z.astype(np.float32))
+    Wh = oracle.f32_from_bf16(oracle.dequantize(packed, S, Z, K, g, sym)).astype(np.float64)
+    expect = (q - np.repeat(z, g, 1)) * np.repeat(s, g, 1)      # ≤ 8 significant bits: exact
+    assert np.array_equal(Wh, expect)
+
+
+# ------------------------------------------------------------------ reference matmul
+def _bounded_bf16(rng, shape, emin=-6, emax=6):
+    mant = rng.integers(128, 256, size=shape)                  # 8 significant bits
+    e = rng.integers(emin, emax + 1, size=shape)
+    sign = rng.choice([-1, 1], size=shape)
+    v = sign * mant * 2.0 ** (e - 7)
+    return oracle.bf16_from_f32(v.astype(np.float32))
+
+
+@pytest.mark.parametrize("M,N,K", [(1, 1, 1), (3, 5, 7), (4, 16, 16), (7, 3, 33)])
+def test_gemm_f64_exact_rational_bruteforce(M, N, K):
+    rng = np.random.default_rng(M * 100 + N * 10 + K)
+    X = _bounded_bf16(rng, (M, K))
+    W = _bounded_bf16(rng, (N, K))
+    Y = oracle.gemm_f64(X, W)
+    xf, wf = oracle.f32_from_bf16(X), oracle.f32_from_bf16(W)
+    for m in range(M):
+        for n in range(N):
+            exact = sum(Fraction(float(xf[m, k])) * Fraction(float(wf[n, k])) for k in range(K))
+            assert Y[m, n] == float(exact)         # exact: bounded exponents fit binary64
+
+
+def test_gemm_one_hot_reduces_to_dequantize():
+    W = workloads.bits(workloads.make_weight(24, 256, 0.02, seed=9))
+    for sym in (False, True):
+        P, S, Z = oracle.quantize(W, 128, sym)
+        Wh = oracle.dequantize(P, S, Z, 256, 128, sym)
+        ks = np.array([0, 1, 127, 128, 200, 255])
+        X = np.zeros((ks.size, 256), np.float32)
+        X[np.arange(ks.size), ks] = 1.0
+        Y = oracle.gemm_w4a16(oracle.bf16_from_f32(X), P, S, Z, 128, sym)
+        assert np.array_equal(oracle.bf16_from_f64(Y), Wh[:, ks].T)
+
+
+def test_gemm_all_ones_gives_row_sums():
+    W = workloads.bits(workloads.make_weight(9, 128, 0.02, seed=4))
+    P, S, Z = oracle.quantize(W, 32, False)
+    Wh = oracle.f32_from_bf16(oracle.dequantize(P, S, Z, 128, 32, False))
+    X = oracle.bf16_from_f32(np.ones((2, 128), np.float32))
+    Y = oracle.gemm_w4a16(X, P, S, Z, 32, False)
+    for n in range(9):
+        exact = sum(Fraction(float(v)) for v in Wh[n])
+        assert Y[0, n] == float(exact) and Y[1, n] == float(exact)
+
+
+def test_gemm_sampled_equals_full():
+    W = workloads.bits(workloads.make_weight(40, 384, 0.02, seed=2))
+    X = workloads.bits(workloads.make_activation(5, 384, seed=3, outlier_frac=0.02,
+                                                 outlier_mode="set"))
+    for sym in (False, True):
+        P, S, Z = oracle.quantize(W, 64, sym)
+        full = oracle.gemm_w4a16(X, P, S, Z, 64, sym)
+        ms = np.array([0, 4, 2, 3, 1, 4])
+        ns = np.array([0, 39, 17, 5, 38, 1])
+        assert np.array_equal(oracle.gemm_sampled(X, P, S, Z, 64, sym, ms, ns), full[ms, ns])
+
+
+def test_quantize_rejects_bad_shapes():
+    W = np.zeros((2, 96), np.uint16)
+    with pytest.raises(ValueError):
+        oracle.quantize(W, 64, False)           # K % g != 0
