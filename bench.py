@@ -1,0 +1,657 @@
+"""Benchmark of the W4A16 fused GEMM on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+                    [--workload decode7b|decode70b|prefill] [--no-extras]
+
+Metric: W4A16 GEMM HBM GB/s at M=1 and TFLOPS at M=2048, as % of the B200
+roofline.  The headline line (default workload) is the M=1 decode of the two
+Llama-2-7B-shaped layers (K=4096,N=11008 and K=11008,N=4096; g=128, asym):
+one step = both fused GEMMs, through the library's dispatch, on synthetic
+seeded weights/activations of that shape.  `value` is algorithmic bytes per
+step (packed weights + scales + zeros + X read once + Y written once) times
+steps, over the device time of the timed region, summed over ranks and
+divided by the max over ranks.  The same JSON line carries the M=2048 prefill
+TFLOPS (K=N=8192) with its tensor-core roofline, a dense bf16 cuBLAS GEMM and
+the unfused dequantize-then-GEMM at the same shapes, the end-to-end number
+through the public API with host buffers, and the host oracle on the CPU.
+
+Timing: W warm-up steps, then K steps replayed from CUDA graphs (one graph per
+rotation slot, so launch cost stays off the device timeline), bracketed by a
+barrier and torch.cuda.synchronize() on both sides, CUDA events on the
+launching stream.  Weight copies rotate so the bytes touched between reuses
+exceed twice the L2 size: every step streams its weights from HBM.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import torch  # noqa: E402
+
+import workloads  # noqa: E402
+
+METRIC = "W4A16 GEMM HBM GB/s at M=1 and TFLOPS at M=2048, as % of B200 roofline"
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+L2_BYTES_FALLBACK = 126 * 1024 * 1024
+
+
+# ---------------------------------------------------------------------------- helpers
+def load_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            p = json.load(f)
+        return {k: float(p[k]) for k in FALLBACK_PEAKS}, "measured"
+    except (OSError, KeyError, ValueError):
+        return dict(FALLBACK_PEAKS), "fallback"
+
+
+def algorithmic_bytes(M: int, N: int, K: int, g: int, sym: bool) -> int:
+    """Packed codes + scales (+ zeros if asymmetric) + X read once + Y written once."""
+    return N * K // 2 + 2 * N * (K // g) * (1 if sym else 2) + 2 * M * K + 2 * M * N
+
+
+def kernel_source_digest() -> str:
+    h = hashlib.sha256()
+    csrc = os.path.join(ROOT, "weight_only_quantization_rtn_b200", "csrc")
+    for name in sorted(os.listdir(csrc)):
+        with open(os.path.join(csrc, name), "rb") as f:
+            h.update(name.encode())
+            h.update(f.read())
+    return h.hexdigest()[:16]
+
+
+def ncu_traffic(kernel_key: str):
+    """DRAM bytes per launch from a committed ncu capture of the current kernel
+    source, or None when the capture is missing or the kernel changed since."""
+    path = os.path.join(ROOT, "profiles", "ncu_traffic.json")
+    try:
+        with open(path) as f:
+            table = json.load(f)
+        entry = table[kernel_key]
+        if entry.get("kernel_source_digest") != kernel_source_digest():
+            return None
+        return float(entry["dram_bytes_per_launch"])
+    except (OSError, KeyError, ValueError):
+        return None
+
+
+class ClockSampler:
+    """nvidia-smi sampling of SM clock and throttle reasons while it runs."""
+    FIELDS = ("clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.hw_slowdown,"
+              "clocks_event_reasons.hw_thermal_slowdown,clocks_event_reasons.sw_thermal_slowdown,"
+              "clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, index: int):
+        self.index = index
+        self.proc = None
+        self.t0 = self.t1 = None
+
+    def __enter__(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(self.index), f"--query-gpu=timestamp,{self.FIELDS}",
+                 "--format=csv,noheader,nounits", "-lms", "50"],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+            time.sleep(0.3)
+        except OSError:
+            self.proc = None
+        self.t0 = time.time()
+        return self
+
+    def mark_end(self):
+        self.t1 = time.time()
+
+    def __exit__(self, *exc):
+        self.lines = []
+        if self.proc is not None:
+            time.sleep(0.12)
+            self.proc.terminate()
+            try:
+                out, _ = self.proc.communicate(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+                out, _ = self.proc.communicate()
+            self.lines = [l for l in out.splitlines() if l.strip()]
+        return False
+
+    def summary(self):
+        import datetime
+        rows = []
+        for l in self.lines:
+            parts = [p.strip() for p in l.split(",")]
+            if len(parts) < 8:
+                continue
+            try:
+                ts = datetime.datetime.strptime(parts[0], "%Y/%m/%d %H:%M:%S.%f").timestamp()
+                if self.t1 is not None and not (self.t0 - 0.06 <= ts <= self.t1 + 0.06):
+                    continue                      # keep the samples taken in the timed region
+                rows.append((float(parts[1]), float(parts[2]), parts[4:8]))
+            except ValueError:
+                continue
+        if not rows:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": [], "samples": 0}
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({names[i] for _, _, r in rows for i, v in enumerate(r) if v == "Active"})
+        return {"sm_mhz": statistics.median(r[0] for r in rows),
+                "sm_max_mhz": max(r[1] for r in rows), "reasons": reasons, "samples": len(rows)}
+
+
+# ---------------------------------------------------------------------------- dist
+def dist_setup(n_gpus: int):
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        torch.cuda.set_device(local)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=torch.device("cuda", local))
+    else:
+        torch.cuda.set_device(0)
+    return world, rank, local
+
+
+def barrier(world):
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+
+
+def max_over_ranks(world, value: float) -> float:
+    if world == 1:
+        return value
+    import torch.distributed as dist
+    t = torch.tensor([value], dtype=torch.float64, device="cuda")
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def sum_over_ranks(world, value: float) -> float:
+    if world == 1:
+        return value
+    import torch.distributed as dist
+    t = torch.tensor([value], dtype=torch.float64, device="cuda")
+    dist.all_reduce(t, op=dist.ReduceOp.SUM)
+    return float(t.item())
+
+
+# ---------------------------------------------------------------------------- workloads
+class GemmCase:
+    """One layer of a workload, resident on the device, with `copies` rotating
+    copies of the quantized weights (and activations)."""
+
+    def __init__(self, w4, layer, M, g, sym, copies, dev):
+        self.layer, self.M, self.g, self.sym = layer, M, g, sym
+        self.N, self.K = layer.N, layer.K
+        W = layer.weight().to(dev)
+        P, S, Z = w4.quantize(W, g, sym)
+        self.W_dense = W
+        self.P = [P] + [P.clone() for _ in range(copies - 1)]
+        self.S = [S] + [S.clone() for _ in range(copies - 1)]
+        self.Z = [Z] + [Z.clone() for _ in range(copies - 1)]
+        X = layer.activation(M).to(dev)
+        self.X = [X] + [X.clone() for _ in range(copies - 1)]
+        self.Y = [torch.empty(M, self.N, dtype=torch.bfloat16, device=dev) for _ in range(copies)]
+        self.bytes = algorithmic_bytes(M, self.N, self.K, g, sym)
+        self.flops = 2 * M * self.N * self.K
+
+    def call(self, w4, i):
+        j = i % len(self.P)
+        w4.gemm(self.X[j], self.P[j], self.S[j], self.Z[j], self.g, self.sym, out=self.Y[j])
+
+
+def copies_for(bytes_per_step: int, l2: int) -> int:
+    return max(2, -(-2 * l2 // max(bytes_per_step, 1)) + 1)
+
+
+def capture_step_graphs(w4, cases, copies, with_events):
+    """One CUDA graph per rotation slot; each runs one step (every case once).
+    With events, external timing events bracket every GEMM inside the graph."""
+    graphs, events = [], []
+    stream = torch.cuda.Stream()
+    stream.wait_stream(torch.cuda.current_stream())
+    with torch.cuda.stream(stream):
+        for i in range(copies):          # compile plans and set kernel attributes before capture
+            for c in cases:
+                c.call(w4, i)
+    torch.cuda.current_stream().wait_stream(stream)
+    torch.cuda.synchronize()
+    for i in range(copies):
+        g = torch.cuda.CUDAGraph()
+        ev = [torch.cuda.Event(enable_timing=True, external=True) for _ in range(len(cases) + 1)]
+        with torch.cuda.graph(g, stream=stream):
+            if with_events:
+                ev[0].record()
+            for ci, c in enumerate(cases):
+                c.call(w4, i)
+                if with_events:
+                    ev[ci + 1].record()
+        graphs.append(g)
+        events.append(ev)
+    torch.cuda.synchronize()
+    return graphs, events
+
+
+def run_timed(world, graphs, steps, warmup, sampler_index=None):
+    for s in range(warmup):
+        graphs[s % len(graphs)].replay()
+    torch.cuda.synchronize()
+    barrier(world)
+    torch.cuda.synchronize()
+    start = torch.cuda.Event(enable_timing=True)
+    end = torch.cuda.Event(enable_timing=True)
+    sampler = ClockSampler(sampler_index) if sampler_index is not None else None
+    if sampler:
+        sampler.__enter__()
+    start.record()
+    for s in range(steps):
+        graphs[s % len(graphs)].replay()
+    end.record()
+    end.synchronize()
+    if sampler:
+        sampler.mark_end()
+        sampler.__exit__(None, None, None)
+    torch.cuda.synchronize()
+    barrier(world)
+    ms = start.elapsed_time(end)
+    return ms, (sampler.summary() if sampler else None)
+
+
+def per_kernel_ms(events, n_cases):
+    """Average duration of each case's GEMM over the last replay of every slot."""
+    out = [[] for _ in range(n_cases)]
+    for ev in events:
+        for ci in range(n_cases):
+            out[ci].append(ev[ci].elapsed_time(ev[ci + 1]))
+    return [statistics.mean(v) for v in out]
+
+
+def time_callable(fn, iters, warmup=3):
+    for _ in range(warmup):
+        fn()
+    torch.cuda.synchronize()
+    a = torch.cuda.Event(enable_timing=True)
+    b = torch.cuda.Event(enable_timing=True)
+    a.record()
+    for _ in range(iters):
+        fn()
+    b.record()
+    b.synchronize()
+    return a.elapsed_time(b) / iters
+
+
+def graph_of(fn, copies):
+    """CUDA graphs of fn(i) for each rotation slot i (for comparison timings)."""
+    stream = torch.cuda.Stream()
+    stream.wait_stream(torch.cuda.current_stream())
+    with torch.cuda.stream(stream):
+        for i in range(copies):
+            fn(i)
+    torch.cuda.current_stream().wait_stream(stream)
+    torch.cuda.synchronize()
+    gs = []
+    for i in range(copies):
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g, stream=stream):
+            fn(i)
+        gs.append(g)
+    torch.cuda.synchronize()
+    return gs
+
+
+def time_graphs(gs, iters):
+    for i in range(3):
+        gs[i % len(gs)].replay()
+    torch.cuda.synchronize()
+    a = torch.cuda.Event(enable_timing=True)
+    b = torch.cuda.Event(enable_timing=True)
+    a.record()
+    for i in range(iters):
+        gs[i % len(gs)].replay()
+    b.record()
+    b.synchronize()
+    return a.elapsed_time(b) / iters
+
+
+# ---------------------------------------------------------------------------- oracle baseline
+def cpu_baseline(layers, M, g, sym, unit_bytes: bool, budget_s: float = 6.0):
+    """The host oracle as it stands (dequantize + binary64 matmul from the packed
+    form) on the same layer shapes; repeats the whole workload until budget_s."""
+    import oracle
+    oracle.build()
+    prepared = []
+    for layer in layers:
+        Wb = workloads.bits(layer.weight())
+        Xb = workloads.bits(layer.activation(M))
+        P, S, Z = oracle.quantize(Wb, g, sym)
+        prepared.append((layer, Xb, P, S, Z))
+    reps, t0 = 0, time.perf_counter()
+    while True:
+        for layer, Xb, P, S, Z in prepared:
+            oracle.gemm_w4a16(Xb, P, S, Z, g, sym)
+        reps += 1
+        el = time.perf_counter() - t0
+        if el >= budget_s or reps >= 50:
+            break
+    per_step = el / reps
+    if unit_bytes:
+        work = sum(algorithmic_bytes(M, l.N, l.K, g, sym) for l in layers)
+        value, unit = work / per_step / 1e9, "GB/s"
+    else:
+        work = sum(2 * M * l.N * l.K for l in layers)
+        value, unit = work / per_step / 1e12, "TFLOP/s"
+    return {"value": value, "unit": unit, "cores": oracle.num_threads(), "kind": "oracle",
+            "sample": f"{reps} full step(s) of the workload ({len(layers)} layer GEMM(s), "
+                      f"dequantize + binary64 matmul from the packed form) in {el:.2f} s",
+            "s_per_step": per_step}
+
+
+def cpu_baseline_sampled(layer, M, g, sym, rows: int):
+    """Oracle on a bounded sample of output rows (for workloads far beyond a
+    minute of CPU time); throughput scaled per output row."""
+    import numpy as np
+    import oracle
+    oracle.build()
+    Wb = workloads.bits(layer.weight())
+    Xb = workloads.bits(layer.activation(M))
+    P, S, Z = oracle.quantize(Wb, g, sym)
+    ns = np.arange(rows, dtype=np.int64)
+    ms = np.zeros(rows, dtype=np.int64)
+    mm, nn = np.meshgrid(np.arange(M), ns, indexing="ij")
+    t0 = time.perf_counter()
+    oracle.gemm_sampled(Xb, P, S, Z, g, sym, mm.ravel(), nn.ravel())
+    el = time.perf_counter() - t0
+    frac = rows / layer.N
+    flops = 2 * M * layer.N * layer.K * frac
+    return {"value": flops / el / 1e12, "unit": "TFLOP/s", "cores": oracle.num_threads(),
+            "kind": "oracle",
+            "sample": f"{rows} of {layer.N} output columns x all {M} rows "
+                      f"({frac * 100:.2f}% of the outputs) in {el:.2f} s",
+            "s_per_step": el / frac}
+
+
+# ---------------------------------------------------------------------------- main arms
+WORKLOAD_DEFS = {
+    # name: (workload, M, g, sym, metric half)
+    "decode7b": (workloads.DECODE_7B, 1, 128, False, "hbm"),
+    "decode70b": (workloads.DECODE_70B, 1, 128, False, "hbm"),
+    "prefill": (workloads.PREFILL, 2048, 128, False, "tensor"),
+}
+
+
+def run_ours(args):
+    world, rank, local = dist_setup(args.gpus)
+    dev = torch.device("cuda", local)
+    import weight_only_quantization_rtn_b200 as w4
+    from weight_only_quantization_rtn_b200 import build as w4build
+    if rank == 0:
+        w4build.build()
+    barrier(world)
+    w4.lib()
+    peaks, peak_src = load_peaks()
+    props = torch.cuda.get_device_properties(dev)
+    l2 = getattr(props, "L2_cache_size", 0) or L2_BYTES_FALLBACK
+
+    wl, M, g, sym, half = WORKLOAD_DEFS[args.workload]
+    bytes_step = sum(algorithmic_bytes(M, l.N, l.K, g, sym) for l in wl.layers)
+    flops_step = sum(2 * M * l.N * l.K for l in wl.layers)
+    in_bytes_step = sum(l.N * l.K // 2 + 2 * l.N * (l.K // g) * (1 if sym else 2) + 2 * M * l.K
+                        for l in wl.layers)
+    copies = copies_for(in_bytes_step, l2)
+    cases = [GemmCase(w4, l, M, g, sym, copies, dev) for l in wl.layers]
+    graphs, events = capture_step_graphs(w4, cases, copies, with_events=True)
+    ms, clocks = run_timed(world, graphs, args.steps, args.warmup, sampler_index=local)
+    kms = per_kernel_ms(events, len(cases))
+    ms_max = max_over_ranks(world, ms)
+    total_bytes = sum_over_ranks(world, bytes_step * args.steps)
+    total_flops = sum_over_ranks(world, flops_step * args.steps)
+    sec = ms_max / 1e3
+    if half == "hbm":
+        value, unit = total_bytes / sec / 1e9, "GB/s"
+    else:
+        value, unit = total_flops / sec / 1e12, "TFLOP/s"
+
+    plans = [w4.plan(M, c.N, c.K, g, sym) for c in cases]
+    kernel_name = "gemv_decode_kernel" if plans[0]["path"] == "decode" else "gemm_tc_kernel"
+    k_bytes = sum(c.bytes for c in cases)
+    k_flops = sum(c.flops for c in cases)
+    k_sec = sum(kms) / 1e3
+    if half == "hbm":
+        achieved = k_bytes / k_sec / 1e9
+        roof = {"bound": "hbm", "achieved": achieved, "peak": peaks["hbm_gbs"], "unit": "GB/s",
+                "frac": achieved / peaks["hbm_gbs"], "peak_source": peak_src}
+    else:
+        achieved = k_flops / k_sec / 1e12
+        pk = peaks["bf16_tflops"]
+        roof = {"bound": "tensor", "achieved": achieved, "peak": pk, "unit": "TFLOP/s",
+                "frac": achieved / pk, "peak_source": peak_src + " (burst)"}
+    traffic = ncu_traffic(f"{kernel_name}:{args.workload}")
+    roof["traffic"] = traffic
+    roof["kernel"] = kernel_name
+    roof["per_launch_us"] = [round(x * 1e3, 3) for x in kms]
+    roof["algorithmic_bytes_per_launch"] = [c.bytes for c in cases]
+
+    line = {
+        "metric": METRIC, "value": value, "unit": unit, "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": ms_max / args.steps, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+        "config": {
+            "workload": f"{wl.name}_M{M}", "M": M,
+            "layers_KxN": [[l.K, l.N] for l in wl.layers], "g": g,
+            "mode": "sym" if sym else "asym", "description": wl.description,
+            "l2": f"{copies} rotating copies of weights+activations "
+                  f"({copies * in_bytes_step / 2**20:.0f} MiB, > 2x L2 of {l2 / 2**20:.0f} MiB)",
+            "parallelism": f"replicas x{world} (independent problems, no collective)",
+            "plan": plans, "algorithmic_bytes_per_step": bytes_step,
+            "flops_per_step": flops_step,
+        },
+        "roofline": roof,
+        "gpu_launches": len(cases) * args.steps,
+        "clocks": clocks,
+    }
+
+    # ------------------------------------------------ end to end through the public API
+    pinned = [c.X[0].cpu().pin_memory() for c in cases]
+    h2d = sum(x.numel() * 2 for x in pinned)
+    d2h = sum(c.M * c.N * 2 for c in cases)
+    e2e_steps = min(args.steps, 200)
+
+    def e2e_step(i):
+        for c, xh in zip(cases, pinned):
+            j = i % copies
+            w4.gemm(xh, c.P[j], c.S[j], c.Z[j], c.g, c.sym)   # host X in, host Y out
+
+    for i in range(args.warmup):
+        e2e_step(i)
+    torch.cuda.synchronize()
+    barrier(world)
+    torch.cuda.synchronize()
+    a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    a.record()
+    for i in range(e2e_steps):
+        e2e_step(i)
+    b.record()
+    b.synchronize()
+    barrier(world)
+    e2e_ms = max_over_ranks(world, a.elapsed_time(b))
+    e2e_total = sum_over_ranks(world, (bytes_step if half == "hbm" else flops_step) * e2e_steps)
+    e2e_val = e2e_total / (e2e_ms / 1e3) / (1e9 if half == "hbm" else 1e12)
+    line["e2e"] = {"value": e2e_val, "unit": unit, "h2d_bytes_per_step": h2d,
+                   "d2h_bytes_per_step": d2h, "steps": e2e_steps,
+                   "ms_per_step": e2e_ms / e2e_steps}
+
+    # ------------------------------------------------ comparisons and the other metric half
+    if not args.no_extras:
+        line["comparisons"] = comparisons(w4, cases, copies, l2, half)
+        if args.workload != "prefill":
+            line["prefill"] = prefill_extra(w4, peaks, peak_src, l2, dev)
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        cb = cpu_baseline(wl.layers, M, g, sym, unit_bytes=(half == "hbm")) \
+            if half == "hbm" else cpu_baseline_sampled(wl.layers[0], M, g, sym, rows=16)
+        line["cpu_baseline"] = cb
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        import torch.distributed as dist
+        del graphs
+        torch.cuda.synchronize()
+        dist.destroy_process_group()
+
+
+def comparisons(w4, cases, copies, l2, half):
+    """Dense bf16 cuBLAS GEMM and the unfused dequantize-then-GEMM at the same
+    shapes, timed the same way (graphs, rotation past L2)."""
+    out = {}
+    dense_bytes = sum(c.N * c.K * 2 for c in cases)
+    dcopies = max(2, -(-2 * l2 // dense_bytes) + 1)
+    Wd = [[c.W_dense] + [c.W_dense.clone() for _ in range(dcopies - 1)] for c in cases]
+
+    def dense(i):
+        for c, ws in zip(cases, Wd):
+            torch.matmul(c.X[0], ws[i % dcopies].t(), out=c.Y[0])
+
+    gs = graph_of(dense, dcopies)
+    ms = time_graphs(gs, 200)
+    out["dense_bf16_cublas"] = {"ms_per_step": ms, "bytes_per_step": dense_bytes}
+    del gs
+    Wh = [torch.empty_like(c.W_dense) for c in cases]
+
+    def unfused(i):
+        for c, wh in zip(cases, Wh):
+            j = i % copies
+            w4.dequantize(c.P[j], c.S[j], c.Z[j], c.g, c.sym, out=wh)
+            torch.matmul(c.X[j], wh.t(), out=c.Y[j])
+
+    gs = graph_of(unfused, copies)
+    out["unfused_dequant_then_cublas"] = {"ms_per_step": time_graphs(gs, 100)}
+    del gs
+    fused = graph_of(lambda i: [c.call(w4, i) for c in cases], copies)
+    out["fused_w4a16"] = {"ms_per_step": time_graphs(fused, 200)}
+    out["speedup_vs_dense"] = out["dense_bf16_cublas"]["ms_per_step"] / out["fused_w4a16"]["ms_per_step"]
+    out["speedup_vs_unfused"] = (out["unfused_dequant_then_cublas"]["ms_per_step"] /
+                                 out["fused_w4a16"]["ms_per_step"])
+    del Wd
+    torch.cuda.empty_cache()
+    return out
+
+
+def prefill_extra(w4, peaks, peak_src, l2, dev, iters=50):
+    """The metric's other half: TFLOPS at M=2048, K=N=8192 (g=128, asym)."""
+    layer = workloads.PREFILL.layers[0]
+    M = 2048
+    in_bytes = layer.N * layer.K // 2 + 4 * layer.N * (layer.K // 128) + 2 * M * layer.K
+    copies = copies_for(in_bytes, l2)
+    case = GemmCase(w4, layer, M, 128, False, copies, dev)
+    graphs, events = capture_step_graphs(w4, [case], copies, with_events=True)
+    for s in range(3):
+        graphs[s % copies].replay()
+    torch.cuda.synchronize()
+    a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    a.record()
+    for s in range(iters):
+        graphs[s % copies].replay()
+    b.record()
+    b.synchronize()
+    ms = a.elapsed_time(b) / iters
+    kms = per_kernel_ms(events, 1)[0]
+    tflops = case.flops / (kms / 1e3) / 1e12
+    pk = peaks["bf16_tflops"]
+    res = {"workload": "prefill_2048x8192x8192_g128_asym", "ms_per_step": ms,
+           "TFLOP/s": case.flops / (ms / 1e3) / 1e12,
+           "roofline": {"bound": "tensor", "achieved": tflops, "peak": pk, "unit": "TFLOP/s",
+                        "frac": tflops / pk, "peak_source": peak_src + " (burst)",
+                        "traffic": ncu_traffic("gemm_tc_kernel:prefill"),
+                        "kernel": "gemm_tc_kernel", "per_launch_us": kms * 1e3},
+           "plan": w4.plan(M, layer.N, layer.K, 128, False)}
+    dcopies = max(2, -(-2 * l2 // (layer.N * layer.K * 2 + 2 * M * layer.K)) + 1)
+    Wd = [case.W_dense] + [case.W_dense.clone() for _ in range(dcopies - 1)]
+    Xd = [case.X[0]] + [case.X[0].clone() for _ in range(dcopies - 1)]
+    gs = graph_of(lambda i: torch.matmul(Xd[i % dcopies], Wd[i % dcopies].t(), out=case.Y[0]),
+                  dcopies)
+    dms = time_graphs(gs, iters)
+    res["dense_bf16_cublas"] = {"ms_per_step": dms, "TFLOP/s": case.flops / (dms / 1e3) / 1e12}
+    del gs, Wd, Xd, graphs, case
+    torch.cuda.empty_cache()
+    return res
+
+
+def run_reference(args):
+    """The reference arm: the host oracle as it stands, timed on this machine's
+    cores, on the same workload and metric; each step a bounded sample."""
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return
+    wl, M, g, sym, half = WORKLOAD_DEFS[args.workload]
+    if half == "hbm":
+        import oracle
+        oracle.build()
+        prepared = []
+        for layer in wl.layers:
+            Wb = workloads.bits(layer.weight())
+            Xb = workloads.bits(layer.activation(M))
+            P, S, Z = oracle.quantize(Wb, g, sym)
+            prepared.append((Xb, P, S, Z))
+        bytes_step = sum(algorithmic_bytes(M, l.N, l.K, g, sym) for l in wl.layers)
+        for _ in range(min(args.warmup, 1)):
+            for Xb, P, S, Z in prepared:
+                oracle.gemm_w4a16(Xb, P, S, Z, g, sym)
+        steps = max(1, min(args.steps, 20))
+        t0 = time.perf_counter()
+        for _ in range(steps):
+            for Xb, P, S, Z in prepared:
+                oracle.gemm_w4a16(Xb, P, S, Z, g, sym)
+        el = time.perf_counter() - t0
+        value, unit = bytes_step * steps / el / 1e9, "GB/s"
+        sample = f"{steps} full step(s): both layer GEMMs, dequantize + binary64 matmul"
+        cores = oracle.num_threads()
+    else:
+        cb = cpu_baseline_sampled(wl.layers[0], M, g, sym, rows=16)
+        steps, el = 1, cb["s_per_step"]
+        value, unit, sample, cores = cb["value"], cb["unit"], cb["sample"], cb["cores"]
+    line = {"impl": "reference", "metric": METRIC, "value": value, "unit": unit, "n_gpus": world,
+            "steps": steps, "warmup": args.warmup, "ms_per_step": el / steps * 1e3,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+            "data": "synthetic",
+            "config": {"workload": f"{wl.name}_M{M}", "M": M,
+                       "layers_KxN": [[l.K, l.N] for l in wl.layers], "g": g,
+                       "mode": "sym" if sym else "asym"},
+            "cpu_baseline": {"value": value, "unit": unit, "cores": cores, "kind": "oracle",
+                             "sample": sample},
+            "e2e": {"value": value, "unit": unit, "h2d_bytes_per_step": 0,
+                    "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+
+
+def main():
+    ap = argparse.ArgumentParser(description=__doc__.split("\n")[0])
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=50000)
+    ap.add_argument("--warmup", type=int, default=50)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--workload", choices=sorted(WORKLOAD_DEFS), default="decode7b")
+    ap.add_argument("--no-extras", action="store_true",
+                    help="skip comparisons and the prefill half (profiling runs)")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    if args.warmup < 3:
+        ap.error("--warmup must be at least 3")
+    if args.impl == "reference":
+        run_reference(args)
+    else:
+        run_ours(args)
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,166 @@
+/*
+ * w4a16.h — C ABI of the B200 (sm_100a) W4A16 weight-only RTN library.
+ *
+ * W4A16: weights stored as 4-bit integer codes, activations kept in 16-bit
+ * floating point (bf16 here).  The method, as the pages describe it:
+ *
+ *  - qwbw.cn, "推理优化中“用精度换性能“的核心技术：量化":
+ *      §2.2  INT4 holds [−8, 7] or [0, 15];
+ *      §2.3  x_int = round(x_float / s) + z,  x̂_float = (x_int − z) × s;
+ *      §3.3  symmetric:  s = max|x| / max_int, z = 0;
+ *            asymmetric: s = (max(x) − min(x)) / (2^b − 1), z = round(−min(x)/s);
+ *      §3.4  group-wise granularity: each group of 128 weights shares one
+ *            16-bit scale and an optional 16-bit zero point (4.25 bits/weight);
+ *      §3.2  weight-only inference: load INT4 from memory, dequantize to
+ *            16-bit, multiply with 16-bit activations.
+ *  - meko1.github.io, "量化实战深入（GPTQ / AWQ / SmoothQuant / KV 量化）",
+ *      §二  q = round(x/s) + z, x ≈ s·(q − z); absmax s = max|x| / (2^(b−1) − 1);
+ *           per-group = one scale per 128 elements.
+ *  - offer.aigcbaba.com, "大模型推理中 Weight-only、W8A8 和 FP8 量化有什么区别？",
+ *      §二  a fused kernel reads INT4, unpacks and scales in registers or shared
+ *           memory, and multiplies with the high-precision activations.
+ *  - mianshidashi.cn, "LLM 量化中 W4A16 表示什么…", 显存收益主要来自权重 / 性能取决于 kernel:
+ *           0.5 byte per INT4 weight; dequantize inside the GEMM while reading
+ *           INT4, rather than expanding the whole matrix first.
+ *
+ * Readings fixed by this library where the pages leave a step open:
+ *  round() is round-half-to-even in binary32; s is computed in binary32 and
+ *  rounded to bf16, and z and q use that bf16 s; codes are clamped to the INT4
+ *  range; the asymmetric range is widened to contain 0 (so z is an integer in
+ *  [0, 15] and 0 is on the grid); a group whose s rounds to 0 gets z = q = 0;
+ *  symmetric codes are 4-bit two's complement and s = max|x| / 7; groups run
+ *  along K (input channels); the dequantized weight is bf16_rn((q − z)·s).
+ *
+ * Layouts (all row-major, contiguous, every pointer 16-byte aligned):
+ *  W       bf16  [N, K]      weights, N = output features, K = input features
+ *  X       bf16  [M, K]      activations
+ *  Y       bf16  [M, N]      Y = X · Ŵᵀ, fp32 accumulation, rounded once to bf16
+ *  packed  uint8 [N, K/2]    byte i of a row holds element 2i in its low nibble
+ *                            and element 2i+1 in its high nibble
+ *  scales  bf16  [N, K/g]    one scale per group of g consecutive elements of a row
+ *  zeros   bf16  [N, K/g]    zero point per group (an integer 0..15 stored in bf16);
+ *                            all 0 in symmetric mode
+ *
+ * Supported: g ∈ {32, 64, 128}, K a positive multiple of g, N ≥ 0, M ≥ 0
+ * (M = 0 or N = 0 is a no-op), N, K, M < 2^31.  Every pointer is a DEVICE
+ * pointer owned by the caller; the library allocates no device memory and keeps
+ * no state beyond per-device constants (device properties, tensor-map encoder).
+ * Each call is asynchronous on `stream` (a cudaStream_t; NULL = legacy default
+ * stream).  Arguments are checked on the host before any launch; a rejected
+ * call launches nothing and returns W4A16_EINVAL.  No call aborts, throws or
+ * falls back to the CPU.
+ */
+#ifndef W4A16_H_
+#define W4A16_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#define W4A16_ABI_VERSION 1
+
+typedef enum w4a16_status {
+    W4A16_OK = 0,
+    W4A16_EINVAL = 1,        /* bad size, group, mode, alignment or null pointer; nothing launched */
+    W4A16_EUNSUPPORTED = 2,  /* valid request the current device cannot run (needs sm_100) */
+    W4A16_ECUDA = 3,         /* the CUDA runtime reported an error while launching */
+    W4A16_EWORKSPACE = 4,    /* workspace smaller than w4a16_gemm_workspace_size() */
+    W4A16_EDEVICE = 5        /* a kernel gave up a bounded wait (see w4a16_device_error) */
+} w4a16_status;
+
+/* GEMM kernel choice (roofline-driven: decode is weight-bandwidth bound, prefill
+ * is tensor-core bound — Quantization & Acceleration page, 关键判据; the
+ * aigcbaba selection page, §二 and §五). */
+typedef enum w4a16_path {
+    W4A16_PATH_AUTO = 0,       /* choose from (M, N, K, g) */
+    W4A16_PATH_DECODE = 1,     /* small-M split-K kernel: 128-bit packed loads, in-register
+                                  dequantization, bf16 MMA with fp32 accumulation, split-K
+                                  partial sums reduced through thread-block-cluster shared
+                                  memory; supports M ≤ 16 */
+    W4A16_PATH_TENSORCORE = 2  /* large-M kernel: TMA-fed INT4 tile dequantized into shared
+                                  memory and fed to tcgen05 bf16 MMA with TMEM accumulators */
+} w4a16_path;
+
+/* The launch a GEMM call would make (filled by w4a16_gemm_plan). */
+typedef struct w4a16_plan {
+    int32_t path;        /* w4a16_path actually used (never AUTO) */
+    int32_t split_k;     /* decode: CTAs per cluster splitting K (1..8) */
+    int32_t tile_m;      /* tensor-core: activation rows per CTA tile (32/64/128/256);
+                            decode: 8 or 16 (MMA columns) */
+    int32_t tile_n;      /* output features per CTA tile */
+    int64_t grid;        /* CTAs launched */
+    int32_t threads;     /* threads per CTA */
+    int32_t smem_bytes;  /* dynamic shared memory per CTA */
+} w4a16_plan;
+
+/* Quantize W[N, K] group-wise by RTN (asymmetric when sym == 0, symmetric when
+ * sym == 1) and pack two codes per byte.
+ *   W       in   bf16 [N, K]
+ *   packed  out  uint8 [N, K/2]
+ *   scales  out  bf16 [N, K/g]
+ *   zeros   out  bf16 [N, K/g]; may be NULL when sym == 1 (else written as 0)
+ * Inputs must be finite.  Bit-exact with the host oracle. */
+w4a16_status w4a16_quantize(const void* W, int64_t N, int64_t K, int32_t g, int32_t sym,
+                            void* packed, void* scales, void* zeros, void* stream);
+
+/* Expand packed codes to Ŵ[n, k] = bf16_rn((q − z)·s) (qwbw.cn page §2.3).
+ * This is the unfused form the fused GEMM avoids; it is provided for checking
+ * and for callers that need Ŵ.
+ *   packed, scales in; zeros in (ignored, may be NULL, when sym == 1)
+ *   W_hat   out  bf16 [N, K] */
+w4a16_status w4a16_dequantize(const void* packed, const void* scales, const void* zeros,
+                              int64_t N, int64_t K, int32_t g, int32_t sym, void* W_hat,
+                              void* stream);
+
+/* Bytes of device workspace w4a16_gemm needs for this shape.  Every current
+ * kernel reduces split-K partial sums on chip, so this returns 0; the argument
+ * pair stays in the ABI so a future kernel can ask for scratch. */
+size_t w4a16_gemm_workspace_size(int64_t M, int64_t N, int64_t K, int32_t g);
+
+/* Fused W4A16 GEMM: Y[M, N] = X[M, K] · Ŵ[N, K]ᵀ with Ŵ = bf16_rn((q − z)·s)
+ * formed in registers/shared memory from the packed codes, fp32 accumulation,
+ * one rounding of each output to bf16.  Never materialises Ŵ in global memory.
+ *   X in bf16 [M, K]; packed/scales/zeros as produced by w4a16_quantize
+ *   (zeros ignored, may be NULL, when sym == 1); Y out bf16 [M, N].
+ *   workspace/workspace_bytes: device scratch of at least
+ *   w4a16_gemm_workspace_size() bytes (may be NULL/0 when that is 0).
+ * Results are deterministic: the same inputs give bitwise-equal Y. */
+w4a16_status w4a16_gemm(const void* X, int64_t M, int64_t K, const void* packed,
+                        const void* scales, const void* zeros, int64_t N, int32_t g,
+                        int32_t sym, void* Y, void* workspace, size_t workspace_bytes,
+                        void* stream);
+
+/* w4a16_gemm with the dispatch decision overridden: `path` forces a kernel
+ * (AUTO = same as w4a16_gemm) and `split_k` (decode only, 0 = automatic,
+ * else 1..8) forces the number of CTAs splitting K.  Used by tests, benchmarks
+ * and profiling to exercise both kernels at the same shape.  Returns
+ * W4A16_EINVAL if the forced kernel cannot run the shape (e.g. DECODE with M > 16). */
+w4a16_status w4a16_gemm_ex(const void* X, int64_t M, int64_t K, const void* packed,
+                           const void* scales, const void* zeros, int64_t N, int32_t g,
+                           int32_t sym, void* Y, void* workspace, size_t workspace_bytes,
+                           int32_t path, int32_t split_k, void* stream);
+
+/* Host-only: report the launch w4a16_gemm_ex would make (no device access).
+ * Returns W4A16_EINVAL for shapes or forced paths it would reject. */
+w4a16_status w4a16_gemm_plan(int64_t M, int64_t N, int64_t K, int32_t g, int32_t sym,
+                             int32_t path, int32_t split_k, w4a16_plan* plan);
+
+/* Read and clear the current device's error word, written by a kernel that gave
+ * up a bounded wait (a pipeline barrier that did not complete within about one
+ * second).  *code = 0 when no kernel reported one.  Synchronizes the device. */
+w4a16_status w4a16_device_error(int32_t* code);
+
+/* Human-readable name of a status code (static string, never NULL). */
+const char* w4a16_status_string(w4a16_status status);
+
+/* W4A16_ABI_VERSION of the loaded library. */
+int32_t w4a16_abi_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* W4A16_H_ */

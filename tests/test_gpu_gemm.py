@@ -1,0 +1,189 @@
+"""GPU parity of the fused W4A16 GEMM against the oracle.
+
+Y is compared with the oracle's binary64 matmul Y64 over the dequantized
+weights: max|Y − Y64| ≤ 4e-3·max|Y64| and ‖Y − bf16(Y64)‖_F ≤ 1e-3·‖bf16(Y64)‖_F
+(tests/helpers.py explains which reference each bar uses).  Where a result is exact (one-hot activations
+select single dequantized weights) the comparison is bit-exact.  Both kernels
+(decode and tensor-core) are forced at the same shapes; the full-size
+workloads run in the launch configuration the benchmark times and are checked
+on sampled outputs the oracle computes one by one."""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+import workloads
+import weight_only_quantization_rtn_b200 as w4
+from weight_only_quantization_rtn_b200 import build as w4build
+from helpers import assert_y_close
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module", autouse=True)
+def _built():
+    w4build.build()
+    oracle.build()
+    yield
+    assert w4.device_error() == 0
+
+
+def _quantized(N, K, g, sym, seed, outlier=True):
+    W = workloads.make_weight(N, K, 0.02, seed, outlier_frac=0.01 if outlier else 0.0,
+                              outlier_scale=20.0)
+    Wd = W.cuda()
+    P, S, Z = w4.quantize(Wd, g, sym)
+    return P, S, Z
+
+
+def _check_full(M, N, K, g, sym, path, seed=0, split_k=0, x_outliers=True):
+    P, S, Z = _quantized(N, K, g, sym, seed)
+    X = workloads.make_activation(M, K, seed + 1, outlier_frac=0.01 if x_outliers else 0.0,
+                                  outlier_mode="set")
+    Y = w4.gemm(X.cuda(), P, S, Z, g, sym, path=path, split_k=split_k)
+    torch.cuda.synchronize()
+    Y64 = oracle.gemm_w4a16(workloads.bits(X), P.cpu().numpy(), workloads.bits(S),
+                            workloads.bits(Z), g, sym)
+    assert_y_close(workloads.bits(Y), Y64, f"M={M} N={N} K={K} g={g} sym={sym} {path}")
+    return Y
+
+
+# ------------------------------------------------------------------ small shapes, both paths
+DECODE_SHAPES = [(1, 256, 256), (1, 1, 128), (2, 37, 384), (3, 100, 1152), (5, 64, 32 * 7),
+                 (8, 128, 4096), (9, 96, 640), (13, 257, 1024), (16, 512, 2048)]
+
+
+@pytest.mark.parametrize("sym", [False, True])
+@pytest.mark.parametrize("g", [32, 64, 128])
+@pytest.mark.parametrize("M,N,K", DECODE_SHAPES)
+def test_decode_path_small(M, N, K, g, sym):
+    if K % g:
+        pytest.skip("K not a multiple of g")
+    _check_full(M, N, K, g, sym, "decode", seed=M + N + K)
+
+
+@pytest.mark.parametrize("split_k", [1, 2, 3, 5, 8])
+def test_decode_forced_split_k(split_k):
+    _check_full(4, 300, 8 * 128 * 3, 128, False, "decode", seed=5, split_k=split_k)
+
+
+TC_SHAPES = [(1, 128, 64 * 3), (17, 200, 256), (32, 128, 128), (33, 384, 512), (64, 129, 96),
+             (100, 256, 1024), (128, 640, 320), (200, 128, 2048), (256, 256, 256),
+             (257, 384, 768), (300, 130, 128 * 5), (600, 1000, 1024)]
+
+
+@pytest.mark.parametrize("sym", [False, True])
+@pytest.mark.parametrize("g", [32, 64, 128])
+@pytest.mark.parametrize("M,N,K", TC_SHAPES)
+def test_tensorcore_path_small(M, N, K, g, sym):
+    if K % g:
+        pytest.skip("K not a multiple of g")
+    _check_full(M, N, K, g, sym, "tensorcore", seed=M * 3 + N + K)
+
+
+# ------------------------------------------------------------------ exact special cases
+@pytest.mark.parametrize("path", ["decode", "tensorcore"])
+@pytest.mark.parametrize("sym", [False, True])
+@pytest.mark.parametrize("g", [32, 128])
+def test_one_hot_activations_select_dequantized_weights_bit_exact(path, sym, g):
+    """X = one-hot rows: Y[m, n] = Ŵ[n, k_m] exactly (a single nonzero product,
+    exact in fp32, and already a bf16 value), so the fused dequantization of
+    every code position is checked bit for bit."""
+    N, K = 160, 512
+    P, S, Z = _quantized(N, K, g, sym, seed=11)
+    Wh = w4.dequantize(P, S, Z, g, sym)
+    ks = torch.arange(0, K, dtype=torch.long)
+    for start in range(0, K, 16):
+        kk = ks[start:start + 16]
+        X = torch.zeros(kk.numel(), K, dtype=torch.bfloat16)
+        X[torch.arange(kk.numel()), kk] = 1.0
+        Y = w4.gemm(X.cuda(), P, S, Z, g, sym, path=path)
+        assert torch.equal(Y, Wh[:, kk.cuda()].t().contiguous()), f"k in {start}..{start + 15}"
+
+
+@pytest.mark.parametrize("path", ["decode", "tensorcore"])
+def test_deterministic_bitwise(path):
+    P, S, Z = _quantized(1000, 4096, 128, False, seed=3)
+    X = workloads.make_activation(16, 4096, 4).cuda()
+    ys = [w4.gemm(X, P, S, Z, 128, False, path=path) for _ in range(3)]
+    assert all(torch.equal(ys[0], y) for y in ys[1:])
+
+
+def test_paths_agree_closely():
+    P, S, Z = _quantized(384, 2048, 64, True, seed=8)
+    X = workloads.make_activation(16, 2048, 9, outlier_frac=0.01, outlier_mode="set").cuda()
+    a = w4.gemm(X, P, S, Z, 64, True, path="decode").float()
+    b = w4.gemm(X, P, S, Z, 64, True, path="tensorcore").float()
+    assert torch.max(torch.abs(a - b)) <= 4e-3 * torch.max(torch.abs(a))
+
+
+def test_empty_problems_are_noops():
+    P, S, Z = _quantized(64, 256, 128, False, seed=1)
+    Y = w4.gemm(torch.empty(0, 256, dtype=torch.bfloat16, device="cuda"), P, S, Z, 128, False)
+    assert Y.shape == (0, 64)
+
+
+def test_host_buffers_end_to_end():
+    P, S, Z = _quantized(256, 512, 128, False, seed=12)
+    X = workloads.make_activation(2, 512, 13).pin_memory()
+    Y = w4.gemm(X, P, S, Z, 128, False)
+    assert not Y.is_cuda
+    Yd = w4.gemm(X.cuda(), P, S, Z, 128, False)
+    assert torch.equal(Y, Yd.cpu())
+
+
+# ------------------------------------------------------------------ full-size workloads
+def _check_sampled(layer, M, g, sym, path="auto", n_samples=3072, seed=0):
+    W = layer.weight()
+    X = layer.activation(M)
+    P, S, Z = w4.quantize(W.cuda(), g, sym)
+    Y = w4.gemm(X.cuda(), P, S, Z, g, sym, path=path)
+    torch.cuda.synchronize()
+    rng = np.random.default_rng(seed + M)
+    N = layer.N
+    ms = rng.integers(0, M, n_samples)
+    ns = rng.integers(0, N, n_samples)
+    # always include the first and last rows/columns
+    ms[:4] = [0, M - 1, 0, M - 1]
+    ns[:4] = [0, 0, N - 1, N - 1]
+    ref = oracle.gemm_sampled(workloads.bits(X), P.cpu().numpy(), workloads.bits(S),
+                              workloads.bits(Z), g, sym, ms, ns)
+    got = workloads.bits(Y)[ms, ns]
+    assert_y_close(got, ref, f"{layer.name} M={M} g={g} sym={sym}")
+
+
+@pytest.mark.parametrize("M", workloads.DECODE_7B.Ms)
+@pytest.mark.parametrize("li", [0, 1])
+def test_7b_decode_full_size(li, M):
+    _check_sampled(workloads.DECODE_7B.layers[li], M, 128, False)
+
+
+@pytest.mark.parametrize("sym", [False, True])
+@pytest.mark.parametrize("M", workloads.DECODE_70B.Ms)
+@pytest.mark.parametrize("li", [0, 1])
+def test_70b_decode_full_size(li, M, sym):
+    _check_sampled(workloads.DECODE_70B.layers[li], M, 128, sym)
+
+
+def test_prefill_full_size():
+    _check_sampled(workloads.PREFILL.layers[0], 2048, 128, False, n_samples=4096)
+
+
+@pytest.mark.parametrize("M,g,sym", [(1, 32, False), (2, 64, True), (16, 128, False),
+                                     (32, 32, True), (64, 64, False), (128, 128, True),
+                                     (256, 32, False), (512, 64, True), (1024, 128, False),
+                                     (4096, 32, True)])
+def test_crossover_full_size(M, g, sym):
+    _check_sampled(workloads.CROSSOVER.layers[0], M, g, sym, n_samples=2048)
+
+
+def test_tiny_config_full_compare():
+    layer = workloads.TINY.layers[0]
+    for path in ("decode", "tensorcore"):
+        W = layer.weight()
+        X = layer.activation(1)
+        P, S, Z = w4.quantize(W.cuda(), 128, False)
+        Y = w4.gemm(X.cuda(), P, S, Z, 128, False, path=path)
+        ref = oracle.gemm_w4a16(workloads.bits(X), P.cpu().numpy(), workloads.bits(S),
+                                workloads.bits(Z), 128, False)
+        assert_y_close(workloads.bits(Y), ref, f"tiny {path}")

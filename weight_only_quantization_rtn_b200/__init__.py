@@ -1,0 +1,213 @@
+"""W4A16 weight-only RTN quantization and fused INT4 x bf16 GEMM for B200 (sm_100a).
+
+A thin binding over the C ABI in ``include/w4a16.h`` (``libw4a16.so``, built
+in-tree by ``python -m weight_only_quantization_rtn_b200.build``).  PyTorch is
+used only for device memory and the current CUDA stream; every step of the
+computation runs in the library's CUDA kernels.  There is no CPU fallback:
+the first call raises ImportError if the library is missing.
+
+    packed, scales, zeros = quantize(W, g=128, sym=False)   # W: bf16 [N, K] on cuda
+    Y = gemm(X, packed, scales, zeros, g=128, sym=False)      # X: bf16 [M, K] -> Y [M, N]
+    W_hat = dequantize(packed, scales, zeros, g=128, sym=False)
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+
+import torch
+
+__all__ = ["lib", "quantize", "dequantize", "gemm", "plan", "workspace_size", "device_error",
+           "W4A16Error", "PATH_AUTO", "PATH_DECODE", "PATH_TENSORCORE", "LIB_PATH"]
+
+LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libw4a16.so")
+
+PATH_AUTO, PATH_DECODE, PATH_TENSORCORE = 0, 1, 2
+_PATHS = {"auto": PATH_AUTO, "decode": PATH_DECODE, "tensorcore": PATH_TENSORCORE}
+_STATUS = {0: "OK", 1: "EINVAL", 2: "EUNSUPPORTED", 3: "ECUDA", 4: "EWORKSPACE", 5: "EDEVICE"}
+
+
+class W4A16Error(RuntimeError):
+    def __init__(self, status: int, what: str):
+        self.status = status
+        super().__init__(f"{what}: {lib().w4a16_status_string(status).decode()}")
+
+
+class Plan(ctypes.Structure):
+    _fields_ = [("path", ctypes.c_int32), ("split_k", ctypes.c_int32),
+                ("tile_m", ctypes.c_int32), ("tile_n", ctypes.c_int32),
+                ("grid", ctypes.c_int64), ("threads", ctypes.c_int32),
+                ("smem_bytes", ctypes.c_int32)]
+
+
+def _load() -> ctypes.CDLL:
+    if not os.path.exists(LIB_PATH):
+        raise ImportError(f"W4A16 CUDA library not built: {LIB_PATH} is missing "
+                          "(run `python -m weight_only_quantization_rtn_b200.build`)")
+    lib = ctypes.CDLL(LIB_PATH)
+    vp, i64, i32, sz = ctypes.c_void_p, ctypes.c_int64, ctypes.c_int32, ctypes.c_size_t
+    lib.w4a16_quantize.argtypes = [vp, i64, i64, i32, i32, vp, vp, vp, vp]
+    lib.w4a16_dequantize.argtypes = [vp, vp, vp, i64, i64, i32, i32, vp, vp]
+    lib.w4a16_gemm_workspace_size.argtypes = [i64, i64, i64, i32]
+    lib.w4a16_gemm_workspace_size.restype = sz
+    lib.w4a16_gemm.argtypes = [vp, i64, i64, vp, vp, vp, i64, i32, i32, vp, vp, sz, vp]
+    lib.w4a16_gemm_ex.argtypes = [vp, i64, i64, vp, vp, vp, i64, i32, i32, vp, vp, sz, i32, i32,
+                                  vp]
+    lib.w4a16_gemm_plan.argtypes = [i64, i64, i64, i32, i32, i32, i32, ctypes.POINTER(Plan)]
+    lib.w4a16_device_error.argtypes = [ctypes.POINTER(ctypes.c_int32)]
+    lib.w4a16_status_string.argtypes = [ctypes.c_int]
+    lib.w4a16_status_string.restype = ctypes.c_char_p
+    lib.w4a16_abi_version.restype = ctypes.c_int32
+    for name in ("w4a16_quantize", "w4a16_dequantize", "w4a16_gemm", "w4a16_gemm_ex",
+                 "w4a16_gemm_plan", "w4a16_device_error"):
+        getattr(lib, name).restype = ctypes.c_int
+    return lib
+
+
+_lib = None
+
+
+def lib() -> ctypes.CDLL:
+    """The loaded C library; raises ImportError if it has not been built."""
+    global _lib
+    if _lib is None:
+        _lib = _load()
+    return _lib
+
+
+def _check(status: int, what: str) -> None:
+    if status != 0:
+        raise W4A16Error(status, what)
+
+
+def _ptr(t: torch.Tensor | None):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _stream(dev: torch.device):
+    return ctypes.c_void_p(torch.cuda.current_stream(dev).cuda_stream)
+
+
+def _need(t: torch.Tensor, dtype: torch.dtype, name: str, ndim: int = 2) -> None:
+    if not isinstance(t, torch.Tensor):
+        raise TypeError(f"{name} must be a torch.Tensor")
+    if t.dtype != dtype:
+        raise TypeError(f"{name} must be {dtype}, got {t.dtype}")
+    if t.dim() != ndim:
+        raise ValueError(f"{name} must be {ndim}-D, got shape {tuple(t.shape)}")
+    if not t.is_cuda:
+        raise ValueError(f"{name} must be on a CUDA device")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+
+
+def quantize(W: torch.Tensor, g: int = 128, sym: bool = False):
+    """Group-wise RTN quantization of W[N, K] (bf16, cuda).
+
+    Returns (packed uint8 [N, K/2], scales bf16 [N, K/g], zeros bf16 [N, K/g]);
+    zeros are all 0 when ``sym``."""
+    _need(W, torch.bfloat16, "W")
+    N, K = W.shape
+    if g <= 0 or K % g:
+        raise ValueError(f"K={K} must be a multiple of g={g}")
+    packed = torch.empty((N, K // 2), dtype=torch.uint8, device=W.device)
+    scales = torch.empty((N, K // g), dtype=torch.bfloat16, device=W.device)
+    zeros = torch.empty((N, K // g), dtype=torch.bfloat16, device=W.device)
+    with torch.cuda.device(W.device):
+        _check(lib().w4a16_quantize(_ptr(W), N, K, g, int(bool(sym)), _ptr(packed), _ptr(scales),
+                                   _ptr(zeros), _stream(W.device)), "w4a16_quantize")
+    return packed, scales, zeros
+
+
+def dequantize(packed: torch.Tensor, scales: torch.Tensor, zeros: torch.Tensor | None,
+               g: int = 128, sym: bool = False, out: torch.Tensor | None = None) -> torch.Tensor:
+    """Ŵ[N, K] = bf16_rn((q − z)·s), materialised (the unfused form)."""
+    _need(packed, torch.uint8, "packed")
+    _need(scales, torch.bfloat16, "scales")
+    if not sym:
+        _need(zeros, torch.bfloat16, "zeros")
+    N, K = packed.shape[0], packed.shape[1] * 2
+    if out is None:
+        W_hat = torch.empty((N, K), dtype=torch.bfloat16, device=packed.device)
+    else:
+        _need(out, torch.bfloat16, "out")
+        if tuple(out.shape) != (N, K):
+            raise ValueError("out has the wrong shape")
+        W_hat = out
+    with torch.cuda.device(packed.device):
+        _check(lib().w4a16_dequantize(_ptr(packed), _ptr(scales), _ptr(zeros if not sym else None),
+                                     N, K, g, int(bool(sym)), _ptr(W_hat),
+                                     _stream(packed.device)), "w4a16_dequantize")
+    return W_hat
+
+
+def workspace_size(M: int, N: int, K: int, g: int) -> int:
+    return int(lib().w4a16_gemm_workspace_size(M, N, K, g))
+
+
+def plan(M: int, N: int, K: int, g: int = 128, sym: bool = False, path: str | int = "auto",
+         split_k: int = 0) -> dict:
+    """The launch w4a16_gemm would make for this shape (host only)."""
+    p = Plan()
+    pid = _PATHS[path] if isinstance(path, str) else int(path)
+    _check(lib().w4a16_gemm_plan(M, N, K, g, int(bool(sym)), pid, split_k, ctypes.byref(p)),
+           "w4a16_gemm_plan")
+    return {"path": {v: k for k, v in _PATHS.items()}[p.path], "split_k": p.split_k,
+            "tile_m": p.tile_m, "tile_n": p.tile_n, "grid": p.grid, "threads": p.threads,
+            "smem_bytes": p.smem_bytes}
+
+
+_workspaces: dict = {}
+
+
+def gemm(X: torch.Tensor, packed: torch.Tensor, scales: torch.Tensor,
+         zeros: torch.Tensor | None, g: int = 128, sym: bool = False, path: str | int = "auto",
+         split_k: int = 0, out: torch.Tensor | None = None) -> torch.Tensor:
+    """Fused W4A16 GEMM: Y[M, N] = X[M, K] · Ŵ[N, K]ᵀ (bf16 in/out, fp32 accumulation).
+
+    If X lives in host memory (ideally pinned) it is copied to the weights'
+    device and Y is copied back to the host: the end-to-end form of the call."""
+    host_in = not X.is_cuda
+    dev = packed.device
+    if host_in:
+        Xd = X.to(dev, non_blocking=True)
+    else:
+        Xd = X
+    _need(Xd, torch.bfloat16, "X")
+    _need(packed, torch.uint8, "packed")
+    _need(scales, torch.bfloat16, "scales")
+    if not sym:
+        _need(zeros, torch.bfloat16, "zeros")
+    M, K = Xd.shape
+    N = packed.shape[0]
+    if packed.shape[1] * 2 != K:
+        raise ValueError(f"packed has K={packed.shape[1] * 2}, X has K={K}")
+    if out is None:
+        out = torch.empty((M, N), dtype=torch.bfloat16, device=dev)
+    else:
+        _need(out, torch.bfloat16, "out")
+        if tuple(out.shape) != (M, N):
+            raise ValueError("out has the wrong shape")
+    ws_bytes = workspace_size(M, N, K, g)
+    ws = None
+    if ws_bytes:
+        ws = _workspaces.get(dev)
+        if ws is None or ws.numel() < ws_bytes:
+            ws = torch.zeros(ws_bytes, dtype=torch.uint8, device=dev)
+            _workspaces[dev] = ws
+    pid = _PATHS[path] if isinstance(path, str) else int(path)
+    with torch.cuda.device(dev):
+        _check(lib().w4a16_gemm_ex(_ptr(Xd), M, K, _ptr(packed), _ptr(scales),
+                                  _ptr(zeros if not sym else None), N, g, int(bool(sym)),
+                                  _ptr(out), _ptr(ws), ws_bytes, pid, split_k, _stream(dev)),
+               "w4a16_gemm")
+    if host_in:
+        return out.to("cpu")
+    return out
+
+
+def device_error() -> int:
+    """Read and clear the device error word (0 = no kernel gave up a wait)."""
+    code = ctypes.c_int32(0)
+    _check(lib().w4a16_device_error(ctypes.byref(code)), "w4a16_device_error")
+    return int(code.value)

@@ -1,0 +1,139 @@
+// Quantize/pack and dequantize kernels (HBM-bound, one pass each).
+//
+// Quantization follows qwbw.cn, "推理优化中“用精度换性能“的核心技术：量化",
+// §2.3 (x_int = round(x/s) + z) and §3.3 (asymmetric s = (max − min)/(2^b − 1),
+// z = round(−min/s); symmetric s = max|x|/max_int, z = 0), with b = 4 and
+// groups of g elements along K (§3.4).  Arithmetic is binary32 with IEEE
+// round-to-nearest division (__fdiv_rn) and round-half-to-even (rintf); the
+// scale is rounded to bf16 before z and q are formed, the asymmetric range is
+// widened to contain 0, and codes are clamped to the INT4 range.
+#pragma once
+
+#include "common.cuh"
+
+namespace w4a16 {
+
+// Clamp in binary32 before converting to an integer.
+__device__ __forceinline__ float clampf(float r, float lo, float hi) {
+    return r < lo ? lo : (r > hi ? hi : r);
+}
+
+// One thread owns 8 consecutive elements (one 16-byte load, one 32-bit packed
+// store); TPG = G/8 consecutive lanes own one group and combine their min/max
+// with butterfly shuffles.  Loops are warp-uniform so every shuffle has all 32
+// lanes present.
+template <int G, bool SYM>
+__global__ void __launch_bounds__(256) quantize_pack_kernel(const uint16_t* __restrict__ W,
+                                                            int64_t total_chunks,
+                                                            uint32_t* __restrict__ packed32,
+                                                            uint16_t* __restrict__ scales,
+                                                            uint16_t* __restrict__ zeros) {
+    constexpr int TPG = G / 8;
+    const int lane = threadIdx.x & 31;
+    const int64_t warp0 = ((int64_t)blockIdx.x * blockDim.x + threadIdx.x) >> 5;
+    const int64_t nwarps = ((int64_t)gridDim.x * blockDim.x) >> 5;
+    for (int64_t base = warp0 * 32; base < total_chunks; base += nwarps * 32) {
+        const int64_t c = base + lane;
+        const bool valid = c < total_chunks;
+        uint4 v = make_uint4(0, 0, 0, 0);
+        if (valid) v = ldg_stream(W + c * 8);
+        const uint32_t wv[4] = {v.x, v.y, v.z, v.w};
+        float x[8];
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+            x[2 * i] = __uint_as_float(wv[i] << 16);
+            x[2 * i + 1] = __uint_as_float(wv[i] & 0xFFFF0000u);
+        }
+        uint32_t word = 0;
+        uint32_t s_bits;
+        int32_t z = 0;
+        if (!SYM) {
+            float mn = 0.0f, mx = 0.0f;                 // range widened to contain 0
+#pragma unroll
+            for (int i = 0; i < 8; ++i) {
+                mn = x[i] < mn ? x[i] : mn;
+                mx = x[i] > mx ? x[i] : mx;
+            }
+#pragma unroll
+            for (int o = 1; o < TPG; o <<= 1) {
+                const float omn = __shfl_xor_sync(0xffffffffu, mn, o);
+                const float omx = __shfl_xor_sync(0xffffffffu, mx, o);
+                mn = omn < mn ? omn : mn;
+                mx = omx > mx ? omx : mx;
+            }
+            const float s32 = __fdiv_rn(__fsub_rn(mx, mn), 15.0f);
+            s_bits = f32_to_bf16_bits_rn(s32);
+            const float s = bf16_bits_to_f32(s_bits);
+            if (s != 0.0f) {
+                z = (int32_t)clampf(rintf(__fdiv_rn(-mn, s)), 0.0f, 15.0f);
+#pragma unroll
+                for (int i = 0; i < 8; ++i) {
+                    const float r = clampf(rintf(__fdiv_rn(x[i], s)), -32.0f, 32.0f);
+                    int32_t q = (int32_t)r + z;
+                    q = q < 0 ? 0 : (q > 15 ? 15 : q);
+                    word |= (uint32_t)q << (4 * i);
+                }
+            }
+        } else {
+            float amax = 0.0f;
+#pragma unroll
+            for (int i = 0; i < 8; ++i) {
+                const float a = fabsf(x[i]);
+                amax = a > amax ? a : amax;
+            }
+#pragma unroll
+            for (int o = 1; o < TPG; o <<= 1) {
+                const float oa = __shfl_xor_sync(0xffffffffu, amax, o);
+                amax = oa > amax ? oa : amax;
+            }
+            const float s32 = __fdiv_rn(amax, 7.0f);
+            s_bits = f32_to_bf16_bits_rn(s32);
+            const float s = bf16_bits_to_f32(s_bits);
+            if (s != 0.0f) {
+#pragma unroll
+                for (int i = 0; i < 8; ++i) {
+                    const float r = clampf(rintf(__fdiv_rn(x[i], s)), -32.0f, 32.0f);
+                    int32_t q = (int32_t)r;
+                    q = q < -8 ? -8 : (q > 7 ? 7 : q);
+                    word |= ((uint32_t)q & 0xFu) << (4 * i);   // 4-bit two's complement
+                }
+            }
+        }
+        if (valid) {
+            packed32[c] = word;
+            if ((lane & (TPG - 1)) == 0) {
+                const int64_t grp = c / TPG;
+                scales[grp] = (uint16_t)s_bits;
+                if (zeros != nullptr) zeros[grp] = (uint16_t)f32_to_bf16_bits_rn((float)z);
+            }
+        }
+    }
+}
+
+// Ŵ = bf16_rn((q − z)·s): one thread expands 32 codes (one 16-byte load) into
+// 64 bytes of bf16; the 32 codes always lie in one group since g ≥ 32.
+template <int G, bool SYM>
+__global__ void __launch_bounds__(256) dequantize_kernel(const uint4* __restrict__ packed16,
+                                                         const uint16_t* __restrict__ scales,
+                                                         const uint16_t* __restrict__ zeros,
+                                                         int64_t total_chunks,
+                                                         uint4* __restrict__ W_hat) {
+    constexpr int CPG = G / 32;   // 32-code chunks per group
+    const int64_t stride = (int64_t)gridDim.x * blockDim.x;
+    for (int64_t c = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; c < total_chunks;
+         c += stride) {
+        const uint4 v = ldg_stream(packed16 + c);
+        const int64_t grp = c / CPG;
+        const uint32_t ss = dup16(ldg_u16(scales + grp));
+        const uint32_t zz = zero_pair<SYM>(SYM ? 0u : (uint32_t)ldg_u16(zeros + grp));
+        const uint32_t wv[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+            uint32_t d[4];
+            dequant8_natural<SYM>(wv[i], zz, ss, d);
+            W_hat[c * 4 + i] = make_uint4(d[0], d[1], d[2], d[3]);
+        }
+    }
+}
+
+}  // namespace w4a16
