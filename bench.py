@@ -15,11 +15,14 @@ TFLOPS (K=N=8192) with its tensor-core roofline, a dense bf16 cuBLAS GEMM and
 the unfused dequantize-then-GEMM at the same shapes, the end-to-end number
 through the public API with host buffers, and the host oracle on the CPU.
 
-Timing: W warm-up steps, then K steps replayed from CUDA graphs (one graph per
-rotation slot, so launch cost stays off the device timeline), bracketed by a
-barrier and torch.cuda.synchronize() on both sides, CUDA events on the
-launching stream.  Weight copies rotate so the bytes touched between reuses
-exceed twice the L2 size: every step streams its weights from HBM.
+Timing: W warm-up steps, then exactly K steps replayed from CUDA graphs (one
+graph holds a full rotation over the weight copies, so graph launches are
+amortized; leftover steps replay one-step graphs), bracketed by a barrier and
+torch.cuda.synchronize() on both sides, CUDA events on the launching stream.
+Weight copies rotate so the bytes touched between reuses exceed twice the L2
+size: every step streams its weights from HBM.  The timed region contains only
+the workload's GEMM launches, so the average launch duration behind the
+roofline figure is the region's time over its launches.
 """
 from __future__ import annotations
 
@@ -168,22 +171,33 @@ def barrier(world):
         dist.barrier()
 
 
-def max_over_ranks(world, value: float) -> float:
+def _reduce_scalar(world, value: float, op) -> float:
     if world == 1:
         return value
     import torch.distributed as dist
-    t = torch.tensor([value], dtype=torch.float64, device="cuda")
-    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    dev = "cuda" if dist.get_backend() == "nccl" else "cpu"
+    t = torch.tensor([value], dtype=torch.float64, device=dev)
+    dist.all_reduce(t, op=op)
     return float(t.item())
+
+
+def max_over_ranks(world, value: float) -> float:
+    """Timing is the slowest rank's: max of the per-rank device times."""
+    import torch.distributed as dist
+    return value if world == 1 else _reduce_scalar(world, value, dist.ReduceOp.MAX)
 
 
 def sum_over_ranks(world, value: float) -> float:
-    if world == 1:
-        return value
+    """Work is the whole job's: sum of the per-rank bytes or flops."""
     import torch.distributed as dist
-    t = torch.tensor([value], dtype=torch.float64, device="cuda")
-    dist.all_reduce(t, op=dist.ReduceOp.SUM)
-    return float(t.item())
+    return value if world == 1 else _reduce_scalar(world, value, dist.ReduceOp.SUM)
+
+
+def job_throughput(world, per_rank_work: float, per_rank_ms: float, scale: float) -> float:
+    """Whole-job throughput: all ranks' work over the max of their times."""
+    total = sum_over_ranks(world, per_rank_work)
+    ms = max_over_ranks(world, per_rank_ms)
+    return total / (ms / 1e3) / scale
 
 
 # ---------------------------------------------------------------------------- workloads
@@ -211,41 +225,54 @@ class GemmCase:
         w4.gemm(self.X[j], self.P[j], self.S[j], self.Z[j], self.g, self.sym, out=self.Y[j])
 
 
+def launches_per_call(plan: dict) -> int:
+    """Kernels one GEMM call launches: the decode path adds a fixup kernel when
+    its stream-K partition splits a row block (a host-side property of the plan)."""
+    return int(plan["kernels"])
+
+
 def copies_for(bytes_per_step: int, l2: int) -> int:
     return max(2, -(-2 * l2 // max(bytes_per_step, 1)) + 1)
 
 
-def capture_step_graphs(w4, cases, copies, with_events):
-    """One CUDA graph per rotation slot; each runs one step (every case once).
-    With events, external timing events bracket every GEMM inside the graph."""
-    graphs, events = [], []
+def capture_rotation_graph(w4, cases, copies):
+    """One CUDA graph holding a full rotation: `copies` steps, step i running
+    every case on weight copy i.  Replaying it back to back keeps consecutive
+    steps on different copies, and amortizes the graph launch over the steps."""
     stream = torch.cuda.Stream()
     stream.wait_stream(torch.cuda.current_stream())
     with torch.cuda.stream(stream):
-        for i in range(copies):          # compile plans and set kernel attributes before capture
+        for i in range(copies):          # plans, tensor maps and kernel attributes before capture
             for c in cases:
                 c.call(w4, i)
     torch.cuda.current_stream().wait_stream(stream)
     torch.cuda.synchronize()
+    rot = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(rot, stream=stream):
+        for i in range(copies):
+            for c in cases:
+                c.call(w4, i)
+    singles = []
     for i in range(copies):
         g = torch.cuda.CUDAGraph()
-        ev = [torch.cuda.Event(enable_timing=True, external=True) for _ in range(len(cases) + 1)]
         with torch.cuda.graph(g, stream=stream):
-            if with_events:
-                ev[0].record()
-            for ci, c in enumerate(cases):
+            for c in cases:
                 c.call(w4, i)
-                if with_events:
-                    ev[ci + 1].record()
-        graphs.append(g)
-        events.append(ev)
+        singles.append(g)
     torch.cuda.synchronize()
-    return graphs, events
+    return rot, singles
 
 
-def run_timed(world, graphs, steps, warmup, sampler_index=None):
-    for s in range(warmup):
-        graphs[s % len(graphs)].replay()
+def replay_steps(rot, singles, copies, steps):
+    """Exactly `steps` steps: whole rotations, then single steps for the rest."""
+    for _ in range(steps // copies):
+        rot.replay()
+    for i in range(steps % copies):
+        singles[i].replay()
+
+
+def run_timed(world, rot, singles, copies, steps, warmup, sampler_index=None):
+    replay_steps(rot, singles, copies, warmup)
     torch.cuda.synchronize()
     barrier(world)
     torch.cuda.synchronize()
@@ -255,8 +282,7 @@ def run_timed(world, graphs, steps, warmup, sampler_index=None):
     if sampler:
         sampler.__enter__()
     start.record()
-    for s in range(steps):
-        graphs[s % len(graphs)].replay()
+    replay_steps(rot, singles, copies, steps)
     end.record()
     end.synchronize()
     if sampler:
@@ -268,13 +294,22 @@ def run_timed(world, graphs, steps, warmup, sampler_index=None):
     return ms, (sampler.summary() if sampler else None)
 
 
-def per_kernel_ms(events, n_cases):
-    """Average duration of each case's GEMM over the last replay of every slot."""
-    out = [[] for _ in range(n_cases)]
-    for ev in events:
-        for ci in range(n_cases):
-            out[ci].append(ev[ci].elapsed_time(ev[ci + 1]))
-    return [statistics.mean(v) for v in out]
+def per_layer_ms(w4, cases, copies, reps=50):
+    """Diagnostic outside the timed region: each case alone, replayed from a
+    rotation graph, so its own average duration (launch gaps included)."""
+    out = []
+    for c in cases:
+        rot, singles = capture_rotation_graph(w4, [c], copies)
+        replay_steps(rot, singles, copies, copies * 3)
+        torch.cuda.synchronize()
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record()
+        replay_steps(rot, singles, copies, copies * reps)
+        b.record()
+        b.synchronize()
+        out.append(a.elapsed_time(b) / (copies * reps))
+        del rot, singles
+    return out
 
 
 def time_callable(fn, iters, warmup=3):
@@ -410,9 +445,8 @@ def run_ours(args):
                         for l in wl.layers)
     copies = copies_for(in_bytes_step, l2)
     cases = [GemmCase(w4, l, M, g, sym, copies, dev) for l in wl.layers]
-    graphs, events = capture_step_graphs(w4, cases, copies, with_events=True)
-    ms, clocks = run_timed(world, graphs, args.steps, args.warmup, sampler_index=local)
-    kms = per_kernel_ms(events, len(cases))
+    rot, singles = capture_rotation_graph(w4, cases, copies)
+    ms, clocks = run_timed(world, rot, singles, copies, args.steps, args.warmup, sampler_index=local)
     ms_max = max_over_ranks(world, ms)
     total_bytes = sum_over_ranks(world, bytes_step * args.steps)
     total_flops = sum_over_ranks(world, flops_step * args.steps)
@@ -421,25 +455,28 @@ def run_ours(args):
         value, unit = total_bytes / sec / 1e9, "GB/s"
     else:
         value, unit = total_flops / sec / 1e12, "TFLOP/s"
+    kms = per_layer_ms(w4, cases, copies)
 
     plans = [w4.plan(M, c.N, c.K, g, sym) for c in cases]
     kernel_name = "gemv_decode_kernel" if plans[0]["path"] == "decode" else "gemm_tc_kernel"
-    k_bytes = sum(c.bytes for c in cases)
-    k_flops = sum(c.flops for c in cases)
-    k_sec = sum(kms) / 1e3
+    # The timed region holds only this workload's GEMM launches, so the kernel's
+    # average launch duration is the region's time over its launches.
+    launches = len(cases) * args.steps
+    k_sec = (ms / 1e3) / args.steps
     if half == "hbm":
-        achieved = k_bytes / k_sec / 1e9
+        achieved = bytes_step / k_sec / 1e9
         roof = {"bound": "hbm", "achieved": achieved, "peak": peaks["hbm_gbs"], "unit": "GB/s",
                 "frac": achieved / peaks["hbm_gbs"], "peak_source": peak_src}
     else:
-        achieved = k_flops / k_sec / 1e12
+        achieved = flops_step / k_sec / 1e12
         pk = peaks["bf16_tflops"]
         roof = {"bound": "tensor", "achieved": achieved, "peak": pk, "unit": "TFLOP/s",
                 "frac": achieved / pk, "peak_source": peak_src + " (burst)"}
     traffic = ncu_traffic(f"{kernel_name}:{args.workload}")
     roof["traffic"] = traffic
     roof["kernel"] = kernel_name
-    roof["per_launch_us"] = [round(x * 1e3, 3) for x in kms]
+    roof["avg_launch_us"] = k_sec / len(cases) * 1e6
+    roof["per_layer_us_alone"] = [round(x * 1e3, 3) for x in kms]
     roof["algorithmic_bytes_per_launch"] = [c.bytes for c in cases]
 
     line = {
@@ -457,7 +494,7 @@ def run_ours(args):
             "flops_per_step": flops_step,
         },
         "roofline": roof,
-        "gpu_launches": len(cases) * args.steps,
+        "gpu_launches": sum(launches_per_call(p) for p in plans) * args.steps,
         "clocks": clocks,
     }
 
@@ -504,7 +541,7 @@ def run_ours(args):
         print(json.dumps(line), flush=True)
     if world > 1:
         import torch.distributed as dist
-        del graphs
+        del rot, singles
         torch.cuda.synchronize()
         dist.destroy_process_group()
 
@@ -553,18 +590,16 @@ def prefill_extra(w4, peaks, peak_src, l2, dev, iters=50):
     in_bytes = layer.N * layer.K // 2 + 4 * layer.N * (layer.K // 128) + 2 * M * layer.K
     copies = copies_for(in_bytes, l2)
     case = GemmCase(w4, layer, M, 128, False, copies, dev)
-    graphs, events = capture_step_graphs(w4, [case], copies, with_events=True)
-    for s in range(3):
-        graphs[s % copies].replay()
+    rot, singles = capture_rotation_graph(w4, [case], copies)
+    replay_steps(rot, singles, copies, 3)
     torch.cuda.synchronize()
     a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     a.record()
-    for s in range(iters):
-        graphs[s % copies].replay()
+    replay_steps(rot, singles, copies, iters)
     b.record()
     b.synchronize()
     ms = a.elapsed_time(b) / iters
-    kms = per_kernel_ms(events, 1)[0]
+    kms = ms
     tflops = case.flops / (kms / 1e3) / 1e12
     pk = peaks["bf16_tflops"]
     res = {"workload": "prefill_2048x8192x8192_g128_asym", "ms_per_step": ms,
@@ -581,7 +616,7 @@ def prefill_extra(w4, peaks, peak_src, l2, dev, iters=50):
                   dcopies)
     dms = time_graphs(gs, iters)
     res["dense_bf16_cublas"] = {"ms_per_step": dms, "TFLOP/s": case.flops / (dms / 1e3) / 1e12}
-    del gs, Wd, Xd, graphs, case
+    del gs, Wd, Xd, rot, singles, case
     torch.cuda.empty_cache()
     return res
 

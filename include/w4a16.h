@@ -45,6 +45,7 @@
  * (M = 0 or N = 0 is a no-op), N, K, M < 2^31.  Every pointer is a DEVICE
  * pointer owned by the caller; the library allocates no device memory and keeps
  * no state beyond per-device constants (device properties, tensor-map encoder).
+ * Device scratch, where a kernel needs it, is the caller's `workspace`.
  * Each call is asynchronous on `stream` (a cudaStream_t; NULL = legacy default
  * stream).  Arguments are checked on the host before any launch; a rejected
  * call launches nothing and returns W4A16_EINVAL.  No call aborts, throws or
@@ -75,25 +76,29 @@ typedef enum w4a16_status {
  * is tensor-core bound — Quantization & Acceleration page, 关键判据; the
  * aigcbaba selection page, §二 and §五). */
 typedef enum w4a16_path {
-    W4A16_PATH_AUTO = 0,       /* choose from (M, N, K, g) */
-    W4A16_PATH_DECODE = 1,     /* small-M split-K kernel: 128-bit packed loads, in-register
-                                  dequantization, bf16 MMA with fp32 accumulation, split-K
-                                  partial sums reduced through thread-block-cluster shared
-                                  memory; supports M ≤ 16 */
+    W4A16_PATH_AUTO = 0,       /* choose from M (roofline: M ≤ 16 is weight-bandwidth bound) */
+    W4A16_PATH_DECODE = 1,     /* small-M kernel, M ≤ 16: persistent stream-K grid; TMA streams
+                                  packed codes and X into a shared-memory ring; in-register
+                                  dequantization feeds bf16 MMAs with fp32 accumulation; row
+                                  blocks split across CTAs are added in a fixed order by a
+                                  second small kernel */
     W4A16_PATH_TENSORCORE = 2  /* large-M kernel: TMA-fed INT4 tile dequantized into shared
                                   memory and fed to tcgen05 bf16 MMA with TMEM accumulators */
 } w4a16_path;
 
 /* The launch a GEMM call would make (filled by w4a16_gemm_plan). */
 typedef struct w4a16_plan {
-    int32_t path;        /* w4a16_path actually used (never AUTO) */
-    int32_t split_k;     /* decode: CTAs per cluster splitting K (1..8) */
-    int32_t tile_m;      /* tensor-core: activation rows per CTA tile (32/64/128/256);
-                            decode: 8 or 16 (MMA columns) */
-    int32_t tile_n;      /* output features per CTA tile */
-    int64_t grid;        /* CTAs launched */
-    int32_t threads;     /* threads per CTA */
-    int32_t smem_bytes;  /* dynamic shared memory per CTA */
+    int32_t path;            /* w4a16_path actually used (never AUTO) */
+    int32_t tile_m;          /* activation rows per tile (decode: 8 or 16 MMA columns;
+                                tensor core: 32/64/128/256) */
+    int32_t tile_n;          /* output features per tile */
+    int32_t threads;         /* threads per CTA */
+    int64_t grid;            /* CTAs launched */
+    int32_t smem_bytes;      /* dynamic shared memory per CTA */
+    int32_t stages;          /* shared-memory pipeline depth */
+    int32_t kernels;         /* kernels the call launches (decode: 2 when its stream-K
+                                partition splits a row block between CTAs, else 1) */
+    int64_t workspace_bytes; /* device workspace this launch needs */
 } w4a16_plan;
 
 /* Quantize W[N, K] group-wise by RTN (asymmetric when sym == 0, symmetric when
@@ -115,9 +120,13 @@ w4a16_status w4a16_dequantize(const void* packed, const void* scales, const void
                               int64_t N, int64_t K, int32_t g, int32_t sym, void* W_hat,
                               void* stream);
 
-/* Bytes of device workspace w4a16_gemm needs for this shape.  Every current
- * kernel reduces split-K partial sums on chip, so this returns 0; the argument
- * pair stays in the ABI so a future kernel can ask for scratch. */
+/* Bytes of device workspace w4a16_gemm needs for this shape (0 for the
+ * tensor-core path).  The decode path stores there the fp32 partial sums of the
+ * 32-row blocks that its stream-K partition splits between CTAs; a second,
+ * small kernel adds them in a fixed order.  The contents are scratch: no
+ * initialization is needed and nothing is kept between calls, but two calls
+ * that may run at the same time (for instance on two streams) need two
+ * workspaces.  Uses the current device's SM count. */
 size_t w4a16_gemm_workspace_size(int64_t M, int64_t N, int64_t K, int32_t g);
 
 /* Fused W4A16 GEMM: Y[M, N] = X[M, K] · Ŵ[N, K]ᵀ with Ŵ = bf16_rn((q − z)·s)
@@ -126,7 +135,7 @@ size_t w4a16_gemm_workspace_size(int64_t M, int64_t N, int64_t K, int32_t g);
  *   X in bf16 [M, K]; packed/scales/zeros as produced by w4a16_quantize
  *   (zeros ignored, may be NULL, when sym == 1); Y out bf16 [M, N].
  *   workspace/workspace_bytes: device scratch of at least
- *   w4a16_gemm_workspace_size() bytes (may be NULL/0 when that is 0).
+ *   w4a16_gemm_workspace_size() bytes, 16-byte aligned (see there).
  * Results are deterministic: the same inputs give bitwise-equal Y. */
 w4a16_status w4a16_gemm(const void* X, int64_t M, int64_t K, const void* packed,
                         const void* scales, const void* zeros, int64_t N, int32_t g,
@@ -134,19 +143,23 @@ w4a16_status w4a16_gemm(const void* X, int64_t M, int64_t K, const void* packed,
                         void* stream);
 
 /* w4a16_gemm with the dispatch decision overridden: `path` forces a kernel
- * (AUTO = same as w4a16_gemm) and `split_k` (decode only, 0 = automatic,
- * else 1..8) forces the number of CTAs splitting K.  Used by tests, benchmarks
- * and profiling to exercise both kernels at the same shape.  Returns
- * W4A16_EINVAL if the forced kernel cannot run the shape (e.g. DECODE with M > 16). */
+ * (AUTO = same as w4a16_gemm) and `ctas` (decode only; 0 = automatic, one or
+ * two CTAs per SM) sets the size of the persistent grid, hence where the
+ * stream-K partition splits row blocks.  Used by tests, benchmarks and
+ * profiling to exercise both kernels and many partitions at the same shape.
+ * Returns W4A16_EINVAL if the forced kernel cannot run the shape (DECODE with
+ * M > 16, or `ctas` given for the tensor-core path), W4A16_EWORKSPACE if the
+ * workspace is smaller than the plan's workspace_bytes. */
 w4a16_status w4a16_gemm_ex(const void* X, int64_t M, int64_t K, const void* packed,
                            const void* scales, const void* zeros, int64_t N, int32_t g,
                            int32_t sym, void* Y, void* workspace, size_t workspace_bytes,
-                           int32_t path, int32_t split_k, void* stream);
+                           int32_t path, int32_t ctas, void* stream);
 
-/* Host-only: report the launch w4a16_gemm_ex would make (no device access).
- * Returns W4A16_EINVAL for shapes or forced paths it would reject. */
+/* Host-only: report the launch w4a16_gemm_ex would make, including the
+ * workspace it needs.  Returns W4A16_EINVAL for shapes or overrides it would
+ * reject. */
 w4a16_status w4a16_gemm_plan(int64_t M, int64_t N, int64_t K, int32_t g, int32_t sym,
-                             int32_t path, int32_t split_k, w4a16_plan* plan);
+                             int32_t path, int32_t ctas, w4a16_plan* plan);
 
 /* Read and clear the current device's error word, written by a kernel that gave
  * up a bounded wait (a pipeline barrier that did not complete within about one

@@ -61,15 +61,15 @@ FAKE = 0x10000          # 16-byte aligned, never dereferenced on the host
 
 
 def _gemm(lib, M=1, K=128, N=64, g=128, sym=0, X=FAKE, P=FAKE, S=FAKE, Z=FAKE, Y=FAKE,
-          path=0, split=0, ws=None, ws_bytes=0):
-    return lib.w4a16_gemm_ex(X, M, K, P, S, Z, N, g, sym, Y, ws, ws_bytes, path, split, None)
+          path=0, ctas=0, ws=FAKE, ws_bytes=1 << 30):
+    return lib.w4a16_gemm_ex(X, M, K, P, S, Z, N, g, sym, Y, ws, ws_bytes, path, ctas, None)
 
 
 @pytest.mark.parametrize("kw", [
     dict(g=48), dict(g=16), dict(g=256), dict(K=96), dict(K=0), dict(M=-1), dict(N=-2),
     dict(sym=2), dict(X=None), dict(P=None), dict(S=None), dict(Y=None), dict(Z=None),
     dict(X=FAKE + 8), dict(P=FAKE + 4), dict(Y=FAKE + 2), dict(S=FAKE + 2),
-    dict(M=17, path=1), dict(path=3), dict(split=9), dict(split=2, path=2),
+    dict(M=17, path=1), dict(path=3), dict(ctas=-1), dict(ctas=70000), dict(ctas=2, path=2),
     dict(K=2 ** 31),
 ])
 def test_gemm_rejects_invalid_arguments(lib, kw):
@@ -95,9 +95,24 @@ def test_quantize_and_dequantize_reject_invalid(lib):
     assert d(FAKE, FAKE, FAKE, 4, 128, 32, 0, FAKE + 1, None) == EINVAL
 
 
-def test_workspace_size_is_zero(lib):
-    assert w4.workspace_size(1, 4096, 4096, 128) == 0
+def test_workspace_sizes(lib):
+    # tensor-core path needs none; decode needs counters + partial row blocks
     assert w4.workspace_size(2048, 8192, 8192, 32) == 0
+    assert w4.workspace_size(17, 8192, 8192, 32) == 0
+    rb = 4096 // 32
+    p = w4.plan(1, 4096, 4096, 128)
+    assert p["workspace_bytes"] == (rb + p["grid"]) * 256 * 4
+    p16 = w4.plan(16, 4096, 4096, 128)
+    assert p16["workspace_bytes"] == (rb + p16["grid"]) * 512 * 4
+    assert w4.workspace_size(1, 4096, 4096, 128) == p["workspace_bytes"]
+
+
+def test_decode_rejects_small_workspace(lib):
+    need = w4.plan(1, 64, 128, 128)["workspace_bytes"]
+    assert need > 0
+    assert _gemm(lib, ws_bytes=need - 1) == EWORKSPACE
+    assert _gemm(lib, ws=None) == EINVAL
+    assert _gemm(lib, ws=FAKE + 8) == EINVAL
 
 
 def test_dispatch_plans():
@@ -106,18 +121,111 @@ def test_dispatch_plans():
     assert w4.plan(17, 4096, 4096)["path"] == "tensorcore"
     p = w4.plan(2048, 8192, 8192)
     assert p["path"] == "tensorcore" and p["tile_m"] == 256 and p["grid"] == 64 * 8
-    assert p["smem_bytes"] <= 232448
+    assert p["smem_bytes"] <= 232448 and p["workspace_bytes"] == 0
     for M, bm in ((17, 32), (32, 32), (33, 64), (64, 64), (65, 128), (128, 128), (129, 256)):
         assert w4.plan(M, 8192, 8192)["tile_m"] == bm
     for M in (1, 8):
         assert w4.plan(M, 4096, 4096)["tile_m"] == 8
     assert w4.plan(9, 4096, 4096)["tile_m"] == 16
-    p = w4.plan(1, 4096, 11008, split_k=3)
-    assert p["split_k"] == 3 and p["grid"] == 3 * 4096 // 32
-    for N, K in ((11008, 4096), (4096, 11008), (28672, 8192), (8192, 28672), (256, 256)):
-        p = w4.plan(1, N, K)
-        assert 1 <= p["split_k"] <= 8
-        assert p["grid"] % p["split_k"] == 0
-        assert (K + 127) // 128 >= p["split_k"]
+
+
+def test_decode_persistent_grid_and_smem():
+    for M, N, K in ((1, 11008, 4096), (1, 4096, 11008), (1, 28672, 8192), (8, 8192, 28672),
+                    (16, 8192, 8192), (1, 256, 256)):
+        p = w4.plan(M, N, K)
+        units = -(-N // 32) * -(-K // 1024)
+        per_sm = 2 if (M <= 8 and p["smem_bytes"] * 2 + 2048 <= 233472) else 1
+        assert p["grid"] == min(units, 148 * per_sm)
+        assert p["smem_bytes"] <= 232448 and p["stages"] >= 2
+        assert p["threads"] == 288
+    # forced grid sizes (any positive count, capped at the number of units)
+    assert w4.plan(1, 4096, 11008, ctas=7)["grid"] == 7
+    assert w4.plan(1, 64, 1024, ctas=50)["grid"] == 2          # 2 row blocks x 1 K block
     with pytest.raises(w4.W4A16Error):
         w4.plan(17, 4096, 4096, path="decode")
+    with pytest.raises(w4.W4A16Error):
+        w4.plan(64, 4096, 4096, path="tensorcore", ctas=4)
+
+
+def _owner(u, U, C):
+    return ((u + 1) * C - 1) // U
+
+
+@pytest.mark.parametrize("U,C", [(10, 3), (1376, 296), (1408, 296), (7, 7), (5, 1), (100, 99)])
+def test_stream_k_partition_arithmetic(U, C):
+    """The kernel's split u_c = floor(c·U/C) and its inverse owner(u): every
+    unit has exactly one owner, owners are contiguous and non-decreasing, the
+    partial-sum slot rb + c of a split row block never collides, and the fixup
+    kernel's rule (boundary b handles the row block it falls in iff b is the
+    row block's first owner) finishes every split row block exactly once."""
+    starts = [c * U // C for c in range(C + 1)]
+    for c in range(C):
+        for u in range(starts[c], starts[c + 1]):
+            assert _owner(u, U, C) == c
+    for kbn in (1, 3, 4, 11):
+        if U % kbn:
+            continue
+        rbs = U // kbn
+        used = set()
+        for rb in range(rbs):
+            cf, cl = _owner(rb * kbn, U, C), _owner(rb * kbn + kbn - 1, U, C)
+            for c in range(cf, cl + 1):
+                slot = rb + c
+                assert slot not in used and slot < rbs + C
+                used.add(slot)
+        handled = []
+        for b in range(C - 1):
+            u_next = (b + 1) * U // C
+            if u_next % kbn == 0:
+                continue
+            rb = u_next // kbn
+            if _owner(rb * kbn, U, C) == b:
+                handled.append(rb)
+        split = [rb for rb in range(rbs)
+                 if _owner(rb * kbn, U, C) != _owner(rb * kbn + kbn - 1, U, C)]
+        assert sorted(handled) == split
+
+
+def _walk(u0, u1, kbn):
+    """Mirror of the decode kernel's unit visiting order (UnitWalk)."""
+    rb_first = u0 // kbn
+    rb, kb = rb_first, u0 - rb_first * kbn
+    rb_last = (u1 - 1) // kbn
+    kb_last_end = (u1 - 1) - rb_last * kbn + 1
+    two, phase, out = rb_last != rb_first, 0, []
+    for i in range(u1 - u0):
+        if i > 0:
+            if phase == 0 and two and kb == kbn - 1:
+                phase, rb, kb = 1, rb_last, 0
+            elif phase == 1 and kb == kb_last_end - 1:
+                phase, rb, kb = 2, rb_first + 1, 0
+            elif phase == 2 and kb == kbn - 1:
+                rb, kb = rb + 1, 0
+            else:
+                kb += 1
+        if phase == 0:
+            end = (kb == kbn - 1) if two else (kb == kb_last_end - 1)
+        elif phase == 1:
+            end = kb == kb_last_end - 1
+        else:
+            end = kb == kbn - 1
+        out.append((rb, kb, end))
+    return out
+
+
+@pytest.mark.parametrize("kbn", [1, 2, 3, 4, 8, 11, 28])
+def test_stream_k_unit_walk(kbn):
+    """Each CTA visits its units exactly once, each row block contiguously,
+    and marks the end of every row block it touches exactly once (after its
+    last unit there): the split first and last segments come first."""
+    for rbs in (1, 2, 3, 7, 20):
+        U = rbs * kbn
+        for C in range(1, min(U, 40) + 1):
+            for c in range(C):
+                u0, u1 = c * U // C, (c + 1) * U // C
+                w = _walk(u0, u1, kbn)
+                assert sorted(rb * kbn + kb for rb, kb, _ in w) == list(range(u0, u1))
+                for rb in set(r for r, _, _ in w):
+                    idx = [i for i, (r, _, _) in enumerate(w) if r == rb]
+                    assert idx == list(range(idx[0], idx[-1] + 1))
+                    assert [i for i in idx if w[i][2]] == [idx[-1]]

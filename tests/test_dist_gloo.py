@@ -1,0 +1,57 @@
+"""Multi-rank host logic of bench.py on CPU with the gloo backend (world size 2):
+the timed value is all ranks' work over the slowest rank's time, and the
+reference arm prints from rank 0 only."""
+import json
+import os
+import subprocess
+import sys
+
+import pytest
+import torch.multiprocessing as mp
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def _worker(rank, world, port, q):
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port), RANK=str(rank),
+                      WORLD_SIZE=str(world))
+    sys.path.insert(0, ROOT)
+    import torch.distributed as dist
+    import bench
+    dist.init_process_group("gloo", rank=rank, world_size=world)
+    # rank r did (r+1)·100 bytes of work in (r+1)·2 ms
+    work, ms = (rank + 1) * 100.0, (rank + 1) * 2.0
+    q.put((rank, bench.max_over_ranks(world, ms), bench.sum_over_ranks(world, work),
+           bench.job_throughput(world, work, ms, 1.0)))
+    dist.barrier()
+    dist.destroy_process_group()
+
+
+def test_max_and_sum_over_ranks_gloo():
+    ctx = mp.get_context("spawn")
+    q = ctx.Queue()
+    port = 29600 + os.getpid() % 1000
+    procs = [ctx.Process(target=_worker, args=(r, 2, port, q)) for r in range(2)]
+    for p in procs:
+        p.start()
+    for p in procs:
+        p.join(timeout=120)
+        assert p.exitcode == 0
+    res = sorted(q.get(timeout=10) for _ in range(2))
+    for rank, mx, total, thr in res:
+        assert mx == 4.0 and total == 300.0
+        assert thr == pytest.approx(300.0 / 0.004)      # 300 bytes over the slowest 4 ms
+
+
+def test_reference_arm_prints_once_under_torchrun():
+    cmd = [sys.executable, "-m", "torch.distributed.run", "--nnodes=1", "--nproc-per-node=2",
+           "--master-addr=127.0.0.1", f"--master-port={29700 + os.getpid() % 1000}",
+           os.path.join(ROOT, "bench.py"), "--impl", "reference", "--gpus", "2", "--steps", "1",
+           "--warmup", "3"]
+    r = subprocess.run(cmd, cwd=ROOT, capture_output=True, text=True, timeout=600)
+    assert r.returncode == 0, r.stderr[-2000:]
+    lines = [l for l in r.stdout.splitlines() if l.startswith("{")]
+    assert len(lines) == 1
+    line = json.loads(lines[0])
+    assert line["impl"] == "reference" and line["n_gpus"] == 2
+    assert line["cpu_baseline"]["kind"] == "oracle" and line["e2e"]["h2d_bytes_per_step"] == 0

@@ -36,11 +36,11 @@ def _quantized(N, K, g, sym, seed, outlier=True):
     return P, S, Z
 
 
-def _check_full(M, N, K, g, sym, path, seed=0, split_k=0, x_outliers=True):
+def _check_full(M, N, K, g, sym, path, seed=0, ctas=0, x_outliers=True):
     P, S, Z = _quantized(N, K, g, sym, seed)
     X = workloads.make_activation(M, K, seed + 1, outlier_frac=0.01 if x_outliers else 0.0,
                                   outlier_mode="set")
-    Y = w4.gemm(X.cuda(), P, S, Z, g, sym, path=path, split_k=split_k)
+    Y = w4.gemm(X.cuda(), P, S, Z, g, sym, path=path, ctas=ctas)
     torch.cuda.synchronize()
     Y64 = oracle.gemm_w4a16(workloads.bits(X), P.cpu().numpy(), workloads.bits(S),
                             workloads.bits(Z), g, sym)
@@ -62,9 +62,13 @@ def test_decode_path_small(M, N, K, g, sym):
     _check_full(M, N, K, g, sym, "decode", seed=M + N + K)
 
 
-@pytest.mark.parametrize("split_k", [1, 2, 3, 5, 8])
-def test_decode_forced_split_k(split_k):
-    _check_full(4, 300, 8 * 128 * 3, 128, False, "decode", seed=5, split_k=split_k)
+@pytest.mark.parametrize("ctas", [1, 2, 3, 5, 7, 13, 40, 97, 300])
+@pytest.mark.parametrize("M", [1, 12])
+def test_decode_stream_k_partitions(ctas, M):
+    """Many persistent-grid sizes: row blocks split 0..n times between CTAs,
+    finished by the last arrival; counters must be back at zero afterwards."""
+    _check_full(M, 300, 1024 * 5 + 256, 128, False, "decode", seed=5, ctas=ctas)
+    _check_full(M, 300, 1024 * 5 + 256, 128, False, "decode", seed=6, ctas=ctas)
 
 
 TC_SHAPES = [(1, 128, 64 * 3), (17, 200, 256), (32, 128, 128), (33, 384, 512), (64, 129, 96),

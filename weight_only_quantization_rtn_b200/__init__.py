@@ -34,10 +34,11 @@ class W4A16Error(RuntimeError):
 
 
 class Plan(ctypes.Structure):
-    _fields_ = [("path", ctypes.c_int32), ("split_k", ctypes.c_int32),
-                ("tile_m", ctypes.c_int32), ("tile_n", ctypes.c_int32),
-                ("grid", ctypes.c_int64), ("threads", ctypes.c_int32),
-                ("smem_bytes", ctypes.c_int32)]
+    _fields_ = [("path", ctypes.c_int32), ("tile_m", ctypes.c_int32),
+                ("tile_n", ctypes.c_int32), ("threads", ctypes.c_int32),
+                ("grid", ctypes.c_int64), ("smem_bytes", ctypes.c_int32),
+                ("stages", ctypes.c_int32), ("kernels", ctypes.c_int32),
+                ("workspace_bytes", ctypes.c_int64)]
 
 
 def _load() -> ctypes.CDLL:
@@ -146,33 +147,44 @@ def workspace_size(M: int, N: int, K: int, g: int) -> int:
 
 
 def plan(M: int, N: int, K: int, g: int = 128, sym: bool = False, path: str | int = "auto",
-         split_k: int = 0) -> dict:
+         ctas: int = 0) -> dict:
     """The launch w4a16_gemm would make for this shape (host only)."""
     p = Plan()
     pid = _PATHS[path] if isinstance(path, str) else int(path)
-    _check(lib().w4a16_gemm_plan(M, N, K, g, int(bool(sym)), pid, split_k, ctypes.byref(p)),
+    _check(lib().w4a16_gemm_plan(M, N, K, g, int(bool(sym)), pid, ctas, ctypes.byref(p)),
            "w4a16_gemm_plan")
-    return {"path": {v: k for k, v in _PATHS.items()}[p.path], "split_k": p.split_k,
-            "tile_m": p.tile_m, "tile_n": p.tile_n, "grid": p.grid, "threads": p.threads,
-            "smem_bytes": p.smem_bytes}
+    return {"path": {v: k for k, v in _PATHS.items()}[p.path], "tile_m": p.tile_m,
+            "tile_n": p.tile_n, "grid": p.grid, "threads": p.threads,
+            "smem_bytes": p.smem_bytes, "stages": p.stages, "kernels": p.kernels,
+            "workspace_bytes": p.workspace_bytes}
 
 
 _workspaces: dict = {}
 
 
+def _workspace(dev: torch.device, nbytes: int):
+    """A scratch buffer per (device, stream), grown on demand; calls on one
+    stream never overlap, so they can share it."""
+    if nbytes == 0:
+        return None
+    key = (dev, torch.cuda.current_stream(dev).cuda_stream)
+    ws = _workspaces.get(key)
+    if ws is None or ws.numel() < nbytes:
+        ws = torch.empty(nbytes, dtype=torch.uint8, device=dev)
+        _workspaces[key] = ws
+    return ws
+
+
 def gemm(X: torch.Tensor, packed: torch.Tensor, scales: torch.Tensor,
          zeros: torch.Tensor | None, g: int = 128, sym: bool = False, path: str | int = "auto",
-         split_k: int = 0, out: torch.Tensor | None = None) -> torch.Tensor:
+         ctas: int = 0, out: torch.Tensor | None = None) -> torch.Tensor:
     """Fused W4A16 GEMM: Y[M, N] = X[M, K] · Ŵ[N, K]ᵀ (bf16 in/out, fp32 accumulation).
 
     If X lives in host memory (ideally pinned) it is copied to the weights'
     device and Y is copied back to the host: the end-to-end form of the call."""
     host_in = not X.is_cuda
     dev = packed.device
-    if host_in:
-        Xd = X.to(dev, non_blocking=True)
-    else:
-        Xd = X
+    Xd = X.to(dev, non_blocking=True) if host_in else X
     _need(Xd, torch.bfloat16, "X")
     _need(packed, torch.uint8, "packed")
     _need(scales, torch.bfloat16, "scales")
@@ -188,18 +200,13 @@ def gemm(X: torch.Tensor, packed: torch.Tensor, scales: torch.Tensor,
         _need(out, torch.bfloat16, "out")
         if tuple(out.shape) != (M, N):
             raise ValueError("out has the wrong shape")
-    ws_bytes = workspace_size(M, N, K, g)
-    ws = None
-    if ws_bytes:
-        ws = _workspaces.get(dev)
-        if ws is None or ws.numel() < ws_bytes:
-            ws = torch.zeros(ws_bytes, dtype=torch.uint8, device=dev)
-            _workspaces[dev] = ws
     pid = _PATHS[path] if isinstance(path, str) else int(path)
     with torch.cuda.device(dev):
+        ws_bytes = plan(M, N, K, g, sym, pid, ctas)["workspace_bytes"] if M and N else 0
+        ws = _workspace(dev, ws_bytes)
         _check(lib().w4a16_gemm_ex(_ptr(Xd), M, K, _ptr(packed), _ptr(scales),
-                                  _ptr(zeros if not sym else None), N, g, int(bool(sym)),
-                                  _ptr(out), _ptr(ws), ws_bytes, pid, split_k, _stream(dev)),
+                                   _ptr(zeros if not sym else None), N, g, int(bool(sym)),
+                                   _ptr(out), _ptr(ws), ws_bytes, pid, ctas, _stream(dev)),
                "w4a16_gemm")
     if host_in:
         return out.to("cpu")

@@ -72,6 +72,12 @@ __device__ __forceinline__ uint32_t bf16x2_sub(uint32_t a, uint32_t b) {
     return d;
 }
 
+__device__ __forceinline__ uint32_t bf16x2_add(uint32_t a, uint32_t b) {
+    uint32_t d;
+    asm("add.rn.bf16x2 %0, %1, %2;" : "=r"(d) : "r"(a), "r"(b));
+    return d;
+}
+
 __device__ __forceinline__ uint32_t bf16x2_mul(uint32_t a, uint32_t b) {
     uint32_t d;
     asm("mul.rn.bf16x2 %0, %1, %2;" : "=r"(d) : "r"(a), "r"(b));
@@ -87,10 +93,23 @@ __device__ __forceinline__ uint32_t zero_pair(uint32_t z_bits) {
     return (0x4300u | (z & 0xFu)) * 0x00010001u;
 }
 
-// OR (asym) or XOR (sym) of the bf16 exponent pattern into isolated nibbles.
+// (a & mask) | magic  (asym)  or  (a & mask) ^ magic  (sym), as one LOP3.
 template <bool SYM>
-__device__ __forceinline__ uint32_t magic(uint32_t nibbles_0x000F000F) {
-    return SYM ? (nibbles_0x000F000F ^ 0x43084308u) : (nibbles_0x000F000F | 0x43004300u);
+__device__ __forceinline__ uint32_t isolate_magic(uint32_t a, uint32_t mask) {
+    uint32_t d;
+    if (SYM) {
+        asm("lop3.b32 %0, %1, %2, %3, 0x6A;" : "=r"(d) : "r"(a), "r"(mask), "n"(0x43084308));
+    } else {
+        asm("lop3.b32 %0, %1, %2, %3, 0xEA;" : "=r"(d) : "r"(a), "r"(mask), "n"(0x43004300));
+    }
+    return d;
+}
+
+// One bf16x2 of bf16_rn((q − z)·s) from codes isolated into the low nibble of
+// each 16-bit half of `a` (the other bits of `a` are masked off).
+template <bool SYM>
+__device__ __forceinline__ uint32_t dq_pair(uint32_t a, uint32_t zz, uint32_t ss) {
+    return bf16x2_mul(bf16x2_sub(isolate_magic<SYM>(a, 0x000F000Fu), zz), ss);
 }
 
 // Eight codes of one 32-bit word (code i in nibble i) -> four bf16x2 values of
@@ -99,10 +118,7 @@ template <bool SYM>
 __device__ __forceinline__ void dequant8_interleaved(uint32_t w, uint32_t zz, uint32_t ss,
                                                      uint32_t out[4]) {
 #pragma unroll
-    for (int j = 0; j < 4; ++j) {
-        uint32_t p = magic<SYM>((w >> (4 * j)) & 0x000F000Fu);
-        out[j] = bf16x2_mul(bf16x2_sub(p, zz), ss);
-    }
+    for (int j = 0; j < 4; ++j) out[j] = dq_pair<SYM>(w >> (4 * j), zz, ss);
 }
 
 // Same values in NATURAL order: (q0,q1) (q2,q3) (q4,q5) (q6,q7).
@@ -115,8 +131,7 @@ __device__ __forceinline__ void dequant8_natural(uint32_t w, uint32_t zz, uint32
     for (int j = 0; j < 4; ++j) {
         // bytes: [lo.j, 0, hi.j, 0] — selector 8|x replicates the (zero) sign bit
         const uint32_t sel = (uint32_t)j | 0x80u | ((uint32_t)(4 + j) << 8) | 0xC000u;
-        uint32_t p = magic<SYM>(__byte_perm(lo, hi, sel) & 0x000F000Fu);
-        out[j] = bf16x2_mul(bf16x2_sub(p, zz), ss);
+        out[j] = dq_pair<SYM>(__byte_perm(lo, hi, sel), zz, ss);
     }
 }
 
@@ -134,6 +149,34 @@ __device__ __forceinline__ void mma_bf16_16816(float c[4], uint32_t a0, uint32_t
 // ------------------------------------------------------------------ shared memory / mbarrier
 __device__ __forceinline__ uint32_t smem_u32(const void* p) {
     return static_cast<uint32_t>(__cvta_generic_to_shared(p));
+}
+
+__device__ __forceinline__ uint4 lds128(const void* p) {
+    uint4 v;
+    asm volatile("ld.shared.v4.u32 {%0,%1,%2,%3}, [%4];"
+                 : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
+                 : "r"(smem_u32(p)));
+    return v;
+}
+
+__device__ __forceinline__ uint32_t lds_u16(const void* p) {
+    unsigned short v;
+    asm volatile("ld.shared.u16 %0, [%1];" : "=h"(v) : "r"(smem_u32(p)));
+    return v;
+}
+
+__device__ __forceinline__ uint32_t lds_u32(const void* p) {
+    uint32_t v;
+    asm volatile("ld.shared.u32 %0, [%1];" : "=r"(v) : "r"(smem_u32(p)));
+    return v;
+}
+
+__device__ __forceinline__ void sts_u32(void* p, uint32_t v) {
+    asm volatile("st.shared.u32 [%0], %1;" ::"r"(smem_u32(p)), "r"(v) : "memory");
+}
+
+__device__ __forceinline__ void named_bar_sync(int id, int count) {
+    asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(count) : "memory");
 }
 
 __device__ __forceinline__ void mbar_init(uint32_t bar, uint32_t count) {
@@ -165,16 +208,27 @@ __device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
     return ok != 0;
 }
 
+// try_wait that lets the hardware suspend the thread until the phase completes
+// (or about `hint_ns` pass), so that waiting warps take no issue slots.
+__device__ __forceinline__ bool mbar_try_wait_sleep(uint32_t bar, uint32_t parity, uint32_t hint_ns) {
+    uint32_t ok;
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t}"
+        : "=r"(ok)
+        : "r"(bar), "r"(parity), "r"(hint_ns)
+        : "memory");
+    return ok != 0;
+}
+
 // Wait for the phase with the given parity to complete; give up after about a
 // second, record the error and return false.
 __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity) {
     if (mbar_try_wait(bar, parity)) return true;
     const uint64_t t0 = global_timer_ns();
     while (true) {
-#pragma unroll 1
-        for (int i = 0; i < 64; ++i) {
-            if (mbar_try_wait(bar, parity)) return true;
-        }
+        if (mbar_try_wait_sleep(bar, parity, 20000u)) return true;
         if (global_timer_ns() - t0 > kWaitTimeoutNs) {
             report_error(kErrMbarTimeout);
             return false;

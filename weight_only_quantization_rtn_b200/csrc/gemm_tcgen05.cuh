@@ -12,9 +12,12 @@
 // weights as the UMMA A operand (M = 128) and the activations as B (N = BM).
 //
 // Warp roles (6 warps):
-//   warp 0      TMA producer: per 64-wide K block, one TMA load of the X tile
-//               (BM x 64 bf16, 128-byte swizzle) and one of the packed tile
-//               (128 rows x 32 bytes), completing on the stage's "full" barrier.
+//   warp 0      producer: per 64-wide K block, one lane issues a TMA load of the
+//               X tile (BM x 64 bf16, 128-byte swizzle) and one of the packed
+//               tile (128 rows x 32 bytes); all 32 lanes copy the block's scales
+//               and zero points (one aligned pair of groups per row) into the
+//               stage with 4-byte cp.async copies.  Both complete on the stage's
+//               "full" barrier, so the dequantizers never wait on global loads.
 //   warp 1      TMEM allocator and, on one elected lane, the MMA issuer: waits
 //               for the stage's X tile and dequantized A tile, issues four
 //               tcgen05.mma (K = 16 each), and commits to the stage's "empty"
@@ -46,7 +49,8 @@ struct TcConfig {
     static constexpr int kXBytes = BM * kTcBlockK * 2;          // X tile
     static constexpr int kABytes = kTcTileN * kTcBlockK * 2;    // dequantized weight tile
     static constexpr int kPBytes = kTcTileN * kTcBlockK / 2;    // packed codes tile
-    static constexpr int kStageBytes = kXBytes + kABytes + kPBytes;
+    static constexpr int kSZBytes = 2 * kTcTileN * 4;              // scale and zero pairs per row
+    static constexpr int kStageBytes = kXBytes + kABytes + kPBytes + kSZBytes;
     static constexpr int kBudget = 220 * 1024;
     static constexpr int kStagesRaw = kBudget / kStageBytes;
     static constexpr int kStages = kStagesRaw > 8 ? 8 : kStagesRaw;
@@ -59,7 +63,7 @@ template <int BM, bool SYM, int G>
 __global__ void __launch_bounds__(kTcThreads, 1)
     gemm_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ CUtensorMap tmP,
                    const uint16_t* __restrict__ scales, const uint16_t* __restrict__ zeros,
-                   uint16_t* __restrict__ Y, int M, int N, int K) {
+                   uint16_t* __restrict__ Y, int M, int N, int K, int sz_async) {
     using Cfg = TcConfig<BM>;
     constexpr int S = Cfg::kStages;
     static_assert(S >= 2, "pipeline needs at least two stages");
@@ -71,7 +75,8 @@ __global__ void __launch_bounds__(kTcThreads, 1)
     uint8_t* xs = smem;                                   // S x kXBytes
     uint8_t* as = xs + S * Cfg::kXBytes;                  // S x kABytes
     uint8_t* ps = as + S * Cfg::kABytes;                  // S x kPBytes
-    uint64_t* bars = reinterpret_cast<uint64_t*>(ps + S * Cfg::kPBytes);
+    uint32_t* szs = reinterpret_cast<uint32_t*>(ps + S * Cfg::kPBytes);   // S x [2][128] u32 pairs
+    uint64_t* bars = reinterpret_cast<uint64_t*>(szs + S * 2 * kTcTileN);
     uint64_t* full = bars;             // TMA bytes landed
     uint64_t* afull = bars + S;        // dequantized A tile written
     uint64_t* empty = bars + 2 * S;    // MMAs reading the stage retired
@@ -87,7 +92,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
 
     if (threadIdx.x == 0) {
         for (int s = 0; s < S; ++s) {
-            mbar_init(smem_u32(&full[s]), 1);
+            mbar_init(smem_u32(&full[s]), 1 + 32);   // TMA expect_tx arrive + 32 scale lanes
             mbar_init(smem_u32(&afull[s]), 128);
             mbar_init(smem_u32(&empty[s]), 1);
         }
@@ -108,20 +113,53 @@ __global__ void __launch_bounds__(kTcThreads, 1)
     const uint32_t tmem_d = *tmem_holder;
 
     if (warp == 0) {
-        // ------------------------------------------------------------ TMA producer
-        if (lane == 0) {
-            int issued = 0;
-            for (int kb = 0; kb < num_kb; ++kb) {
-                const int s = kb % S;
-                const uint32_t ph = (uint32_t)(kb / S) & 1u;
-                if (!mbar_wait(smem_u32(&empty[s]), ph ^ 1u)) break;
-                mbar_arrive_expect_tx(smem_u32(&full[s]), Cfg::kXBytes + Cfg::kPBytes);
-                tma_load_2d(smem_u32(xs + s * Cfg::kXBytes), &tmX, kb * kTcBlockK, m0,
-                            smem_u32(&full[s]));
-                tma_load_2d(smem_u32(ps + s * Cfg::kPBytes), &tmP, kb * (kTcBlockK / 2), n0,
-                            smem_u32(&full[s]));
-                ++issued;
+        // ------------------------------------------------------------ producer
+        int issued = 0;
+        for (int kb = 0; kb < num_kb; ++kb) {
+            const int s = kb % S;
+            const uint32_t ph = (uint32_t)(kb / S) & 1u;
+            bool ok = true;
+            if (lane == 0) ok = mbar_wait(smem_u32(&empty[s]), ph ^ 1u);   // one lane waits
+            if (!__shfl_sync(0xffffffffu, ok ? 1 : 0, 0)) break;
+            const uint32_t bar = smem_u32(&full[s]);
+            if (lane == 0) {
+                mbar_arrive_expect_tx(bar, Cfg::kXBytes + Cfg::kPBytes);
+                tma_load_2d(smem_u32(xs + s * Cfg::kXBytes), &tmX, kb * kTcBlockK, m0, bar);
+                tma_load_2d(smem_u32(ps + s * Cfg::kPBytes), &tmP, kb * (kTcBlockK / 2), n0, bar);
             }
+            // the aligned pair of groups holding this block's group(s), per row and array
+            const int jpair = ((kb * kTcBlockK) / G) & ~1;
+            uint32_t* dst = szs + s * 2 * kTcTileN;
+            if (sz_async) {
+#pragma unroll
+                for (int e = lane; e < 2 * kTcTileN; e += 32) {
+                    const int arr = e / kTcTileN, r = e % kTcTileN;
+                    const int n = n0 + r;
+                    const bool in = n < N && !(SYM && arr == 1);
+                    const uint16_t* src = (arr == 0 ? scales : zeros) +
+                                          (in ? (int64_t)n * Gn + jpair : 0);
+                    asm volatile("cp.async.ca.shared.global [%0], [%1], 4, %2;" ::"r"(smem_u32(dst + e)),
+                                 "l"(in ? src : scales), "r"(in ? 4u : 0u)
+                                 : "memory");
+                }
+                asm volatile("cp.async.mbarrier.arrive.noinc.shared::cta.b64 [%0];" ::"r"(bar) : "memory");
+            } else {
+                for (int e = lane; e < 2 * kTcTileN; e += 32) {
+                    const int arr = e / kTcTileN, r = e % kTcTileN;
+                    const int n = n0 + r;
+                    uint32_t v = 0;
+                    if (n < N && !(SYM && arr == 1)) {
+                        const uint16_t* src = (arr == 0 ? scales : zeros) + (int64_t)n * Gn + jpair;
+                        v = ldg_u16(src);
+                        if (jpair + 1 < Gn) v |= (uint32_t)ldg_u16(src + 1) << 16;
+                    }
+                    dst[e] = v;
+                }
+                mbar_arrive(bar);
+            }
+            ++issued;
+        }
+        if (lane == 0) {
             // Do not leave while copies into this CTA's shared memory are in flight.
             for (int kb = (issued > S ? issued - S : 0); kb < issued; ++kb) {
                 if (!mbar_wait(smem_u32(&full[kb % S]), (uint32_t)(kb / S) & 1u)) break;
@@ -156,36 +194,25 @@ __global__ void __launch_bounds__(kTcThreads, 1)
         const int r = (warp & 3) * 32 + lane;   // weight row within the tile == TMEM lane
         const int n = n0 + r;
         const bool row_ok = n < N;
-        const uint16_t* srow = scales + (int64_t)(row_ok ? n : 0) * Gn;
-        const uint16_t* zrow = SYM ? nullptr : zeros + (int64_t)(row_ok ? n : 0) * Gn;
-        auto load_sz = [&](int kb, uint32_t sv[2], uint32_t zv[2]) {
-#pragma unroll
-            for (int h = 0; h < 2; ++h) {
-                const int grp = (kb * kTcBlockK + 32 * h) / G;
-                const bool ok = row_ok && kb < num_kb && grp < Gn;
-                sv[h] = ok ? (uint32_t)ldg_u16(srow + grp) : 0u;
-                zv[h] = (ok && !SYM) ? (uint32_t)ldg_u16(zrow + grp) : 0u;
-            }
-        };
-        uint32_t s_cur[2], z_cur[2];
-        load_sz(0, s_cur, z_cur);
         bool ok = true;
         for (int kb = 0; kb < num_kb; ++kb) {
             const int s = kb % S;
             const uint32_t ph = (uint32_t)(kb / S) & 1u;
-            uint32_t s_nxt[2], z_nxt[2];
-            load_sz(kb + 1, s_nxt, z_nxt);           // prefetch next block's scale/zero
             if (!mbar_wait(smem_u32(&full[s]), ph)) {
                 ok = false;
                 break;
             }
-            const uint4* prow = reinterpret_cast<const uint4*>(ps + s * Cfg::kPBytes + r * 32);
-            uint8_t* arow = as + s * Cfg::kABytes + r * 128;
+            const uint32_t spair = lds_u32(szs + s * 2 * kTcTileN + r);
+            const uint32_t zpair = SYM ? 0u : lds_u32(szs + s * 2 * kTcTileN + kTcTileN + r);
+            const uint8_t* prow = ps + s * Cfg::kPBytes + r * 32;
+            const uint32_t arow = smem_u32(as + s * Cfg::kABytes + r * 128);
 #pragma unroll
             for (int h = 0; h < 2; ++h) {
-                const uint4 v = prow[h];
-                const uint32_t ss = dup16(s_cur[h]);
-                const uint32_t zz = zero_pair<SYM>(z_cur[h]);
+                const uint4 v = lds128(prow + 16 * h);
+                const int half = ((kb * kTcBlockK + 32 * h) / G) & 1;   // position in the pair
+                const uint32_t ss = dup16(spair >> (16 * half));
+                const uint32_t zz = SYM ? 0x43084308u
+                                        : bf16x2_add(dup16(zpair >> (16 * half)), 0x43004300u);
                 const uint32_t wv[4] = {v.x, v.y, v.z, v.w};
 #pragma unroll
                 for (int i = 0; i < 4; ++i) {
@@ -193,15 +220,13 @@ __global__ void __launch_bounds__(kTcThreads, 1)
                     dequant8_natural<SYM>(wv[i], zz, ss, d);
                     const int chunk = 4 * h + i;                 // 16-byte chunk: k = 8·chunk
                     const int phys = chunk ^ (r & 7);            // 128-byte swizzle
-                    *reinterpret_cast<uint4*>(arow + phys * 16) = make_uint4(d[0], d[1], d[2], d[3]);
+                    asm volatile("st.shared.v4.u32 [%0], {%1, %2, %3, %4};" ::"r"(arow + phys * 16),
+                                 "r"(d[0]), "r"(d[1]), "r"(d[2]), "r"(d[3])
+                                 : "memory");
                 }
             }
             fence_proxy_async_smem();
             mbar_arrive(smem_u32(&afull[s]));
-            s_cur[0] = s_nxt[0];
-            s_cur[1] = s_nxt[1];
-            z_cur[0] = z_nxt[0];
-            z_cur[1] = z_nxt[1];
         }
         // ------------------------------------------------------------ epilogue
         if (ok && mbar_wait(smem_u32(accf), 0)) {

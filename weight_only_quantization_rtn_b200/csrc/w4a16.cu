@@ -72,19 +72,71 @@ w4a16_status launch_status() {
 }
 
 // ---------------------------------------------------------------- plans
-// Decode kernel tiling: 16-row warp tiles, two per CTA; S CTAs of a cluster
-// split K when the row tiles alone would leave SMs idle.
-constexpr int kDecodeTPW = 2;
-constexpr int kDecodeRows = 16 * kDecodeTPW;
+constexpr int kSmemPerSm = 233472;        // shared memory per SM (228 KB)
+constexpr int kSmemPerBlockMax = 232448;  // opt-in maximum per CTA (227 KB)
+constexpr int kSmemReservedPerCta = 1024; // reserved by the system per resident CTA
+constexpr int kMaxCtas = 65535;
 
-int decode_split(int64_t N, int64_t K, int sm_count) {
-    const int64_t row_blocks = (N + kDecodeRows - 1) / kDecodeRows;
-    const int64_t chunks = (K + 127) / 128;
-    // Aim for about 4 CTAs per SM; keep at least 2 K chunks per warp per CTA.
-    const int64_t want = (int64_t)sm_count * 4;
-    int s = 1;
-    while (s < 8 && row_blocks * s < want && chunks / (s + 1) >= 2 * kDecodeWarps) ++s;
-    return s;
+// Decode kernel geometry for (M, N, K, g): 32-row x 1024-K units, a ring of
+// shared-memory stages sized to fit one or two CTAs per SM.
+struct DecodeGeometry {
+    int mb;            // n8 MMA column blocks (1: M ≤ 8, 2: M ≤ 16)
+    int rb;            // row blocks of 32 rows
+    int kbn;           // K blocks of 1024
+    int64_t units;     // rb · kbn
+    int stage_bytes;   // packed tile + X slice, multiple of 1024
+    int stages;
+    int ctas_per_sm;
+    int smem_bytes;    // dynamic shared memory per CTA
+};
+
+int decode_fixed_smem(int mb) {
+    return kDecConsumers * 2 * mb * 128 * 4     // per-warp partial tiles
+           + 2 * kDecMaxStages * 8 + 16         // barriers and flags
+           + 1024;                              // alignment slack
+}
+
+// Stage: packed tile (16 KB) | X slice (M x 1024 bf16) | scales + zeros (2 x 32 x 1024/g bf16).
+int decode_sz_offset(int64_t M) { return kDecPBytes + (int)M * 2048; }
+
+int decode_stage_bytes(int64_t M, int g) {
+    const int raw = decode_sz_offset(M) + 2 * kDecRows * (kDecBlockK / g) * 2;
+    return (raw + 1023) / 1024 * 1024;
+}
+
+DecodeGeometry decode_geometry(int64_t M, int64_t N, int64_t K, int g) {
+    DecodeGeometry d{};
+    d.mb = M <= 8 ? 1 : 2;
+    d.rb = (int)((N + kDecRows - 1) / kDecRows);
+    d.kbn = (int)((K + kDecBlockK - 1) / kDecBlockK);
+    d.units = (int64_t)d.rb * d.kbn;
+    d.stage_bytes = decode_stage_bytes(M, g);
+    const int fixed = decode_fixed_smem(d.mb);
+    const int two = (kSmemPerSm / 2 - kSmemReservedPerCta - fixed) / d.stage_bytes;
+    if (d.mb == 1 && two >= 3) {
+        d.ctas_per_sm = 2;
+        d.stages = two < kDecMaxStages ? two : kDecMaxStages;
+    } else {
+        const int one = (kSmemPerBlockMax - fixed) / d.stage_bytes;
+        d.ctas_per_sm = 1;
+        d.stages = one < kDecMaxStages ? one : kDecMaxStages;
+    }
+    d.smem_bytes = d.stages * d.stage_bytes + fixed;
+    return d;
+}
+
+// Workspace: (rb + ctas) fp32 partial row blocks of 256·MB values; slot rb + c
+// holds CTA c's part of a row block that the stream-K partition splits.  It is
+// scratch: no initialization is needed and nothing survives a call.
+int64_t decode_workspace_bytes(const DecodeGeometry& d, int64_t ctas) {
+    return (int64_t)(d.rb + ctas) * 256 * d.mb * 4;
+}
+
+// True if some boundary of the even unit split falls inside a row block.
+bool decode_has_split(const DecodeGeometry& d, int64_t ctas) {
+    for (int64_t b = 1; b < ctas; ++b)
+        if ((b * d.units / ctas) % d.kbn != 0) return true;
+    return false;
 }
 
 int tc_tile_m(int64_t M) {
@@ -112,86 +164,61 @@ w4a16_status check_shape(int64_t M, int64_t N, int64_t K, int32_t g, int32_t sym
     return W4A16_OK;
 }
 
+// M-dispatch: small M streams the weights (HBM-bound) with the decode kernel;
+// larger M is tensor-core bound and goes to the tcgen05 kernel.
+int choose_path(int64_t M) { return M <= 16 ? W4A16_PATH_DECODE : W4A16_PATH_TENSORCORE; }
+
 w4a16_status make_plan(int64_t M, int64_t N, int64_t K, int32_t g, int32_t sym, int32_t path,
-                       int32_t split_k, int sm_count, w4a16_plan* p) {
+                       int32_t ctas, int sm_count, w4a16_plan* p) {
     w4a16_status st = check_shape(M, N, K, g, sym);
     if (st != W4A16_OK) return st;
     if (path < W4A16_PATH_AUTO || path > W4A16_PATH_TENSORCORE) return W4A16_EINVAL;
-    if (split_k < 0 || split_k > 8) return W4A16_EINVAL;
-    int chosen = path;
-    if (chosen == W4A16_PATH_AUTO) chosen = M <= 16 ? W4A16_PATH_DECODE : W4A16_PATH_TENSORCORE;
+    if (ctas < 0 || ctas > kMaxCtas) return W4A16_EINVAL;
+    const int chosen = path == W4A16_PATH_AUTO ? choose_path(M) : path;
     if (chosen == W4A16_PATH_DECODE && M > 16) return W4A16_EINVAL;
-    if (chosen == W4A16_PATH_TENSORCORE && split_k > 1) return W4A16_EINVAL;
+    if (chosen == W4A16_PATH_TENSORCORE && ctas != 0) return W4A16_EINVAL;
     *p = w4a16_plan{};
     p->path = chosen;
     if (chosen == W4A16_PATH_DECODE) {
-        const int64_t row_blocks = (N + kDecodeRows - 1) / kDecodeRows;
-        p->split_k = split_k > 0 ? split_k : decode_split(N, K, sm_count);
-        p->tile_m = M <= 8 ? 8 : 16;
-        p->tile_n = kDecodeRows;
-        p->grid = row_blocks * p->split_k;
-        p->threads = kDecodeThreads;
-        p->smem_bytes = 0;
+        const DecodeGeometry d = decode_geometry(M, N, K, g);
+        int64_t grid = ctas > 0 ? ctas : (int64_t)sm_count * d.ctas_per_sm;
+        if (grid > d.units) grid = d.units;
+        if (grid < 1) grid = 1;
+        p->tile_m = 8 * d.mb;
+        p->tile_n = kDecRows;
+        p->grid = grid;
+        p->threads = kDecThreads;
+        p->smem_bytes = d.smem_bytes;
+        p->stages = d.stages;
+        p->kernels = decode_has_split(d, grid) ? 2 : 1;
+        p->workspace_bytes = decode_workspace_bytes(d, grid);
     } else {
         const int bm = tc_tile_m(M);
-        p->split_k = 1;
         p->tile_m = bm;
         p->tile_n = kTcTileN;
         p->grid = ((N + kTcTileN - 1) / kTcTileN) * ((M + bm - 1) / bm);
         p->threads = kTcThreads;
         p->smem_bytes = tc_smem_bytes(bm);
+        p->stages = TcConfig<256>::kStages;
+        switch (bm) {
+            case 32: p->stages = TcConfig<32>::kStages; break;
+            case 64: p->stages = TcConfig<64>::kStages; break;
+            case 128: p->stages = TcConfig<128>::kStages; break;
+            default: break;
+        }
+        p->kernels = 1;
+        p->workspace_bytes = 0;
     }
     return W4A16_OK;
 }
 
-// ---------------------------------------------------------------- launches
-template <int MB, bool SYM, int G>
-w4a16_status launch_decode_t(const w4a16_plan& p, const void* X, int M, int64_t K,
-                             const void* packed, const void* scales, const void* zeros, int64_t N,
-                             void* Y, cudaStream_t stream) {
-    const int total_chunks = (int)((K + 127) / 128);
-    const int cps = (total_chunks + p.split_k - 1) / p.split_k;
-    cudaLaunchConfig_t cfg = {};
-    cfg.gridDim = dim3((unsigned)p.grid, 1, 1);
-    cfg.blockDim = dim3(kDecodeThreads, 1, 1);
-    cfg.dynamicSmemBytes = 0;
-    cfg.stream = stream;
-    cudaLaunchAttribute attr[1];
-    attr[0].id = cudaLaunchAttributeClusterDimension;
-    attr[0].val.clusterDim.x = (unsigned)p.split_k;
-    attr[0].val.clusterDim.y = 1;
-    attr[0].val.clusterDim.z = 1;
-    cfg.attrs = attr;
-    cfg.numAttrs = 1;
-    cudaError_t e = cudaLaunchKernelEx(
-        &cfg, gemv_decode_kernel<MB, kDecodeTPW, SYM, G>, static_cast<const uint16_t*>(X), M, K,
-        static_cast<const uint8_t*>(packed), static_cast<const uint16_t*>(scales),
-        static_cast<const uint16_t*>(zeros), N, static_cast<uint16_t*>(Y), (int)p.split_k, cps);
-    return e == cudaSuccess ? W4A16_OK : W4A16_ECUDA;
-}
-
-template <bool SYM, int G>
-w4a16_status launch_decode_g(const w4a16_plan& p, const void* X, int M, int64_t K,
-                             const void* packed, const void* scales, const void* zeros, int64_t N,
-                             void* Y, cudaStream_t stream) {
-    if (p.tile_m == 8) return launch_decode_t<1, SYM, G>(p, X, M, K, packed, scales, zeros, N, Y, stream);
-    return launch_decode_t<2, SYM, G>(p, X, M, K, packed, scales, zeros, N, Y, stream);
-}
-
-w4a16_status launch_decode(const w4a16_plan& p, const void* X, int M, int64_t K,
-                           const void* packed, const void* scales, const void* zeros, int64_t N,
-                           int32_t g, int32_t sym, void* Y, cudaStream_t stream) {
-#define W4A16_DECODE_CASE(GG)                                                                 \
-    case GG:                                                                                  \
-        return sym ? launch_decode_g<true, GG>(p, X, M, K, packed, scales, zeros, N, Y, stream) \
-                   : launch_decode_g<false, GG>(p, X, M, K, packed, scales, zeros, N, Y, stream);
-    switch (g) {
-        W4A16_DECODE_CASE(32)
-        W4A16_DECODE_CASE(64)
-        W4A16_DECODE_CASE(128)
-        default: return W4A16_EINVAL;
-    }
-#undef W4A16_DECODE_CASE
+int current_sm_count() {
+    int dev = 0, sms = 0;
+    if (cudaGetDevice(&dev) == cudaSuccess &&
+        cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) == cudaSuccess && sms > 0)
+        return sms;
+    cudaGetLastError();
+    return 148;
 }
 
 w4a16_status encode_2d(CUtensorMap* map, CUtensorMapDataType dtype, const void* base,
@@ -210,11 +237,98 @@ w4a16_status encode_2d(CUtensorMap* map, CUtensorMapDataType dtype, const void* 
     return r == CUDA_SUCCESS ? W4A16_OK : W4A16_ECUDA;
 }
 
+// ---------------------------------------------------------------- decode launch
+template <int MB, bool SYM, int G>
+w4a16_status launch_decode_t(const w4a16_plan& p, const CUtensorMap& tmP, const CUtensorMap& tmX,
+                             const DecodeArgs& args, bool has_split, cudaStream_t stream) {
+    auto kern = gemv_decode_kernel<MB, SYM, G>;
+    static bool attr_set[kMaxDevices] = {};
+    int dev = 0;
+    cudaGetDevice(&dev);
+    if (!attr_set[dev]) {
+        if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 kSmemPerBlockMax) != cudaSuccess)
+            return W4A16_ECUDA;
+        attr_set[dev] = true;
+    }
+    // Programmatic dependent launch: the kernel may start while the previous
+    // grid on the stream drains; it reads only weights before its dependency wait.
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3((unsigned)p.grid, 1, 1);
+    cfg.blockDim = dim3(kDecThreads, 1, 1);
+    cfg.dynamicSmemBytes = (size_t)p.smem_bytes;
+    cfg.stream = stream;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    if (cudaLaunchKernelEx(&cfg, kern, tmP, tmX, args) != cudaSuccess) return W4A16_ECUDA;
+    if (has_split) {
+        cudaLaunchConfig_t fcfg = cfg;
+        fcfg.gridDim = dim3((unsigned)(p.grid - 1), 1, 1);
+        fcfg.blockDim = dim3(256, 1, 1);
+        fcfg.dynamicSmemBytes = 0;
+        if (cudaLaunchKernelEx(&fcfg, decode_fixup_kernel<MB>, args, (int64_t)p.grid) != cudaSuccess)
+            return W4A16_ECUDA;
+    }
+    return W4A16_OK;
+}
+
+w4a16_status launch_decode(const w4a16_plan& p, const void* X, int64_t M, int64_t K,
+                           const void* packed, const void* scales, const void* zeros, int64_t N,
+                           int32_t g, int32_t sym, void* Y, void* workspace, cudaStream_t stream) {
+    const DecodeGeometry d = decode_geometry(M, N, K, g);
+    CUtensorMap tmP, tmX;
+    w4a16_status st = encode_2d(&tmP, CU_TENSOR_MAP_DATA_TYPE_UINT8, packed, (uint64_t)(K / 2),
+                                (uint64_t)N, (uint64_t)(K / 2), 128, kDecRows,
+                                CU_TENSOR_MAP_SWIZZLE_128B);
+    if (st != W4A16_OK) return st;
+    st = encode_2d(&tmX, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, X, (uint64_t)K, (uint64_t)M,
+                   (uint64_t)K * 2, 256, (uint32_t)M, CU_TENSOR_MAP_SWIZZLE_NONE);
+    if (st != W4A16_OK) return st;
+    DecodeArgs args{};
+    args.scales = static_cast<const uint16_t*>(scales);
+    args.zeros = static_cast<const uint16_t*>(zeros);
+    args.Y = static_cast<uint16_t*>(Y);
+    args.ws_part = static_cast<float*>(workspace);
+    args.M = (int)M;
+    args.N = (int)N;
+    args.K = (int)K;
+    args.RB = d.rb;
+    args.KBn = d.kbn;
+    args.stages = d.stages;
+    args.stage_bytes = d.stage_bytes;
+    args.sz_offset = decode_sz_offset(M);
+    args.sz_async = ((K / g) % 2 == 0) ? 1 : 0;   // 4-byte aligned scale rows
+    args.U = d.units;
+    const bool split = p.kernels > 1;
+    if (d.mb == 1) {
+        if (sym) {
+            if (g == 32) return launch_decode_t<1, true, 32>(p, tmP, tmX, args, split, stream);
+            if (g == 64) return launch_decode_t<1, true, 64>(p, tmP, tmX, args, split, stream);
+            return launch_decode_t<1, true, 128>(p, tmP, tmX, args, split, stream);
+        }
+        if (g == 32) return launch_decode_t<1, false, 32>(p, tmP, tmX, args, split, stream);
+        if (g == 64) return launch_decode_t<1, false, 64>(p, tmP, tmX, args, split, stream);
+        return launch_decode_t<1, false, 128>(p, tmP, tmX, args, split, stream);
+    }
+    if (sym) {
+        if (g == 32) return launch_decode_t<2, true, 32>(p, tmP, tmX, args, split, stream);
+        if (g == 64) return launch_decode_t<2, true, 64>(p, tmP, tmX, args, split, stream);
+        return launch_decode_t<2, true, 128>(p, tmP, tmX, args, split, stream);
+    }
+    if (g == 32) return launch_decode_t<2, false, 32>(p, tmP, tmX, args, split, stream);
+    if (g == 64) return launch_decode_t<2, false, 64>(p, tmP, tmX, args, split, stream);
+    return launch_decode_t<2, false, 128>(p, tmP, tmX, args, split, stream);
+}
+
 template <int BM, bool SYM, int G>
 w4a16_status launch_tc_t(const w4a16_plan& p, const CUtensorMap& tmX, const CUtensorMap& tmP,
                          const void* scales, const void* zeros, void* Y, int M, int N, int K,
                          cudaStream_t stream) {
     auto kern = gemm_tc_kernel<BM, SYM, G>;
+    const int sz_async = ((K / G) % 2 == 0) ? 1 : 0;   // 4-byte aligned scale rows
     static bool attr_set[kMaxDevices] = {};
     int dev = 0;
     cudaGetDevice(&dev);
@@ -227,7 +341,7 @@ w4a16_status launch_tc_t(const w4a16_plan& p, const CUtensorMap& tmX, const CUte
     dim3 grid((unsigned)((N + kTcTileN - 1) / kTcTileN), (unsigned)((M + BM - 1) / BM), 1);
     kern<<<grid, kTcThreads, TcConfig<BM>::kSmemBytes, stream>>>(
         tmX, tmP, static_cast<const uint16_t*>(scales), static_cast<const uint16_t*>(zeros),
-        static_cast<uint16_t*>(Y), M, N, K);
+        static_cast<uint16_t*>(Y), M, N, K, sz_async);
     return launch_status();
 }
 
@@ -359,42 +473,36 @@ w4a16_status w4a16_dequantize(const void* packed, const void* scales, const void
 }
 
 size_t w4a16_gemm_workspace_size(int64_t M, int64_t N, int64_t K, int32_t g) {
-    (void)M;
-    (void)N;
-    (void)K;
-    (void)g;
-    return 0;
+    w4a16_plan p;
+    if (make_plan(M, N, K, g, 0, W4A16_PATH_AUTO, 0, current_sm_count(), &p) != W4A16_OK) return 0;
+    return (size_t)p.workspace_bytes;
 }
 
 w4a16_status w4a16_gemm_plan(int64_t M, int64_t N, int64_t K, int32_t g, int32_t sym,
-                             int32_t path, int32_t split_k, w4a16_plan* plan) {
+                             int32_t path, int32_t ctas, w4a16_plan* plan) {
     if (!plan) return W4A16_EINVAL;
-    return make_plan(M, N, K, g, sym, path, split_k, 148, plan);
+    return make_plan(M, N, K, g, sym, path, ctas, current_sm_count(), plan);
 }
 
 w4a16_status w4a16_gemm_ex(const void* X, int64_t M, int64_t K, const void* packed,
                            const void* scales, const void* zeros, int64_t N, int32_t g,
                            int32_t sym, void* Y, void* workspace, size_t workspace_bytes,
-                           int32_t path, int32_t split_k, void* stream) {
-    (void)workspace;
+                           int32_t path, int32_t ctas, void* stream) {
     w4a16_plan p;
-    w4a16_status st = make_plan(M, N, K, g, sym, path, split_k, 148, &p);
+    w4a16_status st = make_plan(M, N, K, g, sym, path, ctas, current_sm_count(), &p);
     if (st != W4A16_OK) return st;
-    if (workspace_bytes < w4a16_gemm_workspace_size(M, N, K, g)) return W4A16_EWORKSPACE;
     if (M == 0 || N == 0) return W4A16_OK;
     if (!X || !packed || !scales || !Y || (!sym && !zeros)) return W4A16_EINVAL;
     if (!aligned16(X) || !aligned16(packed) || !aligned16(scales) || !aligned16(Y) ||
         (!sym && !aligned16(zeros)))
         return W4A16_EINVAL;
+    if (workspace_bytes < (size_t)p.workspace_bytes) return W4A16_EWORKSPACE;
+    if (p.workspace_bytes > 0 && (workspace == nullptr || !aligned16(workspace))) return W4A16_EINVAL;
     DeviceInfo di;
     if ((st = device_info(&di)) != W4A16_OK) return st;
-    if (di.sm_count != 148) {
-        st = make_plan(M, N, K, g, sym, path, split_k, di.sm_count, &p);
-        if (st != W4A16_OK) return st;
-    }
     cudaStream_t s = static_cast<cudaStream_t>(stream);
     if (p.path == W4A16_PATH_DECODE)
-        return launch_decode(p, X, (int)M, K, packed, scales, zeros, N, g, sym, Y, s);
+        return launch_decode(p, X, M, K, packed, scales, zeros, N, g, sym, Y, workspace, s);
     return launch_tc(p, X, M, K, packed, scales, zeros, N, g, sym, Y, s);
 }
 
