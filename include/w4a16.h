@@ -161,6 +161,32 @@ w4a16_status w4a16_gemm_ex(const void* X, int64_t M, int64_t K, const void* pack
 w4a16_status w4a16_gemm_plan(int64_t M, int64_t N, int64_t K, int32_t g, int32_t sym,
                              int32_t path, int32_t ctas, w4a16_plan* plan);
 
+/* Size of the built-in device scratch used by w4a16_gemm_decode_noalloc. */
+#define W4A16_NOALLOC_SCRATCH_BYTES ((size_t)8 << 20)
+
+/* Decode-path GEMM (M ≤ 16) that allocates nothing and takes no workspace.
+ * The pages have no counterpart: this exists for callers that cannot allocate
+ * device memory — code running while a CUDA graph is being captured (where
+ * cudaMalloc is not allowed), plug-ins whose host framework owns every device
+ * allocation through its own pool, and hosts that forbid allocation after
+ * start-up so that memory use stays fixed.
+ * Same arguments, result and determinism as w4a16_gemm_ex with
+ * path = W4A16_PATH_DECODE and ctas = 0, minus the workspace: the split-K
+ * partial sums live in a file-scope device array of
+ * W4A16_NOALLOC_SCRATCH_BYTES that every GPU which loads the library keeps
+ * until the process exits.  Returns W4A16_EWORKSPACE, launching nothing, when
+ * the problem needs more scratch than that (its plan's workspace_bytes), and
+ * W4A16_EINVAL for M > 16 or any argument w4a16_gemm_ex would reject.
+ * The first call on a device looks up the array's device address for that
+ * device (cudaGetSymbolAddress, with the device current); make that first
+ * call before any stream capture.  All calls share the one array and it keeps
+ * the last call's contents; nothing in it needs to start at zero.  Calls that
+ * overlap on the GPU (other streams, other threads, other graph branches)
+ * race on it: serialize them. */
+w4a16_status w4a16_gemm_decode_noalloc(const void* X, int64_t M, int64_t K, const void* packed,
+                                       const void* scales, const void* zeros, int64_t N,
+                                       int32_t g, int32_t sym, void* Y, void* stream);
+
 /* Read and clear the current device's error word, written by a kernel that gave
  * up a bounded wait (a pipeline barrier that did not complete within about one
  * second).  *code = 0 when no kernel reported one.  Synchronizes the device. */

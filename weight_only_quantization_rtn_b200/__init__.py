@@ -17,8 +17,8 @@ import os
 
 import torch
 
-__all__ = ["lib", "quantize", "dequantize", "gemm", "plan", "workspace_size", "device_error",
-           "W4A16Error", "PATH_AUTO", "PATH_DECODE", "PATH_TENSORCORE", "LIB_PATH"]
+__all__ = ["lib", "quantize", "dequantize", "gemm", "gemm_decode_noalloc", "plan",
+           "workspace_size", "device_error", "W4A16Error", "PATH_AUTO", "PATH_DECODE", "PATH_TENSORCORE", "LIB_PATH"]
 
 LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libw4a16.so")
 
@@ -55,6 +55,8 @@ def _load() -> ctypes.CDLL:
     lib.w4a16_gemm_ex.argtypes = [vp, i64, i64, vp, vp, vp, i64, i32, i32, vp, vp, sz, i32, i32,
                                   vp]
     lib.w4a16_gemm_plan.argtypes = [i64, i64, i64, i32, i32, i32, i32, ctypes.POINTER(Plan)]
+    lib.w4a16_gemm_decode_noalloc.argtypes = [vp, i64, i64, vp, vp, vp, i64, i32, i32, vp, vp]
+    lib.w4a16_gemm_decode_noalloc.restype = ctypes.c_int
     lib.w4a16_device_error.argtypes = [ctypes.POINTER(ctypes.c_int32)]
     lib.w4a16_status_string.argtypes = [ctypes.c_int]
     lib.w4a16_status_string.restype = ctypes.c_char_p
@@ -210,6 +212,31 @@ def gemm(X: torch.Tensor, packed: torch.Tensor, scales: torch.Tensor,
                "w4a16_gemm")
     if host_in:
         return out.to("cpu")
+    return out
+
+
+def gemm_decode_noalloc(X: torch.Tensor, packed: torch.Tensor, scales: torch.Tensor,
+                        zeros: torch.Tensor | None, g: int = 128, sym: bool = False,
+                        out: torch.Tensor | None = None) -> torch.Tensor:
+    """Decode-path GEMM (M ≤ 16, device tensors) through the entry point that
+    allocates no device memory of its own: its split-K scratch is a fixed
+    array inside the library, shared by every call, so calls must not overlap
+    on the GPU.  Only ``out`` is allocated here, and only when it is None."""
+    _need(X, torch.bfloat16, "X")
+    _need(packed, torch.uint8, "packed")
+    _need(scales, torch.bfloat16, "scales")
+    if not sym:
+        _need(zeros, torch.bfloat16, "zeros")
+    M, K = X.shape
+    N = packed.shape[0]
+    dev = packed.device
+    if out is None:
+        out = torch.empty((M, N), dtype=torch.bfloat16, device=dev)
+    with torch.cuda.device(dev):
+        _check(lib().w4a16_gemm_decode_noalloc(_ptr(X), M, K, _ptr(packed), _ptr(scales),
+                                               _ptr(zeros if not sym else None), N, g,
+                                               int(bool(sym)), _ptr(out), _stream(dev)),
+               "w4a16_gemm_decode_noalloc")
     return out
 
 

@@ -388,6 +388,28 @@ int grid_for(int64_t work_items, int threads, int sm_count) {
     return (int)(blocks < cap ? (blocks < 1 ? 1 : blocks) : cap);
 }
 
+// Built-in scratch for w4a16_gemm_decode_noalloc (callers that cannot
+// allocate).  In host code this name is only a host-side stand-in; the device
+// address comes from cudaGetSymbolAddress, looked up once per device.
+static __device__ __align__(256) unsigned char g_noalloc_scratch[W4A16_NOALLOC_SCRATCH_BYTES];
+void* g_noalloc_ptr[kMaxDevices] = {};
+
+w4a16_status noalloc_scratch(void** out) {
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return W4A16_ECUDA;
+    std::lock_guard<std::mutex> lock(g_mutex);
+    if (g_noalloc_ptr[dev] == nullptr) {
+        void* p = nullptr;
+        if (cudaGetSymbolAddress(&p, g_noalloc_scratch) != cudaSuccess || p == nullptr) {
+            cudaGetLastError();
+            return W4A16_ECUDA;
+        }
+        g_noalloc_ptr[dev] = p;
+    }
+    *out = g_noalloc_ptr[dev];
+    return W4A16_OK;
+}
+
 }  // namespace
 
 // ==================================================================== ABI
@@ -512,6 +534,26 @@ w4a16_status w4a16_gemm(const void* X, int64_t M, int64_t K, const void* packed,
                         void* stream) {
     return w4a16_gemm_ex(X, M, K, packed, scales, zeros, N, g, sym, Y, workspace,
                          workspace_bytes, W4A16_PATH_AUTO, 0, stream);
+}
+
+w4a16_status w4a16_gemm_decode_noalloc(const void* X, int64_t M, int64_t K, const void* packed,
+                                       const void* scales, const void* zeros, int64_t N,
+                                       int32_t g, int32_t sym, void* Y, void* stream) {
+    w4a16_plan p;
+    w4a16_status st = make_plan(M, N, K, g, sym, W4A16_PATH_DECODE, 0, current_sm_count(), &p);
+    if (st != W4A16_OK) return st;
+    if (M == 0 || N == 0) return W4A16_OK;
+    if (!X || !packed || !scales || !Y || (!sym && !zeros)) return W4A16_EINVAL;
+    if (!aligned16(X) || !aligned16(packed) || !aligned16(scales) || !aligned16(Y) ||
+        (!sym && !aligned16(zeros)))
+        return W4A16_EINVAL;
+    if ((size_t)p.workspace_bytes > W4A16_NOALLOC_SCRATCH_BYTES) return W4A16_EWORKSPACE;
+    DeviceInfo di;
+    if ((st = device_info(&di)) != W4A16_OK) return st;
+    void* scratch = nullptr;
+    if ((st = noalloc_scratch(&scratch)) != W4A16_OK) return st;
+    return launch_decode(p, X, M, K, packed, scales, zeros, N, g, sym, Y, scratch,
+                         static_cast<cudaStream_t>(stream));
 }
 
 w4a16_status w4a16_device_error(int32_t* code) {
