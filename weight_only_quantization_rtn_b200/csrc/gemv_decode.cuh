@@ -127,6 +127,7 @@ struct DecodeArgs {
     int stage_bytes;      // packed + X + scale/zero bytes per stage (multiple of 1024)
     int sz_offset;        // offset of the scale/zero block inside a stage
     int sz_async;         // 1: scale rows are 4-byte aligned, copy with cp.async
+    int sz_tma;           // 1: scale rows are 16-byte aligned, copy with TMA (tmS, tmZ)
     int64_t U;            // units = RB · KBn
 };
 
@@ -144,7 +145,9 @@ __device__ __forceinline__ void cp_async_arrive_noinc(uint32_t bar) {
 template <int MB, bool SYM, int G>
 __global__ void __launch_bounds__(kDecThreads, MB == 1 ? 2 : 1)
     gemv_decode_kernel(const __grid_constant__ CUtensorMap tmP,
-                       const __grid_constant__ CUtensorMap tmX, const DecodeArgs a) {
+                       const __grid_constant__ CUtensorMap tmX,
+                       const __grid_constant__ CUtensorMap tmS,
+                       const __grid_constant__ CUtensorMap tmZ, const DecodeArgs a) {
     constexpr int GB = kDecBlockK / G;                 // groups per row per unit
     constexpr int RED = 2 * MB * 128;                  // partial elements per row block
 
@@ -171,7 +174,8 @@ __global__ void __launch_bounds__(kDecThreads, MB == 1 ? 2 : 1)
 
     if (threadIdx.x == 0) {
         for (int s = 0; s < S; ++s) {
-            mbar_init(smem_u32(&full[s]), 1 + 32);     // TMA expect_tx arrive + 32 scale lanes
+            // TMA expect_tx arrive (+ 32 scale-copying lanes when scales are not copied by TMA)
+            mbar_init(smem_u32(&full[s]), a.sz_tma ? 1 : 1 + 32);
             mbar_init(smem_u32(&empty[s]), kDecConsumers);
         }
         *abort_flag = 0;
@@ -185,8 +189,13 @@ __global__ void __launch_bounds__(kDecThreads, MB == 1 ? 2 : 1)
         if (lane == 0) {
             prefetch_tensormap(&tmP);
             prefetch_tensormap(&tmX);
+            if (a.sz_tma) {
+                prefetch_tensormap(&tmS);
+                if (!SYM) prefetch_tensormap(&tmZ);
+            }
         }
-        const uint32_t tx = (uint32_t)kDecPBytes + 4u * xbox_bytes;
+        const uint32_t sz_tx = a.sz_tma ? (uint32_t)((SYM ? 1 : 2) * kDecRows * GB * 2) : 0u;
+        const uint32_t tx = (uint32_t)kDecPBytes + 4u * xbox_bytes + sz_tx;
         // Weights (packed codes, scales, zeros) never depend on the preceding
         // kernel, so the first ring's worth is requested before waiting for it;
         // X, and everything this grid writes, comes after the wait.
@@ -222,11 +231,17 @@ __global__ void __launch_bounds__(kDecThreads, MB == 1 ? 2 : 1)
                 }
             }
             if (i < pre) pre_kb[i] = kb;
-            // scales (and zeros): 32 rows x GB groups; lane -> consecutive group pairs of a row
+            // scales (and zeros): 32 rows x GB groups
             uint16_t* sz = reinterpret_cast<uint16_t*>(st + a.sz_offset);
             const int g0 = kb * GB;
             const int arrays = SYM ? 1 : 2;
-            if (a.sz_async) {
+            if (a.sz_tma) {
+                if (lane == 0) {
+                    tma_load_2d(smem_u32(sz), &tmS, g0, rb * kDecRows, bar);
+                    if (!SYM) tma_load_2d(smem_u32(sz + kDecRows * GB), &tmZ, g0, rb * kDecRows, bar);
+                }
+            } else if (a.sz_async) {
+                // lane -> consecutive group pairs of a row
 #pragma unroll 1
                 for (int e = lane; e < kDecRows * (GB / 2); e += 32) {
                     const int r = e / (GB / 2);
@@ -350,32 +365,37 @@ __global__ void __launch_bounds__(kDecThreads, MB == 1 ? 2 : 1)
                     }
                 }
             }
-            // A fragments: rows 16t + g + 8h, 16 bytes at chunk c of the unit (128-byte swizzle)
+            // A fragments: rows 16t + g + 8h, 16 bytes at chunk c of the unit (128-byte swizzle).
+            // Both 16-row tiles are loaded first and their MMA chains interleaved.
             const uint8_t* pb = st + (c >> 1) * 4096 + ((((c & 1) << 2) | q) ^ g) * 16 + g * 128;
+            uint32_t w[2][2][4];
+            uint32_t ss[2][2], zz[2][2];
 #pragma unroll
             for (int t = 0; t < 2; ++t) {
-                const uint4 w0v = lds128(pb + (16 * t) * 128);
-                const uint4 w1v = lds128(pb + (16 * t + 8) * 128);
-                const int r0 = 16 * t + g, r1 = r0 + 8;
-                const uint32_t ss0 = dup16(lds_u16(ssm + r0 * GB + grp_local));
-                const uint32_t ss1 = dup16(lds_u16(ssm + r1 * GB + grp_local));
-                const uint32_t zz0 =
-                    SYM ? 0x43084308u : bf16x2_add(dup16(lds_u16(zsm + r0 * GB + grp_local)), 0x43004300u);
-                const uint32_t zz1 =
-                    SYM ? 0x43084308u : bf16x2_add(dup16(lds_u16(zsm + r1 * GB + grp_local)), 0x43004300u);
-                const uint32_t w0[4] = {w0v.x, w0v.y, w0v.z, w0v.w};
-                const uint32_t w1[4] = {w1v.x, w1v.y, w1v.z, w1v.w};
 #pragma unroll
-                for (int ii = 0; ii < 4; ++ii) {
+                for (int hr = 0; hr < 2; ++hr) {
+                    const uint4 v = lds128(pb + (16 * t + 8 * hr) * 128);
+                    w[t][hr][0] = v.x; w[t][hr][1] = v.y; w[t][hr][2] = v.z; w[t][hr][3] = v.w;
+                    const int r = 16 * t + 8 * hr + g;
+                    ss[t][hr] = __byte_perm(lds_u16(ssm + r * GB + grp_local), 0, 0x1010);
+                    zz[t][hr] = SYM ? 0x43084308u
+                                    : bf16x2_add(__byte_perm(lds_u16(zsm + r * GB + grp_local), 0, 0x1010),
+                                                 0x43004300u);
+                }
+            }
 #pragma unroll
-                    for (int hh = 0; hh < 2; ++hh) {
+            for (int ii = 0; ii < 4; ++ii) {
+#pragma unroll
+                for (int hh = 0; hh < 2; ++hh) {
+#pragma unroll
+                    for (int t = 0; t < 2; ++t) {
                         // fragment registers produced in the order the MMA reads them:
                         // (row g, k-pair lo) (row g+8, lo) (row g, hi) (row g+8, hi)
                         uint32_t fa[4];
-                        fa[0] = dq_pair<SYM>(w0[ii] >> (8 * hh), zz0, ss0);
-                        fa[1] = dq_pair<SYM>(w1[ii] >> (8 * hh), zz1, ss1);
-                        fa[2] = dq_pair<SYM>(w0[ii] >> (8 * hh + 4), zz0, ss0);
-                        fa[3] = dq_pair<SYM>(w1[ii] >> (8 * hh + 4), zz1, ss1);
+                        fa[0] = dq_pair<SYM>(w[t][0][ii] >> (8 * hh), zz[t][0], ss[t][0]);
+                        fa[1] = dq_pair<SYM>(w[t][1][ii] >> (8 * hh), zz[t][1], ss[t][1]);
+                        fa[2] = dq_pair<SYM>(w[t][0][ii] >> (8 * hh + 4), zz[t][0], ss[t][0]);
+                        fa[3] = dq_pair<SYM>(w[t][1][ii] >> (8 * hh + 4), zz[t][1], ss[t][1]);
 #pragma unroll
                         for (int mb = 0; mb < MB; ++mb)
                             mma_bf16_16816(acc[t][mb], fa[0], fa[1], fa[2], fa[3], bf[mb][ii][hh][0],
@@ -409,18 +429,17 @@ __global__ void __launch_bounds__(kDecThreads, MB == 1 ? 2 : 1)
                 for (int w = 0; w < kDecConsumers; ++w) sum += red[w * RED + e];
                 v[k] = sum;
             }
+            // The row block is whole here iff all its units lie in this CTA's range.
             const int64_t first_u = (int64_t)rb * a.KBn;
-            const int64_t c_first = owner_of(first_u, a.U, C);
-            const int64_t c_last = owner_of(first_u + a.KBn - 1, a.U, C);
-            if (c_first != c_last) {
+            const bool whole = first_u >= u0 && first_u + a.KBn <= u1;
+            if (!whole) {
                 // split row block: publish this CTA's part; the fixup kernel adds the parts
                 float* part = a.ws_part + (int64_t)(rb + cta) * RED;
 #pragma unroll
                 for (int k = 0; k < MB; ++k) part[tid + 256 * k] = v[k];
             }
             named_bar_sync(1, kDecConsumers * 32);   // red[] is rewritten at the next row block
-            const bool write_now = c_first == c_last;
-            if (write_now) {
+            if (whole) {
 #pragma unroll
                 for (int k = 0; k < MB; ++k) {
                     const int e = tid + 256 * k;

@@ -240,7 +240,8 @@ w4a16_status encode_2d(CUtensorMap* map, CUtensorMapDataType dtype, const void* 
 // ---------------------------------------------------------------- decode launch
 template <int MB, bool SYM, int G>
 w4a16_status launch_decode_t(const w4a16_plan& p, const CUtensorMap& tmP, const CUtensorMap& tmX,
-                             const DecodeArgs& args, bool has_split, cudaStream_t stream) {
+                             const CUtensorMap& tmS, const CUtensorMap& tmZ, const DecodeArgs& args,
+                             bool has_split, cudaStream_t stream) {
     auto kern = gemv_decode_kernel<MB, SYM, G>;
     static bool attr_set[kMaxDevices] = {};
     int dev = 0;
@@ -263,7 +264,7 @@ w4a16_status launch_decode_t(const w4a16_plan& p, const CUtensorMap& tmP, const 
     cfg.stream = stream;
     cfg.attrs = attr;
     cfg.numAttrs = 1;
-    if (cudaLaunchKernelEx(&cfg, kern, tmP, tmX, args) != cudaSuccess) return W4A16_ECUDA;
+    if (cudaLaunchKernelEx(&cfg, kern, tmP, tmX, tmS, tmZ, args) != cudaSuccess) return W4A16_ECUDA;
     if (has_split) {
         cudaLaunchConfig_t fcfg = cfg;
         fcfg.gridDim = dim3((unsigned)(p.grid - 1), 1, 1);
@@ -301,26 +302,42 @@ w4a16_status launch_decode(const w4a16_plan& p, const void* X, int64_t M, int64_
     args.stage_bytes = d.stage_bytes;
     args.sz_offset = decode_sz_offset(M);
     args.sz_async = ((K / g) % 2 == 0) ? 1 : 0;   // 4-byte aligned scale rows
+    args.sz_tma = ((K / g) % 8 == 0) ? 1 : 0;     // 16-byte aligned scale rows
     args.U = d.units;
     const bool split = p.kernels > 1;
+    // Scales and zeros [N][K/g]: boxes of 32 rows x (1024/g) groups, when their rows are
+    // 16-byte aligned; otherwise the kernel copies them with cp.async and these are unused.
+    CUtensorMap tmS = tmP, tmZ = tmP;
+    if (args.sz_tma) {
+        st = encode_2d(&tmS, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, scales, (uint64_t)(K / g),
+                       (uint64_t)N, (uint64_t)(K / g) * 2, (uint32_t)(kDecBlockK / g), kDecRows,
+                       CU_TENSOR_MAP_SWIZZLE_NONE);
+        if (st != W4A16_OK) return st;
+        if (!sym) {
+            st = encode_2d(&tmZ, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, zeros, (uint64_t)(K / g),
+                           (uint64_t)N, (uint64_t)(K / g) * 2, (uint32_t)(kDecBlockK / g), kDecRows,
+                           CU_TENSOR_MAP_SWIZZLE_NONE);
+            if (st != W4A16_OK) return st;
+        }
+    }
     if (d.mb == 1) {
         if (sym) {
-            if (g == 32) return launch_decode_t<1, true, 32>(p, tmP, tmX, args, split, stream);
-            if (g == 64) return launch_decode_t<1, true, 64>(p, tmP, tmX, args, split, stream);
-            return launch_decode_t<1, true, 128>(p, tmP, tmX, args, split, stream);
+            if (g == 32) return launch_decode_t<1, true, 32>(p, tmP, tmX, tmS, tmZ, args, split, stream);
+            if (g == 64) return launch_decode_t<1, true, 64>(p, tmP, tmX, tmS, tmZ, args, split, stream);
+            return launch_decode_t<1, true, 128>(p, tmP, tmX, tmS, tmZ, args, split, stream);
         }
-        if (g == 32) return launch_decode_t<1, false, 32>(p, tmP, tmX, args, split, stream);
-        if (g == 64) return launch_decode_t<1, false, 64>(p, tmP, tmX, args, split, stream);
-        return launch_decode_t<1, false, 128>(p, tmP, tmX, args, split, stream);
+        if (g == 32) return launch_decode_t<1, false, 32>(p, tmP, tmX, tmS, tmZ, args, split, stream);
+        if (g == 64) return launch_decode_t<1, false, 64>(p, tmP, tmX, tmS, tmZ, args, split, stream);
+        return launch_decode_t<1, false, 128>(p, tmP, tmX, tmS, tmZ, args, split, stream);
     }
     if (sym) {
-        if (g == 32) return launch_decode_t<2, true, 32>(p, tmP, tmX, args, split, stream);
-        if (g == 64) return launch_decode_t<2, true, 64>(p, tmP, tmX, args, split, stream);
-        return launch_decode_t<2, true, 128>(p, tmP, tmX, args, split, stream);
+        if (g == 32) return launch_decode_t<2, true, 32>(p, tmP, tmX, tmS, tmZ, args, split, stream);
+        if (g == 64) return launch_decode_t<2, true, 64>(p, tmP, tmX, tmS, tmZ, args, split, stream);
+        return launch_decode_t<2, true, 128>(p, tmP, tmX, tmS, tmZ, args, split, stream);
     }
-    if (g == 32) return launch_decode_t<2, false, 32>(p, tmP, tmX, args, split, stream);
-    if (g == 64) return launch_decode_t<2, false, 64>(p, tmP, tmX, args, split, stream);
-    return launch_decode_t<2, false, 128>(p, tmP, tmX, args, split, stream);
+    if (g == 32) return launch_decode_t<2, false, 32>(p, tmP, tmX, tmS, tmZ, args, split, stream);
+    if (g == 64) return launch_decode_t<2, false, 64>(p, tmP, tmX, tmS, tmZ, args, split, stream);
+    return launch_decode_t<2, false, 128>(p, tmP, tmX, tmS, tmZ, args, split, stream);
 }
 
 template <int BM, bool SYM, int G>
