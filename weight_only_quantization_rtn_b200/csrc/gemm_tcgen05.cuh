@@ -11,25 +11,29 @@
 // i.e. the CTA computes a 128 (n) x BM (m) tile of Yᵀ, with the dequantized
 // weights as the UMMA A operand (M = 128) and the activations as B (N = BM).
 //
-// Warp roles (6 warps):
+// Warp roles (10 warps):
 //   warp 0      producer: per 64-wide K block, one lane issues a TMA load of the
 //               X tile (BM x 64 bf16, 128-byte swizzle) and one of the packed
-//               tile (128 rows x 32 bytes); all 32 lanes copy the block's scales
-//               and zero points (one aligned pair of groups per row) into the
-//               stage with 4-byte cp.async copies.  Both complete on the stage's
-//               "full" barrier, so the dequantizers never wait on global loads.
+//               tile (128 rows x 32 bytes, 32-byte swizzle).  Scales and zero
+//               points arrive by TMA in slabs of 8 groups x 128 rows (one slab
+//               serves g/8 K blocks, a two-slot ring with its own barriers) when
+//               their rows are 16-byte aligned; otherwise all 32 lanes copy the
+//               block's aligned pair of groups per row into the stage with 4-byte
+//               cp.async copies that complete on the stage's "full" barrier.
 //   warp 1      TMEM allocator and, on one elected lane, the MMA issuer: waits
 //               for the stage's X tile and dequantized A tile, issues four
 //               tcgen05.mma (K = 16 each), and commits to the stage's "empty"
 //               barrier so producer and dequantizers may reuse it.
-//   warps 2..5  dequantizers, one weight row per thread: nibbles from the packed
-//               tile -> bf16 pairs (q − z)·s -> 16-byte chunks written into the
-//               A tile in the 128-byte swizzled K-major layout the UMMA
-//               descriptor expects; fence.proxy.async makes the generic-proxy
-//               writes visible to the tensor core before the "a_full" arrive.
-//               After the K loop the same warps drain TMEM (tcgen05.ld), round
-//               to bf16 and store Y.  Warp w reads TMEM lanes 32·(w%4)..+31,
-//               which are the rows it dequantized.
+//   warps 2..9  dequantizers, two per SM sub-partition: thread (w, l) takes
+//               weight row 32·(w%4) + l and K half (w−2)/4 of the block: nibbles
+//               from the packed tile -> bf16 pairs (q − z)·s -> 16-byte chunks
+//               written into the A tile in the 128-byte swizzled K-major layout
+//               the UMMA descriptor expects; fence.proxy.async makes the
+//               generic-proxy writes visible to the tensor core before the
+//               "a_full" arrive.  After the K loop the same warps drain TMEM
+//               (tcgen05.ld), round to bf16 and store Y: warp w reads TMEM lanes
+//               32·(w%4)..+31, the rows it dequantized, and every other 32-column
+//               block of the accumulator.
 //
 // Every barrier wait is bounded (about one second); a timeout records an error
 // in the device error word and the role stops issuing work, then the CTA
@@ -40,7 +44,8 @@
 
 namespace w4a16 {
 
-constexpr int kTcThreads = 192;
+constexpr int kTcDequantWarps = 8;
+constexpr int kTcThreads = (2 + kTcDequantWarps) * 32;
 constexpr int kTcBlockK = 64;                 // K per pipeline stage (one 128-byte swizzle row)
 constexpr int kTcTileN = 128;                 // UMMA M: weight rows per CTA
 
@@ -51,11 +56,13 @@ struct TcConfig {
     static constexpr int kPBytes = kTcTileN * kTcBlockK / 2;    // packed codes tile
     static constexpr int kSZBytes = 2 * kTcTileN * 4;              // scale and zero pairs per row
     static constexpr int kStageBytes = kXBytes + kABytes + kPBytes + kSZBytes;
-    static constexpr int kBudget = 220 * 1024;
+    static constexpr int kSlabBytes = 2 * 2 * kTcTileN * 8 * 2;  // two slots of scale + zero slabs
+    static constexpr int kBudget = 220 * 1024 - kSlabBytes;
     static constexpr int kStagesRaw = kBudget / kStageBytes;
     static constexpr int kStages = kStagesRaw > 8 ? 8 : kStagesRaw;
     static constexpr int kBarrierBytes = 1024;
-    static constexpr int kSmemBytes = kStages * kStageBytes + kBarrierBytes + 1024;  // + align slack
+    static constexpr int kSmemBytes =
+        kStages * kStageBytes + kSlabBytes + kBarrierBytes + 1024;   // + align slack
     static constexpr int kTmemCols = BM < 32 ? 32 : BM;
 };
 
@@ -63,7 +70,9 @@ template <int BM, bool SYM, int G>
 __global__ void __launch_bounds__(kTcThreads, 1)
     gemm_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ CUtensorMap tmP,
                    const uint16_t* __restrict__ scales, const uint16_t* __restrict__ zeros,
-                   uint16_t* __restrict__ Y, int M, int N, int K, int sz_async) {
+                   uint16_t* __restrict__ Y, int M, int N, int K, int sz_async,
+                   const __grid_constant__ CUtensorMap tmS, const __grid_constant__ CUtensorMap tmZ,
+                   int sz_tma) {
     using Cfg = TcConfig<BM>;
     constexpr int S = Cfg::kStages;
     static_assert(S >= 2, "pipeline needs at least two stages");
@@ -76,12 +85,16 @@ __global__ void __launch_bounds__(kTcThreads, 1)
     uint8_t* as = xs + S * Cfg::kXBytes;                  // S x kABytes
     uint8_t* ps = as + S * Cfg::kABytes;                  // S x kPBytes
     uint32_t* szs = reinterpret_cast<uint32_t*>(ps + S * Cfg::kPBytes);   // S x [2][128] u32 pairs
-    uint64_t* bars = reinterpret_cast<uint64_t*>(szs + S * 2 * kTcTileN);
+    uint16_t* slab = reinterpret_cast<uint16_t*>(szs + S * 2 * kTcTileN); // 2 x [2][128][8] u16
+    uint64_t* bars = reinterpret_cast<uint64_t*>(slab + 2 * 2 * kTcTileN * 8);
     uint64_t* full = bars;             // TMA bytes landed
     uint64_t* afull = bars + S;        // dequantized A tile written
     uint64_t* empty = bars + 2 * S;    // MMAs reading the stage retired
     uint64_t* accf = bars + 3 * S;     // all MMAs retired
-    uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(bars + 3 * S + 1);
+    uint64_t* slab_full = bars + 3 * S + 1;    // [2] slab of scales/zeros landed
+    uint64_t* slab_empty = bars + 3 * S + 3;   // [2] dequantizers done with the slab
+    uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(bars + 3 * S + 5);
+    constexpr int kSlabKb = 8 * G / kTcBlockK;   // K blocks served by one slab of 8 groups
 
     const int warp = threadIdx.x >> 5;
     const int lane = threadIdx.x & 31;
@@ -92,16 +105,24 @@ __global__ void __launch_bounds__(kTcThreads, 1)
 
     if (threadIdx.x == 0) {
         for (int s = 0; s < S; ++s) {
-            mbar_init(smem_u32(&full[s]), 1 + 32);   // TMA expect_tx arrive + 32 scale lanes
-            mbar_init(smem_u32(&afull[s]), 128);
+            mbar_init(smem_u32(&full[s]), sz_tma ? 1 : 1 + 32);   // TMA arrive (+ 32 scale lanes)
+            mbar_init(smem_u32(&afull[s]), kTcDequantWarps);
             mbar_init(smem_u32(&empty[s]), 1);
         }
         mbar_init(smem_u32(accf), 1);
+        for (int t = 0; t < 2; ++t) {
+            mbar_init(smem_u32(&slab_full[t]), 1);
+            mbar_init(smem_u32(&slab_empty[t]), kTcDequantWarps);
+        }
         fence_mbar_init();
     }
     if (warp == 0 && lane == 0) {
         prefetch_tensormap(&tmX);
         prefetch_tensormap(&tmP);
+        if (sz_tma) {
+            prefetch_tensormap(&tmS);
+            if (!SYM) prefetch_tensormap(&tmZ);
+        }
     }
     if (warp == 1) {
         tmem_alloc(smem_u32(tmem_holder), Cfg::kTmemCols);
@@ -122,6 +143,20 @@ __global__ void __launch_bounds__(kTcThreads, 1)
             if (lane == 0) ok = mbar_wait(smem_u32(&empty[s]), ph ^ 1u);   // one lane waits
             if (!__shfl_sync(0xffffffffu, ok ? 1 : 0, 0)) break;
             const uint32_t bar = smem_u32(&full[s]);
+            if (sz_tma && kb % kSlabKb == 0) {
+                // next slab of scales/zeros: its slot is free once the dequantizers
+                // finished the slab two back
+                const int t = kb / kSlabKb, slot = t & 1;
+                if (lane == 0) ok = mbar_wait(smem_u32(&slab_empty[slot]), ((uint32_t)(t >> 1) & 1u) ^ 1u);
+                if (!__shfl_sync(0xffffffffu, ok ? 1 : 0, 0)) break;
+                if (lane == 0) {
+                    const uint32_t sb = smem_u32(&slab_full[slot]);
+                    uint16_t* dsl = slab + slot * 2 * kTcTileN * 8;
+                    mbar_arrive_expect_tx(sb, (SYM ? 1 : 2) * kTcTileN * 8 * 2);
+                    tma_load_2d(smem_u32(dsl), &tmS, t * 8, n0, sb);
+                    if (!SYM) tma_load_2d(smem_u32(dsl + kTcTileN * 8), &tmZ, t * 8, n0, sb);
+                }
+            }
             if (lane == 0) {
                 mbar_arrive_expect_tx(bar, Cfg::kXBytes + Cfg::kPBytes);
                 tma_load_2d(smem_u32(xs + s * Cfg::kXBytes), &tmX, kb * kTcBlockK, m0, bar);
@@ -130,7 +165,9 @@ __global__ void __launch_bounds__(kTcThreads, 1)
             // the aligned pair of groups holding this block's group(s), per row and array
             const int jpair = ((kb * kTcBlockK) / G) & ~1;
             uint32_t* dst = szs + s * 2 * kTcTileN;
-            if (sz_async) {
+            if (sz_tma) {
+                // scales/zeros come with the slab
+            } else if (sz_async) {
 #pragma unroll
                 for (int e = lane; e < 2 * kTcTileN; e += 32) {
                     const int arr = e / kTcTileN, r = e % kTcTileN;
@@ -164,6 +201,11 @@ __global__ void __launch_bounds__(kTcThreads, 1)
             for (int kb = (issued > S ? issued - S : 0); kb < issued; ++kb) {
                 if (!mbar_wait(smem_u32(&full[kb % S]), (uint32_t)(kb / S) & 1u)) break;
             }
+            if (sz_tma && issued > 0) {
+                const int slabs = (issued - 1) / kSlabKb + 1;   // slabs requested so far
+                for (int t = (slabs > 2 ? slabs - 2 : 0); t < slabs; ++t)
+                    if (!mbar_wait(smem_u32(&slab_full[t & 1]), (uint32_t)(t >> 1) & 1u)) break;
+            }
         }
     } else if (warp == 1) {
         // ------------------------------------------------------------ MMA issuer
@@ -192,27 +234,46 @@ __global__ void __launch_bounds__(kTcThreads, 1)
     } else {
         // ------------------------------------------------------------ dequantize
         const int r = (warp & 3) * 32 + lane;   // weight row within the tile == TMEM lane
+        const int h = (warp - 2) >> 2;          // K half of each 64-wide block
         const int n = n0 + r;
         const bool row_ok = n < N;
         bool ok = true;
         for (int kb = 0; kb < num_kb; ++kb) {
             const int s = kb % S;
             const uint32_t ph = (uint32_t)(kb / S) & 1u;
+            const int t = kb / kSlabKb, slot = t & 1;
+            if (sz_tma && kb % kSlabKb == 0 &&
+                !mbar_wait(smem_u32(&slab_full[slot]), (uint32_t)(t >> 1) & 1u)) {
+                ok = false;
+                break;
+            }
             if (!mbar_wait(smem_u32(&full[s]), ph)) {
                 ok = false;
                 break;
             }
-            const uint32_t spair = lds_u32(szs + s * 2 * kTcTileN + r);
-            const uint32_t zpair = SYM ? 0u : lds_u32(szs + s * 2 * kTcTileN + kTcTileN + r);
+            uint32_t spair = 0u, zpair = 0u;
+            if (!sz_tma) {
+                spair = lds_u32(szs + s * 2 * kTcTileN + r);
+                zpair = SYM ? 0u : lds_u32(szs + s * 2 * kTcTileN + kTcTileN + r);
+            }
+            const uint16_t* srow = slab + slot * 2 * kTcTileN * 8 + r * 8;
             const uint8_t* prow = ps + s * Cfg::kPBytes + r * 32;
             const uint32_t arow = smem_u32(as + s * Cfg::kABytes + r * 128);
-#pragma unroll
-            for (int h = 0; h < 2; ++h) {
-                const uint4 v = lds128(prow + 16 * h);
-                const int half = ((kb * kTcBlockK + 32 * h) / G) & 1;   // position in the pair
-                const uint32_t ss = dup16(spair >> (16 * half));
-                const uint32_t zz = SYM ? 0x43084308u
-                                        : bf16x2_add(dup16(zpair >> (16 * half)), 0x43004300u);
+            {
+                // 32-byte swizzle: chunk h of row r sits at position h ^ bit 2 of r
+                const uint4 v = lds128(prow + 16 * (h ^ ((r >> 2) & 1)));
+                uint32_t ss, zz;
+                if (sz_tma) {
+                    const int gi = ((kb * kTcBlockK + 32 * h) / G) % 8;   // group within the slab
+                    ss = __byte_perm(lds_u16(srow + gi), 0, 0x1010);
+                    zz = SYM ? 0x43084308u
+                             : bf16x2_add(__byte_perm(lds_u16(srow + kTcTileN * 8 + gi), 0, 0x1010),
+                                          0x43004300u);
+                } else {
+                    const int half = ((kb * kTcBlockK + 32 * h) / G) & 1;   // position in the pair
+                    ss = dup16(spair >> (16 * half));
+                    zz = SYM ? 0x43084308u : bf16x2_add(dup16(zpair >> (16 * half)), 0x43004300u);
+                }
                 const uint32_t wv[4] = {v.x, v.y, v.z, v.w};
 #pragma unroll
                 for (int i = 0; i < 4; ++i) {
@@ -226,14 +287,18 @@ __global__ void __launch_bounds__(kTcThreads, 1)
                 }
             }
             fence_proxy_async_smem();
-            mbar_arrive(smem_u32(&afull[s]));
+            __syncwarp();
+            if (lane == 0) mbar_arrive(smem_u32(&afull[s]));
+            if (sz_tma && (kb % kSlabKb == kSlabKb - 1 || kb == num_kb - 1)) {
+                if (lane == 0) mbar_arrive(smem_u32(&slab_empty[slot]));
+            }
         }
         // ------------------------------------------------------------ epilogue
         if (ok && mbar_wait(smem_u32(accf), 0)) {
             tc_fence_after();
             const uint32_t t_lane = (uint32_t)((warp & 3) * 32) << 16;
 #pragma unroll 1
-            for (int cb = 0; cb < BM / 32; ++cb) {
+            for (int cb = h; cb < BM / 32; cb += 2) {
                 uint32_t v[32];
                 tmem_ld_32x32b_x32(tmem_d + t_lane + cb * 32, v);
                 tmem_wait_ld();

@@ -342,6 +342,7 @@ w4a16_status launch_decode(const w4a16_plan& p, const void* X, int64_t M, int64_
 
 template <int BM, bool SYM, int G>
 w4a16_status launch_tc_t(const w4a16_plan& p, const CUtensorMap& tmX, const CUtensorMap& tmP,
+                         const CUtensorMap& tmS, const CUtensorMap& tmZ, int sz_tma,
                          const void* scales, const void* zeros, void* Y, int M, int N, int K,
                          cudaStream_t stream) {
     auto kern = gemm_tc_kernel<BM, SYM, G>;
@@ -358,20 +359,24 @@ w4a16_status launch_tc_t(const w4a16_plan& p, const CUtensorMap& tmX, const CUte
     dim3 grid((unsigned)((N + kTcTileN - 1) / kTcTileN), (unsigned)((M + BM - 1) / BM), 1);
     kern<<<grid, kTcThreads, TcConfig<BM>::kSmemBytes, stream>>>(
         tmX, tmP, static_cast<const uint16_t*>(scales), static_cast<const uint16_t*>(zeros),
-        static_cast<uint16_t*>(Y), M, N, K, sz_async);
+        static_cast<uint16_t*>(Y), M, N, K, sz_async, tmS, tmZ, sz_tma);
     return launch_status();
 }
 
 template <bool SYM, int G>
 w4a16_status launch_tc_g(const w4a16_plan& p, const CUtensorMap& tmX, const CUtensorMap& tmP,
+                         const CUtensorMap& tmS, const CUtensorMap& tmZ, int sz_tma,
                          const void* scales, const void* zeros, void* Y, int M, int N, int K,
                          cudaStream_t stream) {
+#define W4A16_TC_TILE(BMV) \
+    launch_tc_t<BMV, SYM, G>(p, tmX, tmP, tmS, tmZ, sz_tma, scales, zeros, Y, M, N, K, stream)
     switch (p.tile_m) {
-        case 32: return launch_tc_t<32, SYM, G>(p, tmX, tmP, scales, zeros, Y, M, N, K, stream);
-        case 64: return launch_tc_t<64, SYM, G>(p, tmX, tmP, scales, zeros, Y, M, N, K, stream);
-        case 128: return launch_tc_t<128, SYM, G>(p, tmX, tmP, scales, zeros, Y, M, N, K, stream);
-        default: return launch_tc_t<256, SYM, G>(p, tmX, tmP, scales, zeros, Y, M, N, K, stream);
+        case 32: return W4A16_TC_TILE(32);
+        case 64: return W4A16_TC_TILE(64);
+        case 128: return W4A16_TC_TILE(128);
+        default: return W4A16_TC_TILE(256);
     }
+#undef W4A16_TC_TILE
 }
 
 w4a16_status launch_tc(const w4a16_plan& p, const void* X, int64_t M, int64_t K,
@@ -383,13 +388,29 @@ w4a16_status launch_tc(const w4a16_plan& p, const void* X, int64_t M, int64_t K,
                                 CU_TENSOR_MAP_SWIZZLE_128B);
     if (st != W4A16_OK) return st;
     st = encode_2d(&tmP, CU_TENSOR_MAP_DATA_TYPE_UINT8, packed, (uint64_t)(K / 2), (uint64_t)N,
-                   (uint64_t)(K / 2), kTcBlockK / 2, kTcTileN, CU_TENSOR_MAP_SWIZZLE_NONE);
+                   (uint64_t)(K / 2), kTcBlockK / 2, kTcTileN, CU_TENSOR_MAP_SWIZZLE_32B);
     if (st != W4A16_OK) return st;
+    // Scales and zeros [N][K/g] in slabs of 8 groups x 128 rows, when their rows are
+    // 16-byte aligned; otherwise the kernel copies them with cp.async.
+    const int sz_tma = ((K / g) % 8 == 0) ? 1 : 0;
+    CUtensorMap tmS = tmP, tmZ = tmP;
+    if (sz_tma) {
+        st = encode_2d(&tmS, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, scales, (uint64_t)(K / g), (uint64_t)N,
+                       (uint64_t)(K / g) * 2, 8, kTcTileN, CU_TENSOR_MAP_SWIZZLE_NONE);
+        if (st != W4A16_OK) return st;
+        if (!sym) {
+            st = encode_2d(&tmZ, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, zeros, (uint64_t)(K / g),
+                           (uint64_t)N, (uint64_t)(K / g) * 2, 8, kTcTileN, CU_TENSOR_MAP_SWIZZLE_NONE);
+            if (st != W4A16_OK) return st;
+        }
+    }
     const int m = (int)M, n = (int)N, k = (int)K;
-#define W4A16_TC_CASE(GG)                                                                     \
-    case GG:                                                                                  \
-        return sym ? launch_tc_g<true, GG>(p, tmX, tmP, scales, zeros, Y, m, n, k, stream)      \
-                   : launch_tc_g<false, GG>(p, tmX, tmP, scales, zeros, Y, m, n, k, stream);
+#define W4A16_TC_CASE(GG)                                                                      \
+    case GG:                                                                                   \
+        return sym ? launch_tc_g<true, GG>(p, tmX, tmP, tmS, tmZ, sz_tma, scales, zeros, Y, m, n, \
+                                           k, stream)                                          \
+                   : launch_tc_g<false, GG>(p, tmX, tmP, tmS, tmZ, sz_tma, scales, zeros, Y, m, n, \
+                                            k, stream);
     switch (g) {
         W4A16_TC_CASE(32)
         W4A16_TC_CASE(64)
