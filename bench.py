@@ -63,10 +63,18 @@ def algorithmic_bytes(M: int, N: int, K: int, g: int, sym: bool) -> int:
     return N * K // 2 + 2 * N * (K // g) * (1 if sym else 2) + 2 * M * K + 2 * M * N
 
 
-def kernel_source_digest() -> str:
+# Sources each timed kernel is built from (its device code, the shared device
+# helpers, and the host file that chooses its launch configuration).
+KERNEL_SOURCES = {
+    "gemv_decode_kernel": ("common.cuh", "gemv_decode.cuh", "w4a16.cu"),
+    "gemm_tc_kernel": ("common.cuh", "gemm_tcgen05.cuh", "w4a16.cu"),
+}
+
+
+def kernel_source_digest(kernel: str) -> str:
     h = hashlib.sha256()
     csrc = os.path.join(ROOT, "weight_only_quantization_rtn_b200", "csrc")
-    for name in sorted(os.listdir(csrc)):
+    for name in KERNEL_SOURCES[kernel]:
         with open(os.path.join(csrc, name), "rb") as f:
             h.update(name.encode())
             h.update(f.read())
@@ -75,13 +83,14 @@ def kernel_source_digest() -> str:
 
 def ncu_traffic(kernel_key: str):
     """DRAM bytes per launch from a committed ncu capture of the current kernel
-    source, or None when the capture is missing or the kernel changed since."""
+    source (profiles/ncu_traffic.json, key "<kernel>:<workload>"), or None when
+    the capture is missing or the kernel's sources changed since."""
     path = os.path.join(ROOT, "profiles", "ncu_traffic.json")
     try:
         with open(path) as f:
             table = json.load(f)
         entry = table[kernel_key]
-        if entry.get("kernel_source_digest") != kernel_source_digest():
+        if entry.get("kernel_source_digest") != kernel_source_digest(kernel_key.split(":")[0]):
             return None
         return float(entry["dram_bytes_per_launch"])
     except (OSError, KeyError, ValueError):
@@ -621,6 +630,62 @@ def prefill_extra(w4, peaks, peak_src, l2, dev, iters=50):
     return res
 
 
+def crossover_sweep(args):
+    """M-dispatch evidence: at K=N=8192 time each kernel that can run each M
+    (decode for M <= 16, tensor-core for every M) and a dense bf16 cuBLAS GEMM
+    of the same shape, with inputs rotated over copies larger than L2.  Prints
+    one JSON object {"crossover": [...]}; not a benchmark line."""
+    import weight_only_quantization_rtn_b200 as w4
+    from weight_only_quantization_rtn_b200 import build as w4build
+    w4build.build()
+    w4.lib()
+    dev = torch.device("cuda", 0)
+    props = torch.cuda.get_device_properties(dev)
+    l2 = getattr(props, "L2_cache_size", 0) or L2_BYTES_FALLBACK
+    layer = workloads.CROSSOVER.layers[0]
+    N, K = layer.N, layer.K
+    W = layer.weight().to(dev)
+    rows = []
+    for g, sym in ((128, False), (128, True), (64, False), (32, False)):
+        P, S, Z = w4.quantize(W, g, sym)
+        wbytes = N * K // 2 + 2 * N * (K // g) * (1 if sym else 2)
+        for M in workloads.CROSSOVER.Ms:
+            copies = copies_for(wbytes + 2 * M * K, l2)
+            Ps = [P] + [P.clone() for _ in range(copies - 1)]
+            Ss = [S] + [S.clone() for _ in range(copies - 1)]
+            Zs = [Z] + [Z.clone() for _ in range(copies - 1)]
+            X = layer.activation(M).to(dev)
+            Xs = [X] + [X.clone() for _ in range(copies - 1)]
+            Y = torch.empty(M, N, dtype=torch.bfloat16, device=dev)
+            iters = 40 if M <= 1024 else 12
+            row = {"g": g, "mode": "sym" if sym else "asym", "M": M, "N": N, "K": K,
+                   "dispatch": w4.plan(M, N, K, g, sym)["path"],
+                   "algorithmic_bytes": algorithmic_bytes(M, N, K, g, sym), "flops": 2 * M * N * K}
+            for path in ("decode", "tensorcore"):
+                if path == "decode" and M > 16:
+                    continue
+                gs = graph_of(lambda i, path=path: w4.gemm(Xs[i % copies], Ps[i % copies],
+                                                           Ss[i % copies], Zs[i % copies], g, sym,
+                                                           path=path, out=Y), copies)
+                row[path + "_us"] = time_graphs(gs, iters) * 1e3
+                del gs
+            if g == 128 and not sym:
+                dcopies = max(2, -(-2 * l2 // (N * K * 2 + 2 * M * K)) + 1)
+                Wd = [W] + [W.clone() for _ in range(dcopies - 1)]
+                Xd = Xs[:1] + [X.clone() for _ in range(dcopies - 1)]
+                gs = graph_of(lambda i: torch.matmul(Xd[i % dcopies], Wd[i % dcopies].t(), out=Y),
+                              dcopies)
+                row["dense_bf16_cublas_us"] = time_graphs(gs, iters) * 1e3
+                del gs, Wd, Xd
+            cand = {k[:-3]: v for k, v in row.items() if k in ("decode_us", "tensorcore_us")}
+            row["fastest"] = min(cand, key=cand.get)
+            rows.append(row)
+            del Ps, Ss, Zs, Xs, X, Y
+            torch.cuda.empty_cache()
+        del P, S, Z
+    print(json.dumps({"crossover": rows}))
+
+
 def run_reference(args):
     """The reference arm: the host oracle as it stands, timed on this machine's
     cores, on the same workload and metric; each step a bounded sample."""
@@ -679,10 +744,14 @@ def main():
     ap.add_argument("--no-extras", action="store_true",
                     help="skip comparisons and the prefill half (profiling runs)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--crossover", action="store_true",
+                    help="print the M-dispatch sweep at K=N=8192 instead of a benchmark line")
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be at least 3")
-    if args.impl == "reference":
+    if args.crossover:
+        crossover_sweep(args)
+    elif args.impl == "reference":
         run_reference(args)
     else:
         run_ours(args)

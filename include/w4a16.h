@@ -120,10 +120,13 @@ w4a16_status w4a16_dequantize(const void* packed, const void* scales, const void
                               int64_t N, int64_t K, int32_t g, int32_t sym, void* W_hat,
                               void* stream);
 
-/* Bytes of device workspace w4a16_gemm needs for this shape (0 for the
- * tensor-core path).  The decode path stores there the fp32 partial sums of the
- * 32-row blocks that its stream-K partition splits between CTAs; a second,
- * small kernel adds them in a fixed order.  The contents are scratch: no
+/* Bytes of device workspace w4a16_gemm needs for this shape.  The decode path
+ * stores there the fp32 partial sums of the 32-row blocks that its stream-K
+ * partition splits between CTAs; the tensor-core path, when its output tiles
+ * are fewer than the SMs and it splits K into S parts, stores S fp32 partial
+ * results of M x N (each rounded up to a multiple of 4 elements), and 0 bytes
+ * are needed otherwise.  In both cases a second, small kernel adds the parts in
+ * a fixed order.  The contents are scratch: no
  * initialization is needed and nothing is kept between calls, but two calls
  * that may run at the same time (for instance on two streams) need two
  * workspaces.  Uses the current device's SM count. */

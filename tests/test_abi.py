@@ -96,9 +96,13 @@ def test_quantize_and_dequantize_reject_invalid(lib):
 
 
 def test_workspace_sizes(lib):
-    # tensor-core path needs none; decode needs counters + partial row blocks
+    # tensor-core path: none with enough output tiles to fill the SMs, else S fp32
+    # partial M x N results (split-K); decode: partial row blocks
     assert w4.workspace_size(2048, 8192, 8192, 32) == 0
-    assert w4.workspace_size(17, 8192, 8192, 32) == 0
+    p17 = w4.plan(17, 8192, 8192, 32)
+    splits = p17["grid"] // ((8192 // 128) * 1)
+    assert splits == 2 and p17["kernels"] == 2
+    assert w4.workspace_size(17, 8192, 8192, 32) == splits * (17 * 8192) * 4
     rb = 4096 // 32
     p = w4.plan(1, 4096, 4096, 128)
     assert p["workspace_bytes"] == (rb + p["grid"]) * 256 * 4
@@ -121,7 +125,7 @@ def test_dispatch_plans():
     assert w4.plan(17, 4096, 4096)["path"] == "tensorcore"
     p = w4.plan(2048, 8192, 8192)
     assert p["path"] == "tensorcore" and p["tile_m"] == 256 and p["grid"] == 64 * 8
-    assert p["smem_bytes"] <= 232448 and p["workspace_bytes"] == 0
+    assert p["smem_bytes"] <= 232448 and p["workspace_bytes"] == 0 and p["kernels"] == 1
     for M, bm in ((17, 32), (32, 32), (33, 64), (64, 64), (65, 128), (128, 128), (129, 256)):
         assert w4.plan(M, 8192, 8192)["tile_m"] == bm
     for M in (1, 8):

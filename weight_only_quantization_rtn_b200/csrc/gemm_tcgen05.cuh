@@ -35,6 +35,11 @@
 //               32·(w%4)..+31, the rows it dequantized, and every other 32-column
 //               block of the accumulator.
 //
+// Split-K: when there are fewer (n, m) tiles than SMs, gridDim.z CTAs share each
+// tile's K range (CTA z takes K blocks [z·kb_split, (z+1)·kb_split)), each writes
+// its fp32 partial tile to the workspace, and tc_splitk_reduce_kernel, chained by
+// programmatic dependent launch, adds the partials in z order and writes Y.
+//
 // Every barrier wait is bounded (about one second); a timeout records an error
 // in the device error word and the role stops issuing work, then the CTA
 // drains and frees its TMEM before returning.
@@ -72,7 +77,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
                    const uint16_t* __restrict__ scales, const uint16_t* __restrict__ zeros,
                    uint16_t* __restrict__ Y, int M, int N, int K, int sz_async,
                    const __grid_constant__ CUtensorMap tmS, const __grid_constant__ CUtensorMap tmZ,
-                   int sz_tma) {
+                   int sz_tma, int kb_split, float* __restrict__ partials) {
     using Cfg = TcConfig<BM>;
     constexpr int S = Cfg::kStages;
     static_assert(S >= 2, "pipeline needs at least two stages");
@@ -101,6 +106,9 @@ __global__ void __launch_bounds__(kTcThreads, 1)
     const int n0 = blockIdx.x * kTcTileN;
     const int m0 = blockIdx.y * BM;
     const int num_kb = (K + kTcBlockK - 1) / kTcBlockK;
+    // this CTA's K blocks [kb0, kb0 + nkb); kb0 is a multiple of the slab length
+    const int kb0 = (int)blockIdx.z * kb_split;
+    const int nkb = min(num_kb - kb0, kb_split);
     const int Gn = K / G;
 
     if (threadIdx.x == 0) {
@@ -110,6 +118,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
             mbar_init(smem_u32(&empty[s]), 1);
         }
         mbar_init(smem_u32(accf), 1);
+        grid_launch_dependents();          // the split-K reduction may start as this grid drains
         for (int t = 0; t < 2; ++t) {
             mbar_init(smem_u32(&slab_full[t]), 1);
             mbar_init(smem_u32(&slab_empty[t]), kTcDequantWarps);
@@ -136,25 +145,26 @@ __global__ void __launch_bounds__(kTcThreads, 1)
     if (warp == 0) {
         // ------------------------------------------------------------ producer
         int issued = 0;
-        for (int kb = 0; kb < num_kb; ++kb) {
-            const int s = kb % S;
-            const uint32_t ph = (uint32_t)(kb / S) & 1u;
+        for (int i = 0; i < nkb; ++i) {
+            const int kb = kb0 + i;
+            const int s = i % S;
+            const uint32_t ph = (uint32_t)(i / S) & 1u;
             bool ok = true;
             if (lane == 0) ok = mbar_wait(smem_u32(&empty[s]), ph ^ 1u);   // one lane waits
             if (!__shfl_sync(0xffffffffu, ok ? 1 : 0, 0)) break;
             const uint32_t bar = smem_u32(&full[s]);
-            if (sz_tma && kb % kSlabKb == 0) {
+            if (sz_tma && i % kSlabKb == 0) {
                 // next slab of scales/zeros: its slot is free once the dequantizers
                 // finished the slab two back
-                const int t = kb / kSlabKb, slot = t & 1;
+                const int t = i / kSlabKb, slot = t & 1;
                 if (lane == 0) ok = mbar_wait(smem_u32(&slab_empty[slot]), ((uint32_t)(t >> 1) & 1u) ^ 1u);
                 if (!__shfl_sync(0xffffffffu, ok ? 1 : 0, 0)) break;
                 if (lane == 0) {
                     const uint32_t sb = smem_u32(&slab_full[slot]);
                     uint16_t* dsl = slab + slot * 2 * kTcTileN * 8;
                     mbar_arrive_expect_tx(sb, (SYM ? 1 : 2) * kTcTileN * 8 * 2);
-                    tma_load_2d(smem_u32(dsl), &tmS, t * 8, n0, sb);
-                    if (!SYM) tma_load_2d(smem_u32(dsl + kTcTileN * 8), &tmZ, t * 8, n0, sb);
+                    tma_load_2d(smem_u32(dsl), &tmS, (kb / kSlabKb) * 8, n0, sb);
+                    if (!SYM) tma_load_2d(smem_u32(dsl + kTcTileN * 8), &tmZ, (kb / kSlabKb) * 8, n0, sb);
                 }
             }
             if (lane == 0) {
@@ -198,8 +208,8 @@ __global__ void __launch_bounds__(kTcThreads, 1)
         }
         if (lane == 0) {
             // Do not leave while copies into this CTA's shared memory are in flight.
-            for (int kb = (issued > S ? issued - S : 0); kb < issued; ++kb) {
-                if (!mbar_wait(smem_u32(&full[kb % S]), (uint32_t)(kb / S) & 1u)) break;
+            for (int i = (issued > S ? issued - S : 0); i < issued; ++i) {
+                if (!mbar_wait(smem_u32(&full[i % S]), (uint32_t)(i / S) & 1u)) break;
             }
             if (sz_tma && issued > 0) {
                 const int slabs = (issued - 1) / kSlabKb + 1;   // slabs requested so far
@@ -211,9 +221,9 @@ __global__ void __launch_bounds__(kTcThreads, 1)
         // ------------------------------------------------------------ MMA issuer
         if (lane == 0) {
             constexpr uint32_t idesc = idesc_bf16_f32(kTcTileN, BM);
-            for (int kb = 0; kb < num_kb; ++kb) {
-                const int s = kb % S;
-                const uint32_t ph = (uint32_t)(kb / S) & 1u;
+            for (int i = 0; i < nkb; ++i) {
+                const int s = i % S;
+                const uint32_t ph = (uint32_t)(i / S) & 1u;
                 if (!mbar_wait(smem_u32(&full[s]), ph)) break;
                 if (!mbar_wait(smem_u32(&afull[s]), ph)) break;
                 tc_fence_after();
@@ -223,7 +233,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
                 for (int kk = 0; kk < kTcBlockK / 16; ++kk) {
                     tc_mma_bf16(tmem_d, sw128_kmajor_desc(a_base + kk * 32),
                                 sw128_kmajor_desc(x_base + kk * 32), idesc,
-                                (kb | kk) != 0 ? 1u : 0u);
+                                (i | kk) != 0 ? 1u : 0u);
                 }
                 tc_commit(smem_u32(&empty[s]));
             }
@@ -238,11 +248,12 @@ __global__ void __launch_bounds__(kTcThreads, 1)
         const int n = n0 + r;
         const bool row_ok = n < N;
         bool ok = true;
-        for (int kb = 0; kb < num_kb; ++kb) {
-            const int s = kb % S;
-            const uint32_t ph = (uint32_t)(kb / S) & 1u;
-            const int t = kb / kSlabKb, slot = t & 1;
-            if (sz_tma && kb % kSlabKb == 0 &&
+        for (int i = 0; i < nkb; ++i) {
+            const int kb = kb0 + i;
+            const int s = i % S;
+            const uint32_t ph = (uint32_t)(i / S) & 1u;
+            const int t = i / kSlabKb, slot = t & 1;
+            if (sz_tma && i % kSlabKb == 0 &&
                 !mbar_wait(smem_u32(&slab_full[slot]), (uint32_t)(t >> 1) & 1u)) {
                 ok = false;
                 break;
@@ -289,7 +300,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
             fence_proxy_async_smem();
             __syncwarp();
             if (lane == 0) mbar_arrive(smem_u32(&afull[s]));
-            if (sz_tma && (kb % kSlabKb == kSlabKb - 1 || kb == num_kb - 1)) {
+            if (sz_tma && (i % kSlabKb == kSlabKb - 1 || i == nkb - 1)) {
                 if (lane == 0) mbar_arrive(smem_u32(&slab_empty[slot]));
             }
         }
@@ -302,13 +313,21 @@ __global__ void __launch_bounds__(kTcThreads, 1)
                 uint32_t v[32];
                 tmem_ld_32x32b_x32(tmem_d + t_lane + cb * 32, v);
                 tmem_wait_ld();
-                if (row_ok) {
+                if (row_ok && partials == nullptr) {
 #pragma unroll
                     for (int j = 0; j < 32; ++j) {
                         const int m = m0 + cb * 32 + j;
                         if (m < M)
                             Y[(int64_t)m * N + n] =
                                 (uint16_t)f32_to_bf16_bits_rn(__uint_as_float(v[j]));
+                    }
+                } else if (row_ok) {
+                    // split-K: this CTA's fp32 part, [z][round_up(M·N, 4)] row-major in (m, n)
+                    float* part = partials + (int64_t)blockIdx.z * (((int64_t)M * N + 3) & ~(int64_t)3);
+#pragma unroll
+                    for (int j = 0; j < 32; ++j) {
+                        const int m = m0 + cb * 32 + j;
+                        if (m < M) part[(int64_t)m * N + n] = __uint_as_float(v[j]);
                     }
                 }
             }
@@ -319,6 +338,34 @@ __global__ void __launch_bounds__(kTcThreads, 1)
     if (warp == 1) {
         tc_fence_after();
         tmem_dealloc(tmem_d, Cfg::kTmemCols);
+    }
+}
+
+// Adds the split-K partial tiles in z order and rounds to bf16: Y = Σ_z part[z].
+// Four elements per thread, grid-stride; the parts are the preceding grid's output.
+__global__ void __launch_bounds__(256) tc_splitk_reduce_kernel(const float* __restrict__ partials,
+                                                               int splits, int64_t mn,
+                                                               uint16_t* __restrict__ Y) {
+    grid_dependency_wait();
+    const int64_t stride = ((mn + 3) & ~(int64_t)3);
+    const int64_t step = (int64_t)gridDim.x * blockDim.x * 4;
+    for (int64_t e = ((int64_t)blockIdx.x * blockDim.x + threadIdx.x) * 4; e < mn; e += step) {
+        if (e + 4 <= mn) {
+            float4 acc = __ldcg(reinterpret_cast<const float4*>(partials + e));
+            for (int z = 1; z < splits; ++z) {
+                const float4 v = __ldcg(reinterpret_cast<const float4*>(partials + z * stride + e));
+                acc.x += v.x; acc.y += v.y; acc.z += v.z; acc.w += v.w;
+            }
+            const uint32_t lo = f32_to_bf16_bits_rn(acc.x) | (f32_to_bf16_bits_rn(acc.y) << 16);
+            const uint32_t hi = f32_to_bf16_bits_rn(acc.z) | (f32_to_bf16_bits_rn(acc.w) << 16);
+            *reinterpret_cast<uint2*>(Y + e) = make_uint2(lo, hi);
+        } else {
+            for (int64_t i = e; i < mn; ++i) {
+                float acc = __ldcg(partials + i);
+                for (int z = 1; z < splits; ++z) acc += __ldcg(partials + z * stride + i);
+                Y[i] = (uint16_t)f32_to_bf16_bits_rn(acc);
+            }
+        }
     }
 }
 

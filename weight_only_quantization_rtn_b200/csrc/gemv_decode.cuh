@@ -105,14 +105,6 @@ struct UnitWalk {
     }
 };
 
-__device__ __forceinline__ void grid_dependency_wait() {
-    asm volatile("griddepcontrol.wait;" ::: "memory");
-}
-
-__device__ __forceinline__ void grid_launch_dependents() {
-    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
-}
-
 struct DecodeArgs {
     const uint16_t* scales;
     const uint16_t* zeros;

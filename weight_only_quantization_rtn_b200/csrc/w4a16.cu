@@ -146,6 +146,32 @@ int tc_tile_m(int64_t M) {
     return 256;
 }
 
+// Split-K for the tensor-core path: when the (n, m) tiles are fewer than the SMs,
+// split each tile's K blocks over up to sm_count / tiles CTAs (at most 8, at
+// least 4 K blocks each); split boundaries are multiples of the scale slab
+// (g/8 blocks) when scales come by TMA.  Returns K blocks per split.
+int tc_kb_split(int num_kb, int splits, int g, bool sz_tma) {
+    int kbs = (num_kb + splits - 1) / splits;
+    const int slab = sz_tma ? g / 8 : 1;
+    return (kbs + slab - 1) / slab * slab;
+}
+
+void tc_split(int64_t M, int64_t N, int64_t K, int g, int bm, int sm_count, int* splits,
+              int* kb_split) {
+    const int64_t tiles = ((N + kTcTileN - 1) / kTcTileN) * ((M + bm - 1) / bm);
+    const int num_kb = (int)((K + kTcBlockK - 1) / kTcBlockK);
+    const bool sz_tma = (K / g) % 8 == 0;
+    int s = 1;
+    if (tiles < sm_count) {
+        s = (int)(sm_count / tiles);
+        if (s > 8) s = 8;
+        if (s > num_kb / 4) s = num_kb / 4;
+        if (s < 1) s = 1;
+    }
+    *kb_split = tc_kb_split(num_kb, s, g, sz_tma);
+    *splits = (num_kb + *kb_split - 1) / *kb_split;
+}
+
 int tc_smem_bytes(int bm) {
     switch (bm) {
         case 32: return TcConfig<32>::kSmemBytes;
@@ -194,9 +220,11 @@ w4a16_status make_plan(int64_t M, int64_t N, int64_t K, int32_t g, int32_t sym, 
         p->workspace_bytes = decode_workspace_bytes(d, grid);
     } else {
         const int bm = tc_tile_m(M);
+        int splits = 1, kb_split = 0;
+        tc_split(M, N, K, g, bm, sm_count, &splits, &kb_split);
         p->tile_m = bm;
         p->tile_n = kTcTileN;
-        p->grid = ((N + kTcTileN - 1) / kTcTileN) * ((M + bm - 1) / bm);
+        p->grid = ((N + kTcTileN - 1) / kTcTileN) * ((M + bm - 1) / bm) * splits;
         p->threads = kTcThreads;
         p->smem_bytes = tc_smem_bytes(bm);
         p->stages = TcConfig<256>::kStages;
@@ -206,8 +234,8 @@ w4a16_status make_plan(int64_t M, int64_t N, int64_t K, int32_t g, int32_t sym, 
             case 128: p->stages = TcConfig<128>::kStages; break;
             default: break;
         }
-        p->kernels = 1;
-        p->workspace_bytes = 0;
+        p->kernels = splits > 1 ? 2 : 1;
+        p->workspace_bytes = splits > 1 ? (int64_t)splits * ((M * N + 3) / 4 * 4) * 4 : 0;
     }
     return W4A16_OK;
 }
@@ -344,7 +372,7 @@ template <int BM, bool SYM, int G>
 w4a16_status launch_tc_t(const w4a16_plan& p, const CUtensorMap& tmX, const CUtensorMap& tmP,
                          const CUtensorMap& tmS, const CUtensorMap& tmZ, int sz_tma,
                          const void* scales, const void* zeros, void* Y, int M, int N, int K,
-                         cudaStream_t stream) {
+                         void* workspace, cudaStream_t stream) {
     auto kern = gemm_tc_kernel<BM, SYM, G>;
     const int sz_async = ((K / G) % 2 == 0) ? 1 : 0;   // 4-byte aligned scale rows
     static bool attr_set[kMaxDevices] = {};
@@ -356,20 +384,45 @@ w4a16_status launch_tc_t(const w4a16_plan& p, const CUtensorMap& tmX, const CUte
             return W4A16_ECUDA;
         attr_set[dev] = true;
     }
-    dim3 grid((unsigned)((N + kTcTileN - 1) / kTcTileN), (unsigned)((M + BM - 1) / BM), 1);
+    const int64_t tiles = (int64_t)((N + kTcTileN - 1) / kTcTileN) * ((M + BM - 1) / BM);
+    const int splits = (int)(p.grid / tiles);
+    const int num_kb = (K + kTcBlockK - 1) / kTcBlockK;
+    const int kb_split = tc_kb_split(num_kb, splits, G, sz_tma != 0);
+    float* partials = splits > 1 ? static_cast<float*>(workspace) : nullptr;
+    dim3 grid((unsigned)((N + kTcTileN - 1) / kTcTileN), (unsigned)((M + BM - 1) / BM),
+              (unsigned)splits);
     kern<<<grid, kTcThreads, TcConfig<BM>::kSmemBytes, stream>>>(
         tmX, tmP, static_cast<const uint16_t*>(scales), static_cast<const uint16_t*>(zeros),
-        static_cast<uint16_t*>(Y), M, N, K, sz_async, tmS, tmZ, sz_tma);
-    return launch_status();
+        static_cast<uint16_t*>(Y), M, N, K, sz_async, tmS, tmZ, sz_tma, kb_split, partials);
+    w4a16_status st = launch_status();
+    if (st != W4A16_OK || splits == 1) return st;
+    // Sum of the partial tiles, chained by programmatic dependent launch.
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cudaLaunchConfig_t cfg = {};
+    const int64_t mn = (int64_t)M * N;
+    int64_t blocks = (mn / 4 + 255) / 256 + 1;
+    if (blocks > 148 * 8) blocks = 148 * 8;
+    cfg.gridDim = dim3((unsigned)blocks, 1, 1);
+    cfg.blockDim = dim3(256, 1, 1);
+    cfg.stream = stream;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    if (cudaLaunchKernelEx(&cfg, tc_splitk_reduce_kernel, static_cast<const float*>(partials),
+                           splits, mn, static_cast<uint16_t*>(Y)) != cudaSuccess)
+        return W4A16_ECUDA;
+    return W4A16_OK;
 }
 
 template <bool SYM, int G>
 w4a16_status launch_tc_g(const w4a16_plan& p, const CUtensorMap& tmX, const CUtensorMap& tmP,
                          const CUtensorMap& tmS, const CUtensorMap& tmZ, int sz_tma,
                          const void* scales, const void* zeros, void* Y, int M, int N, int K,
-                         cudaStream_t stream) {
+                         void* workspace, cudaStream_t stream) {
 #define W4A16_TC_TILE(BMV) \
-    launch_tc_t<BMV, SYM, G>(p, tmX, tmP, tmS, tmZ, sz_tma, scales, zeros, Y, M, N, K, stream)
+    launch_tc_t<BMV, SYM, G>(p, tmX, tmP, tmS, tmZ, sz_tma, scales, zeros, Y, M, N, K, workspace, \
+                             stream)
     switch (p.tile_m) {
         case 32: return W4A16_TC_TILE(32);
         case 64: return W4A16_TC_TILE(64);
@@ -381,7 +434,7 @@ w4a16_status launch_tc_g(const w4a16_plan& p, const CUtensorMap& tmX, const CUte
 
 w4a16_status launch_tc(const w4a16_plan& p, const void* X, int64_t M, int64_t K,
                        const void* packed, const void* scales, const void* zeros, int64_t N,
-                       int32_t g, int32_t sym, void* Y, cudaStream_t stream) {
+                       int32_t g, int32_t sym, void* Y, void* workspace, cudaStream_t stream) {
     CUtensorMap tmX, tmP;
     w4a16_status st = encode_2d(&tmX, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, X, (uint64_t)K,
                                 (uint64_t)M, (uint64_t)K * 2, kTcBlockK, (uint32_t)p.tile_m,
@@ -408,9 +461,9 @@ w4a16_status launch_tc(const w4a16_plan& p, const void* X, int64_t M, int64_t K,
 #define W4A16_TC_CASE(GG)                                                                      \
     case GG:                                                                                   \
         return sym ? launch_tc_g<true, GG>(p, tmX, tmP, tmS, tmZ, sz_tma, scales, zeros, Y, m, n, \
-                                           k, stream)                                          \
+                                           k, workspace, stream)                               \
                    : launch_tc_g<false, GG>(p, tmX, tmP, tmS, tmZ, sz_tma, scales, zeros, Y, m, n, \
-                                            k, stream);
+                                            k, workspace, stream);
     switch (g) {
         W4A16_TC_CASE(32)
         W4A16_TC_CASE(64)
@@ -563,7 +616,7 @@ w4a16_status w4a16_gemm_ex(const void* X, int64_t M, int64_t K, const void* pack
     cudaStream_t s = static_cast<cudaStream_t>(stream);
     if (p.path == W4A16_PATH_DECODE)
         return launch_decode(p, X, M, K, packed, scales, zeros, N, g, sym, Y, workspace, s);
-    return launch_tc(p, X, M, K, packed, scales, zeros, N, g, sym, Y, s);
+    return launch_tc(p, X, M, K, packed, scales, zeros, N, g, sym, Y, workspace, s);
 }
 
 w4a16_status w4a16_gemm(const void* X, int64_t M, int64_t K, const void* packed,
