@@ -98,11 +98,12 @@ def test_quantize_and_dequantize_reject_invalid(lib):
 def test_workspace_sizes(lib):
     # tensor-core path: none with enough output tiles to fill the SMs, else S fp32
     # partial M x N results (split-K); decode: partial row blocks
-    assert w4.workspace_size(2048, 8192, 8192, 32) == 0
+    assert w4.workspace_size(4096, 8192, 8192, 32) == 0          # 1024 tiles: last wave 92% full
     p17 = w4.plan(17, 8192, 8192, 32)
     splits = p17["grid"] // ((8192 // 128) * 1)
     assert splits == 2 and p17["kernels"] == 2
-    assert w4.workspace_size(17, 8192, 8192, 32) == splits * (17 * 8192) * 4
+    # tile-local parts: [split][tile][32 activation rows][128 weight rows] fp32
+    assert w4.workspace_size(17, 8192, 8192, 32) == splits * 64 * 32 * 128 * 4
     rb = 4096 // 32
     p = w4.plan(1, 4096, 4096, 128)
     assert p["workspace_bytes"] == (rb + p["grid"]) * 256 * 4
@@ -124,13 +125,42 @@ def test_dispatch_plans():
     assert w4.plan(16, 4096, 11008)["path"] == "decode"
     assert w4.plan(17, 4096, 4096)["path"] == "tensorcore"
     p = w4.plan(2048, 8192, 8192)
-    assert p["path"] == "tensorcore" and p["tile_m"] == 256 and p["grid"] == 64 * 8
-    assert p["smem_bytes"] <= 232448 and p["workspace_bytes"] == 0 and p["kernels"] == 1
+    # 512 tiles on 148 SMs: three full waves unsplit, the 68-tile last wave split in two
+    assert p["path"] == "tensorcore" and p["tile_m"] == 256 and p["grid"] == 444 + 68 * 2
+    assert p["smem_bytes"] <= 232448 and p["kernels"] == 3
+    assert p["workspace_bytes"] == 2 * 68 * 256 * 128 * 4
     for M, bm in ((17, 32), (32, 32), (33, 64), (64, 64), (65, 128), (128, 128), (129, 256)):
         assert w4.plan(M, 8192, 8192)["tile_m"] == bm
     for M in (1, 8):
         assert w4.plan(M, 4096, 4096)["tile_m"] == 8
     assert w4.plan(9, 4096, 4096)["tile_m"] == 16
+
+
+def _tc_schedule(M, N, K, g, sms=148):
+    """Mirror of the tensor-core launch schedule: (head tiles, tail tiles, splits)."""
+    bm = 32 if M <= 32 else 64 if M <= 64 else 128 if M <= 128 else 256
+    tiles = -(-N // 128) * -(-M // bm)
+    num_kb = -(-K // 64)
+    tail = tiles if tiles < sms else (tiles % sms if 0 < tiles % sms <= sms // 2 else 0)
+    s = max(1, min(sms // tail, 8, num_kb // 4)) if tail else 1
+    slab = g // 8 if (K // g) % 8 == 0 else 1
+    kbs = -(-(-(-num_kb // s)) // slab) * slab
+    splits = -(-num_kb // kbs)
+    if splits < 2:
+        return tiles, 0, 1, bm
+    return tiles - tail, tail, splits, bm
+
+
+@pytest.mark.parametrize("M,N,K,g", [(17, 8192, 8192, 32), (64, 4096, 4096, 128), (256, 11008, 4096, 64),
+                                     (2048, 8192, 8192, 128), (4096, 8192, 8192, 128),
+                                     (1024, 28672, 8192, 128), (20, 37, 96, 32), (200, 4096, 1152, 32)])
+def test_tensorcore_schedule(M, N, K, g):
+    head, tail, splits, bm = _tc_schedule(M, N, K, g)
+    p = w4.plan(M, N, K, g, path="tensorcore")
+    assert p["tile_m"] == bm
+    assert p["grid"] == head + tail * splits
+    assert p["kernels"] == (1 if head else 0) + (2 if tail else 0)
+    assert p["workspace_bytes"] == (splits * tail * bm * 128 * 4 if tail else 0)
 
 
 def test_decode_persistent_grid_and_smem():

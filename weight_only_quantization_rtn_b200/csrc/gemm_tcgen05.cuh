@@ -35,10 +35,14 @@
 //               32·(w%4)..+31, the rows it dequantized, and every other 32-column
 //               block of the accumulator.
 //
-// Split-K: when there are fewer (n, m) tiles than SMs, gridDim.z CTAs share each
-// tile's K range (CTA z takes K blocks [z·kb_split, (z+1)·kb_split)), each writes
-// its fp32 partial tile to the workspace, and tc_splitk_reduce_kernel, chained by
-// programmatic dependent launch, adds the partials in z order and writes Y.
+// Tiles and split-K: CTA (x, z) of a launch computes output tile t = tile_base + x
+// (n-tile t % tiles_n, m-tile t / tiles_n).  When a launch splits K, gridDim.z
+// CTAs share each tile's K range (CTA z takes K blocks [z·kb_split,
+// (z+1)·kb_split)), each writes its fp32 partial tile to the workspace, and
+// tc_splitk_reduce_kernel, chained by programmatic dependent launch, adds the
+// partials in z order and writes Y.  The host splits K when the tiles are fewer
+// than the SMs, and splits only the last, partial wave of tiles (a second launch)
+// when that wave would leave most SMs idle.
 //
 // Every barrier wait is bounded (about one second); a timeout records an error
 // in the device error word and the role stops issuing work, then the CTA
@@ -77,7 +81,8 @@ __global__ void __launch_bounds__(kTcThreads, 1)
                    const uint16_t* __restrict__ scales, const uint16_t* __restrict__ zeros,
                    uint16_t* __restrict__ Y, int M, int N, int K, int sz_async,
                    const __grid_constant__ CUtensorMap tmS, const __grid_constant__ CUtensorMap tmZ,
-                   int sz_tma, int kb_split, float* __restrict__ partials) {
+                   int sz_tma, int kb_split, float* __restrict__ partials, int tile_base,
+                   int tiles_n) {
     using Cfg = TcConfig<BM>;
     constexpr int S = Cfg::kStages;
     static_assert(S >= 2, "pipeline needs at least two stages");
@@ -103,8 +108,9 @@ __global__ void __launch_bounds__(kTcThreads, 1)
 
     const int warp = threadIdx.x >> 5;
     const int lane = threadIdx.x & 31;
-    const int n0 = blockIdx.x * kTcTileN;
-    const int m0 = blockIdx.y * BM;
+    const int tile = tile_base + (int)blockIdx.x;
+    const int n0 = (tile % tiles_n) * kTcTileN;
+    const int m0 = (tile / tiles_n) * BM;
     const int num_kb = (K + kTcBlockK - 1) / kTcBlockK;
     // this CTA's K blocks [kb0, kb0 + nkb); kb0 is a multiple of the slab length
     const int kb0 = (int)blockIdx.z * kb_split;
@@ -321,14 +327,12 @@ __global__ void __launch_bounds__(kTcThreads, 1)
                             Y[(int64_t)m * N + n] =
                                 (uint16_t)f32_to_bf16_bits_rn(__uint_as_float(v[j]));
                     }
-                } else if (row_ok) {
-                    // split-K: this CTA's fp32 part, [z][round_up(M·N, 4)] row-major in (m, n)
-                    float* part = partials + (int64_t)blockIdx.z * (((int64_t)M * N + 3) & ~(int64_t)3);
+                } else if (partials != nullptr) {
+                    // split-K: this CTA's fp32 part of its tile, [z][tile of the launch][BM][128]
+                    float* part = partials +
+                                  ((int64_t)blockIdx.z * gridDim.x + blockIdx.x) * (BM * kTcTileN);
 #pragma unroll
-                    for (int j = 0; j < 32; ++j) {
-                        const int m = m0 + cb * 32 + j;
-                        if (m < M) part[(int64_t)m * N + n] = __uint_as_float(v[j]);
-                    }
+                    for (int j = 0; j < 32; ++j) part[(cb * 32 + j) * kTcTileN + r] = __uint_as_float(v[j]);
                 }
             }
         }
@@ -339,33 +343,41 @@ __global__ void __launch_bounds__(kTcThreads, 1)
         tc_fence_after();
         tmem_dealloc(tmem_d, Cfg::kTmemCols);
     }
+    // A launch that started early behind another tile launch does not complete
+    // before it: work queued after this launch may then rely on both.
+    if (threadIdx.x == 0) grid_dependency_wait();
 }
 
-// Adds the split-K partial tiles in z order and rounds to bf16: Y = Σ_z part[z].
-// Four elements per thread, grid-stride; the parts are the preceding grid's output.
-__global__ void __launch_bounds__(256) tc_splitk_reduce_kernel(const float* __restrict__ partials,
-                                                               int splits, int64_t mn,
-                                                               uint16_t* __restrict__ Y) {
+// Adds the split-K partial tiles in z order and rounds to bf16: for each tile of the
+// preceding launch, Y[m0 + m][n0 + r] = Σ_z part[z][tile][m][r].  Four consecutive
+// rows r per thread, grid-stride; the parts are the preceding grid's output.
+__global__ void __launch_bounds__(256) tc_splitk_reduce_kernel(
+    const float* __restrict__ partials, int splits, int tiles, int tile_base, int tiles_n, int bm,
+    int M, int N, uint16_t* __restrict__ Y) {
     grid_dependency_wait();
-    const int64_t stride = ((mn + 3) & ~(int64_t)3);
-    const int64_t step = (int64_t)gridDim.x * blockDim.x * 4;
-    for (int64_t e = ((int64_t)blockIdx.x * blockDim.x + threadIdx.x) * 4; e < mn; e += step) {
-        if (e + 4 <= mn) {
-            float4 acc = __ldcg(reinterpret_cast<const float4*>(partials + e));
-            for (int z = 1; z < splits; ++z) {
-                const float4 v = __ldcg(reinterpret_cast<const float4*>(partials + z * stride + e));
-                acc.x += v.x; acc.y += v.y; acc.z += v.z; acc.w += v.w;
-            }
-            const uint32_t lo = f32_to_bf16_bits_rn(acc.x) | (f32_to_bf16_bits_rn(acc.y) << 16);
-            const uint32_t hi = f32_to_bf16_bits_rn(acc.z) | (f32_to_bf16_bits_rn(acc.w) << 16);
-            *reinterpret_cast<uint2*>(Y + e) = make_uint2(lo, hi);
-        } else {
-            for (int64_t i = e; i < mn; ++i) {
-                float acc = __ldcg(partials + i);
-                for (int z = 1; z < splits; ++z) acc += __ldcg(partials + z * stride + i);
-                Y[i] = (uint16_t)f32_to_bf16_bits_rn(acc);
-            }
+    const int64_t per_tile = (int64_t)bm * kTcTileN;
+    const int64_t stride = (int64_t)tiles * per_tile;          // one split's parts
+    const int64_t items = stride / 4;
+    for (int64_t e = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; e < items;
+         e += (int64_t)gridDim.x * blockDim.x) {
+        const int64_t idx = 4 * e;
+        const int tl = (int)(idx / per_tile);
+        const int within = (int)(idx - (int64_t)tl * per_tile);
+        const int m_local = within / kTcTileN, r = within % kTcTileN;
+        const int t = tile_base + tl;
+        const int m = (t / tiles_n) * bm + m_local;
+        const int n = (t % tiles_n) * kTcTileN + r;
+        if (m >= M || n >= N) continue;
+        float4 acc = __ldcg(reinterpret_cast<const float4*>(partials + idx));
+        for (int z = 1; z < splits; ++z) {
+            const float4 v = __ldcg(reinterpret_cast<const float4*>(partials + z * stride + idx));
+            acc.x += v.x; acc.y += v.y; acc.z += v.z; acc.w += v.w;
         }
+        const float a4[4] = {acc.x, acc.y, acc.z, acc.w};
+        uint16_t* y = Y + (int64_t)m * N + n;
+#pragma unroll
+        for (int q = 0; q < 4; ++q)
+            if (n + q < N) y[q] = (uint16_t)f32_to_bf16_bits_rn(a4[q]);
     }
 }
 

@@ -325,7 +325,7 @@ __global__ void __launch_bounds__(kDecThreads, MB == 1 ? 2 : 1)
             wk.advance();
             if (++s == S) { s = 0; ph ^= 1u; }
         }
-        const int rb = wk.rb, kb = wk.kb;
+        const int rb = wk.rb;
 
         // Once any wait has been given up, skip the remaining work but keep the
         // row-block barrier protocol below, so every consumer warp finishes.

@@ -156,20 +156,50 @@ int tc_kb_split(int num_kb, int splits, int g, bool sz_tma) {
     return (kbs + slab - 1) / slab * slab;
 }
 
-void tc_split(int64_t M, int64_t N, int64_t K, int g, int bm, int sm_count, int* splits,
-              int* kb_split) {
-    const int64_t tiles = ((N + kTcTileN - 1) / kTcTileN) * ((M + bm - 1) / bm);
+// Tensor-core launch schedule.  Output tiles (128 weight rows x bm activation
+// rows) run unsplit in a "head" launch; K is split over `splits` CTAs per tile for
+// the "tail" tiles, whose partials a reduce kernel adds.  All tiles are tail when
+// they are fewer than the SMs; otherwise only a last partial wave that would leave
+// more than half of the SMs idle becomes the tail.  Splits: up to sm_count / tail
+// tiles, at most 8, at least 4 K blocks each.
+struct TcSchedule {
+    int tiles_n;      // n-tiles (128 weight rows each)
+    int64_t head;     // unsplit tiles [0, head)
+    int64_t tail;     // split tiles [head, head + tail)
+    int splits;       // K splits of each tail tile (1 when there is no tail)
+    int kb_split;     // K blocks per split
+};
+
+TcSchedule tc_schedule(int64_t M, int64_t N, int64_t K, int g, int bm, int sm_count) {
+    TcSchedule t{};
+    t.tiles_n = (int)((N + kTcTileN - 1) / kTcTileN);
+    const int64_t tiles = (int64_t)t.tiles_n * ((M + bm - 1) / bm);
     const int num_kb = (int)((K + kTcBlockK - 1) / kTcBlockK);
     const bool sz_tma = (K / g) % 8 == 0;
-    int s = 1;
+    int64_t tail = 0;
     if (tiles < sm_count) {
-        s = (int)(sm_count / tiles);
+        tail = tiles;
+    } else {
+        const int64_t rem = tiles % sm_count;
+        if (rem > 0 && rem <= sm_count / 2) tail = rem;
+    }
+    int s = 1;
+    if (tail > 0) {
+        s = (int)(sm_count / tail);
         if (s > 8) s = 8;
         if (s > num_kb / 4) s = num_kb / 4;
         if (s < 1) s = 1;
     }
-    *kb_split = tc_kb_split(num_kb, s, g, sz_tma);
-    *splits = (num_kb + *kb_split - 1) / *kb_split;
+    t.kb_split = tc_kb_split(num_kb, s, g, sz_tma);
+    t.splits = (num_kb + t.kb_split - 1) / t.kb_split;
+    if (t.splits < 2) {                       // nothing to split: one unsplit launch
+        t.splits = 1;
+        t.kb_split = num_kb;
+        tail = 0;
+    }
+    t.head = tiles - tail;
+    t.tail = tail;
+    return t;
 }
 
 int tc_smem_bytes(int bm) {
@@ -220,11 +250,10 @@ w4a16_status make_plan(int64_t M, int64_t N, int64_t K, int32_t g, int32_t sym, 
         p->workspace_bytes = decode_workspace_bytes(d, grid);
     } else {
         const int bm = tc_tile_m(M);
-        int splits = 1, kb_split = 0;
-        tc_split(M, N, K, g, bm, sm_count, &splits, &kb_split);
+        const TcSchedule ts = tc_schedule(M, N, K, g, bm, sm_count);
         p->tile_m = bm;
         p->tile_n = kTcTileN;
-        p->grid = ((N + kTcTileN - 1) / kTcTileN) * ((M + bm - 1) / bm) * splits;
+        p->grid = ts.head + ts.tail * ts.splits;
         p->threads = kTcThreads;
         p->smem_bytes = tc_smem_bytes(bm);
         p->stages = TcConfig<256>::kStages;
@@ -234,8 +263,8 @@ w4a16_status make_plan(int64_t M, int64_t N, int64_t K, int32_t g, int32_t sym, 
             case 128: p->stages = TcConfig<128>::kStages; break;
             default: break;
         }
-        p->kernels = splits > 1 ? 2 : 1;
-        p->workspace_bytes = splits > 1 ? (int64_t)splits * ((M * N + 3) / 4 * 4) * 4 : 0;
+        p->kernels = (ts.head > 0 ? 1 : 0) + (ts.tail > 0 ? 2 : 0);
+        p->workspace_bytes = ts.tail > 0 ? (int64_t)ts.splits * ts.tail * bm * kTcTileN * 4 : 0;
     }
     return W4A16_OK;
 }
@@ -384,33 +413,47 @@ w4a16_status launch_tc_t(const w4a16_plan& p, const CUtensorMap& tmX, const CUte
             return W4A16_ECUDA;
         attr_set[dev] = true;
     }
-    const int64_t tiles = (int64_t)((N + kTcTileN - 1) / kTcTileN) * ((M + BM - 1) / BM);
-    const int splits = (int)(p.grid / tiles);
+    // the same schedule make_plan reported (it used this device's SM count)
+    const TcSchedule ts = tc_schedule(M, N, K, G, BM, current_sm_count());
+    const auto* sc = static_cast<const uint16_t*>(scales);
+    const auto* ze = static_cast<const uint16_t*>(zeros);
+    auto* y = static_cast<uint16_t*>(Y);
     const int num_kb = (K + kTcBlockK - 1) / kTcBlockK;
-    const int kb_split = tc_kb_split(num_kb, splits, G, sz_tma != 0);
-    float* partials = splits > 1 ? static_cast<float*>(workspace) : nullptr;
-    dim3 grid((unsigned)((N + kTcTileN - 1) / kTcTileN), (unsigned)((M + BM - 1) / BM),
-              (unsigned)splits);
-    kern<<<grid, kTcThreads, TcConfig<BM>::kSmemBytes, stream>>>(
-        tmX, tmP, static_cast<const uint16_t*>(scales), static_cast<const uint16_t*>(zeros),
-        static_cast<uint16_t*>(Y), M, N, K, sz_async, tmS, tmZ, sz_tma, kb_split, partials);
-    w4a16_status st = launch_status();
-    if (st != W4A16_OK || splits == 1) return st;
-    // Sum of the partial tiles, chained by programmatic dependent launch.
+    if (ts.head > 0) {
+        kern<<<dim3((unsigned)ts.head, 1, 1), kTcThreads, TcConfig<BM>::kSmemBytes, stream>>>(
+            tmX, tmP, sc, ze, y, M, N, K, sz_async, tmS, tmZ, sz_tma, num_kb, nullptr, 0, ts.tiles_n);
+        w4a16_status st = launch_status();
+        if (st != W4A16_OK) return st;
+    }
+    if (ts.tail == 0) return W4A16_OK;
+    float* partials = static_cast<float*>(workspace);
+    // The tail may start while the head drains (programmatic dependent launch);
+    // the reduce waits for the tail, and the tail waits for the head before it ends.
     cudaLaunchAttribute attr[1];
     attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
     attr[0].val.programmaticStreamSerializationAllowed = 1;
     cudaLaunchConfig_t cfg = {};
-    const int64_t mn = (int64_t)M * N;
-    int64_t blocks = (mn / 4 + 255) / 256 + 1;
-    if (blocks > 148 * 8) blocks = 148 * 8;
-    cfg.gridDim = dim3((unsigned)blocks, 1, 1);
-    cfg.blockDim = dim3(256, 1, 1);
+    cfg.gridDim = dim3((unsigned)ts.tail, 1, (unsigned)ts.splits);
+    cfg.blockDim = dim3(kTcThreads, 1, 1);
+    cfg.dynamicSmemBytes = TcConfig<BM>::kSmemBytes;
     cfg.stream = stream;
     cfg.attrs = attr;
-    cfg.numAttrs = 1;
-    if (cudaLaunchKernelEx(&cfg, tc_splitk_reduce_kernel, static_cast<const float*>(partials),
-                           splits, mn, static_cast<uint16_t*>(Y)) != cudaSuccess)
+    cfg.numAttrs = ts.head > 0 ? 1 : 0;
+    if (cudaLaunchKernelEx(&cfg, kern, tmX, tmP, sc, ze, y, M, N, K, sz_async, tmS, tmZ, sz_tma,
+                           ts.kb_split, partials, (int)ts.head, ts.tiles_n) != cudaSuccess)
+        return W4A16_ECUDA;
+    // Sum of the partial tiles, chained by programmatic dependent launch.
+    const int64_t items = ts.tail * BM * kTcTileN / 4;
+    int64_t blocks = (items + 255) / 256;
+    if (blocks > 148 * 8) blocks = 148 * 8;
+    cudaLaunchConfig_t rcfg = {};
+    rcfg.gridDim = dim3((unsigned)blocks, 1, 1);
+    rcfg.blockDim = dim3(256, 1, 1);
+    rcfg.stream = stream;
+    rcfg.attrs = attr;
+    rcfg.numAttrs = 1;
+    if (cudaLaunchKernelEx(&rcfg, tc_splitk_reduce_kernel, static_cast<const float*>(partials),
+                           ts.splits, (int)ts.tail, (int)ts.head, ts.tiles_n, BM, M, N, y) != cudaSuccess)
         return W4A16_ECUDA;
     return W4A16_OK;
 }
