@@ -540,8 +540,17 @@ def run_ours(args):
     # ------------------------------------------------ comparisons and the other metric half
     if not args.no_extras:
         line["comparisons"] = comparisons(w4, cases, copies, l2, half)
+        if half == "hbm":
+            ro = read_only_stream_gbs(dev)
+            roof["read_only_stream_gbs"] = ro
+            roof["frac_of_read_only_stream"] = roof["achieved"] / ro
+            roof["frac_of_nominal"] = roof["achieved"] / NOMINAL_HBM_GBS
+        else:
+            roof["frac_of_nominal"] = roof["achieved"] / NOMINAL_BF16_TFLOPS
         if args.workload != "prefill":
             line["prefill"] = prefill_extra(w4, peaks, peak_src, l2, dev)
+            pr = line["prefill"]["roofline"]
+            pr["frac_of_nominal"] = pr["achieved"] / NOMINAL_BF16_TFLOPS
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         cb = cpu_baseline(wl.layers, M, g, sym, unit_bytes=(half == "hbm")) \
             if half == "hbm" else cpu_baseline_sampled(wl.layers[0], M, g, sym, rows=16)
@@ -553,6 +562,31 @@ def run_ours(args):
         del rot, singles
         torch.cuda.synchronize()
         dist.destroy_process_group()
+
+
+# Nominal B200 figures (for context beside the measured denominators).
+NOMINAL_HBM_GBS = 8000.0
+NOMINAL_BF16_TFLOPS = 2250.0
+
+
+def read_only_stream_gbs(dev, nbytes: int = 2 << 30, iters: int = 10) -> float:
+    """HBM read bandwidth of a plain streaming reduction (torch.sum over a buffer
+    16x the L2), the read-only counterpart of the measured copy bandwidth."""
+    buf = torch.ones(nbytes // 4, dtype=torch.float32, device=dev)
+    out = torch.empty((), dtype=torch.float32, device=dev)
+    for _ in range(3):
+        torch.sum(buf, dim=0, out=out)
+    torch.cuda.synchronize()
+    a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    a.record()
+    for _ in range(iters):
+        torch.sum(buf, dim=0, out=out)
+    b.record()
+    b.synchronize()
+    gbs = nbytes * iters / (a.elapsed_time(b) / 1e3) / 1e9
+    del buf
+    torch.cuda.empty_cache()
+    return gbs
 
 
 def comparisons(w4, cases, copies, l2, half):

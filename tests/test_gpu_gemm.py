@@ -113,6 +113,34 @@ def test_deterministic_bitwise(path):
     assert all(torch.equal(ys[0], y) for y in ys[1:])
 
 
+@pytest.mark.parametrize("M,N,K,g,sym", [
+    (300, 10240, 2048, 32, False),    # 160 tiles: 148 unsplit + a 12-tile tail split 8 ways
+    (2048, 8192, 2048, 128, True),    # 512 tiles: 444 unsplit + a 68-tile tail split 2 ways
+    (48, 1000, 4352, 64, False),      # 8 tiles, all split (ragged N, K not a slab multiple)
+])
+def test_tensorcore_head_and_split_tail(M, N, K, g, sym):
+    """Tiles that run unsplit and tiles whose K is split (partials added by the
+    reduce kernel) both match the oracle on sampled outputs, including the last
+    rows and columns, and two runs are bitwise identical."""
+    plan = w4.plan(M, N, K, g, sym, path="tensorcore")
+    assert plan["kernels"] >= 2 and plan["workspace_bytes"] > 0
+    P, S, Z = _quantized(N, K, g, sym, seed=M)
+    X = workloads.make_activation(M, K, M + 1, outlier_frac=0.01, outlier_mode="set")
+    Xd = X.cuda()
+    Y = w4.gemm(Xd, P, S, Z, g, sym, path="tensorcore")
+    Y2 = w4.gemm(Xd, P, S, Z, g, sym, path="tensorcore")
+    torch.cuda.synchronize()
+    assert torch.equal(Y, Y2)
+    rng = np.random.default_rng(M)
+    ms = rng.integers(0, M, 2048)
+    ns = rng.integers(0, N, 2048)
+    ms[:4] = [0, M - 1, 0, M - 1]
+    ns[:4] = [0, 0, N - 1, N - 1]
+    ref = oracle.gemm_sampled(workloads.bits(X), P.cpu().numpy(), workloads.bits(S),
+                              workloads.bits(Z), g, sym, ms, ns)
+    assert_y_close(workloads.bits(Y)[ms, ns], ref, f"M={M} N={N} K={K} g={g} sym={sym}")
+
+
 def test_paths_agree_closely():
     P, S, Z = _quantized(384, 2048, 64, True, seed=8)
     X = workloads.make_activation(16, 2048, 9, outlier_frac=0.01, outlier_mode="set").cuda()
