@@ -551,6 +551,7 @@ def run_ours(args):
             line["prefill"] = prefill_extra(w4, peaks, peak_src, l2, dev)
             pr = line["prefill"]["roofline"]
             pr["frac_of_nominal"] = pr["achieved"] / NOMINAL_BF16_TFLOPS
+            line["quantize_dequantize"] = elementwise_extras(w4, peaks, l2, dev)
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         cb = cpu_baseline(wl.layers, M, g, sym, unit_bytes=(half == "hbm")) \
             if half == "hbm" else cpu_baseline_sampled(wl.layers[0], M, g, sym, rows=16)
@@ -587,6 +588,33 @@ def read_only_stream_gbs(dev, nbytes: int = 2 << 30, iters: int = 10) -> float:
     del buf
     torch.cuda.empty_cache()
     return gbs
+
+
+def elementwise_extras(w4, peaks, l2, dev, iters=20):
+    """Quantize/pack and standalone dequantize of a 7B-shaped weight (K=4096,
+    N=11008, g=128, asym): single HBM passes, reported against the measured copy
+    bandwidth.  Bytes: quantize reads W (2 B/weight) and writes codes, scales and
+    zeros; dequantize reads those and writes Ŵ (2 B/weight)."""
+    layer = workloads.DECODE_7B.layers[0]
+    N, K, g = layer.N, layer.K, 128
+    W = layer.weight().to(dev)
+    packed_bytes = N * K // 2 + 4 * N * (K // g)
+    copies = max(2, -(-2 * l2 // (N * K * 2)) + 1)
+    Ws = [W] + [W.clone() for _ in range(copies - 1)]
+    outs = [w4.quantize(w, g, False) for w in Ws]
+    gs = graph_of(lambda i: w4.quantize(Ws[i % copies], g, False), copies)
+    qms = time_graphs(gs, iters)
+    del gs
+    Wh = torch.empty(N, K, dtype=torch.bfloat16, device=dev)
+    gs = graph_of(lambda i: w4.dequantize(*outs[i % copies], g, False, out=Wh), copies)
+    dms = time_graphs(gs, iters)
+    del gs, Ws, outs, Wh, W
+    torch.cuda.empty_cache()
+    pk = peaks["hbm_gbs"]
+    qb, db = N * K * 2 + packed_bytes, packed_bytes + N * K * 2
+    return {"shape": f"N={N},K={K},g={g},asym",
+            "quantize": {"us": qms * 1e3, "GB/s": qb / (qms / 1e3) / 1e9, "frac": qb / (qms / 1e3) / 1e9 / pk},
+            "dequantize": {"us": dms * 1e3, "GB/s": db / (dms / 1e3) / 1e9, "frac": db / (dms / 1e3) / 1e9 / pk}}
 
 
 def comparisons(w4, cases, copies, l2, half):
