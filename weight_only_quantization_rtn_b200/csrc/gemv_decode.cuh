@@ -37,10 +37,10 @@
 //    the parts in CTA (= K) order and writes Y.  No CTA ever waits on another,
 //    so the split costs no synchronization latency inside the streaming kernel,
 //    and the result is deterministic.
-//  * Programmatic dependent launch also lets the next kernel on the stream start
-//    while this one drains: the producer requests its first stages of weights
-//    (which no preceding kernel writes) before griddepcontrol.wait, and X, Y and
-//    the workspace are touched only after it.
+//  * Programmatic dependent launch lets the next kernel on the stream start
+//    while this one drains: its CTAs are placed, set up their barriers and
+//    prefetch their tensor maps, then wait (griddepcontrol.wait) before any
+//    memory access.
 #pragma once
 
 #include "common.cuh"
@@ -188,17 +188,17 @@ __global__ void __launch_bounds__(kDecThreads, MB == 1 ? 2 : 1)
         }
         const uint32_t sz_tx = a.sz_tma ? (uint32_t)((SYM ? 1 : 2) * kDecRows * GB * 2) : 0u;
         const uint32_t tx = (uint32_t)kDecPBytes + 4u * xbox_bytes + sz_tx;
-        // Weights (packed codes, scales, zeros) never depend on the preceding
-        // kernel, so the first ring's worth is requested before waiting for it;
-        // X, and everything this grid writes, comes after the wait.
-        const int pre = nunits < S ? nunits : S;
-        int pre_kb[kDecMaxStages];
+        // Nothing is requested before the preceding grid has completed.  Weights
+        // do not depend on it, but requesting them early was measured to be
+        // slower: CTAs that start while the previous grid drains would prefetch
+        // their ring while the last-placed CTAs start cold, which staggers their
+        // finish, and the early requests compete with the drain for HBM.
+        grid_dependency_wait();
         UnitWalk wk;
         wk.init(u0, u1, a.KBn);
         int issued = 0;
         int s = 0;
         uint32_t ph = 0;
-        bool failed = false;
         for (int i = 0; i < nunits; ++i) {
             if (i > 0) {
                 wk.advance();
@@ -207,7 +207,7 @@ __global__ void __launch_bounds__(kDecThreads, MB == 1 ? 2 : 1)
             const int rb = wk.rb, kb = wk.kb;
             bool ok = true;
             if (lane == 0) ok = mbar_wait(smem_u32(&empty[s]), ph ^ 1u);   // one lane waits
-            if (!__shfl_sync(0xffffffffu, ok ? 1 : 0, 0)) { failed = true; break; }
+            if (!__shfl_sync(0xffffffffu, ok ? 1 : 0, 0)) break;
             uint8_t* st = stages + s * a.stage_bytes;
             const uint32_t bar = smem_u32(&full[s]);
             if (lane == 0) {
@@ -215,14 +215,11 @@ __global__ void __launch_bounds__(kDecThreads, MB == 1 ? 2 : 1)
 #pragma unroll
                 for (int b = 0; b < 4; ++b)
                     tma_load_2d(smem_u32(st + b * 4096), &tmP, kb * 512 + b * 128, rb * kDecRows, bar);
-                if (i >= pre) {
 #pragma unroll
-                    for (int b = 0; b < 4; ++b)
-                        tma_load_2d(smem_u32(st + kDecPBytes + b * xbox_bytes), &tmX,
-                                    kb * kDecBlockK + b * 256, 0, bar);
-                }
+                for (int b = 0; b < 4; ++b)
+                    tma_load_2d(smem_u32(st + kDecPBytes + b * xbox_bytes), &tmX,
+                                kb * kDecBlockK + b * 256, 0, bar);
             }
-            if (i < pre) pre_kb[i] = kb;
             // scales (and zeros): 32 rows x GB groups
             uint16_t* sz = reinterpret_cast<uint16_t*>(st + a.sz_offset);
             const int g0 = kb * GB;
@@ -263,32 +260,6 @@ __global__ void __launch_bounds__(kDecThreads, MB == 1 ? 2 : 1)
                 mbar_arrive(bar);
             }
             ++issued;
-            if (i == pre - 1) {
-                grid_dependency_wait();
-                if (lane == 0) {
-                    for (int j = 0; j < pre; ++j) {
-                        uint8_t* sj = stages + j * a.stage_bytes;
-#pragma unroll
-                        for (int b = 0; b < 4; ++b)
-                            tma_load_2d(smem_u32(sj + kDecPBytes + b * xbox_bytes), &tmX,
-                                        pre_kb[j] * kDecBlockK + b * 256, 0, smem_u32(&full[j]));
-                    }
-                }
-            }
-        }
-        if (failed && issued > 0 && issued < pre) {
-            // The loop stopped before X of the prefetched units was requested:
-            // request it now so that their barriers, and the drain below, complete.
-            grid_dependency_wait();
-            if (lane == 0) {
-                for (int j = 0; j < issued; ++j) {
-                    uint8_t* sj = stages + j * a.stage_bytes;
-#pragma unroll
-                    for (int b = 0; b < 4; ++b)
-                        tma_load_2d(smem_u32(sj + kDecPBytes + b * xbox_bytes), &tmX,
-                                    pre_kb[j] * kDecBlockK + b * 256, 0, smem_u32(&full[j]));
-                }
-            }
         }
         // Do not leave while copies into this CTA's shared memory are in flight.
         for (int i = (issued > S ? issued - S : 0); i < issued; ++i) {
