@@ -118,21 +118,21 @@ __global__ void __launch_bounds__(256) dequantize_kernel(const uint4* __restrict
                                                          const uint16_t* __restrict__ zeros,
                                                          int64_t total_chunks,
                                                          uint4* __restrict__ W_hat) {
-    constexpr int CPG = G / 32;   // 32-code chunks per group
+    // One 4-byte word (8 codes) per thread and step, so that a warp's loads are
+    // 128 contiguous bytes and its stores (8 bf16 = 16 bytes each) 512.
+    constexpr int WPG = G / 8;   // words per group
+    const uint32_t* packed = reinterpret_cast<const uint32_t*>(packed16);
+    const int64_t total_words = total_chunks * 4;
     const int64_t stride = (int64_t)gridDim.x * blockDim.x;
-    for (int64_t c = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; c < total_chunks;
-         c += stride) {
-        const uint4 v = ldg_stream(packed16 + c);
-        const int64_t grp = c / CPG;
+    for (int64_t w = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; w < total_words; w += stride) {
+        uint32_t v;
+        asm volatile("ld.global.nc.L1::no_allocate.u32 %0, [%1];" : "=r"(v) : "l"(packed + w));
+        const int64_t grp = w / WPG;
         const uint32_t ss = dup16(ldg_u16(scales + grp));
         const uint32_t zz = zero_pair<SYM>(SYM ? 0u : (uint32_t)ldg_u16(zeros + grp));
-        const uint32_t wv[4] = {v.x, v.y, v.z, v.w};
-#pragma unroll
-        for (int i = 0; i < 4; ++i) {
-            uint32_t d[4];
-            dequant8_natural<SYM>(wv[i], zz, ss, d);
-            W_hat[c * 4 + i] = make_uint4(d[0], d[1], d[2], d[3]);
-        }
+        uint32_t d[4];
+        dequant8_natural<SYM>(v, zz, ss, d);
+        W_hat[w] = make_uint4(d[0], d[1], d[2], d[3]);
     }
 }
 
