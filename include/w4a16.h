@@ -44,8 +44,9 @@
  * Supported: g ∈ {32, 64, 128}, K a positive multiple of g, N ≥ 0, M ≥ 0
  * (M = 0 or N = 0 is a no-op), N, K, M < 2^31.  Every pointer is a DEVICE
  * pointer owned by the caller; the library allocates no device memory and keeps
- * no state beyond per-device constants (device properties, tensor-map encoder).
- * Device scratch, where a kernel needs it, is the caller's `workspace`.
+ * no state beyond per-device constants (device properties, tensor-map encoder)
+ * and the fixed scratch array of w4a16_gemm_decode_noalloc.  Device scratch,
+ * where a kernel needs it, is otherwise the caller's `workspace`.
  * Each call is asynchronous on `stream` (a cudaStream_t; NULL = legacy default
  * stream).  Arguments are checked on the host before any launch; a rejected
  * call launches nothing and returns W4A16_EINVAL.  No call aborts, throws or
@@ -61,7 +62,7 @@
 extern "C" {
 #endif
 
-#define W4A16_ABI_VERSION 1
+#define W4A16_ABI_VERSION 2   /* 2: the tensor-core path may need a workspace (split K) */
 
 typedef enum w4a16_status {
     W4A16_OK = 0,
@@ -83,7 +84,10 @@ typedef enum w4a16_path {
                                   blocks split across CTAs are added in a fixed order by a
                                   second small kernel */
     W4A16_PATH_TENSORCORE = 2  /* large-M kernel: TMA-fed INT4 tile dequantized into shared
-                                  memory and fed to tcgen05 bf16 MMA with TMEM accumulators */
+                                  memory and fed to tcgen05 bf16 MMA with TMEM accumulators;
+                                  when the output tiles are fewer than the SMs, or the last
+                                  wave of tiles would leave most SMs idle, those tiles split
+                                  K and a reduce kernel adds the parts in a fixed order */
 } w4a16_path;
 
 /* The launch a GEMM call would make (filled by w4a16_gemm_plan). */
@@ -96,8 +100,10 @@ typedef struct w4a16_plan {
     int64_t grid;            /* CTAs launched */
     int32_t smem_bytes;      /* dynamic shared memory per CTA */
     int32_t stages;          /* shared-memory pipeline depth */
-    int32_t kernels;         /* kernels the call launches (decode: 2 when its stream-K
-                                partition splits a row block between CTAs, else 1) */
+    int32_t kernels;         /* kernels the call launches: decode 2 when its stream-K
+                                partition splits a row block between CTAs, else 1;
+                                tensor core 1 unsplit, 2 when every tile splits K (+ the
+                                reduce), 3 with an unsplit head, a split tail and the reduce */
     int64_t workspace_bytes; /* device workspace this launch needs */
 } w4a16_plan;
 

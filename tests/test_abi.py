@@ -52,7 +52,7 @@ def test_library_is_sm100a_only_and_links_no_cudart_dso(lib):
 
 
 def test_status_strings_and_version(lib):
-    assert lib.w4a16_abi_version() == 1
+    assert lib.w4a16_abi_version() == 2
     for s in range(6):
         assert lib.w4a16_status_string(s).startswith(b"W4A16")
 

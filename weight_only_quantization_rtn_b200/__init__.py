@@ -22,6 +22,8 @@ __all__ = ["lib", "quantize", "dequantize", "gemm", "gemm_decode_noalloc", "plan
 
 LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libw4a16.so")
 
+# W4A16_ABI_VERSION in include/w4a16.h that the argument lists below follow
+ABI_VERSION = 2
 PATH_AUTO, PATH_DECODE, PATH_TENSORCORE = 0, 1, 2
 _PATHS = {"auto": PATH_AUTO, "decode": PATH_DECODE, "tensorcore": PATH_TENSORCORE}
 _STATUS = {0: "OK", 1: "EINVAL", 2: "EUNSUPPORTED", 3: "ECUDA", 4: "EWORKSPACE", 5: "EDEVICE"}
@@ -64,6 +66,9 @@ def _load() -> ctypes.CDLL:
     for name in ("w4a16_quantize", "w4a16_dequantize", "w4a16_gemm", "w4a16_gemm_ex",
                  "w4a16_gemm_plan", "w4a16_device_error"):
         getattr(lib, name).restype = ctypes.c_int
+    if lib.w4a16_abi_version() != ABI_VERSION:
+        raise ImportError(f"{LIB_PATH} has ABI version {lib.w4a16_abi_version()}, this binding "
+                          f"expects {ABI_VERSION}: rebuild it")
     return lib
 
 
