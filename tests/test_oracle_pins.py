@@ -285,6 +285,64 @@ def test_on_grid_matrix_is_recovered_exactly(g):
     assert np.array_equal(Wh, Wb)
 
 
+# ------------------------------------------------------------------ per-channel (g = K)
+@pytest.mark.parametrize("sym", [False, True])
+def test_hand_computed_rows_per_channel(sym):
+    """Per-channel granularity (one scale per output row; meko1 page, 量化粒度
+    table; qwbw.cn page §3.4) is g = K: each row of a [rows, 4] matrix is one of
+    the hand-computed groups and must get that group's s, z, codes and x̂."""
+    cases = [c for c in CASES if (c["mode"] == "sym") == sym]
+    assert cases
+    W = oracle.bf16_from_f32(np.stack([_f32(c["x"]) for c in cases]))
+    P, S, Z = oracle.quantize(W, 4, sym)
+    assert S.shape == (len(cases), 1) and Z.shape == (len(cases), 1)
+    Wh = oracle.f32_from_bf16(oracle.dequantize(P, S, Z, 4, 4, sym))
+    for r, c in enumerate(cases):
+        assert S[r, 0] == int(c["s_bits"], 16)
+        assert float(oracle.f32_from_bf16(Z[r, :1])[0]) == (0.0 if sym else c["z"])
+        assert list(P[r]) == [int(b, 16) for b in c["packed"]]
+        assert list(Wh[r]) == [float(v) for v in c["x_hat"]]
+
+
+def test_on_grid_rows_per_channel_recovered_exactly():
+    """Closed form at g = K: rows (q − z)·s with one s and z per row, each row
+    using codes 0 and 15, re-quantize to exactly (s, z, q) and dequantize to W."""
+    rng = np.random.default_rng(17)
+    N, K = 7, 416
+    q = rng.integers(0, 16, size=(N, K))
+    q[:, 3] = 0
+    q[:, K - 2] = 15
+    z = rng.integers(0, 16, size=(N, 1))
+    s = rng.choice([8, 9, 11, 13, 15], size=(N, 1)) * 2.0 ** rng.integers(-14, -6, size=(N, 1))
+    x = (q - z) * s
+    Wb = oracle.bf16_from_f32(x.astype(np.float32))
+    assert np.array_equal(oracle.f32_from_bf16(Wb).astype(np.float64), x)
+    P, S, Z = oracle.quantize(Wb, K, sym=False)
+    assert np.array_equal(oracle.f32_from_bf16(S).astype(np.float64), s)
+    assert np.array_equal(oracle.f32_from_bf16(Z).astype(np.int64), z)
+    assert np.array_equal(oracle.unpack_codes(P.reshape(-1), N * K, False).reshape(N, K), q)
+    assert np.array_equal(oracle.dequantize(P, S, Z, K, K, False), Wb)
+
+
+def test_per_channel_equals_groups_with_equal_ranges():
+    """Invariant: when every 32-wide group of a row holds the row's minimum and
+    maximum (hence also its max|x|), grouped (g = 32) and per-channel (g = K)
+    quantization give the same codes, and the grouped scales and zeros are the
+    per-channel ones repeated."""
+    rng = np.random.default_rng(23)
+    N, K = 5, 256
+    x = rng.standard_normal((N, K)) * 0.02
+    lo, hi = x.min(1, keepdims=True) - 0.01, x.max(1, keepdims=True) + 0.01
+    x[:, 0::32], x[:, 1::32] = lo, hi
+    Wb = oracle.bf16_from_f32(x.astype(np.float32))
+    for sym in (False, True):
+        Pg, Sg, Zg = oracle.quantize(Wb, 32, sym)
+        Pc, Sc, Zc = oracle.quantize(Wb, K, sym)
+        assert np.array_equal(Pg, Pc)
+        assert np.array_equal(Sg, np.repeat(Sc, K // 32, 1))
+        assert np.array_equal(Zg, np.repeat(Zc, K // 32, 1))
+
+
 @pytest.mark.parametrize("sym", [False, True])
 def test_dequantize_closed_form_indexing(sym):
     """Hand-built packed/scales/zeros whose products (q − z)·s are exact in bf16:
