@@ -58,9 +58,20 @@ def load_peaks():
         return dict(FALLBACK_PEAKS), "fallback"
 
 
+def group_of(g: int, K: int) -> int:
+    """g = 0 in a workload definition means per-channel granularity: one group
+    spanning each row (g = K), one scale and zero per output feature."""
+    return K if g == 0 else g
+
+
+def input_bytes(M: int, N: int, K: int, g: int, sym: bool) -> int:
+    """Packed codes + scales (+ zeros if asymmetric) + X."""
+    return N * K // 2 + 2 * N * (K // g) * (1 if sym else 2) + 2 * M * K
+
+
 def algorithmic_bytes(M: int, N: int, K: int, g: int, sym: bool) -> int:
     """Packed codes + scales (+ zeros if asymmetric) + X read once + Y written once."""
-    return N * K // 2 + 2 * N * (K // g) * (1 if sym else 2) + 2 * M * K + 2 * M * N
+    return input_bytes(M, N, K, g, sym) + 2 * M * N
 
 
 # Sources each timed kernel is built from (its device code, the shared device
@@ -378,19 +389,19 @@ def cpu_baseline(layers, M, g, sym, unit_bytes: bool, budget_s: float = 6.0):
     for layer in layers:
         Wb = workloads.bits(layer.weight())
         Xb = workloads.bits(layer.activation(M))
-        P, S, Z = oracle.quantize(Wb, g, sym)
+        P, S, Z = oracle.quantize(Wb, group_of(g, layer.K), sym)
         prepared.append((layer, Xb, P, S, Z))
     reps, t0 = 0, time.perf_counter()
     while True:
         for layer, Xb, P, S, Z in prepared:
-            oracle.gemm_w4a16(Xb, P, S, Z, g, sym)
+            oracle.gemm_w4a16(Xb, P, S, Z, group_of(g, layer.K), sym)
         reps += 1
         el = time.perf_counter() - t0
         if el >= budget_s or reps >= 50:
             break
     per_step = el / reps
     if unit_bytes:
-        work = sum(algorithmic_bytes(M, l.N, l.K, g, sym) for l in layers)
+        work = sum(algorithmic_bytes(M, l.N, l.K, group_of(g, l.K), sym) for l in layers)
         value, unit = work / per_step / 1e9, "GB/s"
     else:
         work = sum(2 * M * l.N * l.K for l in layers)
@@ -409,6 +420,7 @@ def cpu_baseline_sampled(layer, M, g, sym, rows: int):
     oracle.build()
     Wb = workloads.bits(layer.weight())
     Xb = workloads.bits(layer.activation(M))
+    g = group_of(g, layer.K)
     P, S, Z = oracle.quantize(Wb, g, sym)
     ns = np.arange(rows, dtype=np.int64)
     ms = np.zeros(rows, dtype=np.int64)
@@ -427,11 +439,17 @@ def cpu_baseline_sampled(layer, M, g, sym, rows: int):
 
 # ---------------------------------------------------------------------------- main arms
 WORKLOAD_DEFS = {
-    # name: (workload, M, g, sym, metric half)
+    # name: (workload, M, g, sym, metric half); g = 0: per-channel (g = K)
     "decode7b": (workloads.DECODE_7B, 1, 128, False, "hbm"),
     "decode70b": (workloads.DECODE_70B, 1, 128, False, "hbm"),
     "prefill": (workloads.PREFILL, 2048, 128, False, "tensor"),
+    "decode7b_pc": (workloads.DECODE_7B, 1, 0, False, "hbm"),
+    "prefill_pc": (workloads.PREFILL, 2048, 0, False, "tensor"),
 }
+
+
+def workload_name(wl, M, g) -> str:
+    return f"{wl.name}_M{M}" + ("_per_channel" if g == 0 else "")
 
 
 def run_ours(args):
@@ -448,12 +466,11 @@ def run_ours(args):
     l2 = getattr(props, "L2_cache_size", 0) or L2_BYTES_FALLBACK
 
     wl, M, g, sym, half = WORKLOAD_DEFS[args.workload]
-    bytes_step = sum(algorithmic_bytes(M, l.N, l.K, g, sym) for l in wl.layers)
+    bytes_step = sum(algorithmic_bytes(M, l.N, l.K, group_of(g, l.K), sym) for l in wl.layers)
     flops_step = sum(2 * M * l.N * l.K for l in wl.layers)
-    in_bytes_step = sum(l.N * l.K // 2 + 2 * l.N * (l.K // g) * (1 if sym else 2) + 2 * M * l.K
-                        for l in wl.layers)
+    in_bytes_step = sum(input_bytes(M, l.N, l.K, group_of(g, l.K), sym) for l in wl.layers)
     copies = copies_for(in_bytes_step, l2)
-    cases = [GemmCase(w4, l, M, g, sym, copies, dev) for l in wl.layers]
+    cases = [GemmCase(w4, l, M, group_of(g, l.K), sym, copies, dev) for l in wl.layers]
     rot, singles = capture_rotation_graph(w4, cases, copies)
     ms, clocks = run_timed(world, rot, singles, copies, args.steps, args.warmup, sampler_index=local)
     ms_max = max_over_ranks(world, ms)
@@ -466,7 +483,7 @@ def run_ours(args):
         value, unit = total_flops / sec / 1e12, "TFLOP/s"
     kms = per_layer_ms(w4, cases, copies)
 
-    plans = [w4.plan(M, c.N, c.K, g, sym) for c in cases]
+    plans = [w4.plan(M, c.N, c.K, c.g, sym) for c in cases]
     kernel_name = "gemv_decode_kernel" if plans[0]["path"] == "decode" else "gemm_tc_kernel"
     # The timed region holds only this workload's GEMM launches, so the kernel's
     # average launch duration is the region's time over its launches.
@@ -493,8 +510,8 @@ def run_ours(args):
         "warmup": args.warmup, "ms_per_step": ms_max / args.steps, "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
         "config": {
-            "workload": f"{wl.name}_M{M}", "M": M,
-            "layers_KxN": [[l.K, l.N] for l in wl.layers], "g": g,
+            "workload": workload_name(wl, M, g), "M": M,
+            "layers_KxN": [[l.K, l.N] for l in wl.layers], "g": g if g else "K (per-channel)",
             "mode": "sym" if sym else "asym", "description": wl.description,
             "l2": f"{copies} rotating copies of weights+activations "
                   f"({copies * in_bytes_step / 2**20:.0f} MiB, > 2x L2 of {l2 / 2**20:.0f} MiB)",
@@ -552,6 +569,7 @@ def run_ours(args):
             pr = line["prefill"]["roofline"]
             pr["frac_of_nominal"] = pr["achieved"] / NOMINAL_BF16_TFLOPS
             line["quantize_dequantize"] = elementwise_extras(w4, peaks, l2, dev)
+            line["per_channel"] = per_channel_extras(w4, peaks, peak_src, l2, dev)
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         cb = cpu_baseline(wl.layers, M, g, sym, unit_bytes=(half == "hbm")) \
             if half == "hbm" else cpu_baseline_sampled(wl.layers[0], M, g, sym, rows=16)
@@ -615,6 +633,46 @@ def elementwise_extras(w4, peaks, l2, dev, iters=20):
     return {"shape": f"N={N},K={K},g={g},asym",
             "quantize": {"us": qms * 1e3, "GB/s": qb / (qms / 1e3) / 1e9, "frac": qb / (qms / 1e3) / 1e9 / pk},
             "dequantize": {"us": dms * 1e3, "GB/s": db / (dms / 1e3) / 1e9, "frac": db / (dms / 1e3) / 1e9 / pk}}
+
+
+def per_channel_extras(w4, peaks, peak_src, l2, dev, iters=200):
+    """Per-channel granularity (g = K: one scale and zero per output row) on the
+    7B-shaped decode layers at M=1 and on the prefill shape, timed like the
+    headline: rotation graphs over copies larger than L2, CUDA events on the
+    replay stream.  Bytes per GEMM count one scale (and zero) per row."""
+    out = {}
+    for name in ("decode7b_pc", "prefill_pc"):
+        wl, M, g, sym, half = WORKLOAD_DEFS[name]
+        in_bytes = sum(input_bytes(M, l.N, l.K, l.K, sym) for l in wl.layers)
+        copies = copies_for(in_bytes, l2)
+        cases = [GemmCase(w4, l, M, l.K, sym, copies, dev) for l in wl.layers]
+        rot, singles = capture_rotation_graph(w4, cases, copies)
+        n = iters if half == "hbm" else 30
+        replay_steps(rot, singles, copies, 3)
+        torch.cuda.synchronize()
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record()
+        replay_steps(rot, singles, copies, n)
+        b.record()
+        b.synchronize()
+        ms = a.elapsed_time(b) / n
+        plans = [w4.plan(M, c.N, c.K, c.g, sym) for c in cases]
+        kernel = "gemv_decode_kernel" if plans[0]["path"] == "decode" else "gemm_tc_kernel"
+        if half == "hbm":
+            work = sum(c.bytes for c in cases)
+            ach, pk, unit = work / (ms / 1e3) / 1e9, peaks["hbm_gbs"], "GB/s"
+        else:
+            work = sum(c.flops for c in cases)
+            ach, pk, unit = work / (ms / 1e3) / 1e12, peaks["bf16_tflops"], "TFLOP/s"
+        out[name] = {"workload": workload_name(wl, M, g), "ms_per_step": ms,
+                     "roofline": {"bound": "hbm" if half == "hbm" else "tensor", "achieved": ach,
+                                  "peak": pk, "unit": unit, "frac": ach / pk,
+                                  "peak_source": peak_src + ("" if half == "hbm" else " (burst)"),
+                                  "traffic": ncu_traffic(f"{kernel}:{name}"), "kernel": kernel},
+                     "plan": plans}
+        del rot, singles, cases
+        torch.cuda.empty_cache()
+    return out
 
 
 def comparisons(w4, cases, copies, l2, half):
@@ -763,17 +821,17 @@ def run_reference(args):
         for layer in wl.layers:
             Wb = workloads.bits(layer.weight())
             Xb = workloads.bits(layer.activation(M))
-            P, S, Z = oracle.quantize(Wb, g, sym)
-            prepared.append((Xb, P, S, Z))
-        bytes_step = sum(algorithmic_bytes(M, l.N, l.K, g, sym) for l in wl.layers)
+            P, S, Z = oracle.quantize(Wb, group_of(g, layer.K), sym)
+            prepared.append((Xb, P, S, Z, group_of(g, layer.K)))
+        bytes_step = sum(algorithmic_bytes(M, l.N, l.K, group_of(g, l.K), sym) for l in wl.layers)
         for _ in range(min(args.warmup, 1)):
-            for Xb, P, S, Z in prepared:
-                oracle.gemm_w4a16(Xb, P, S, Z, g, sym)
+            for Xb, P, S, Z, gl in prepared:
+                oracle.gemm_w4a16(Xb, P, S, Z, gl, sym)
         steps = max(1, min(args.steps, 20))
         t0 = time.perf_counter()
         for _ in range(steps):
-            for Xb, P, S, Z in prepared:
-                oracle.gemm_w4a16(Xb, P, S, Z, g, sym)
+            for Xb, P, S, Z, gl in prepared:
+                oracle.gemm_w4a16(Xb, P, S, Z, gl, sym)
         el = time.perf_counter() - t0
         value, unit = bytes_step * steps / el / 1e9, "GB/s"
         sample = f"{steps} full step(s): both layer GEMMs, dequantize + binary64 matmul"
@@ -786,8 +844,9 @@ def run_reference(args):
             "steps": steps, "warmup": args.warmup, "ms_per_step": el / steps * 1e3,
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
             "data": "synthetic",
-            "config": {"workload": f"{wl.name}_M{M}", "M": M,
-                       "layers_KxN": [[l.K, l.N] for l in wl.layers], "g": g,
+            "config": {"workload": workload_name(wl, M, g), "M": M,
+                       "layers_KxN": [[l.K, l.N] for l in wl.layers],
+                       "g": g if g else "K (per-channel)",
                        "mode": "sym" if sym else "asym"},
             "cpu_baseline": {"value": value, "unit": unit, "cores": cores, "kind": "oracle",
                              "sample": sample},

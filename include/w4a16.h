@@ -41,8 +41,10 @@
  *  zeros   bf16  [N, K/g]    zero point per group (an integer 0..15 stored in bf16);
  *                            all 0 in symmetric mode
  *
- * Supported: g ∈ {32, 64, 128}, K a positive multiple of g, N ≥ 0, M ≥ 0
- * (M = 0 or N = 0 is a no-op), N, K, M < 2^31.  Every pointer is a DEVICE
+ * Supported: g ∈ {32, 64, 128} with K a positive multiple of g, or g = K with K
+ * a positive multiple of 32 — per-channel granularity, one scale (and zero) per
+ * output feature, scales/zeros [N, 1] (meko1 page, 量化粒度 table; qwbw.cn page
+ * §3.4); N ≥ 0, M ≥ 0 (M = 0 or N = 0 is a no-op), N, K, M < 2^31.  Every pointer is a DEVICE
  * pointer owned by the caller; the library allocates no device memory and keeps
  * no state beyond per-device constants (device properties, tensor-map encoder)
  * and the fixed scratch array of w4a16_gemm_decode_noalloc.  Device scratch,
@@ -108,7 +110,8 @@ typedef struct w4a16_plan {
 } w4a16_plan;
 
 /* Quantize W[N, K] group-wise by RTN (asymmetric when sym == 0, symmetric when
- * sym == 1) and pack two codes per byte.
+ * sym == 1) and pack two codes per byte.  g = K quantizes per channel: each
+ * row's range is reduced over the whole row.
  *   W       in   bf16 [N, K]
  *   packed  out  uint8 [N, K/2]
  *   scales  out  bf16 [N, K/g]
@@ -128,11 +131,12 @@ w4a16_status w4a16_dequantize(const void* packed, const void* scales, const void
 
 /* Bytes of device workspace w4a16_gemm needs for this shape.  The decode path
  * stores there the fp32 partial sums of the 32-row blocks that its stream-K
- * partition splits between CTAs; the tensor-core path, when its output tiles
- * are fewer than the SMs and it splits K into S parts, stores S fp32 partial
- * results of M x N (each rounded up to a multiple of 4 elements), and 0 bytes
- * are needed otherwise.  In both cases a second, small kernel adds the parts in
- * a fixed order.  The contents are scratch: no
+ * partition splits between CTAs.  The tensor-core path, for the output tiles
+ * whose K it splits into S parts (all tiles when they are fewer than the SMs,
+ * else only a mostly-empty last wave), stores S fp32 partial tiles of
+ * 128 weight rows x tile_m activation rows per split tile, and needs 0 bytes
+ * when it splits nothing.  In both cases a second, small kernel adds the parts
+ * in a fixed order.  The contents are scratch: no
  * initialization is needed and nothing is kept between calls, but two calls
  * that may run at the same time (for instance on two streams) need two
  * workspaces.  Uses the current device's SM count. */

@@ -76,6 +76,34 @@ def test_gemm_rejects_invalid_arguments(lib, kw):
     assert _gemm(lib, **kw) == EINVAL
 
 
+@pytest.mark.parametrize("K,g,ok", [
+    (4096, 4096, True), (11008, 11008, True), (96, 96, True), (512, 512, True),   # g = K
+    (128, 128, True), (4096, 128, True),                                          # grouped
+    (48, 48, False), (200, 200, False),          # per-channel needs K a multiple of 32
+    (4096, 2048, False), (512, 256, False),      # other group sizes are not supported
+])
+def test_per_channel_shape_rules(lib, K, g, ok):
+    """g = K selects per-channel granularity (one scale and zero per row)."""
+    assert (_gemm(lib, M=0, K=K, g=g) == 0) == ok
+    assert (lib.w4a16_quantize(FAKE, 0, K, g, 0, FAKE, FAKE, FAKE, None) == 0) == ok
+    assert (lib.w4a16_dequantize(FAKE, FAKE, FAKE, 0, K, g, 0, FAKE, None) == 0) == ok
+
+
+def test_per_channel_plans():
+    """Per-channel plans cover the same units as grouped ones; the decode stage
+    carries one scale/zero pair per row, so it fits at least as many stages."""
+    for M, N, K in ((1, 11008, 4096), (1, 4096, 11008), (8, 8192, 28672), (16, 4096, 4096)):
+        pc, gr = w4.plan(M, N, K, K), w4.plan(M, N, K, 128)
+        assert pc["path"] == gr["path"] == "decode"
+        assert pc["grid"] == gr["grid"] and pc["kernels"] == gr["kernels"]
+        assert pc["workspace_bytes"] == gr["workspace_bytes"]
+        assert pc["stages"] >= gr["stages"]
+    for M, N, K in ((48, 1000, 4352), (300, 10240, 2048), (2048, 8192, 8192)):
+        head, tail, splits, bm = _tc_schedule(M, N, K, K)
+        p = w4.plan(M, N, K, K)
+        assert p["path"] == "tensorcore" and p["grid"] == head + tail * splits
+
+
 def test_gemm_sym_accepts_null_zeros_validation(lib):
     # with sym=1 a NULL zeros pointer passes validation; M=0 then returns before any launch
     assert _gemm(lib, M=0, sym=1, Z=None) == 0

@@ -65,8 +65,8 @@ def test_decode_path_small(M, N, K, g, sym):
 @pytest.mark.parametrize("ctas", [1, 2, 3, 5, 7, 13, 40, 97, 300])
 @pytest.mark.parametrize("M", [1, 12])
 def test_decode_stream_k_partitions(ctas, M):
-    """Many persistent-grid sizes: row blocks split 0..n times between CTAs,
-    finished by the last arrival; counters must be back at zero afterwards."""
+    """Many persistent-grid sizes: row blocks split 0..n times between CTAs, their
+    parts added by the fixup kernel; two calls in a row reuse the workspace."""
     _check_full(M, 300, 1024 * 5 + 256, 128, False, "decode", seed=5, ctas=ctas)
     _check_full(M, 300, 1024 * 5 + 256, 128, False, "decode", seed=6, ctas=ctas)
 
@@ -88,7 +88,7 @@ def test_tensorcore_path_small(M, N, K, g, sym):
 # ------------------------------------------------------------------ exact special cases
 @pytest.mark.parametrize("path", ["decode", "tensorcore"])
 @pytest.mark.parametrize("sym", [False, True])
-@pytest.mark.parametrize("g", [32, 128])
+@pytest.mark.parametrize("g", [32, 128, 512])     # 512 = K: per-channel
 def test_one_hot_activations_select_dequantized_weights_bit_exact(path, sym, g):
     """X = one-hot rows: Y[m, n] = Ŵ[n, k_m] exactly (a single nonzero product,
     exact in fp32, and already a bf16 value), so the fused dequantization of
@@ -103,6 +103,31 @@ def test_one_hot_activations_select_dequantized_weights_bit_exact(path, sym, g):
         X[torch.arange(kk.numel()), kk] = 1.0
         Y = w4.gemm(X.cuda(), P, S, Z, g, sym, path=path)
         assert torch.equal(Y, Wh[:, kk.cuda()].t().contiguous()), f"k in {start}..{start + 15}"
+
+
+# ------------------------------------------------------------------ per-channel (g = K)
+PC_DECODE_SHAPES = [(1, 256, 256), (1, 1, 160), (3, 100, 1152), (8, 128, 4096), (13, 257, 1056),
+                    (16, 64, 11008)]
+PC_TC_SHAPES = [(17, 128, 96), (48, 1000, 4352), (129, 64, 4096), (300, 700, 1056)]
+
+
+@pytest.mark.parametrize("sym", [False, True])
+@pytest.mark.parametrize("M,N,K", PC_DECODE_SHAPES)
+def test_per_channel_decode(M, N, K, sym):
+    """g = K: one scale and zero per weight row, through the decode kernel."""
+    _check_full(M, N, K, K, sym, "decode", seed=2 * M + N + K)
+
+
+@pytest.mark.parametrize("sym", [False, True])
+@pytest.mark.parametrize("M,N,K", PC_TC_SHAPES)
+def test_per_channel_tensorcore(M, N, K, sym):
+    """g = K through the tensor-core kernel, split-K and unsplit tiles."""
+    _check_full(M, N, K, K, sym, "tensorcore", seed=3 * M + N + K)
+
+
+@pytest.mark.parametrize("ctas", [3, 97])
+def test_per_channel_decode_partitions(ctas):
+    _check_full(5, 300, 1024 * 5 + 256, 1024 * 5 + 256, False, "decode", seed=8, ctas=ctas)
 
 
 @pytest.mark.parametrize("path", ["decode", "tensorcore"])
@@ -207,6 +232,23 @@ def test_prefill_full_size():
                                      (4096, 32, True)])
 def test_crossover_full_size(M, g, sym):
     _check_sampled(workloads.CROSSOVER.layers[0], M, g, sym, n_samples=2048)
+
+
+@pytest.mark.parametrize("li", [0, 1])
+def test_per_channel_7b_decode_full_size(li):
+    layer = workloads.DECODE_7B.layers[li]
+    _check_sampled(layer, 1, layer.K, False)
+
+
+@pytest.mark.parametrize("li", [0, 1])
+def test_per_channel_70b_decode_full_size(li):
+    layer = workloads.DECODE_70B.layers[li]
+    _check_sampled(layer, 2, layer.K, True)
+
+
+def test_per_channel_prefill_full_size():
+    layer = workloads.PREFILL.layers[0]
+    _check_sampled(layer, 2048, layer.K, False, n_samples=2048)
 
 
 def test_tiny_config_full_compare():

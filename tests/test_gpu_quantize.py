@@ -55,12 +55,7 @@ def test_tiny_config_bit_exact():
     _run_and_compare(layer.weight(), 128, False)
 
 
-@pytest.mark.parametrize("sym", [False, True])
-@pytest.mark.parametrize("g", [32, 128])
-def test_degenerate_groups(g, sym):
-    """All-zero groups, one-sided groups, constant groups, exact ties, huge and
-    tiny magnitudes, a single nonzero element."""
-    K = 4 * g
+def _degenerate_rows(K):
     rows = []
     rows.append(np.zeros(K))                                      # all zero: s = 0
     rows.append(np.abs(np.random.default_rng(1).standard_normal(K)) + 0.5)   # all positive
@@ -74,8 +69,34 @@ def test_degenerate_groups(g, sym):
     rows.append(np.random.default_rng(3).standard_normal(K) * 2.0 ** 100)
     rows.append(np.random.default_rng(4).standard_normal(K) * 2.0 ** -100)
     rows.append(np.random.default_rng(5).standard_normal(K) * 1e-39)      # bf16 subnormals
-    W = torch.tensor(np.stack(rows), dtype=torch.float32).to(torch.bfloat16)
-    _run_and_compare(W, g, sym)
+    return torch.tensor(np.stack(rows), dtype=torch.float32).to(torch.bfloat16)
+
+
+@pytest.mark.parametrize("sym", [False, True])
+@pytest.mark.parametrize("g", [32, 128, 160])     # 160 = K: per-channel
+def test_degenerate_groups(g, sym):
+    """All-zero groups, one-sided groups, constant groups, exact ties, huge and
+    tiny magnitudes, a single nonzero element."""
+    K = 4 * g if g != 160 else 160
+    _run_and_compare(_degenerate_rows(K), g, sym)
+
+
+# ------------------------------------------------------------------ per-channel (g = K)
+@pytest.mark.parametrize("sym", [False, True])
+@pytest.mark.parametrize("N,K", [(1, 160), (7, 96), (33, 416), (130, 4096), (517, 1056),
+                                 (64, 11008), (1500, 256)])
+def test_per_channel_bit_exact(N, K, sym):
+    """g = K: one scale and zero per row (a block-wide range reduction per row);
+    1500 rows exceed the row kernel's grid, so CTAs loop over rows."""
+    W = workloads.make_weight(N, K, 0.02, seed=N + 3 * K, outlier_frac=0.02, outlier_scale=20.0)
+    _run_and_compare(W, K, sym)
+
+
+@pytest.mark.parametrize("sym", [False, True])
+@pytest.mark.parametrize("layer_idx", [0, 1])
+def test_per_channel_7b_shaped_bit_exact(layer_idx, sym):
+    layer = workloads.DECODE_7B.layers[layer_idx]
+    _run_and_compare(layer.weight(), layer.K, sym)
 
 
 @pytest.mark.parametrize("layer_idx", [0, 1])

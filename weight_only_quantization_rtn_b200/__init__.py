@@ -110,7 +110,8 @@ def _need(t: torch.Tensor, dtype: torch.dtype, name: str, ndim: int = 2) -> None
 
 
 def quantize(W: torch.Tensor, g: int = 128, sym: bool = False):
-    """Group-wise RTN quantization of W[N, K] (bf16, cuda).
+    """Group-wise RTN quantization of W[N, K] (bf16, cuda); g = K quantizes per
+    channel (one scale and zero per row).
 
     Returns (packed uint8 [N, K/2], scales bf16 [N, K/g], zeros bf16 [N, K/g]);
     zeros are all 0 when ``sym``."""

@@ -104,7 +104,10 @@ __global__ void __launch_bounds__(kTcThreads, 1)
     uint64_t* slab_full = bars + 3 * S + 1;    // [2] slab of scales/zeros landed
     uint64_t* slab_empty = bars + 3 * S + 3;   // [2] dequantizers done with the slab
     uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(bars + 3 * S + 5);
-    constexpr int kSlabKb = 8 * G / kTcBlockK;   // K blocks served by one slab of 8 groups
+    // G == 0: per-channel granularity, one scale (and zero) per row for all of K;
+    // each dequantizing thread reads its row's pair once, nothing is staged.
+    constexpr int kG = G == 0 ? 1 : G;                            // divisor for the grouped forms
+    constexpr int kSlabKb = G == 0 ? 1 : 8 * G / kTcBlockK;       // K blocks served by one slab
 
     const int warp = threadIdx.x >> 5;
     const int lane = threadIdx.x & 31;
@@ -115,11 +118,12 @@ __global__ void __launch_bounds__(kTcThreads, 1)
     // this CTA's K blocks [kb0, kb0 + nkb); kb0 is a multiple of the slab length
     const int kb0 = (int)blockIdx.z * kb_split;
     const int nkb = min(num_kb - kb0, kb_split);
-    const int Gn = K / G;
+    const int Gn = G == 0 ? 1 : K / kG;
 
     if (threadIdx.x == 0) {
         for (int s = 0; s < S; ++s) {
-            mbar_init(smem_u32(&full[s]), sz_tma ? 1 : 1 + 32);   // TMA arrive (+ 32 scale lanes)
+            // TMA arrive (+ 32 scale-copying lanes)
+            mbar_init(smem_u32(&full[s]), (sz_tma || G == 0) ? 1 : 1 + 32);
             mbar_init(smem_u32(&afull[s]), kTcDequantWarps);
             mbar_init(smem_u32(&empty[s]), 1);
         }
@@ -179,10 +183,10 @@ __global__ void __launch_bounds__(kTcThreads, 1)
                 tma_load_2d(smem_u32(ps + s * Cfg::kPBytes), &tmP, kb * (kTcBlockK / 2), n0, bar);
             }
             // the aligned pair of groups holding this block's group(s), per row and array
-            const int jpair = ((kb * kTcBlockK) / G) & ~1;
+            const int jpair = ((kb * kTcBlockK) / kG) & ~1;
             uint32_t* dst = szs + s * 2 * kTcTileN;
-            if (sz_tma) {
-                // scales/zeros come with the slab
+            if (G == 0 || sz_tma) {
+                // per-channel: nothing to stage; grouped: scales/zeros come with the slab
             } else if (sz_async) {
 #pragma unroll
                 for (int e = lane; e < 2 * kTcTileN; e += 32) {
@@ -253,6 +257,11 @@ __global__ void __launch_bounds__(kTcThreads, 1)
         const int h = (warp - 2) >> 2;          // K half of each 64-wide block
         const int n = n0 + r;
         const bool row_ok = n < N;
+        uint32_t row_ss = 0u, row_zz = 0x43084308u;   // per-channel pair of this row
+        if (G == 0 && row_ok) {
+            row_ss = dup16(ldg_u16(scales + n));
+            if (!SYM) row_zz = bf16x2_add(dup16(ldg_u16(zeros + n)), 0x43004300u);
+        }
         bool ok = true;
         for (int i = 0; i < nkb; ++i) {
             const int kb = kb0 + i;
@@ -269,7 +278,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
                 break;
             }
             uint32_t spair = 0u, zpair = 0u;
-            if (!sz_tma) {
+            if (G != 0 && !sz_tma) {
                 spair = lds_u32(szs + s * 2 * kTcTileN + r);
                 zpair = SYM ? 0u : lds_u32(szs + s * 2 * kTcTileN + kTcTileN + r);
             }
@@ -280,14 +289,17 @@ __global__ void __launch_bounds__(kTcThreads, 1)
                 // 32-byte swizzle: chunk h of row r sits at position h ^ bit 2 of r
                 const uint4 v = lds128(prow + 16 * (h ^ ((r >> 2) & 1)));
                 uint32_t ss, zz;
-                if (sz_tma) {
-                    const int gi = ((kb * kTcBlockK + 32 * h) / G) % 8;   // group within the slab
+                if (G == 0) {
+                    ss = row_ss;
+                    zz = row_zz;
+                } else if (sz_tma) {
+                    const int gi = ((kb * kTcBlockK + 32 * h) / kG) % 8;  // group within the slab
                     ss = __byte_perm(lds_u16(srow + gi), 0, 0x1010);
                     zz = SYM ? 0x43084308u
                              : bf16x2_add(__byte_perm(lds_u16(srow + kTcTileN * 8 + gi), 0, 0x1010),
                                           0x43004300u);
                 } else {
-                    const int half = ((kb * kTcBlockK + 32 * h) / G) & 1;   // position in the pair
+                    const int half = ((kb * kTcBlockK + 32 * h) / kG) & 1;  // position in the pair
                     ss = dup16(spair >> (16 * half));
                     zz = SYM ? 0x43084308u : bf16x2_add(dup16(zpair >> (16 * half)), 0x43004300u);
                 }

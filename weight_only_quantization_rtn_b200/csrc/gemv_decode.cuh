@@ -25,11 +25,14 @@
 //    The MMA reduces over K in fragment order, so the nibble pairs are used in
 //    the order the isolation yields them — (q0,q4)(q1,q5)(q2,q6)(q3,q7) — and
 //    the X pairs are permuted to match with PRMT.
-//  * The producer warp's 32 lanes also copy the unit's scales and zero points
-//    into the same stage with 4-byte cp.async copies (zero-filled outside the
-//    matrix) that arrive on the stage's barrier when they land, so consumers
-//    never wait on them; rows whose scale stride is not 4-byte aligned use
-//    plain loads and stores instead.
+//  * The unit's scales and zero points land in the same stage and complete on
+//    the same barrier, so consumers never wait on them: by TMA (boxes of 32
+//    rows x 1024/g groups) when a scale row is 16-byte aligned; otherwise the
+//    producer warp's 32 lanes copy them with 4-byte cp.async copies
+//    (zero-filled outside the matrix), or with plain loads and stores when the
+//    scale stride is not 4-byte aligned.  Per-channel (g = K, template G = 0):
+//    the row block's 32 scales (and zeros) are contiguous, and 4 (8) lanes copy
+//    them with 16-byte cp.async copies.
 //  * At the end of a row block the 8 warps' partial tiles are summed in shared
 //    memory in a fixed order and written to Y.  A row block that the stream-K
 //    partition splits between CTAs is written instead as one fp32 partial per
@@ -129,6 +132,12 @@ __device__ __forceinline__ void cp_async_4(uint32_t dst, const void* src, uint32
                  : "memory");
 }
 
+__device__ __forceinline__ void cp_async_16(uint32_t dst, const void* src, uint32_t src_bytes) {
+    // 16-byte async copy global -> shared; bytes beyond src_bytes (0..16) are zero-filled.
+    asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(dst), "l"(src), "r"(src_bytes)
+                 : "memory");
+}
+
 __device__ __forceinline__ void cp_async_arrive_noinc(uint32_t bar) {
     // Arrive on the barrier once this thread's earlier cp.async copies have landed.
     asm volatile("cp.async.mbarrier.arrive.noinc.shared::cta.b64 [%0];" ::"r"(bar) : "memory");
@@ -140,7 +149,9 @@ __global__ void __launch_bounds__(kDecThreads, MB == 1 ? 2 : 1)
                        const __grid_constant__ CUtensorMap tmX,
                        const __grid_constant__ CUtensorMap tmS,
                        const __grid_constant__ CUtensorMap tmZ, const DecodeArgs a) {
-    constexpr int GB = kDecBlockK / G;                 // groups per row per unit
+    // G == 0: per-channel granularity, one scale (and zero) per row for all of K.
+    constexpr int kG = G == 0 ? 1 : G;                 // divisor for the grouped forms
+    constexpr int GB = G == 0 ? 1 : kDecBlockK / kG;   // groups per row per unit
     constexpr int RED = 2 * MB * 128;                  // partial elements per row block
 
     extern __shared__ uint8_t smem_raw[];
@@ -162,7 +173,7 @@ __global__ void __launch_bounds__(kDecThreads, MB == 1 ? 2 : 1)
     const int nunits = (int)(u1 - u0);
     const int M = a.M;
     const uint32_t xbox_bytes = (uint32_t)M * 512u;
-    const int Gtot = a.K / G;
+    const int Gtot = G == 0 ? 1 : a.K / kG;
 
     if (threadIdx.x == 0) {
         for (int s = 0; s < S; ++s) {
@@ -222,9 +233,20 @@ __global__ void __launch_bounds__(kDecThreads, MB == 1 ? 2 : 1)
             }
             // scales (and zeros): 32 rows x GB groups
             uint16_t* sz = reinterpret_cast<uint16_t*>(st + a.sz_offset);
-            const int g0 = kb * GB;
+            const int g0 = G == 0 ? 0 : kb * GB;
             const int arrays = SYM ? 1 : 2;
-            if (a.sz_tma) {
+            if constexpr (G == 0) {
+                // per-channel: the row block's 32 scales (and zeros) are 64 contiguous,
+                // 16-byte aligned bytes; lanes 0-3 copy the scales, 4-7 the zeros
+                if (lane < 4 * arrays) {
+                    const int arr = lane >> 2, j = lane & 3;
+                    const int n = rb * kDecRows + 8 * j;
+                    const int valid = min(max(a.N - n, 0), 8);
+                    const uint16_t* src = (arr == 0 ? a.scales : a.zeros) + (valid > 0 ? n : 0);
+                    cp_async_16(smem_u32(sz + arr * kDecRows + 8 * j), src, 2u * (uint32_t)valid);
+                }
+                cp_async_arrive_noinc(bar);
+            } else if (a.sz_tma) {
                 if (lane == 0) {
                     tma_load_2d(smem_u32(sz), &tmS, g0, rb * kDecRows, bar);
                     if (!SYM) tma_load_2d(smem_u32(sz + kDecRows * GB), &tmZ, g0, rb * kDecRows, bar);
@@ -273,7 +295,7 @@ __global__ void __launch_bounds__(kDecThreads, MB == 1 ? 2 : 1)
     const int g = lane >> 2;
     const int q = lane & 3;
     const int c = warp;                     // K chunk of the unit: k = 128·c .. 128·c+127
-    const int grp_local = (c * 128 + 32 * q) / G;   // this lane's group inside the unit
+    const int grp_local = G == 0 ? 0 : (c * 128 + 32 * q) / kG;   // this lane's group in the unit
 
     float acc[2][MB][4];
 #pragma unroll

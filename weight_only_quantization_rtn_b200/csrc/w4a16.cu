@@ -32,7 +32,20 @@ PFN_cuTensorMapEncodeTiled_v12000 g_encode_tiled = nullptr;
 
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
-bool valid_group(int32_t g) { return g == 32 || g == 64 || g == 128; }
+// Group sizes along K with kernels of their own.
+bool grouped(int32_t g) { return g == 32 || g == 64 || g == 128; }
+
+// Per-channel granularity: one group spanning the whole row (g == K), one scale
+// and zero point per output feature (meko1 page, 量化粒度 table; qwbw.cn page §3.4).
+// Kernels take it as group size 0.
+bool per_channel(int32_t g, int64_t K) { return !grouped(g) && (int64_t)g == K; }
+
+// g is one of the grouped sizes with K a multiple of it, or g == K with K a
+// multiple of 32 (packed rows of whole 16-byte chunks, as TMA needs).
+bool valid_group(int32_t g, int64_t K) {
+    if (grouped(g)) return K % g == 0;
+    return per_channel(g, K) && K % 32 == 0;
+}
 
 w4a16_status device_info(DeviceInfo* out) {
     int dev = 0;
@@ -96,11 +109,14 @@ int decode_fixed_smem(int mb) {
            + 1024;                              // alignment slack
 }
 
-// Stage: packed tile (16 KB) | X slice (M x 1024 bf16) | scales + zeros (2 x 32 x 1024/g bf16).
+// Stage: packed tile (16 KB) | X slice (M x 1024 bf16) | scales + zeros (2 x 32 x gb bf16).
 int decode_sz_offset(int64_t M) { return kDecPBytes + (int)M * 2048; }
 
-int decode_stage_bytes(int64_t M, int g) {
-    const int raw = decode_sz_offset(M) + 2 * kDecRows * (kDecBlockK / g) * 2;
+// Scale (and zero) groups of one row inside a 1024-wide K block.
+int decode_unit_groups(int32_t g, int64_t K) { return per_channel(g, K) ? 1 : kDecBlockK / g; }
+
+int decode_stage_bytes(int64_t M, int gb) {
+    const int raw = decode_sz_offset(M) + 2 * kDecRows * gb * 2;
     return (raw + 1023) / 1024 * 1024;
 }
 
@@ -110,7 +126,7 @@ DecodeGeometry decode_geometry(int64_t M, int64_t N, int64_t K, int g) {
     d.rb = (int)((N + kDecRows - 1) / kDecRows);
     d.kbn = (int)((K + kDecBlockK - 1) / kDecBlockK);
     d.units = (int64_t)d.rb * d.kbn;
-    d.stage_bytes = decode_stage_bytes(M, g);
+    d.stage_bytes = decode_stage_bytes(M, decode_unit_groups(g, K));
     const int fixed = decode_fixed_smem(d.mb);
     const int two = (kSmemPerSm / 2 - kSmemReservedPerCta - fixed) / d.stage_bytes;
     if (d.mb == 1 && two >= 3) {
@@ -175,7 +191,7 @@ TcSchedule tc_schedule(int64_t M, int64_t N, int64_t K, int g, int bm, int sm_co
     t.tiles_n = (int)((N + kTcTileN - 1) / kTcTileN);
     const int64_t tiles = (int64_t)t.tiles_n * ((M + bm - 1) / bm);
     const int num_kb = (int)((K + kTcBlockK - 1) / kTcBlockK);
-    const bool sz_tma = (K / g) % 8 == 0;
+    const bool sz_tma = !per_channel(g, K) && (K / g) % 8 == 0;
     int64_t tail = 0;
     if (tiles < sm_count) {
         tail = tiles;
@@ -212,11 +228,10 @@ int tc_smem_bytes(int bm) {
 }
 
 w4a16_status check_shape(int64_t M, int64_t N, int64_t K, int32_t g, int32_t sym) {
-    if (!valid_group(g)) return W4A16_EINVAL;
     if (sym != 0 && sym != 1) return W4A16_EINVAL;
     if (M < 0 || N < 0 || K <= 0) return W4A16_EINVAL;
     if (M > kMaxDim || N > kMaxDim || K > kMaxDim) return W4A16_EINVAL;
-    if (K % g != 0) return W4A16_EINVAL;
+    if (!valid_group(g, K)) return W4A16_EINVAL;
     return W4A16_OK;
 }
 
@@ -309,8 +324,9 @@ w4a16_status launch_decode_t(const w4a16_plan& p, const CUtensorMap& tmP, const 
             return W4A16_ECUDA;
         attr_set[dev] = true;
     }
-    // Programmatic dependent launch: the kernel may start while the previous
-    // grid on the stream drains; it reads only weights before its dependency wait.
+    // Programmatic dependent launch: the kernel's CTAs are placed and set up while
+    // the previous grid on the stream drains; they read nothing before their
+    // dependency wait.
     cudaLaunchAttribute attr[1];
     attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
     attr[0].val.programmaticStreamSerializationAllowed = 1;
@@ -358,8 +374,9 @@ w4a16_status launch_decode(const w4a16_plan& p, const void* X, int64_t M, int64_
     args.stages = d.stages;
     args.stage_bytes = d.stage_bytes;
     args.sz_offset = decode_sz_offset(M);
-    args.sz_async = ((K / g) % 2 == 0) ? 1 : 0;   // 4-byte aligned scale rows
-    args.sz_tma = ((K / g) % 8 == 0) ? 1 : 0;     // 16-byte aligned scale rows
+    const bool pc = per_channel(g, K);             // scales [N]: the kernel copies 16-byte runs
+    args.sz_async = (!pc && (K / g) % 2 == 0) ? 1 : 0;   // 4-byte aligned scale rows
+    args.sz_tma = (!pc && (K / g) % 8 == 0) ? 1 : 0;     // 16-byte aligned scale rows
     args.U = d.units;
     const bool split = p.kernels > 1;
     // Scales and zeros [N][K/g]: boxes of 32 rows x (1024/g) groups, when their rows are
@@ -377,33 +394,31 @@ w4a16_status launch_decode(const w4a16_plan& p, const void* X, int64_t M, int64_
             if (st != W4A16_OK) return st;
         }
     }
+    const int gsel = pc ? 0 : g;                   // kernel group size, 0 = per-channel
+#define W4A16_DEC_G(MBV, SYMV)                                                                  \
+    switch (gsel) {                                                                             \
+        case 32: return launch_decode_t<MBV, SYMV, 32>(p, tmP, tmX, tmS, tmZ, args, split, stream); \
+        case 64: return launch_decode_t<MBV, SYMV, 64>(p, tmP, tmX, tmS, tmZ, args, split, stream); \
+        case 128: return launch_decode_t<MBV, SYMV, 128>(p, tmP, tmX, tmS, tmZ, args, split, stream); \
+        case 0: return launch_decode_t<MBV, SYMV, 0>(p, tmP, tmX, tmS, tmZ, args, split, stream);   \
+        default: return W4A16_EINVAL;                                                           \
+    }
     if (d.mb == 1) {
-        if (sym) {
-            if (g == 32) return launch_decode_t<1, true, 32>(p, tmP, tmX, tmS, tmZ, args, split, stream);
-            if (g == 64) return launch_decode_t<1, true, 64>(p, tmP, tmX, tmS, tmZ, args, split, stream);
-            return launch_decode_t<1, true, 128>(p, tmP, tmX, tmS, tmZ, args, split, stream);
-        }
-        if (g == 32) return launch_decode_t<1, false, 32>(p, tmP, tmX, tmS, tmZ, args, split, stream);
-        if (g == 64) return launch_decode_t<1, false, 64>(p, tmP, tmX, tmS, tmZ, args, split, stream);
-        return launch_decode_t<1, false, 128>(p, tmP, tmX, tmS, tmZ, args, split, stream);
+        if (sym) W4A16_DEC_G(1, true)
+        W4A16_DEC_G(1, false)
     }
-    if (sym) {
-        if (g == 32) return launch_decode_t<2, true, 32>(p, tmP, tmX, tmS, tmZ, args, split, stream);
-        if (g == 64) return launch_decode_t<2, true, 64>(p, tmP, tmX, tmS, tmZ, args, split, stream);
-        return launch_decode_t<2, true, 128>(p, tmP, tmX, tmS, tmZ, args, split, stream);
-    }
-    if (g == 32) return launch_decode_t<2, false, 32>(p, tmP, tmX, tmS, tmZ, args, split, stream);
-    if (g == 64) return launch_decode_t<2, false, 64>(p, tmP, tmX, tmS, tmZ, args, split, stream);
-    return launch_decode_t<2, false, 128>(p, tmP, tmX, tmS, tmZ, args, split, stream);
+    if (sym) W4A16_DEC_G(2, true)
+    W4A16_DEC_G(2, false)
+#undef W4A16_DEC_G
 }
 
 template <int BM, bool SYM, int G>
 w4a16_status launch_tc_t(const w4a16_plan& p, const CUtensorMap& tmX, const CUtensorMap& tmP,
                          const CUtensorMap& tmS, const CUtensorMap& tmZ, int sz_tma,
                          const void* scales, const void* zeros, void* Y, int M, int N, int K,
-                         void* workspace, cudaStream_t stream) {
+                         int g, void* workspace, cudaStream_t stream) {
     auto kern = gemm_tc_kernel<BM, SYM, G>;
-    const int sz_async = ((K / G) % 2 == 0) ? 1 : 0;   // 4-byte aligned scale rows
+    const int sz_async = (G != 0 && (K / g) % 2 == 0) ? 1 : 0;   // 4-byte aligned scale rows
     static bool attr_set[kMaxDevices] = {};
     int dev = 0;
     cudaGetDevice(&dev);
@@ -414,7 +429,7 @@ w4a16_status launch_tc_t(const w4a16_plan& p, const CUtensorMap& tmX, const CUte
         attr_set[dev] = true;
     }
     // the same schedule make_plan reported (it used this device's SM count)
-    const TcSchedule ts = tc_schedule(M, N, K, G, BM, current_sm_count());
+    const TcSchedule ts = tc_schedule(M, N, K, g, BM, current_sm_count());
     const auto* sc = static_cast<const uint16_t*>(scales);
     const auto* ze = static_cast<const uint16_t*>(zeros);
     auto* y = static_cast<uint16_t*>(Y);
@@ -462,10 +477,10 @@ template <bool SYM, int G>
 w4a16_status launch_tc_g(const w4a16_plan& p, const CUtensorMap& tmX, const CUtensorMap& tmP,
                          const CUtensorMap& tmS, const CUtensorMap& tmZ, int sz_tma,
                          const void* scales, const void* zeros, void* Y, int M, int N, int K,
-                         void* workspace, cudaStream_t stream) {
+                         int g, void* workspace, cudaStream_t stream) {
 #define W4A16_TC_TILE(BMV) \
-    launch_tc_t<BMV, SYM, G>(p, tmX, tmP, tmS, tmZ, sz_tma, scales, zeros, Y, M, N, K, workspace, \
-                             stream)
+    launch_tc_t<BMV, SYM, G>(p, tmX, tmP, tmS, tmZ, sz_tma, scales, zeros, Y, M, N, K, g, \
+                             workspace, stream)
     switch (p.tile_m) {
         case 32: return W4A16_TC_TILE(32);
         case 64: return W4A16_TC_TILE(64);
@@ -488,7 +503,8 @@ w4a16_status launch_tc(const w4a16_plan& p, const void* X, int64_t M, int64_t K,
     if (st != W4A16_OK) return st;
     // Scales and zeros [N][K/g] in slabs of 8 groups x 128 rows, when their rows are
     // 16-byte aligned; otherwise the kernel copies them with cp.async.
-    const int sz_tma = ((K / g) % 8 == 0) ? 1 : 0;
+    const bool pc = per_channel(g, K);             // per-channel: each row's pair read once
+    const int sz_tma = (!pc && (K / g) % 8 == 0) ? 1 : 0;
     CUtensorMap tmS = tmP, tmZ = tmP;
     if (sz_tma) {
         st = encode_2d(&tmS, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, scales, (uint64_t)(K / g), (uint64_t)N,
@@ -504,13 +520,14 @@ w4a16_status launch_tc(const w4a16_plan& p, const void* X, int64_t M, int64_t K,
 #define W4A16_TC_CASE(GG)                                                                      \
     case GG:                                                                                   \
         return sym ? launch_tc_g<true, GG>(p, tmX, tmP, tmS, tmZ, sz_tma, scales, zeros, Y, m, n, \
-                                           k, workspace, stream)                               \
+                                           k, g, workspace, stream)                            \
                    : launch_tc_g<false, GG>(p, tmX, tmP, tmS, tmZ, sz_tma, scales, zeros, Y, m, n, \
-                                            k, workspace, stream);
-    switch (g) {
+                                            k, g, workspace, stream);
+    switch (pc ? 0 : g) {
         W4A16_TC_CASE(32)
         W4A16_TC_CASE(64)
         W4A16_TC_CASE(128)
+        W4A16_TC_CASE(0)
         default: return W4A16_EINVAL;
     }
 #undef W4A16_TC_CASE
@@ -580,6 +597,12 @@ w4a16_status w4a16_quantize(const void* W, int64_t N, int64_t K, int32_t g, int3
     auto* Pp = static_cast<uint32_t*>(packed);
     auto* Sp = static_cast<uint16_t*>(scales);
     auto* Zp = static_cast<uint16_t*>(zeros);
+    if (per_channel(g, K)) {
+        const int rgrid = (int)(N < (int64_t)di.sm_count * 8 ? N : (int64_t)di.sm_count * 8);
+        if (sym) quantize_rows_kernel<true><<<rgrid, kQuantRowThreads, 0, s>>>(Wp, N, K, Pp, Sp, Zp);
+        else quantize_rows_kernel<false><<<rgrid, kQuantRowThreads, 0, s>>>(Wp, N, K, Pp, Sp, Zp);
+        return launch_status();
+    }
 #define W4A16_Q_CASE(GG)                                                                      \
     case GG:                                                                                  \
         if (sym) quantize_pack_kernel<GG, true><<<grid, 256, 0, s>>>(Wp, chunks, Pp, Sp, Zp); \
@@ -613,6 +636,13 @@ w4a16_status w4a16_dequantize(const void* packed, const void* scales, const void
     auto* Sp = static_cast<const uint16_t*>(scales);
     auto* Zp = static_cast<const uint16_t*>(zeros);
     auto* Wp = static_cast<uint4*>(W_hat);
+    if (per_channel(g, K)) {
+        const int rgrid = (int)(N < (int64_t)di.sm_count * 8 ? N : (int64_t)di.sm_count * 8);
+        const auto* P32 = static_cast<const uint32_t*>(packed);
+        if (sym) dequantize_rows_kernel<true><<<rgrid, 256, 0, s>>>(P32, Sp, Zp, N, K, Wp);
+        else dequantize_rows_kernel<false><<<rgrid, 256, 0, s>>>(P32, Sp, Zp, N, K, Wp);
+        return launch_status();
+    }
 #define W4A16_D_CASE(GG)                                                                       \
     case GG:                                                                                   \
         if (sym) dequantize_kernel<GG, true><<<grid, 256, 0, s>>>(Pp, Sp, Zp, chunks, Wp);     \
