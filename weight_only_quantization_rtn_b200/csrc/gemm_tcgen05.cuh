@@ -16,8 +16,9 @@
 //               X tile (BM x 64 bf16, 128-byte swizzle) and one of the packed
 //               tile (128 rows x 32 bytes, 32-byte swizzle).  Scales and zero
 //               points arrive by TMA in slabs of 8 groups x 128 rows (one slab
-//               serves g/8 K blocks, a two-slot ring with its own barriers) when
-//               their rows are 16-byte aligned; otherwise all 32 lanes copy the
+//               serves g/8 K blocks, a two-slot ring with its own barriers; the
+//               dequantizers copy a landed slab into registers and release it at
+//               once) when their rows are 16-byte aligned; otherwise all 32 lanes copy the
 //               block's aligned pair of groups per row into the stage with 4-byte
 //               cp.async copies that complete on the stage's "full" barrier.
 //   warp 1      TMEM allocator and, on one elected lane, the MMA issuer: waits
@@ -263,15 +264,33 @@ __global__ void __launch_bounds__(kTcThreads, 1)
             if (!SYM) row_zz = bf16x2_add(dup16(ldg_u16(zeros + n)), 0x43004300u);
         }
         bool ok = true;
+        // Scales by TMA slab: when a slab lands, each thread copies its row's 8 scales and
+        // 8 zeros (two 16-byte reads, conflict-free) into registers, adds 128 to the zeros
+        // once, and releases the slot; each K block then picks its pair with one PRMT.
+        uint32_t sreg0 = 0u, sreg1 = 0u, sreg2 = 0u, sreg3 = 0u;   // this row's 8 slab scales
+        uint32_t zreg0 = 0u, zreg1 = 0u, zreg2 = 0u, zreg3 = 0u;   // and 128 + its 8 zeros
         for (int i = 0; i < nkb; ++i) {
             const int kb = kb0 + i;
             const int s = i % S;
             const uint32_t ph = (uint32_t)(i / S) & 1u;
             const int t = i / kSlabKb, slot = t & 1;
-            if (sz_tma && i % kSlabKb == 0 &&
-                !mbar_wait(smem_u32(&slab_full[slot]), (uint32_t)(t >> 1) & 1u)) {
-                ok = false;
-                break;
+            if (sz_tma && i % kSlabKb == 0) {
+                if (!mbar_wait(smem_u32(&slab_full[slot]), (uint32_t)(t >> 1) & 1u)) {
+                    ok = false;
+                    break;
+                }
+                const uint16_t* srow = slab + slot * 2 * kTcTileN * 8 + r * 8;
+                const uint4 sv = lds128(srow);
+                sreg0 = sv.x; sreg1 = sv.y; sreg2 = sv.z; sreg3 = sv.w;
+                if (!SYM) {
+                    const uint4 zv = lds128(srow + kTcTileN * 8);
+                    zreg0 = bf16x2_add(zv.x, 0x43004300u);
+                    zreg1 = bf16x2_add(zv.y, 0x43004300u);
+                    zreg2 = bf16x2_add(zv.z, 0x43004300u);
+                    zreg3 = bf16x2_add(zv.w, 0x43004300u);
+                }
+                __syncwarp();
+                if (lane == 0) mbar_arrive(smem_u32(&slab_empty[slot]));   // slot no longer read
             }
             if (!mbar_wait(smem_u32(&full[s]), ph)) {
                 ok = false;
@@ -282,7 +301,6 @@ __global__ void __launch_bounds__(kTcThreads, 1)
                 spair = lds_u32(szs + s * 2 * kTcTileN + r);
                 zpair = SYM ? 0u : lds_u32(szs + s * 2 * kTcTileN + kTcTileN + r);
             }
-            const uint16_t* srow = slab + slot * 2 * kTcTileN * 8 + r * 8;
             const uint8_t* prow = ps + s * Cfg::kPBytes + r * 32;
             const uint32_t arow = smem_u32(as + s * Cfg::kABytes + r * 128);
             {
@@ -293,11 +311,12 @@ __global__ void __launch_bounds__(kTcThreads, 1)
                     ss = row_ss;
                     zz = row_zz;
                 } else if (sz_tma) {
-                    const int gi = ((kb * kTcBlockK + 32 * h) / kG) % 8;  // group within the slab
-                    ss = __byte_perm(lds_u16(srow + gi), 0, 0x1010);
-                    zz = SYM ? 0x43084308u
-                             : bf16x2_add(__byte_perm(lds_u16(srow + kTcTileN * 8 + gi), 0, 0x1010),
-                                          0x43004300u);
+                    // group within the slab; its 2 bytes of the 8-byte register pair, twice
+                    const int gi = (int)((uint32_t)(kb * kTcBlockK + 32 * h) / (uint32_t)kG) & 7;
+                    const uint32_t sel = 0x1010u + (uint32_t)(gi & 3) * 0x2222u;
+                    const bool up = (gi & 4) != 0;
+                    ss = __byte_perm(up ? sreg2 : sreg0, up ? sreg3 : sreg1, sel);
+                    zz = SYM ? 0x43084308u : __byte_perm(up ? zreg2 : zreg0, up ? zreg3 : zreg1, sel);
                 } else {
                     const int half = ((kb * kTcBlockK + 32 * h) / kG) & 1;  // position in the pair
                     ss = dup16(spair >> (16 * half));
@@ -318,9 +337,6 @@ __global__ void __launch_bounds__(kTcThreads, 1)
             fence_proxy_async_smem();
             __syncwarp();
             if (lane == 0) mbar_arrive(smem_u32(&afull[s]));
-            if (sz_tma && (i % kSlabKb == kSlabKb - 1 || i == nkb - 1)) {
-                if (lane == 0) mbar_arrive(smem_u32(&slab_empty[slot]));
-            }
         }
         // ------------------------------------------------------------ epilogue
         if (ok && mbar_wait(smem_u32(accf), 0)) {
