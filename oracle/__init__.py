@@ -15,6 +15,10 @@ Parity status of each function (what pins it is in ``tests/test_oracle_pins.py``
       nearest-grid-point brute force, error bounds, invariants)
   gemm_f64 / gemm_sampled — pinned (exact rational brute force, one-hot and
       all-ones special cases)
+  group_asym8 / group_sym8 / quantize8 / dequantize8 / gemm_w8a16 /
+      gemm_w8a16_sampled (W8A16: 8-bit codes, one per byte) — pinned
+      (hand-computed 8-bit groups, brute force over all 256 codes, error
+      bounds, on-grid recovery, invariants, one-hot activations)
 """
 from __future__ import annotations
 
@@ -75,6 +79,15 @@ def _load():
             lib.oracle_gemm_w4a16_sampled.argtypes = [vp, i64, i64, vp, vp, vp, i64, i64, i32,
                                                       vp, vp, i64, vp]
             lib.oracle_gemm_w4a16_sampled.restype = ctypes.c_int
+            lib.oracle_group_asym8.argtypes = [vp, i64, vp, vp, vp]
+            lib.oracle_group_sym8.argtypes = [vp, i64, vp, vp]
+            lib.oracle_quantize8.argtypes = [vp, i64, i64, i64, i32, vp, vp, vp]
+            lib.oracle_quantize8.restype = ctypes.c_int
+            lib.oracle_dequantize8.argtypes = [vp, vp, vp, i64, i64, i64, i32, vp]
+            lib.oracle_dequantize8.restype = ctypes.c_int
+            lib.oracle_gemm_w8a16_sampled.argtypes = [vp, i64, i64, vp, vp, vp, i64, i64, i32,
+                                                      vp, vp, i64, vp]
+            lib.oracle_gemm_w8a16_sampled.restype = ctypes.c_int
             lib.oracle_round_to_bf16.argtypes = [vp, i64, vp]
             lib.oracle_f32_array_to_bf16.argtypes = [vp, i64, vp]
             lib.oracle_num_threads.restype = ctypes.c_int
@@ -223,6 +236,80 @@ def gemm_sampled(X_bits, packed, scales, zeros, g: int, sym: bool, ms, ns) -> np
                                        int(bool(sym)), _ptr(ms), _ptr(ns), ms.size, _ptr(out))
     if rc != 0:
         raise ValueError("oracle_gemm_w4a16_sampled rejected its arguments")
+    return out
+
+
+# ---------------------------------------------------------------- W8A16 (8-bit codes)
+def group_asym8(x) -> tuple[int, int, np.ndarray]:
+    """One asymmetric 8-bit group -> (scale bf16 bits, zero point, codes 0..255)."""
+    lib = _load()
+    x = np.ascontiguousarray(x, dtype=np.float32)
+    s = np.zeros(1, dtype=np.uint16)
+    z = np.zeros(1, dtype=np.int32)
+    q = np.zeros(x.size, dtype=np.int32)
+    lib.oracle_group_asym8(_ptr(x), x.size, _ptr(s), _ptr(z), _ptr(q))
+    return int(s[0]), int(z[0]), q
+
+
+def group_sym8(x) -> tuple[int, np.ndarray]:
+    """One symmetric 8-bit group -> (scale bf16 bits, codes −128..127)."""
+    lib = _load()
+    x = np.ascontiguousarray(x, dtype=np.float32)
+    s = np.zeros(1, dtype=np.uint16)
+    q = np.zeros(x.size, dtype=np.int32)
+    lib.oracle_group_sym8(_ptr(x), x.size, _ptr(s), _ptr(q))
+    return int(s[0]), q
+
+
+def quantize8(W_bits, g: int, sym: bool):
+    """W[N, K] bf16 bits -> (codes u8[N, K], scales bf16[N, K/g], zeros bf16[N, K/g])."""
+    lib = _load()
+    W = _u16(W_bits)
+    N, K = W.shape
+    G = K // g
+    codes = np.zeros((N, K), dtype=np.uint8)
+    scales = np.zeros((N, G), dtype=np.uint16)
+    zeros = np.zeros((N, G), dtype=np.uint16)
+    rc = lib.oracle_quantize8(_ptr(W), N, K, g, int(bool(sym)), _ptr(codes), _ptr(scales),
+                              _ptr(zeros))
+    if rc != 0:
+        raise ValueError(f"oracle_quantize8 rejected N={N} K={K} g={g}")
+    return codes, scales, zeros
+
+
+def dequantize8(codes, scales, zeros, g: int, sym: bool) -> np.ndarray:
+    lib = _load()
+    c = np.ascontiguousarray(codes, dtype=np.uint8)
+    s = _u16(scales)
+    z = _u16(zeros) if zeros is not None else np.zeros_like(s)
+    N, K = c.shape
+    out = np.zeros((N, K), dtype=np.uint16)
+    rc = lib.oracle_dequantize8(_ptr(c), _ptr(s), _ptr(z), N, K, g, int(bool(sym)), _ptr(out))
+    if rc != 0:
+        raise ValueError("oracle_dequantize8 rejected its arguments")
+    return out
+
+
+def gemm_w8a16(X_bits, codes, scales, zeros, g: int, sym: bool) -> np.ndarray:
+    """Full W8A16 reference: dequantize the 8-bit codes, then binary64 matmul."""
+    return gemm_f64(_u16(X_bits), dequantize8(codes, scales, zeros, g, sym))
+
+
+def gemm_w8a16_sampled(X_bits, codes, scales, zeros, g: int, sym: bool, ms, ns) -> np.ndarray:
+    lib = _load()
+    X = _u16(X_bits)
+    M, K = X.shape
+    c = np.ascontiguousarray(codes, dtype=np.uint8)
+    s = _u16(scales)
+    z = _u16(zeros) if zeros is not None else np.zeros_like(s)
+    N = c.shape[0]
+    ms = np.ascontiguousarray(ms, dtype=np.int64)
+    ns = np.ascontiguousarray(ns, dtype=np.int64)
+    out = np.zeros(ms.size, dtype=np.float64)
+    rc = lib.oracle_gemm_w8a16_sampled(_ptr(X), M, K, _ptr(c), _ptr(s), _ptr(z), N, g,
+                                       int(bool(sym)), _ptr(ms), _ptr(ns), ms.size, _ptr(out))
+    if rc != 0:
+        raise ValueError("oracle_gemm_w8a16_sampled rejected its arguments")
     return out
 
 

@@ -1,5 +1,6 @@
 /*
- * Host oracle for W4A16 weight-only round-to-nearest (RTN) quantization.
+ * Host oracle for W4A16 weight-only round-to-nearest (RTN) quantization, and
+ * for its 8-bit form W8A16 (the section near the end of this file).
  *
  * TEST INFRASTRUCTURE ONLY.  Only the test suite, the smoke check and the
  * benchmark's CPU-baseline leg may load this code.  It shares no source,
@@ -290,6 +291,166 @@ int oracle_gemm_w4a16_sampled(const uint16_t* X, int64_t M, int64_t K, const uin
             float s = oracle_bf16_to_f32(scales[n * G + j]);
             int32_t z = sym ? 0 : (int32_t)oracle_bf16_to_f32(zeros[n * G + j]);
             uint16_t w = dequant_one(q, z, s);
+            acc += (double)oracle_bf16_to_f32(X[m * K + k]) * (double)oracle_bf16_to_f32(w);
+        }
+        out[i] = acc;
+    }
+    return 0;
+}
+
+/* ---------------------------------------------------------------------------
+ * W8A16: 8-bit codes, one per byte.  [P4] §3.3 states the INT8 form itself:
+ * asymmetric s = (max − min) / 255, z = round(−min / s); symmetric
+ * s = max|x| / max_int with max_int = 2^(8−1) − 1 = 127 ([P3] §二 absmax,
+ * b = 8).  [P2] 详细版 lists W8A16 beside W4A16 as a common scheme.
+ * Readings, as for INT4 with the 8-bit ranges:
+ *  R1, R2, R4, R5, R9 unchanged;
+ *  R3' codes are clamped to [0, 255] (asym) or [−128, 127] (sym);
+ *  R6' sym codes are stored as int8 two's complement, zeros written as 0;
+ *  R7' code of element k is byte k of its row;
+ *  R8' x̂ = bf16_rn((q − z)·s): |q − z| ≤ 255 has 8 significant bits, s has 8,
+ *      so the product is exact in binary32 and is rounded once.
+ *  Zero points are integers 0..255, exact in bf16 (8 significant bits).
+ * ------------------------------------------------------------------------- */
+
+/* Asymmetric 8-bit group: s = (max − min)/255, z = round(−min/s), q = round(x/s) + z. */
+void oracle_group_asym8(const float* x, int64_t g, uint16_t* s_out, int32_t* z_out,
+                        int32_t* q_out) {
+    float mn = 0.0f, mx = 0.0f;                       /* R4: range contains 0 */
+    for (int64_t i = 0; i < g; ++i) {
+        if (x[i] < mn) mn = x[i];
+        if (x[i] > mx) mx = x[i];
+    }
+    float s32 = (mx - mn) / 255.0f;                   /* 2^8 − 1 levels */
+    uint16_t s_bits = oracle_f32_to_bf16_rn(s32);     /* R2 */
+    float s = oracle_bf16_to_f32(s_bits);
+    int32_t z = 0;
+    if (s != 0.0f) {
+        z = (int32_t)clamp_code(rintf(-mn / s), 0.0f, 255.0f);
+    }
+    for (int64_t i = 0; i < g; ++i) {
+        int32_t q = 0;
+        if (s != 0.0f) {                              /* R5 */
+            float r = clamp_code(rintf(x[i] / s), -512.0f, 512.0f);
+            q = (int32_t)r + z;
+            if (q < 0) q = 0;
+            if (q > 255) q = 255;
+        }
+        q_out[i] = q;
+    }
+    *s_out = s_bits;
+    *z_out = z;
+}
+
+/* Symmetric (absmax) 8-bit group: s = max|x| / 127, z = 0, q = round(x/s). */
+void oracle_group_sym8(const float* x, int64_t g, uint16_t* s_out, int32_t* q_out) {
+    float amax = 0.0f;
+    for (int64_t i = 0; i < g; ++i) {
+        float a = fabsf(x[i]);
+        if (a > amax) amax = a;
+    }
+    float s32 = amax / 127.0f;                        /* 2^(8−1) − 1 */
+    uint16_t s_bits = oracle_f32_to_bf16_rn(s32);
+    float s = oracle_bf16_to_f32(s_bits);
+    for (int64_t i = 0; i < g; ++i) {
+        int32_t q = 0;
+        if (s != 0.0f) {
+            float r = clamp_code(rintf(x[i] / s), -512.0f, 512.0f);
+            q = (int32_t)r;
+            if (q < -128) q = -128;
+            if (q > 127) q = 127;
+        }
+        q_out[i] = q;
+    }
+    *s_out = s_bits;
+}
+
+/* Code byte of element k (R6', R7'). */
+static int32_t code8_of(const uint8_t* codes, int64_t idx, int32_t sym) {
+    int32_t q = codes[idx];
+    if (sym && q >= 128) q -= 256;                    /* int8 two's complement */
+    return q;
+}
+
+/* W[N, K] -> codes[N, K] (one byte each), scales/zeros[N, K/g]. */
+int oracle_quantize8(const uint16_t* W, int64_t N, int64_t K, int64_t g, int32_t sym,
+                     uint8_t* codes, uint16_t* scales, uint16_t* zeros) {
+    if (N < 0 || K < 0 || g <= 0 || K % g != 0) return 1;
+    const int64_t G = K / g;
+    int failed = 0;
+    #pragma omp parallel
+    {
+        float* xg = (float*)malloc((size_t)g * sizeof(float));
+        int32_t* qg = (int32_t*)malloc((size_t)g * sizeof(int32_t));
+        if (!xg || !qg) {
+            #pragma omp atomic write
+            failed = 1;
+        }
+        #pragma omp for schedule(static)
+        for (int64_t n = 0; n < N; ++n) {
+            if (!xg || !qg) continue;
+            for (int64_t j = 0; j < G; ++j) {
+                const uint16_t* src = W + n * K + j * g;
+                for (int64_t i = 0; i < g; ++i) xg[i] = oracle_bf16_to_f32(src[i]);
+                uint16_t s_bits;
+                int32_t z = 0;
+                if (sym) {
+                    oracle_group_sym8(xg, g, &s_bits, qg);
+                } else {
+                    oracle_group_asym8(xg, g, &s_bits, &z, qg);
+                }
+                scales[n * G + j] = s_bits;
+                if (zeros) zeros[n * G + j] = oracle_f32_to_bf16_rn((float)z);
+                for (int64_t i = 0; i < g; ++i)
+                    codes[n * K + j * g + i] = (uint8_t)((uint32_t)qg[i] & 0xFFu);
+            }
+        }
+        free(xg);
+        free(qg);
+    }
+    return failed;
+}
+
+/* x̂[n, k] = bf16_rn((q − z)·s) from 8-bit codes (R8'). */
+int oracle_dequantize8(const uint8_t* codes, const uint16_t* scales, const uint16_t* zeros,
+                       int64_t N, int64_t K, int64_t g, int32_t sym, uint16_t* W_hat) {
+    if (N < 0 || K < 0 || g <= 0 || K % g != 0) return 1;
+    const int64_t G = K / g;
+    #pragma omp parallel for schedule(static)
+    for (int64_t n = 0; n < N; ++n) {
+        for (int64_t k = 0; k < K; ++k) {
+            int32_t q = code8_of(codes, n * K + k, sym);
+            int64_t j = k / g;
+            float s = oracle_bf16_to_f32(scales[n * G + j]);
+            int32_t z = sym ? 0 : (int32_t)oracle_bf16_to_f32(zeros[n * G + j]);
+            float prod = (float)(q - z) * s;          /* exact: ≤ 8-bit integer × 8-bit significand */
+            W_hat[n * K + k] = oracle_f32_to_bf16_rn(prod);
+        }
+    }
+    return 0;
+}
+
+/* Y64 at listed (m, n) positions from 8-bit codes, dequantizing row n on the fly. */
+int oracle_gemm_w8a16_sampled(const uint16_t* X, int64_t M, int64_t K, const uint8_t* codes,
+                              const uint16_t* scales, const uint16_t* zeros, int64_t N,
+                              int64_t g, int32_t sym, const int64_t* ms, const int64_t* ns,
+                              int64_t count, double* out) {
+    if (g <= 0 || K % g != 0) return 1;
+    const int64_t G = K / g;
+    #pragma omp parallel for schedule(dynamic, 16)
+    for (int64_t i = 0; i < count; ++i) {
+        int64_t m = ms[i], n = ns[i];
+        double acc = 0.0;
+        if (m < 0 || m >= M || n < 0 || n >= N) {
+            out[i] = NAN;
+            continue;
+        }
+        for (int64_t k = 0; k < K; ++k) {
+            int32_t q = code8_of(codes, n * K + k, sym);
+            int64_t j = k / g;
+            float s = oracle_bf16_to_f32(scales[n * G + j]);
+            int32_t z = sym ? 0 : (int32_t)oracle_bf16_to_f32(zeros[n * G + j]);
+            uint16_t w = oracle_f32_to_bf16_rn((float)(q - z) * s);
             acc += (double)oracle_bf16_to_f32(X[m * K + k]) * (double)oracle_bf16_to_f32(w);
         }
         out[i] = acc;

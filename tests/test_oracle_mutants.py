@@ -27,6 +27,15 @@ MUTANTS = {
     "dequant_truncates": ("return oracle_f32_to_bf16_rn(prod);",
                           "uint32_t u; memcpy(&u, &prod, 4); return (uint16_t)(u >> 16);"),
     "group_index_wraps": ("int64_t j = k / g;", "int64_t j = k % G;"),
+    # 8-bit (W8A16) functions
+    "w8_256_levels": ("(mx - mn) / 255.0f", "(mx - mn) / 256.0f"),
+    "w8_sym_divides_by_128": ("amax / 127.0f", "amax / 128.0f"),
+    "w8_int8_sign_extension": ("if (sym && q >= 128) q -= 256;", "if (sym && q >= 128) q -= 128;"),
+    "w8_code_bytes_reversed": ("codes[n * K + j * g + i] = (uint8_t)",
+                               "codes[n * K + j * g + (g - 1 - i)] = (uint8_t)"),
+    "w8_zero_point_clamped_to_15": ("rintf(-mn / s), 0.0f, 255.0f", "rintf(-mn / s), 0.0f, 15.0f"),
+    "w8_dequant_truncates": ("W_hat[n * K + k] = oracle_f32_to_bf16_rn(prod);",
+                             "uint32_t u; memcpy(&u, &prod, 4); W_hat[n * K + k] = (uint16_t)(u >> 16);"),
 }
 
 

@@ -423,3 +423,185 @@ def test_quantize_rejects_bad_shapes():
     W = np.zeros((2, 96), np.uint16)
     with pytest.raises(ValueError):
         oracle.quantize(W, 64, False)           # K % g != 0
+
+
+# ------------------------------------------------------------------ W8A16 (8-bit codes)
+GOLDEN_W8 = os.path.join(os.path.dirname(__file__), "golden", "hand_groups_w8.json")
+CASES_W8 = json.load(open(GOLDEN_W8))["cases"]
+
+
+@pytest.mark.parametrize("case", CASES_W8, ids=[c["name"] for c in CASES_W8])
+def test_hand_computed_group_w8(case):
+    """8-bit groups worked by hand (INT8 form of qwbw.cn page §3.3; meko1 page
+    §二 absmax with b = 8): scale bits, zero point and codes."""
+    x = _f32(case["x"])
+    if case["mode"] == "sym":
+        s_bits, q = oracle.group_sym8(x)
+        z = 0
+    else:
+        s_bits, z, q = oracle.group_asym8(x)
+    assert s_bits == int(case["s_bits"], 16)
+    assert float(oracle.f32_from_bf16(np.array([s_bits], np.uint16))[0]) == float(case["s"])
+    assert z == case["z"]
+    assert list(q) == case["q"]
+
+
+@pytest.mark.parametrize("case", CASES_W8, ids=[c["name"] for c in CASES_W8])
+def test_hand_computed_group_w8_through_matrix_path(case):
+    """The same groups through quantize8/dequantize8 on a [3, 2g] matrix (two
+    groups per row, in both orders): code bytes, scale and zero slots, x̂."""
+    x = _f32(case["x"])
+    g = x.size
+    sym = case["mode"] == "sym"
+    other = np.linspace(-3.0, 1.0, g).astype(np.float32)
+    rows = [np.concatenate([x, other]), np.concatenate([other, x]), np.concatenate([x, x])]
+    W = oracle.bf16_from_f32(np.stack(rows))
+    C, S, Z = oracle.quantize8(W, g, sym)
+    assert C.shape == (3, 2 * g) and S.shape == (3, 2)
+    exp_codes = [int(b, 16) for b in case["codes"]]
+    for r, slot in ((0, 0), (1, 1), (2, 0), (2, 1)):
+        assert list(C[r, slot * g:(slot + 1) * g]) == exp_codes
+        assert S[r, slot] == int(case["s_bits"], 16)
+        assert float(oracle.f32_from_bf16(Z[r, slot:slot + 1])[0]) == (0.0 if sym else case["z"])
+    xh = oracle.f32_from_bf16(oracle.dequantize8(C, S, Z, g, sym))
+    exp = [float(v) for v in case["x_hat"]]
+    assert list(xh[0, :g]) == exp and list(xh[1, g:]) == exp and list(xh[2, g:]) == exp
+
+
+@pytest.mark.parametrize("g", [4, 32, 128])
+def test_asym8_codes_are_nearest_grid_points(g):
+    """Brute force over all 256 codes: the chosen code minimises |x − (c − z)s|,
+    up to the rounding of the binary32 quotient next to a tie."""
+    for x in _groups(50 + g, g, 240):
+        s_bits, z, q = oracle.group_asym8(x)
+        s = float(oracle.f32_from_bf16(np.array([s_bits], np.uint16))[0])
+        assert 0 <= z <= 255 and np.all((q >= 0) & (q <= 255))
+        if s == 0.0:
+            assert np.all(q == 0) and z == 0
+            continue
+        xs = x.astype(np.float64)
+        grid = (np.arange(256)[None, :] - z) * s
+        dist = np.abs(xs[:, None] - grid)
+        chosen = dist[np.arange(g), q]
+        slack = np.abs(xs) * 2.0**-22 + s * 2.0**-20
+        assert np.all(chosen <= dist.min(1) + slack)
+
+
+@pytest.mark.parametrize("g", [4, 32, 128])
+def test_sym8_codes_are_nearest_grid_points(g):
+    for x in _groups(60 + g, g, 240):
+        s_bits, q = oracle.group_sym8(x)
+        s = float(oracle.f32_from_bf16(np.array([s_bits], np.uint16))[0])
+        assert np.all((q >= -127) & (q <= 127)), "absmax/127 never reaches -128"
+        if s == 0.0:
+            assert np.all(q == 0)
+            continue
+        xs = x.astype(np.float64)
+        grid = np.arange(-128, 128)[None, :] * s
+        dist = np.abs(xs[:, None] - grid)
+        chosen = dist[np.arange(g), q + 128]
+        slack = np.abs(xs) * 2.0**-22 + s * 2.0**-20
+        assert np.all(chosen <= dist.min(1) + slack)
+
+
+@pytest.mark.parametrize("g", [32, 128])
+def test_error_bound_half_step_w8(g):
+    """|x − (q − z)s| ≤ s/2 for unclamped codes; clamped codes exceed it only by
+    the bf16 rounding of s: ≤ s/2 + 255·2^-8·s.  The group minimum maps to code
+    0 and the maximum to 254 or 255."""
+    for x in _groups(70 + g, g, 240):
+        s_bits, z, q = oracle.group_asym8(x)
+        s = float(oracle.f32_from_bf16(np.array([s_bits], np.uint16))[0])
+        if s == 0.0:
+            continue
+        err = np.abs(x.astype(np.float64) - (q - z) * s)
+        inner = (q > 0) & (q < 255)
+        assert np.all(err[inner] <= s / 2 * (1 + 2.0**-20))
+        assert np.all(err <= s / 2 + 255 * 2.0**-8 * s)
+        lo, hi = np.argmin(x), np.argmax(x)
+        if x[lo] < 0:
+            assert q[lo] == 0
+        if x[hi] > 0:
+            assert q[hi] >= 254
+
+
+def test_w8_sym_zeros_and_int8_storage():
+    W = workloads.bits(workloads.make_weight(37, 256, 0.02, seed=15, outlier_frac=0.05,
+                                             outlier_scale=20.0))
+    C, S, Z = oracle.quantize8(W, 64, sym=True)
+    assert np.all(Z == 0)
+    q = C.view(np.int8).astype(np.int64)               # int8 two's complement
+    s = np.repeat(oracle.f32_from_bf16(S).astype(np.float64), 64, axis=1)
+    x = oracle.f32_from_bf16(W).astype(np.float64)
+    assert np.all(np.abs(x - q * s) <= s / 2 * (1 + 2.0**-20))
+    assert q.min() >= -127
+
+
+@pytest.mark.parametrize("sym", [False, True])
+@pytest.mark.parametrize("e", [-9, 6])
+def test_w8_power_of_two_scale_invariance(sym, e):
+    W = workloads.make_weight(16, 256, 0.02, seed=8, outlier_frac=0.02, outlier_scale=20.0)
+    W2 = (W.to(torch.float32) * 2.0**e).to(torch.bfloat16)     # exact scaling
+    C1, S1, Z1 = oracle.quantize8(workloads.bits(W), 32, sym)
+    C2, S2, Z2 = oracle.quantize8(workloads.bits(W2), 32, sym)
+    assert np.array_equal(C1, C2) and np.array_equal(Z1, Z2)
+    assert np.array_equal(oracle.f32_from_bf16(S1) * np.float32(2.0**e), oracle.f32_from_bf16(S2))
+
+
+@pytest.mark.parametrize("g", [32, 128, 512])       # 512 = K: per-channel
+def test_w8_on_grid_matrix_is_recovered_exactly(g):
+    """Closed form: W = (q − z)·s with s a power of two (|q − z| ≤ 255 already
+    takes bf16's 8 significant bits) and each group using codes 0 and 255
+    re-quantizes to exactly (s, z, q) and dequantizes to W."""
+    rng = np.random.default_rng(100 + g)
+    N, K = 6, 512
+    G = K // g
+    q = rng.integers(0, 256, size=(N, K))
+    q[:, 1::g] = 0
+    q[:, 2::g] = 255
+    z = rng.integers(0, 256, size=(N, G))
+    s = 2.0 ** rng.integers(-18, -6, size=(N, G)).astype(np.float64)
+    x = (q - np.repeat(z, g, 1)) * np.repeat(s, g, 1)
+    Wb = oracle.bf16_from_f32(x.astype(np.float32))
+    assert np.array_equal(oracle.f32_from_bf16(Wb).astype(np.float64), x)
+    C, S, Z = oracle.quantize8(Wb, g, sym=False)
+    assert np.array_equal(oracle.f32_from_bf16(S).astype(np.float64), s)
+    assert np.array_equal(oracle.f32_from_bf16(Z).astype(np.int64), z)
+    assert np.array_equal(C.astype(np.int64), q)
+    assert np.array_equal(oracle.dequantize8(C, S, Z, g, False), Wb)
+
+
+@pytest.mark.parametrize("sym", [False, True])
+def test_dequantize8_closed_form_indexing(sym):
+    """Hand-built codes/scales/zeros whose products (q − z)·s are exact in bf16:
+    dequantize8 must place each value at its (row, k)."""
+    rng = np.random.default_rng(31 + sym)
+    N, K, g = 5, 192, 64
+    G = K // g
+    q = rng.integers(-128, 128, size=(N, K)) if sym else rng.integers(0, 256, size=(N, K))
+    z = np.zeros((N, G), np.int64) if sym else rng.integers(0, 256, size=(N, G))
+    s = 2.0 ** rng.integers(-12, 0, size=(N, G)).astype(np.float64)      # powers of two
+    codes = (q & 0xFF).astype(np.uint8)
+    S = oracle.bf16_from_f32(s.astype(np.float32))
+    Z = oracle.bf16_from_f32(z.astype(np.float32))
+    Wh = oracle.f32_from_bf16(oracle.dequantize8(codes, S, Z, g, sym)).astype(np.float64)
+    exp = (q - np.repeat(z, g, 1)) * np.repeat(s, g, 1)     # |q − z| ≤ 255 times a power of two
+    exp_b = oracle.f32_from_bf16(oracle.bf16_from_f32(exp.astype(np.float32))).astype(np.float64)
+    assert np.array_equal(exp, exp_b), "construction: (q − z)·s exact in bf16"
+    assert np.array_equal(Wh, exp)
+
+
+def test_w8_gemm_one_hot_and_sampled():
+    W = workloads.bits(workloads.make_weight(24, 256, 0.02, seed=19))
+    for sym in (False, True):
+        C, S, Z = oracle.quantize8(W, 128, sym)
+        Wh = oracle.dequantize8(C, S, Z, 128, sym)
+        ks = np.array([0, 1, 127, 128, 200, 255])
+        X = np.zeros((ks.size, 256), np.float32)
+        X[np.arange(ks.size), ks] = 1.0
+        Y = oracle.gemm_w8a16(oracle.bf16_from_f32(X), C, S, Z, 128, sym)
+        assert np.array_equal(oracle.bf16_from_f64(Y), Wh[:, ks].T)
+        Xr = workloads.bits(workloads.make_activation(3, 256, 20))
+        Yf = oracle.gemm_w8a16(Xr, C, S, Z, 128, sym)
+        ms, ns = np.array([0, 2, 1, 2]), np.array([0, 23, 7, 11])
+        assert np.array_equal(oracle.gemm_w8a16_sampled(Xr, C, S, Z, 128, sym, ms, ns), Yf[ms, ns])
