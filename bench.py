@@ -1,7 +1,8 @@
 """Benchmark of the W4A16 fused GEMM on B200.
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
-                    [--workload decode7b|decode70b|prefill] [--no-extras]
+                    [--workload decode7b|decode70b|prefill|decode7b_pc|prefill_pc]
+                    [--no-extras] [--no-cpu-baseline] [--crossover]
 
 Metric: W4A16 GEMM HBM GB/s at M=1 and TFLOPS at M=2048, as % of the B200
 roofline.  The headline line (default workload) is the M=1 decode of the two
@@ -14,6 +15,9 @@ divided by the max over ranks.  The same JSON line carries the M=2048 prefill
 TFLOPS (K=N=8192) with its tensor-core roofline, a dense bf16 cuBLAS GEMM and
 the unfused dequantize-then-GEMM at the same shapes, the end-to-end number
 through the public API with host buffers, and the host oracle on the CPU.
+Extras on the same line: standalone quantize/dequantize bandwidth, the
+per-channel (g = K) decode and prefill, and the W8A16 (8-bit code) quantize,
+dequantize and M=1 GEMV.
 
 Timing: W warm-up steps, then exactly K steps replayed from CUDA graphs (one
 graph holds a full rotation over the weight copies, so graph launches are
@@ -570,6 +574,7 @@ def run_ours(args):
             pr["frac_of_nominal"] = pr["achieved"] / NOMINAL_BF16_TFLOPS
             line["quantize_dequantize"] = elementwise_extras(w4, peaks, l2, dev)
             line["per_channel"] = per_channel_extras(w4, peaks, peak_src, l2, dev)
+            line["w8a16"] = w8a16_extras(w4, peaks, l2, dev)
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         cb = cpu_baseline(wl.layers, M, g, sym, unit_bytes=(half == "hbm")) \
             if half == "hbm" else cpu_baseline_sampled(wl.layers[0], M, g, sym, rows=16)
@@ -673,6 +678,59 @@ def per_channel_extras(w4, peaks, peak_src, l2, dev, iters=200):
         del rot, singles, cases
         torch.cuda.empty_cache()
     return out
+
+
+def w8a16_extras(w4, peaks, l2, dev, iters=200):
+    """W8A16 (8-bit codes, one per byte) at g=128 asym: quantize/pack and
+    dequantize of a 7B-shaped weight (N=11008, K=4096), and the fused M=1 GEMV
+    over both 7B-shaped layers, with inputs rotated past L2 and graph-replayed.
+    Bytes: quantize reads W and writes codes + scales + zeros; dequantize the
+    reverse; the GEMV reads codes + scales + zeros + X and writes Y."""
+    g, sym = 128, False
+    layers = workloads.DECODE_7B.layers
+    L0 = layers[0]
+    N, K = L0.N, L0.K
+    pk = peaks["hbm_gbs"]
+    W = L0.weight().to(dev)
+    meta = 4 * N * (K // g)
+    copies = max(2, -(-2 * l2 // (N * K * 2)) + 1)
+    Ws = [W] + [W.clone() for _ in range(copies - 1)]
+    outs = [w4.quantize8(w, g, sym) for w in Ws]
+    gs = graph_of(lambda i: w4.quantize8(Ws[i % copies], g, sym), copies)
+    qms = time_graphs(gs, 20)
+    del gs
+    Wh = torch.empty(N, K, dtype=torch.bfloat16, device=dev)
+    gs = graph_of(lambda i: w4.dequantize8(*outs[i % copies], g, sym, out=Wh), copies)
+    dms = time_graphs(gs, 20)
+    del gs, Ws, outs, Wh, W
+    qb = db = N * K * 2 + N * K + meta
+    # fused GEMV, M=1, both layers per step
+    per_step = sum(l.N * l.K + 4 * l.N * (l.K // g) + 2 * l.K for l in layers)
+    gcopies = copies_for(per_step, l2)
+    sets = []
+    for l in layers:
+        C, S, Z = w4.quantize8(l.weight().to(dev), g, sym)
+        X = l.activation(1).to(dev)
+        Y = torch.empty(1, l.N, dtype=torch.bfloat16, device=dev)
+        sets.append([(C, S, Z, X, Y)] + [(C.clone(), S.clone(), Z.clone(), X.clone(), Y)
+                                         for _ in range(gcopies - 1)])
+
+    def step(i):
+        for cs in sets:
+            C, S, Z, X, Y = cs[i % gcopies]
+            w4.gemm8(X, C, S, Z, g, sym, out=Y)
+
+    gs = graph_of(step, gcopies)
+    gms = time_graphs(gs, iters)
+    del gs, sets
+    torch.cuda.empty_cache()
+    gbytes = sum(algorithmic_bytes(1, l.N, l.K, g, sym) + l.N * l.K // 2 for l in layers)
+    gbs = gbytes / (gms / 1e3) / 1e9
+    return {"shape": f"N={N},K={K},g={g},asym; GEMV: both 7B-shaped layers, M=1",
+            "quantize": {"us": qms * 1e3, "GB/s": qb / (qms / 1e3) / 1e9, "frac": qb / (qms / 1e3) / 1e9 / pk},
+            "dequantize": {"us": dms * 1e3, "GB/s": db / (dms / 1e3) / 1e9, "frac": db / (dms / 1e3) / 1e9 / pk},
+            "gemv_M1": {"us_per_step": gms * 1e3, "bytes_per_step": gbytes, "GB/s": gbs,
+                        "frac": gbs / pk, "kernel": "w8_gemv_kernel"}}
 
 
 def comparisons(w4, cases, copies, l2, half):

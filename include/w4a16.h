@@ -200,6 +200,38 @@ w4a16_status w4a16_gemm_decode_noalloc(const void* X, int64_t M, int64_t K, cons
                                        const void* scales, const void* zeros, int64_t N,
                                        int32_t g, int32_t sym, void* Y, void* stream);
 
+/* ---------------------------------------------------------------------------
+ * W8A16: the same method with 8-bit codes (the INT8 form the qwbw.cn page
+ * states in §3.3: asymmetric s = (max − min)/255, z = round(−min/s); symmetric
+ * s = max|x|/127, meko1 page §二 absmax with b = 8; W8A16 is listed beside
+ * W4A16 on the aigcbaba page, 详细版).  Readings as above with the 8-bit
+ * ranges: codes clamped to [0, 255] (asym) or [−128, 127] (sym, stored as
+ * int8 two's complement); zeros are integers 0..255 stored in bf16.
+ * Layouts: codes uint8 [N, K] (element k of a row in byte k); scales and
+ * zeros bf16 [N, K/g] as for INT4.  Same g and K rules, alignment, stream and
+ * error conventions as the INT4 entry points.
+ * ------------------------------------------------------------------------- */
+
+/* Quantize W[N, K] (bf16) to 8-bit codes: codes uint8 [N, K], scales and zeros
+ * bf16 [N, K/g] (zeros may be NULL when sym == 1, else written as 0).
+ * Bit-exact with the host oracle. */
+w4a16_status w8a16_quantize(const void* W, int64_t N, int64_t K, int32_t g, int32_t sym,
+                            void* codes, void* scales, void* zeros, void* stream);
+
+/* Ŵ[n, k] = bf16_rn((q − z)·s) from 8-bit codes (W_hat bf16 [N, K]). */
+w4a16_status w8a16_dequantize(const void* codes, const void* scales, const void* zeros,
+                              int64_t N, int64_t K, int32_t g, int32_t sym, void* W_hat,
+                              void* stream);
+
+/* Fused W8A16 GEMM for the decode regime, M ≤ 16: Y[M, N] = X[M, K] · Ŵ[N, K]ᵀ
+ * with Ŵ formed in registers, binary32 accumulation, one rounding of each
+ * output to bf16; deterministic.  One warp per weight row streams the row's
+ * codes with 16-byte loads; no workspace.  Returns W4A16_EINVAL for M > 16 (no
+ * large-M W8A16 kernel is built). */
+w4a16_status w8a16_gemm(const void* X, int64_t M, int64_t K, const void* codes,
+                        const void* scales, const void* zeros, int64_t N, int32_t g,
+                        int32_t sym, void* Y, void* stream);
+
 /* Read and clear the current device's error word, written by a kernel that gave
  * up a bounded wait (a pipeline barrier that did not complete within about one
  * second).  *code = 0 when no kernel reported one.  Synchronizes the device. */

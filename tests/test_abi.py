@@ -26,21 +26,22 @@ def lib():
 def declared_functions():
     text = open(HEADER).read()
     text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
-    return sorted(set(re.findall(r"\b(w4a16_[a-z0-9_]+)\s*\(", text)))
+    return sorted(set(re.findall(r"\b(w[48]a16_[a-z0-9_]+)\s*\(", text)))
 
 
 def test_header_declares_the_abi():
     names = declared_functions()
     for n in ("w4a16_quantize", "w4a16_dequantize", "w4a16_gemm", "w4a16_gemm_ex",
               "w4a16_gemm_workspace_size", "w4a16_gemm_plan", "w4a16_status_string",
-              "w4a16_device_error", "w4a16_abi_version"):
+              "w4a16_device_error", "w4a16_abi_version", "w8a16_quantize", "w8a16_dequantize",
+              "w8a16_gemm"):
         assert n in names
 
 
 def test_library_exports_every_declared_symbol(lib):
     out = subprocess.run(["nm", "-D", "--defined-only", w4.LIB_PATH], capture_output=True,
                          text=True, check=True).stdout
-    exported = set(re.findall(r"\sT\s(w4a16_\w+)", out))
+    exported = set(re.findall(r"\sT\s(w[48]a16_\w+)", out))
     for name in declared_functions():
         assert name in exported, f"{name} declared in w4a16.h but not exported"
         assert hasattr(lib, name)
@@ -291,3 +292,26 @@ def test_stream_k_unit_walk(kbn):
                     idx = [i for i, (r, _, _) in enumerate(w) if r == rb]
                     assert idx == list(range(idx[0], idx[-1] + 1))
                     assert [i for i in idx if w[i][2]] == [idx[-1]]
+
+
+# ------------------------------------------------------------------ W8A16 entry points
+def test_w8a16_entry_points_reject_invalid(lib):
+    q, d, gm = lib.w8a16_quantize, lib.w8a16_dequantize, lib.w8a16_gemm
+    assert q(FAKE, 4, 128, 48, 0, FAKE, FAKE, FAKE, None) == EINVAL          # g not supported
+    assert q(FAKE, 4, 200, 200, 0, FAKE, FAKE, FAKE, None) == EINVAL         # per-channel K % 32
+    assert q(FAKE, 4, 128, 128, 0, FAKE, FAKE, None, None) == EINVAL         # asym needs zeros
+    assert q(FAKE + 8, 4, 128, 128, 1, FAKE, FAKE, None, None) == EINVAL     # misaligned W
+    assert q(FAKE, 4, 128, 128, 2, FAKE, FAKE, FAKE, None) == EINVAL         # bad mode
+    assert q(FAKE, 0, 128, 128, 0, FAKE, FAKE, FAKE, None) == 0              # N = 0: nothing to do
+    assert q(FAKE, 0, 4096, 4096, 0, FAKE, FAKE, FAKE, None) == 0            # per-channel accepted
+    assert d(FAKE, FAKE, None, 4, 128, 128, 0, FAKE, None) == EINVAL
+    assert d(FAKE, FAKE, FAKE, 4, 128, 32, 0, FAKE + 2, None) == EINVAL
+    assert d(FAKE, FAKE, FAKE, 0, 96, 96, 0, FAKE, None) == 0
+    X = S = Z = Y = FAKE
+    assert gm(X, 17, 128, FAKE, S, Z, 64, 128, 0, Y, None) == EINVAL         # M > 16: not built
+    assert gm(X, -1, 128, FAKE, S, Z, 64, 128, 0, Y, None) == EINVAL
+    assert gm(X, 1, 96, FAKE, S, Z, 64, 128, 0, Y, None) == EINVAL           # K % g
+    assert gm(X + 8, 1, 128, FAKE, S, Z, 64, 128, 0, Y, None) == EINVAL
+    assert gm(X, 1, 128, FAKE, S, None, 64, 128, 0, Y, None) == EINVAL
+    assert gm(X, 0, 128, FAKE, S, Z, 64, 128, 0, Y, None) == 0              # empty: no launch
+    assert gm(X, 4, 128, FAKE, S, Z, 0, 128, 0, Y, None) == 0

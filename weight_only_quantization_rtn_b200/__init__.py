@@ -18,6 +18,7 @@ import os
 import torch
 
 __all__ = ["lib", "quantize", "dequantize", "gemm", "gemm_decode_noalloc", "plan",
+           "quantize8", "dequantize8", "gemm8",
            "workspace_size", "device_error", "W4A16Error", "PATH_AUTO", "PATH_DECODE", "PATH_TENSORCORE", "LIB_PATH"]
 
 LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libw4a16.so")
@@ -63,8 +64,12 @@ def _load() -> ctypes.CDLL:
     lib.w4a16_status_string.argtypes = [ctypes.c_int]
     lib.w4a16_status_string.restype = ctypes.c_char_p
     lib.w4a16_abi_version.restype = ctypes.c_int32
+    lib.w8a16_quantize.argtypes = [vp, i64, i64, i32, i32, vp, vp, vp, vp]
+    lib.w8a16_dequantize.argtypes = [vp, vp, vp, i64, i64, i32, i32, vp, vp]
+    lib.w8a16_gemm.argtypes = [vp, i64, i64, vp, vp, vp, i64, i32, i32, vp, vp]
     for name in ("w4a16_quantize", "w4a16_dequantize", "w4a16_gemm", "w4a16_gemm_ex",
-                 "w4a16_gemm_plan", "w4a16_device_error"):
+                 "w4a16_gemm_plan", "w4a16_device_error", "w8a16_quantize", "w8a16_dequantize",
+                 "w8a16_gemm"):
         getattr(lib, name).restype = ctypes.c_int
     if lib.w4a16_abi_version() != ABI_VERSION:
         raise ImportError(f"{LIB_PATH} has ABI version {lib.w4a16_abi_version()}, this binding "
@@ -168,6 +173,19 @@ def plan(M: int, N: int, K: int, g: int = 128, sym: bool = False, path: str | in
 
 
 _workspaces: dict = {}
+_plan_bytes: dict = {}
+
+
+def _workspace_bytes(dev: torch.device, M, N, K, g, sym, pid, ctas) -> int:
+    """Workspace of the plan for this shape on this device, asked of the library
+    once per distinct call shape (plans depend only on the shape, the forced
+    kernel and grid, and the device's SM count)."""
+    key = (dev.index, M, N, K, g, bool(sym), pid, ctas)
+    nbytes = _plan_bytes.get(key)
+    if nbytes is None:
+        nbytes = plan(M, N, K, g, sym, pid, ctas)["workspace_bytes"] if M and N else 0
+        _plan_bytes[key] = nbytes
+    return nbytes
 
 
 def _workspace(dev: torch.device, nbytes: int):
@@ -189,7 +207,8 @@ def gemm(X: torch.Tensor, packed: torch.Tensor, scales: torch.Tensor,
     """Fused W4A16 GEMM: Y[M, N] = X[M, K] · Ŵ[N, K]ᵀ (bf16 in/out, fp32 accumulation).
 
     If X lives in host memory (ideally pinned) it is copied to the weights'
-    device and Y is copied back to the host: the end-to-end form of the call."""
+    device and Y is copied back into pinned host memory, waiting for the copy:
+    the end-to-end form of the call."""
     host_in = not X.is_cuda
     dev = packed.device
     Xd = X.to(dev, non_blocking=True) if host_in else X
@@ -210,14 +229,17 @@ def gemm(X: torch.Tensor, packed: torch.Tensor, scales: torch.Tensor,
             raise ValueError("out has the wrong shape")
     pid = _PATHS[path] if isinstance(path, str) else int(path)
     with torch.cuda.device(dev):
-        ws_bytes = plan(M, N, K, g, sym, pid, ctas)["workspace_bytes"] if M and N else 0
+        ws_bytes = _workspace_bytes(dev, M, N, K, g, sym, pid, ctas)
         ws = _workspace(dev, ws_bytes)
         _check(lib().w4a16_gemm_ex(_ptr(Xd), M, K, _ptr(packed), _ptr(scales),
                                    _ptr(zeros if not sym else None), N, g, int(bool(sym)),
                                    _ptr(out), _ptr(ws), ws_bytes, pid, ctas, _stream(dev)),
                "w4a16_gemm")
     if host_in:
-        return out.to("cpu")
+        host = torch.empty((M, N), dtype=torch.bfloat16, pin_memory=True)
+        host.copy_(out, non_blocking=True)
+        torch.cuda.current_stream(dev).synchronize()
+        return host
     return out
 
 
@@ -243,6 +265,70 @@ def gemm_decode_noalloc(X: torch.Tensor, packed: torch.Tensor, scales: torch.Ten
                                                _ptr(zeros if not sym else None), N, g,
                                                int(bool(sym)), _ptr(out), _stream(dev)),
                "w4a16_gemm_decode_noalloc")
+    return out
+
+
+# ---------------------------------------------------------------- W8A16 (8-bit codes)
+def quantize8(W: torch.Tensor, g: int = 128, sym: bool = False):
+    """RTN quantization of W[N, K] (bf16, cuda) to 8-bit codes, one per byte;
+    g = K quantizes per channel.
+
+    Returns (codes uint8 [N, K], scales bf16 [N, K/g], zeros bf16 [N, K/g]);
+    symmetric codes are int8 two's complement and zeros are all 0."""
+    _need(W, torch.bfloat16, "W")
+    N, K = W.shape
+    if g <= 0 or K % g:
+        raise ValueError(f"K={K} must be a multiple of g={g}")
+    codes = torch.empty((N, K), dtype=torch.uint8, device=W.device)
+    scales = torch.empty((N, K // g), dtype=torch.bfloat16, device=W.device)
+    zeros = torch.empty((N, K // g), dtype=torch.bfloat16, device=W.device)
+    with torch.cuda.device(W.device):
+        _check(lib().w8a16_quantize(_ptr(W), N, K, g, int(bool(sym)), _ptr(codes), _ptr(scales),
+                                   _ptr(zeros), _stream(W.device)), "w8a16_quantize")
+    return codes, scales, zeros
+
+
+def dequantize8(codes: torch.Tensor, scales: torch.Tensor, zeros: torch.Tensor | None,
+                g: int = 128, sym: bool = False, out: torch.Tensor | None = None) -> torch.Tensor:
+    """Ŵ[N, K] = bf16_rn((q − z)·s) from 8-bit codes, materialised."""
+    _need(codes, torch.uint8, "codes")
+    _need(scales, torch.bfloat16, "scales")
+    if not sym:
+        _need(zeros, torch.bfloat16, "zeros")
+    N, K = codes.shape
+    if out is None:
+        out = torch.empty((N, K), dtype=torch.bfloat16, device=codes.device)
+    else:
+        _need(out, torch.bfloat16, "out")
+        if tuple(out.shape) != (N, K):
+            raise ValueError("out has the wrong shape")
+    with torch.cuda.device(codes.device):
+        _check(lib().w8a16_dequantize(_ptr(codes), _ptr(scales), _ptr(zeros if not sym else None),
+                                     N, K, g, int(bool(sym)), _ptr(out), _stream(codes.device)),
+               "w8a16_dequantize")
+    return out
+
+
+def gemm8(X: torch.Tensor, codes: torch.Tensor, scales: torch.Tensor,
+          zeros: torch.Tensor | None, g: int = 128, sym: bool = False,
+          out: torch.Tensor | None = None) -> torch.Tensor:
+    """Fused W8A16 GEMM for M ≤ 16: Y[M, N] = X[M, K] · Ŵ[N, K]ᵀ (bf16 in/out,
+    fp32 accumulation), device tensors."""
+    _need(X, torch.bfloat16, "X")
+    _need(codes, torch.uint8, "codes")
+    _need(scales, torch.bfloat16, "scales")
+    if not sym:
+        _need(zeros, torch.bfloat16, "zeros")
+    M, K = X.shape
+    N = codes.shape[0]
+    if codes.shape[1] != K:
+        raise ValueError(f"codes have K={codes.shape[1]}, X has K={K}")
+    if out is None:
+        out = torch.empty((M, N), dtype=torch.bfloat16, device=codes.device)
+    with torch.cuda.device(codes.device):
+        _check(lib().w8a16_gemm(_ptr(X), M, K, _ptr(codes), _ptr(scales),
+                                _ptr(zeros if not sym else None), N, g, int(bool(sym)), _ptr(out),
+                                _stream(codes.device)), "w8a16_gemm")
     return out
 
 

@@ -2,7 +2,8 @@
 
     python -m weight_only_quantization_rtn_b200.build [--verbose]
 
-nvcc compiles the single translation unit csrc/w4a16.cu for sm_100a only
+nvcc compiles the translation units csrc/w4a16.cu (INT4) and csrc/w8a16.cu
+(8-bit codes) into one library for sm_100a only
 (-gencode arch=compute_100a,code=sm_100a), without fast-math (the quantizer's
 division and rounding must be IEEE), with -lineinfo for profiling.  The CUDA
 runtime is linked statically, so the library needs only the driver at run time.
@@ -19,7 +20,7 @@ import sys
 HERE = os.path.dirname(os.path.abspath(__file__))
 ROOT = os.path.dirname(HERE)
 LIB = os.path.join(HERE, "libw4a16.so")
-SRC = os.path.join(HERE, "csrc", "w4a16.cu")
+SRCS = [os.path.join(HERE, "csrc", "w4a16.cu"), os.path.join(HERE, "csrc", "w8a16.cu")]
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
 FLAGS = ["-O3", "-std=c++17", "-lineinfo", "-Xcompiler", "-fPIC", "-shared",
          "--expt-relaxed-constexpr", "-cudart", "static", "-I", os.path.join(ROOT, "include")]
@@ -48,7 +49,7 @@ def build(force: bool = False, verbose: bool = False) -> str:
     if not force and up_to_date():
         return LIB
     tmp = LIB + f".tmp{os.getpid()}"
-    cmd = [nvcc(), *ARCH, *FLAGS, "-o", tmp, SRC]
+    cmd = [nvcc(), *ARCH, *FLAGS, "-o", tmp, *SRCS]
     if verbose:
         cmd.insert(1, "-Xptxas=-v")
     subprocess.check_call(cmd)
