@@ -682,8 +682,9 @@ def per_channel_extras(w4, peaks, peak_src, l2, dev, iters=200):
 
 def w8a16_extras(w4, peaks, l2, dev, iters=200):
     """W8A16 (8-bit codes, one per byte) at g=128 asym: quantize/pack and
-    dequantize of a 7B-shaped weight (N=11008, K=4096), and the fused M=1 GEMV
-    over both 7B-shaped layers, with inputs rotated past L2 and graph-replayed.
+    dequantize of a 7B-shaped weight (N=11008, K=4096), the fused M=1 GEMV over
+    both 7B-shaped layers, and the tensor-core kernel at M=2048, K=N=8192, with
+    inputs rotated past L2 and graph-replayed.
     Bytes: quantize reads W and writes codes + scales + zeros; dequantize the
     reverse; the GEMV reads codes + scales + zeros + X and writes Y."""
     g, sym = 128, False
@@ -726,11 +727,32 @@ def w8a16_extras(w4, peaks, l2, dev, iters=200):
     torch.cuda.empty_cache()
     gbytes = sum(algorithmic_bytes(1, l.N, l.K, g, sym) + l.N * l.K // 2 for l in layers)
     gbs = gbytes / (gms / 1e3) / 1e9
+    # tensor-core kernel with 8-bit codes: prefill M=2048, K=N=8192
+    P = workloads.PREFILL.layers[0]
+    M = 2048
+    pin = P.N * P.K + 4 * P.N * (P.K // g) + 2 * M * P.K
+    pcopies = copies_for(pin, l2)
+    C, S, Z = w4.quantize8(P.weight().to(dev), g, sym)
+    X = P.activation(M).to(dev)
+    Y = torch.empty(M, P.N, dtype=torch.bfloat16, device=dev)
+    psets = [(C, S, Z, X)] + [(C.clone(), S.clone(), Z.clone(), X.clone()) for _ in range(pcopies - 1)]
+    def prefill_step(i):
+        Cc, Sc, Zc, Xc = psets[i % pcopies]
+        w4.gemm8(Xc, Cc, Sc, Zc, g, sym, out=Y)
+
+    gs = graph_of(prefill_step, pcopies)
+    pms = time_graphs(gs, 30)
+    del gs, psets, C, S, Z, X, Y
+    torch.cuda.empty_cache()
+    ptf = 2 * M * P.N * P.K / (pms / 1e3) / 1e12
     return {"shape": f"N={N},K={K},g={g},asym; GEMV: both 7B-shaped layers, M=1",
             "quantize": {"us": qms * 1e3, "GB/s": qb / (qms / 1e3) / 1e9, "frac": qb / (qms / 1e3) / 1e9 / pk},
             "dequantize": {"us": dms * 1e3, "GB/s": db / (dms / 1e3) / 1e9, "frac": db / (dms / 1e3) / 1e9 / pk},
             "gemv_M1": {"us_per_step": gms * 1e3, "bytes_per_step": gbytes, "GB/s": gbs,
-                        "frac": gbs / pk, "kernel": "w8_gemv_kernel"}}
+                        "frac": gbs / pk, "kernel": "w8_gemv_kernel"},
+            "prefill_2048x8192x8192": {"us": pms * 1e3, "TFLOP/s": ptf,
+                                       "frac": ptf / peaks["bf16_tflops"],
+                                       "kernel": "gemm_tc_kernel (8-bit codes)"}}
 
 
 def comparisons(w4, cases, copies, l2, half):

@@ -223,14 +223,23 @@ w4a16_status w8a16_dequantize(const void* codes, const void* scales, const void*
                               int64_t N, int64_t K, int32_t g, int32_t sym, void* W_hat,
                               void* stream);
 
-/* Fused W8A16 GEMM for the decode regime, M ≤ 16: Y[M, N] = X[M, K] · Ŵ[N, K]ᵀ
- * with Ŵ formed in registers, binary32 accumulation, one rounding of each
- * output to bf16; deterministic.  One warp per weight row streams the row's
- * codes with 16-byte loads; no workspace.  Returns W4A16_EINVAL for M > 16 (no
- * large-M W8A16 kernel is built). */
+/* Bytes of device workspace w8a16_gemm needs: 0 for M ≤ 16; for larger M the
+ * tensor-core kernel's split-K partial tiles, as w4a16_gemm_workspace_size
+ * describes.  Uses the current device's SM count; 0 for rejected shapes. */
+size_t w8a16_gemm_workspace_size(int64_t M, int64_t N, int64_t K, int32_t g);
+
+/* Fused W8A16 GEMM: Y[M, N] = X[M, K] · Ŵ[N, K]ᵀ with Ŵ = bf16_rn((q − z)·s)
+ * formed on chip, binary32 accumulation, one rounding of each output to bf16;
+ * deterministic.  M ≤ 16: one warp per weight row streams the row's codes with
+ * 16-byte loads (no workspace).  M > 16: the tensor-core kernel with 8-bit
+ * codes (64-byte code rows per K block, binary32-exact dequantization into the
+ * shared-memory A tile, tcgen05 MMA), split-K as for INT4.  workspace: at least
+ * w8a16_gemm_workspace_size() bytes, 16-byte aligned, when that is nonzero;
+ * W4A16_EWORKSPACE if it is smaller. */
 w4a16_status w8a16_gemm(const void* X, int64_t M, int64_t K, const void* codes,
                         const void* scales, const void* zeros, int64_t N, int32_t g,
-                        int32_t sym, void* Y, void* stream);
+                        int32_t sym, void* Y, void* workspace, size_t workspace_bytes,
+                        void* stream);
 
 /* Read and clear the current device's error word, written by a kernel that gave
  * up a bounded wait (a pipeline barrier that did not complete within about one

@@ -308,10 +308,14 @@ def test_w8a16_entry_points_reject_invalid(lib):
     assert d(FAKE, FAKE, FAKE, 4, 128, 32, 0, FAKE + 2, None) == EINVAL
     assert d(FAKE, FAKE, FAKE, 0, 96, 96, 0, FAKE, None) == 0
     X = S = Z = Y = FAKE
-    assert gm(X, 17, 128, FAKE, S, Z, 64, 128, 0, Y, None) == EINVAL         # M > 16: not built
-    assert gm(X, -1, 128, FAKE, S, Z, 64, 128, 0, Y, None) == EINVAL
-    assert gm(X, 1, 96, FAKE, S, Z, 64, 128, 0, Y, None) == EINVAL           # K % g
-    assert gm(X + 8, 1, 128, FAKE, S, Z, 64, 128, 0, Y, None) == EINVAL
-    assert gm(X, 1, 128, FAKE, S, None, 64, 128, 0, Y, None) == EINVAL
-    assert gm(X, 0, 128, FAKE, S, Z, 64, 128, 0, Y, None) == 0              # empty: no launch
-    assert gm(X, 4, 128, FAKE, S, Z, 0, 128, 0, Y, None) == 0
+    big = 1 << 30
+    assert gm(X, -1, 128, FAKE, S, Z, 64, 128, 0, Y, FAKE, big, None) == EINVAL
+    assert gm(X, 1, 96, FAKE, S, Z, 64, 128, 0, Y, FAKE, big, None) == EINVAL      # K % g
+    assert gm(X + 8, 1, 128, FAKE, S, Z, 64, 128, 0, Y, FAKE, big, None) == EINVAL
+    assert gm(X, 1, 128, FAKE, S, None, 64, 128, 0, Y, FAKE, big, None) == EINVAL
+    assert gm(X, 0, 128, FAKE, S, Z, 64, 128, 0, Y, FAKE, big, None) == 0         # empty: no launch
+    assert gm(X, 4, 128, FAKE, S, Z, 0, 128, 0, Y, FAKE, big, None) == 0
+    ws = lib.w8a16_gemm_workspace_size
+    assert ws(16, 4096, 4096, 128) == 0                     # the GEMV needs none
+    assert ws(17, 8192, 8192, 32) == w4.workspace_size(17, 8192, 8192, 32) > 0
+    assert ws(2048, 8192, 8192, 128) == w4.workspace_size(2048, 8192, 8192, 128)

@@ -1,9 +1,9 @@
 """GPU parity of the W8A16 path (8-bit codes, one per byte) against the oracle.
 
 Codes, scales, zeros and the dequantized weights are integer or once-rounded
-results and must match the oracle's bytes exactly; the fused GEMM (M ≤ 16)
-must meet the same bars as the INT4 GEMM (tests/helpers.py), and is bit-exact
-on one-hot activations."""
+results and must match the oracle's bytes exactly; the fused GEMM (the GEMV for
+M ≤ 16, the tensor-core kernel above) must meet the same bars as the INT4 GEMM
+(tests/helpers.py), and is bit-exact on one-hot activations."""
 import numpy as np
 import pytest
 import torch
@@ -128,7 +128,46 @@ def test_w8_gemm_deterministic_and_7b_full_size():
     assert_y_close(workloads.bits(ys[0])[ms, ns], ref, "W8 7B-shaped layer M=4")
 
 
-def test_w8_rejects_large_m():
-    C, S, Z = w4.quantize8(workloads.make_weight(64, 128, 0.02, seed=1).cuda(), 128, False)
-    with pytest.raises(w4.W4A16Error):
-        w4.gemm8(workloads.make_activation(17, 128, 2).cuda(), C, S, Z, 128, False)
+@pytest.mark.parametrize("sym", [False, True])
+@pytest.mark.parametrize("g", [32, 64, 128, 0])
+@pytest.mark.parametrize("M,N,K", [(17, 128, 96), (33, 384, 512), (48, 1000, 4352),
+                                   (129, 64, 4096), (300, 700, 1056), (600, 1000, 1024)])
+def test_w8_gemm_tensorcore(M, N, K, g, sym):
+    """M > 16: the tensor-core kernel with 8-bit codes (64-byte code rows per K
+    block, 64-byte swizzle), unsplit and split-K tiles, ragged N, M and K."""
+    gg = K if g == 0 else g
+    if K % gg:
+        pytest.skip("K not a multiple of g")
+    _check_gemm(M, N, K, gg, sym, seed=3 * M + N + K)
+
+
+@pytest.mark.parametrize("sym", [False, True])
+@pytest.mark.parametrize("g", [32, 128, 512])
+def test_w8_tensorcore_one_hot_bit_exact(g, sym):
+    """32 one-hot activation rows (M > 16, so the tensor-core kernel): each output
+    is one dequantized weight, exactly."""
+    N, K = 160, 512
+    W = workloads.make_weight(N, K, 0.02, seed=23)
+    C, S, Z = w4.quantize8(W.cuda(), g, sym)
+    Wh = w4.dequantize8(C, S, Z, g, sym)
+    for start in range(0, K, 32):
+        kk = torch.arange(start, start + 32)
+        X = torch.zeros(32, K, dtype=torch.bfloat16)
+        X[torch.arange(32), kk] = 1.0
+        Y = w4.gemm8(X.cuda(), C, S, Z, g, sym)
+        assert torch.equal(Y, Wh[:, kk.cuda()].t().contiguous()), f"k in {start}..{start + 31}"
+
+
+def test_w8_prefill_full_size():
+    layer = workloads.PREFILL.layers[0]                   # M=2048, K=N=8192
+    W, X = layer.weight(), layer.activation(2048)
+    C, S, Z = w4.quantize8(W.cuda(), 128, False)
+    ys = [w4.gemm8(X.cuda(), C, S, Z, 128, False) for _ in range(2)]
+    assert torch.equal(ys[0], ys[1])
+    rng = np.random.default_rng(11)
+    ms = rng.integers(0, 2048, 2048)
+    ns = rng.integers(0, layer.N, 2048)
+    ms[:4], ns[:4] = [0, 2047, 0, 2047], [0, 0, layer.N - 1, layer.N - 1]
+    ref = oracle.gemm_w8a16_sampled(workloads.bits(X), C.cpu().numpy(), workloads.bits(S),
+                                    workloads.bits(Z), 128, False, ms, ns)
+    assert_y_close(workloads.bits(ys[0])[ms, ns], ref, "W8 prefill M=2048")

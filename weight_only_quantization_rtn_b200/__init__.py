@@ -66,7 +66,9 @@ def _load() -> ctypes.CDLL:
     lib.w4a16_abi_version.restype = ctypes.c_int32
     lib.w8a16_quantize.argtypes = [vp, i64, i64, i32, i32, vp, vp, vp, vp]
     lib.w8a16_dequantize.argtypes = [vp, vp, vp, i64, i64, i32, i32, vp, vp]
-    lib.w8a16_gemm.argtypes = [vp, i64, i64, vp, vp, vp, i64, i32, i32, vp, vp]
+    lib.w8a16_gemm.argtypes = [vp, i64, i64, vp, vp, vp, i64, i32, i32, vp, vp, sz, vp]
+    lib.w8a16_gemm_workspace_size.argtypes = [i64, i64, i64, i32]
+    lib.w8a16_gemm_workspace_size.restype = sz
     for name in ("w4a16_quantize", "w4a16_dequantize", "w4a16_gemm", "w4a16_gemm_ex",
                  "w4a16_gemm_plan", "w4a16_device_error", "w8a16_quantize", "w8a16_dequantize",
                  "w8a16_gemm"):
@@ -312,8 +314,10 @@ def dequantize8(codes: torch.Tensor, scales: torch.Tensor, zeros: torch.Tensor |
 def gemm8(X: torch.Tensor, codes: torch.Tensor, scales: torch.Tensor,
           zeros: torch.Tensor | None, g: int = 128, sym: bool = False,
           out: torch.Tensor | None = None) -> torch.Tensor:
-    """Fused W8A16 GEMM for M ≤ 16: Y[M, N] = X[M, K] · Ŵ[N, K]ᵀ (bf16 in/out,
-    fp32 accumulation), device tensors."""
+    """Fused W8A16 GEMM: Y[M, N] = X[M, K] · Ŵ[N, K]ᵀ (bf16 in/out, fp32
+    accumulation), device tensors.  M ≤ 16 runs the warp-per-row GEMV, larger M
+    the tensor-core kernel with 8-bit codes (with a split-K workspace when the
+    library asks for one)."""
     _need(X, torch.bfloat16, "X")
     _need(codes, torch.uint8, "codes")
     _need(scales, torch.bfloat16, "scales")
@@ -325,10 +329,17 @@ def gemm8(X: torch.Tensor, codes: torch.Tensor, scales: torch.Tensor,
         raise ValueError(f"codes have K={codes.shape[1]}, X has K={K}")
     if out is None:
         out = torch.empty((M, N), dtype=torch.bfloat16, device=codes.device)
-    with torch.cuda.device(codes.device):
+    dev = codes.device
+    with torch.cuda.device(dev):
+        key = ("w8", dev.index, M, N, K, g)
+        ws_bytes = _plan_bytes.get(key)
+        if ws_bytes is None:
+            ws_bytes = int(lib().w8a16_gemm_workspace_size(M, N, K, g)) if M and N else 0
+            _plan_bytes[key] = ws_bytes
+        ws = _workspace(dev, ws_bytes)
         _check(lib().w8a16_gemm(_ptr(X), M, K, _ptr(codes), _ptr(scales),
                                 _ptr(zeros if not sym else None), N, g, int(bool(sym)), _ptr(out),
-                                _stream(codes.device)), "w8a16_gemm")
+                                _ptr(ws), ws_bytes, _stream(dev)), "w8a16_gemm")
     return out
 
 

@@ -59,11 +59,13 @@ constexpr int kTcThreads = (2 + kTcDequantWarps) * 32;
 constexpr int kTcBlockK = 64;                 // K per pipeline stage (one 128-byte swizzle row)
 constexpr int kTcTileN = 128;                 // UMMA M: weight rows per CTA
 
-template <int BM>
+// BITS: code width, 4 (two codes per byte) or 8 (W8A16, one code per byte).
+template <int BM, int BITS = 4>
 struct TcConfig {
+    static constexpr int kRowBytes = kTcBlockK * BITS / 8;      // code bytes of a row per K block
     static constexpr int kXBytes = BM * kTcBlockK * 2;          // X tile
     static constexpr int kABytes = kTcTileN * kTcBlockK * 2;    // dequantized weight tile
-    static constexpr int kPBytes = kTcTileN * kTcBlockK / 2;    // packed codes tile
+    static constexpr int kPBytes = kTcTileN * kRowBytes;        // codes tile
     static constexpr int kSZBytes = 2 * kTcTileN * 4;              // scale and zero pairs per row
     static constexpr int kStageBytes = kXBytes + kABytes + kPBytes + kSZBytes;
     static constexpr int kSlabBytes = 2 * 2 * kTcTileN * 8 * 2;  // two slots of scale + zero slabs
@@ -76,7 +78,23 @@ struct TcConfig {
     static constexpr int kTmemCols = BM < 32 ? 32 : BM;
 };
 
-template <int BM, bool SYM, int G>
+// 8-bit codes (one word = 4 codes) -> two bf16x2 of bf16_rn((q − z)·s) in natural
+// order.  2^23 + q is formed exactly by placing the byte in a binary32 mantissa;
+// subtracting zoff = 2^23 + z (exact: < 2^24) leaves q − z, the product with the
+// bf16 scale s is exact in binary32, and the conversion rounds once.
+__device__ __forceinline__ void dequant4_bytes(uint32_t w, float s, float zoff, uint32_t out[2]) {
+    float f[4];
+#pragma unroll
+    for (int i = 0; i < 4; ++i)
+        f[i] = (__uint_as_float(__byte_perm(w, 0x4B000000u, 0x7540u + (uint32_t)i)) - zoff) * s;
+    uint32_t lo, hi;
+    asm("cvt.rn.bf16x2.f32 %0, %1, %2;" : "=r"(lo) : "f"(f[1]), "f"(f[0]));
+    asm("cvt.rn.bf16x2.f32 %0, %1, %2;" : "=r"(hi) : "f"(f[3]), "f"(f[2]));
+    out[0] = lo;
+    out[1] = hi;
+}
+
+template <int BM, bool SYM, int G, int BITS = 4>
 __global__ void __launch_bounds__(kTcThreads, 1)
     gemm_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ CUtensorMap tmP,
                    const uint16_t* __restrict__ scales, const uint16_t* __restrict__ zeros,
@@ -84,7 +102,8 @@ __global__ void __launch_bounds__(kTcThreads, 1)
                    const __grid_constant__ CUtensorMap tmS, const __grid_constant__ CUtensorMap tmZ,
                    int sz_tma, int kb_split, float* __restrict__ partials, int tile_base,
                    int tiles_n) {
-    using Cfg = TcConfig<BM>;
+    static_assert(BITS == 4 || BITS == 8, "4- or 8-bit codes");
+    using Cfg = TcConfig<BM, BITS>;
     constexpr int S = Cfg::kStages;
     static_assert(S >= 2, "pipeline needs at least two stages");
     static_assert(BM % 16 == 0 && BM >= 16 && BM <= 256, "UMMA N must be 16..256, step 16");
@@ -181,7 +200,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
             if (lane == 0) {
                 mbar_arrive_expect_tx(bar, Cfg::kXBytes + Cfg::kPBytes);
                 tma_load_2d(smem_u32(xs + s * Cfg::kXBytes), &tmX, kb * kTcBlockK, m0, bar);
-                tma_load_2d(smem_u32(ps + s * Cfg::kPBytes), &tmP, kb * (kTcBlockK / 2), n0, bar);
+                tma_load_2d(smem_u32(ps + s * Cfg::kPBytes), &tmP, kb * Cfg::kRowBytes, n0, bar);
             }
             // the aligned pair of groups holding this block's group(s), per row and array
             const int jpair = ((kb * kTcBlockK) / kG) & ~1;
@@ -258,17 +277,21 @@ __global__ void __launch_bounds__(kTcThreads, 1)
         const int h = (warp - 2) >> 2;          // K half of each 64-wide block
         const int n = n0 + r;
         const bool row_ok = n < N;
+        // Zero pairs: 128 + z (the INT4 bf16 magic) for 4-bit codes, z itself for 8-bit.
+        auto zero_of = [](uint32_t raw_dup) {
+            return BITS == 4 ? bf16x2_add(raw_dup, 0x43004300u) : raw_dup;
+        };
         uint32_t row_ss = 0u, row_zz = 0x43084308u;   // per-channel pair of this row
         if (G == 0 && row_ok) {
             row_ss = dup16(ldg_u16(scales + n));
-            if (!SYM) row_zz = bf16x2_add(dup16(ldg_u16(zeros + n)), 0x43004300u);
+            if (!SYM) row_zz = zero_of(dup16(ldg_u16(zeros + n)));
         }
         bool ok = true;
         // Scales by TMA slab: when a slab lands, each thread copies its row's 8 scales and
         // 8 zeros (two 16-byte reads, conflict-free) into registers, adds 128 to the zeros
         // once, and releases the slot; each K block then picks its pair with one PRMT.
         uint32_t sreg0 = 0u, sreg1 = 0u, sreg2 = 0u, sreg3 = 0u;   // this row's 8 slab scales
-        uint32_t zreg0 = 0u, zreg1 = 0u, zreg2 = 0u, zreg3 = 0u;   // and 128 + its 8 zeros
+        uint32_t zreg0 = 0u, zreg1 = 0u, zreg2 = 0u, zreg3 = 0u;   // and its 8 zero pairs
         for (int i = 0; i < nkb; ++i) {
             const int kb = kb0 + i;
             const int s = i % S;
@@ -284,10 +307,10 @@ __global__ void __launch_bounds__(kTcThreads, 1)
                 sreg0 = sv.x; sreg1 = sv.y; sreg2 = sv.z; sreg3 = sv.w;
                 if (!SYM) {
                     const uint4 zv = lds128(srow + kTcTileN * 8);
-                    zreg0 = bf16x2_add(zv.x, 0x43004300u);
-                    zreg1 = bf16x2_add(zv.y, 0x43004300u);
-                    zreg2 = bf16x2_add(zv.z, 0x43004300u);
-                    zreg3 = bf16x2_add(zv.w, 0x43004300u);
+                    zreg0 = zero_of(zv.x);
+                    zreg1 = zero_of(zv.y);
+                    zreg2 = zero_of(zv.z);
+                    zreg3 = zero_of(zv.w);
                 }
                 __syncwarp();
                 if (lane == 0) mbar_arrive(smem_u32(&slab_empty[slot]));   // slot no longer read
@@ -301,11 +324,19 @@ __global__ void __launch_bounds__(kTcThreads, 1)
                 spair = lds_u32(szs + s * 2 * kTcTileN + r);
                 zpair = SYM ? 0u : lds_u32(szs + s * 2 * kTcTileN + kTcTileN + r);
             }
-            const uint8_t* prow = ps + s * Cfg::kPBytes + r * 32;
+            const uint8_t* prow = ps + s * Cfg::kPBytes + r * Cfg::kRowBytes;
             const uint32_t arow = smem_u32(as + s * Cfg::kABytes + r * 128);
             {
-                // 32-byte swizzle: chunk h of row r sits at position h ^ bit 2 of r
-                const uint4 v = lds128(prow + 16 * (h ^ ((r >> 2) & 1)));
+                uint4 v, v8 = make_uint4(0, 0, 0, 0);
+                if constexpr (BITS == 4) {
+                    // 32-byte swizzle: chunk h of row r sits at position h ^ bit 2 of r
+                    v = lds128(prow + 16 * (h ^ ((r >> 2) & 1)));
+                } else {
+                    // 64-byte swizzle: 16-byte chunk c of row r sits at c ^ bits 2..1 of r;
+                    // this thread's 32 codes are chunks 2h and 2h + 1
+                    v = lds128(prow + 16 * ((2 * h) ^ ((r >> 1) & 3)));
+                    v8 = lds128(prow + 16 * ((2 * h + 1) ^ ((r >> 1) & 3)));
+                }
                 uint32_t ss, zz;
                 if (G == 0) {
                     ss = row_ss;
@@ -320,13 +351,23 @@ __global__ void __launch_bounds__(kTcThreads, 1)
                 } else {
                     const int half = ((kb * kTcBlockK + 32 * h) / kG) & 1;  // position in the pair
                     ss = dup16(spair >> (16 * half));
-                    zz = SYM ? 0x43084308u : bf16x2_add(dup16(zpair >> (16 * half)), 0x43004300u);
+                    zz = SYM ? 0x43084308u : zero_of(dup16(zpair >> (16 * half)));
                 }
-                const uint32_t wv[4] = {v.x, v.y, v.z, v.w};
+                const uint32_t wv[8] = {v.x, v.y, v.z, v.w, v8.x, v8.y, v8.z, v8.w};
+                // 8-bit: binary32 scale, and 2^23 + z (symmetric codes are flipped to
+                // offset-128 form by XOR with 0x80 and take z = 128)
+                const float s8 = __uint_as_float(ss << 16);
+                const float zoff = SYM ? 8388736.0f : 8388608.0f + __uint_as_float(zz << 16);
 #pragma unroll
                 for (int i = 0; i < 4; ++i) {
                     uint32_t d[4];
-                    dequant8_natural<SYM>(wv[i], zz, ss, d);
+                    if constexpr (BITS == 4) {
+                        dequant8_natural<SYM>(wv[i], zz, ss, d);
+                    } else {
+                        const uint32_t flip = SYM ? 0x80808080u : 0u;
+                        dequant4_bytes(wv[2 * i] ^ flip, s8, zoff, d);
+                        dequant4_bytes(wv[2 * i + 1] ^ flip, s8, zoff, d + 2);
+                    }
                     const int chunk = 4 * h + i;                 // 16-byte chunk: k = 8·chunk
                     const int phys = chunk ^ (r & 7);            // 128-byte swizzle
                     asm volatile("st.shared.v4.u32 [%0], {%1, %2, %3, %4};" ::"r"(arow + phys * 16),

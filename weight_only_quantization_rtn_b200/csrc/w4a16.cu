@@ -14,6 +14,13 @@
 
 using namespace w4a16;
 
+namespace w8 {
+// The 8-bit-code GEMV for M ≤ 16 (csrc/w8a16.cu).
+w4a16_status w8_gemv_launch(const void* X, int64_t M, int64_t K, const void* codes,
+                            const void* scales, const void* zeros, int64_t N, int32_t g,
+                            int32_t sym, void* Y, int sm_count, cudaStream_t stream);
+}
+
 namespace {
 
 constexpr int kMaxDevices = 64;
@@ -218,12 +225,13 @@ TcSchedule tc_schedule(int64_t M, int64_t N, int64_t K, int g, int bm, int sm_co
     return t;
 }
 
-int tc_smem_bytes(int bm) {
+template <int BITS>
+void tc_smem_and_stages(int bm, int* smem, int* stages) {
     switch (bm) {
-        case 32: return TcConfig<32>::kSmemBytes;
-        case 64: return TcConfig<64>::kSmemBytes;
-        case 128: return TcConfig<128>::kSmemBytes;
-        default: return TcConfig<256>::kSmemBytes;
+        case 32: *smem = TcConfig<32, BITS>::kSmemBytes; *stages = TcConfig<32, BITS>::kStages; break;
+        case 64: *smem = TcConfig<64, BITS>::kSmemBytes; *stages = TcConfig<64, BITS>::kStages; break;
+        case 128: *smem = TcConfig<128, BITS>::kSmemBytes; *stages = TcConfig<128, BITS>::kStages; break;
+        default: *smem = TcConfig<256, BITS>::kSmemBytes; *stages = TcConfig<256, BITS>::kStages; break;
     }
 }
 
@@ -239,8 +247,10 @@ w4a16_status check_shape(int64_t M, int64_t N, int64_t K, int32_t g, int32_t sym
 // larger M is tensor-core bound and goes to the tcgen05 kernel.
 int choose_path(int64_t M) { return M <= 16 ? W4A16_PATH_DECODE : W4A16_PATH_TENSORCORE; }
 
+// bits: code width, 4 or 8 (8-bit codes run only on the tensor-core kernel here;
+// their small-M GEMV has its own launcher).
 w4a16_status make_plan(int64_t M, int64_t N, int64_t K, int32_t g, int32_t sym, int32_t path,
-                       int32_t ctas, int sm_count, w4a16_plan* p) {
+                       int32_t ctas, int sm_count, w4a16_plan* p, int bits = 4) {
     w4a16_status st = check_shape(M, N, K, g, sym);
     if (st != W4A16_OK) return st;
     if (path < W4A16_PATH_AUTO || path > W4A16_PATH_TENSORCORE) return W4A16_EINVAL;
@@ -270,14 +280,8 @@ w4a16_status make_plan(int64_t M, int64_t N, int64_t K, int32_t g, int32_t sym, 
         p->tile_n = kTcTileN;
         p->grid = ts.head + ts.tail * ts.splits;
         p->threads = kTcThreads;
-        p->smem_bytes = tc_smem_bytes(bm);
-        p->stages = TcConfig<256>::kStages;
-        switch (bm) {
-            case 32: p->stages = TcConfig<32>::kStages; break;
-            case 64: p->stages = TcConfig<64>::kStages; break;
-            case 128: p->stages = TcConfig<128>::kStages; break;
-            default: break;
-        }
+        if (bits == 8) tc_smem_and_stages<8>(bm, &p->smem_bytes, &p->stages);
+        else tc_smem_and_stages<4>(bm, &p->smem_bytes, &p->stages);
         p->kernels = (ts.head > 0 ? 1 : 0) + (ts.tail > 0 ? 2 : 0);
         p->workspace_bytes = ts.tail > 0 ? (int64_t)ts.splits * ts.tail * bm * kTcTileN * 4 : 0;
     }
@@ -412,19 +416,20 @@ w4a16_status launch_decode(const w4a16_plan& p, const void* X, int64_t M, int64_
 #undef W4A16_DEC_G
 }
 
-template <int BM, bool SYM, int G>
+template <int BM, bool SYM, int G, int BITS>
 w4a16_status launch_tc_t(const w4a16_plan& p, const CUtensorMap& tmX, const CUtensorMap& tmP,
                          const CUtensorMap& tmS, const CUtensorMap& tmZ, int sz_tma,
                          const void* scales, const void* zeros, void* Y, int M, int N, int K,
                          int g, void* workspace, cudaStream_t stream) {
-    auto kern = gemm_tc_kernel<BM, SYM, G>;
+    auto kern = gemm_tc_kernel<BM, SYM, G, BITS>;
+    using Cfg = TcConfig<BM, BITS>;
     const int sz_async = (G != 0 && (K / g) % 2 == 0) ? 1 : 0;   // 4-byte aligned scale rows
     static bool attr_set[kMaxDevices] = {};
     int dev = 0;
     cudaGetDevice(&dev);
     if (!attr_set[dev]) {
         if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                 TcConfig<BM>::kSmemBytes) != cudaSuccess)
+                                 Cfg::kSmemBytes) != cudaSuccess)
             return W4A16_ECUDA;
         attr_set[dev] = true;
     }
@@ -435,7 +440,7 @@ w4a16_status launch_tc_t(const w4a16_plan& p, const CUtensorMap& tmX, const CUte
     auto* y = static_cast<uint16_t*>(Y);
     const int num_kb = (K + kTcBlockK - 1) / kTcBlockK;
     if (ts.head > 0) {
-        kern<<<dim3((unsigned)ts.head, 1, 1), kTcThreads, TcConfig<BM>::kSmemBytes, stream>>>(
+        kern<<<dim3((unsigned)ts.head, 1, 1), kTcThreads, Cfg::kSmemBytes, stream>>>(
             tmX, tmP, sc, ze, y, M, N, K, sz_async, tmS, tmZ, sz_tma, num_kb, nullptr, 0, ts.tiles_n);
         w4a16_status st = launch_status();
         if (st != W4A16_OK) return st;
@@ -450,7 +455,7 @@ w4a16_status launch_tc_t(const w4a16_plan& p, const CUtensorMap& tmX, const CUte
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3((unsigned)ts.tail, 1, (unsigned)ts.splits);
     cfg.blockDim = dim3(kTcThreads, 1, 1);
-    cfg.dynamicSmemBytes = TcConfig<BM>::kSmemBytes;
+    cfg.dynamicSmemBytes = Cfg::kSmemBytes;
     cfg.stream = stream;
     cfg.attrs = attr;
     cfg.numAttrs = ts.head > 0 ? 1 : 0;
@@ -473,13 +478,13 @@ w4a16_status launch_tc_t(const w4a16_plan& p, const CUtensorMap& tmX, const CUte
     return W4A16_OK;
 }
 
-template <bool SYM, int G>
+template <bool SYM, int G, int BITS>
 w4a16_status launch_tc_g(const w4a16_plan& p, const CUtensorMap& tmX, const CUtensorMap& tmP,
                          const CUtensorMap& tmS, const CUtensorMap& tmZ, int sz_tma,
                          const void* scales, const void* zeros, void* Y, int M, int N, int K,
                          int g, void* workspace, cudaStream_t stream) {
 #define W4A16_TC_TILE(BMV) \
-    launch_tc_t<BMV, SYM, G>(p, tmX, tmP, tmS, tmZ, sz_tma, scales, zeros, Y, M, N, K, g, \
+    launch_tc_t<BMV, SYM, G, BITS>(p, tmX, tmP, tmS, tmZ, sz_tma, scales, zeros, Y, M, N, K, g, \
                              workspace, stream)
     switch (p.tile_m) {
         case 32: return W4A16_TC_TILE(32);
@@ -492,14 +497,19 @@ w4a16_status launch_tc_g(const w4a16_plan& p, const CUtensorMap& tmX, const CUte
 
 w4a16_status launch_tc(const w4a16_plan& p, const void* X, int64_t M, int64_t K,
                        const void* packed, const void* scales, const void* zeros, int64_t N,
-                       int32_t g, int32_t sym, void* Y, void* workspace, cudaStream_t stream) {
+                       int32_t g, int32_t sym, void* Y, void* workspace, cudaStream_t stream,
+                       int bits = 4) {
     CUtensorMap tmX, tmP;
     w4a16_status st = encode_2d(&tmX, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, X, (uint64_t)K,
                                 (uint64_t)M, (uint64_t)K * 2, kTcBlockK, (uint32_t)p.tile_m,
                                 CU_TENSOR_MAP_SWIZZLE_128B);
     if (st != W4A16_OK) return st;
-    st = encode_2d(&tmP, CU_TENSOR_MAP_DATA_TYPE_UINT8, packed, (uint64_t)(K / 2), (uint64_t)N,
-                   (uint64_t)(K / 2), kTcBlockK / 2, kTcTileN, CU_TENSOR_MAP_SWIZZLE_32B);
+    // codes [N][K·bits/8]: boxes of 128 rows x one K block (32 bytes with the 32-byte
+    // swizzle for 4-bit codes, 64 bytes with the 64-byte swizzle for 8-bit codes)
+    const uint64_t row_bytes = (uint64_t)K * (uint64_t)bits / 8;
+    st = encode_2d(&tmP, CU_TENSOR_MAP_DATA_TYPE_UINT8, packed, row_bytes, (uint64_t)N, row_bytes,
+                   (uint32_t)(kTcBlockK * bits / 8), kTcTileN,
+                   bits == 8 ? CU_TENSOR_MAP_SWIZZLE_64B : CU_TENSOR_MAP_SWIZZLE_32B);
     if (st != W4A16_OK) return st;
     // Scales and zeros [N][K/g] in slabs of 8 groups x 128 rows, when their rows are
     // 16-byte aligned; otherwise the kernel copies them with cp.async.
@@ -519,10 +529,15 @@ w4a16_status launch_tc(const w4a16_plan& p, const void* X, int64_t M, int64_t K,
     const int m = (int)M, n = (int)N, k = (int)K;
 #define W4A16_TC_CASE(GG)                                                                      \
     case GG:                                                                                   \
-        return sym ? launch_tc_g<true, GG>(p, tmX, tmP, tmS, tmZ, sz_tma, scales, zeros, Y, m, n, \
-                                           k, g, workspace, stream)                            \
-                   : launch_tc_g<false, GG>(p, tmX, tmP, tmS, tmZ, sz_tma, scales, zeros, Y, m, n, \
-                                            k, g, workspace, stream);
+        if (bits == 8)                                                                         \
+            return sym ? launch_tc_g<true, GG, 8>(p, tmX, tmP, tmS, tmZ, sz_tma, scales, zeros, Y, \
+                                                  m, n, k, g, workspace, stream)               \
+                       : launch_tc_g<false, GG, 8>(p, tmX, tmP, tmS, tmZ, sz_tma, scales, zeros, \
+                                                   Y, m, n, k, g, workspace, stream);         \
+        return sym ? launch_tc_g<true, GG, 4>(p, tmX, tmP, tmS, tmZ, sz_tma, scales, zeros, Y, m, n, \
+                                              k, g, workspace, stream)                         \
+                   : launch_tc_g<false, GG, 4>(p, tmX, tmP, tmS, tmZ, sz_tma, scales, zeros, Y, m, \
+                                               n, k, g, workspace, stream);
     switch (pc ? 0 : g) {
         W4A16_TC_CASE(32)
         W4A16_TC_CASE(64)
@@ -718,6 +733,37 @@ w4a16_status w4a16_gemm_decode_noalloc(const void* X, int64_t M, int64_t K, cons
     if ((st = noalloc_scratch(&scratch)) != W4A16_OK) return st;
     return launch_decode(p, X, M, K, packed, scales, zeros, N, g, sym, Y, scratch,
                          static_cast<cudaStream_t>(stream));
+}
+
+size_t w8a16_gemm_workspace_size(int64_t M, int64_t N, int64_t K, int32_t g) {
+    w4a16_plan p;
+    if (M <= 16) return 0;                                  // the GEMV needs no workspace
+    if (make_plan(M, N, K, g, 0, W4A16_PATH_TENSORCORE, 0, current_sm_count(), &p, 8) != W4A16_OK)
+        return 0;
+    return (size_t)p.workspace_bytes;
+}
+
+w4a16_status w8a16_gemm(const void* X, int64_t M, int64_t K, const void* codes, const void* scales,
+                        const void* zeros, int64_t N, int32_t g, int32_t sym, void* Y,
+                        void* workspace, size_t workspace_bytes, void* stream) {
+    w4a16_status st = check_shape(M, N, K, g, sym);
+    if (st != W4A16_OK) return st;
+    if (M == 0 || N == 0) return W4A16_OK;
+    if (!X || !codes || !scales || !Y || (!sym && !zeros)) return W4A16_EINVAL;
+    if (!aligned16(X) || !aligned16(codes) || !aligned16(scales) || !aligned16(Y) ||
+        (!sym && !aligned16(zeros)))
+        return W4A16_EINVAL;
+    DeviceInfo di;
+    if ((st = device_info(&di)) != W4A16_OK) return st;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    if (M <= 16)
+        return w8::w8_gemv_launch(X, M, K, codes, scales, zeros, N, g, sym, Y, di.sm_count, s);
+    w4a16_plan p;
+    st = make_plan(M, N, K, g, sym, W4A16_PATH_TENSORCORE, 0, current_sm_count(), &p, 8);
+    if (st != W4A16_OK) return st;
+    if (workspace_bytes < (size_t)p.workspace_bytes) return W4A16_EWORKSPACE;
+    if (p.workspace_bytes > 0 && (workspace == nullptr || !aligned16(workspace))) return W4A16_EINVAL;
+    return launch_tc(p, X, M, K, codes, scales, zeros, N, g, sym, Y, workspace, s, 8);
 }
 
 w4a16_status w4a16_device_error(int32_t* code) {

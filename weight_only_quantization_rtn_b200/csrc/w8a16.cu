@@ -15,8 +15,10 @@
 //    (G/8 lanes per group, butterfly shuffles) or per-channel (g = K, one CTA
 //    per row, block-wide range reduction and a second pass from L2);
 //  * w8_dequantize_kernel: 8 codes (one 8-byte load) per thread and step;
-//  * w8_gemv_kernel (M ≤ 16): one warp per weight row; each lane streams
-//    16-byte chunks of the row's codes (coalesced 128-bit loads), forms
+//  * w8_gemv_kernel (M ≤ 16; w8a16_gemm launches it through w8_gemv_launch and
+//    runs larger M on the tensor-core kernel with 8-bit codes): one warp per
+//    weight row; each lane streams 16-byte chunks of the row's codes
+//    (coalesced 128-bit loads), forms
 //    x̂ = bf16_rn((q − z)·s) exactly in binary32, and accumulates Σ x·x̂ in
 //    binary32 for every activation row; the lanes' sums are combined by a
 //    fixed butterfly of warp shuffles, so results are deterministic.
@@ -339,6 +341,34 @@ int grid_for(int64_t items, int sm_count) {
 
 w4a16_status launch_status() { return cudaGetLastError() == cudaSuccess ? W4A16_OK : W4A16_ECUDA; }
 
+// Fused GEMV launch for M ≤ 16 (arguments already checked by the caller).
+w4a16_status w8_gemv_launch(const void* X, int64_t M, int64_t K, const void* codes,
+                            const void* scales, const void* zeros, int64_t N, int32_t g,
+                            int32_t sym, void* Y, int sm_count, cudaStream_t s) {
+    const int64_t gl = per_channel(g, K) ? K : (int64_t)g;
+    int64_t grid = (N + kThreads / 32 - 1) / (kThreads / 32);      // one warp per row
+    const int64_t cap = (int64_t)sm_count * 16;
+    if (grid > cap) grid = cap;
+    auto* Xp = static_cast<const uint16_t*>(X);
+    auto* Cp = static_cast<const uint8_t*>(codes);
+    auto* Sp = static_cast<const uint16_t*>(scales);
+    auto* Zp = static_cast<const uint16_t*>(zeros);
+    auto* Yp = static_cast<uint16_t*>(Y);
+    const int m = (int)M;
+#define W8_GEMV(MMV)                                                                           \
+    do {                                                                                       \
+        if (sym) w8_gemv_kernel<MMV, true><<<(unsigned)grid, kThreads, 0, s>>>(Xp, m, K, Cp, Sp, Zp, N, gl, Yp); \
+        else w8_gemv_kernel<MMV, false><<<(unsigned)grid, kThreads, 0, s>>>(Xp, m, K, Cp, Sp, Zp, N, gl, Yp); \
+    } while (0)
+    if (M <= 1) W8_GEMV(1);
+    else if (M <= 2) W8_GEMV(2);
+    else if (M <= 4) W8_GEMV(4);
+    else if (M <= 8) W8_GEMV(8);
+    else W8_GEMV(16);
+#undef W8_GEMV
+    return launch_status();
+}
+
 }  // namespace w8
 
 using namespace w8;
@@ -404,45 +434,6 @@ w4a16_status w8a16_dequantize(const void* codes, const void* scales, const void*
     auto* Wp = static_cast<uint4*>(W_hat);
     if (sym) w8_dequantize_kernel<true><<<grid, kThreads, 0, s>>>(Cp, Sp, Zp, words, gpw, Wp);
     else w8_dequantize_kernel<false><<<grid, kThreads, 0, s>>>(Cp, Sp, Zp, words, gpw, Wp);
-    return launch_status();
-}
-
-w4a16_status w8a16_gemm(const void* X, int64_t M, int64_t K, const void* codes, const void* scales,
-                        const void* zeros, int64_t N, int32_t g, int32_t sym, void* Y,
-                        void* stream) {
-    w4a16_status st = check_shape(N, K, g, sym);
-    if (st != W4A16_OK) return st;
-    if (M < 0 || M > 16) return W4A16_EINVAL;
-    if (M == 0 || N == 0) return W4A16_OK;
-    if (!X || !codes || !scales || !Y || (!sym && !zeros)) return W4A16_EINVAL;
-    if (!aligned16(X) || !aligned16(codes) || !aligned16(scales) || !aligned16(Y) ||
-        (!sym && !aligned16(zeros)))
-        return W4A16_EINVAL;
-    DeviceInfo di;
-    if ((st = device_info(&di)) != W4A16_OK) return st;
-    const int64_t gl = per_channel(g, K) ? K : (int64_t)g;
-    const int64_t warps_needed = N;
-    int64_t grid = (warps_needed + kThreads / 32 - 1) / (kThreads / 32);
-    const int64_t cap = (int64_t)di.sm_count * 16;
-    if (grid > cap) grid = cap;
-    cudaStream_t s = static_cast<cudaStream_t>(stream);
-    auto* Xp = static_cast<const uint16_t*>(X);
-    auto* Cp = static_cast<const uint8_t*>(codes);
-    auto* Sp = static_cast<const uint16_t*>(scales);
-    auto* Zp = static_cast<const uint16_t*>(zeros);
-    auto* Yp = static_cast<uint16_t*>(Y);
-    const int m = (int)M;
-#define W8_GEMV(MMV)                                                                           \
-    do {                                                                                       \
-        if (sym) w8_gemv_kernel<MMV, true><<<(unsigned)grid, kThreads, 0, s>>>(Xp, m, K, Cp, Sp, Zp, N, gl, Yp); \
-        else w8_gemv_kernel<MMV, false><<<(unsigned)grid, kThreads, 0, s>>>(Xp, m, K, Cp, Sp, Zp, N, gl, Yp); \
-    } while (0)
-    if (M <= 1) W8_GEMV(1);
-    else if (M <= 2) W8_GEMV(2);
-    else if (M <= 4) W8_GEMV(4);
-    else if (M <= 8) W8_GEMV(8);
-    else W8_GEMV(16);
-#undef W8_GEMV
     return launch_status();
 }
 
