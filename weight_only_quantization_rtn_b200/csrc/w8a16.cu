@@ -18,7 +18,7 @@
 //  * w8_gemv_kernel (M ≤ 16; w8a16_gemm launches it through w8_gemv_launch and
 //    runs larger M on the tensor-core kernel with 8-bit codes): one warp per
 //    weight row; each lane streams 16-byte chunks of the row's codes
-//    (coalesced 128-bit loads), forms
+//    (coalesced 128-bit loads, four chunks in flight per lane), forms
 //    x̂ = bf16_rn((q − z)·s) exactly in binary32, and accumulates Σ x·x̂ in
 //    binary32 for every activation row; the lanes' sums are combined by a
 //    fixed butterfly of warp shuffles, so results are deterministic.
@@ -238,7 +238,30 @@ __global__ void __launch_bounds__(kThreads) w8_dequantize_kernel(const uint2* __
     }
 }
 
-// Fused GEMV for M ≤ MM (MM ∈ {1, 2, 4, 8, 16}): warp = weight row n.
+// Four 8-bit codes of a word -> their bf16_rn((q − z)·s) values widened to
+// binary32.  The byte placed in a binary32 mantissa gives 2^23 + q exactly;
+// subtracting zoff = 2^23 + z (exact: < 2^24) leaves q − z, the product with s
+// is exact, and cvt.rn.bf16x2 rounds once.  Symmetric words are XORed with
+// 0x80808080 by the caller (offset-128 codes, zoff = 2^23 + 128).
+__device__ __forceinline__ void dequant_word(uint32_t w, float s, float zoff, float out[4]) {
+    float f[4];
+#pragma unroll
+    for (int i = 0; i < 4; ++i)
+        f[i] = (__uint_as_float(__byte_perm(w, 0x4B000000u, 0x7540u + (uint32_t)i)) - zoff) * s;
+#pragma unroll
+    for (int i = 0; i < 4; i += 2) {
+        uint32_t p;
+        asm("cvt.rn.bf16x2.f32 %0, %1, %2;" : "=r"(p) : "f"(f[i + 1]), "f"(f[i]));
+        out[i] = __uint_as_float(p << 16);
+        out[i + 1] = __uint_as_float(p & 0xFFFF0000u);
+    }
+}
+
+// Fused GEMV for M ≤ MM (MM ∈ {1, 2, 4, 8, 16}): warp = weight row n.  Each lane
+// issues the loads of kUnroll 16-code chunks (32 chunks apart) before using
+// any, so a warp keeps 2 KB of codes in flight.
+constexpr int kUnroll = 4;
+
 template <int MM, bool SYM>
 __global__ void __launch_bounds__(kThreads) w8_gemv_kernel(const uint16_t* __restrict__ X, int M,
                                                           int64_t K, const uint8_t* __restrict__ codes,
@@ -251,31 +274,43 @@ __global__ void __launch_bounds__(kThreads) w8_gemv_kernel(const uint16_t* __res
     const int64_t nwarps = ((int64_t)gridDim.x * blockDim.x) >> 5;
     const int64_t Gn = K / g;                      // groups per row
     const int64_t chunks = K / 16;                 // 16-code chunks per row
+    const uint32_t flip = SYM ? 0x80808080u : 0u;
     for (int64_t n = warp0; n < N; n += nwarps) {
         float acc[MM];
 #pragma unroll
         for (int m = 0; m < MM; ++m) acc[m] = 0.0f;
         const uint8_t* row = codes + n * K;
-        for (int64_t c = lane; c < chunks; c += 32) {
-            const uint4 v = ldg16(row + c * 16);
-            const int64_t grp = (c * 16) / g;
-            const float s = bf16_to_f32(__ldg(scales + n * Gn + grp));
-            const int32_t z = SYM ? 0 : (int32_t)bf16_to_f32(__ldg(zeros + n * Gn + grp));
-            const uint32_t wv[4] = {v.x, v.y, v.z, v.w};
-            float w[16];
+        for (int64_t c0 = lane; c0 < chunks; c0 += 32 * kUnroll) {
+            uint4 v[kUnroll];
 #pragma unroll
-            for (int i = 0; i < 16; ++i) w[i] = bf16_to_f32(dequant1(code_of<SYM>(wv[i >> 2], i & 3), z, s));
+            for (int u = 0; u < kUnroll; ++u) {
+                const int64_t c = c0 + 32 * u;
+                v[u] = c < chunks ? ldg16(row + c * 16) : make_uint4(0, 0, 0, 0);
+            }
 #pragma unroll
-            for (int m = 0; m < MM; ++m) {
-                if (m < M) {
-                    const uint16_t* xr = X + (int64_t)m * K + c * 16;
-                    const uint4 xa = __ldg(reinterpret_cast<const uint4*>(xr));
-                    const uint4 xb = __ldg(reinterpret_cast<const uint4*>(xr + 8));
-                    float xf[16];
-                    unpack8(xa, xf);
-                    unpack8(xb, xf + 8);
+            for (int u = 0; u < kUnroll; ++u) {
+                const int64_t c = c0 + 32 * u;
+                if (c >= chunks) break;
+                const int64_t grp = (c * 16) / g;
+                const float s = bf16_to_f32(__ldg(scales + n * Gn + grp));
+                const float zoff = SYM ? 8388736.0f
+                                       : 8388608.0f + bf16_to_f32(__ldg(zeros + n * Gn + grp));
+                const uint32_t wv[4] = {v[u].x, v[u].y, v[u].z, v[u].w};
+                float w[16];
 #pragma unroll
-                    for (int i = 0; i < 16; ++i) acc[m] = fmaf(xf[i], w[i], acc[m]);
+                for (int j = 0; j < 4; ++j) dequant_word(wv[j] ^ flip, s, zoff, w + 4 * j);
+#pragma unroll
+                for (int m = 0; m < MM; ++m) {
+                    if (m < M) {
+                        const uint16_t* xr = X + (int64_t)m * K + c * 16;
+                        const uint4 xa = __ldg(reinterpret_cast<const uint4*>(xr));
+                        const uint4 xb = __ldg(reinterpret_cast<const uint4*>(xr + 8));
+                        float xf[16];
+                        unpack8(xa, xf);
+                        unpack8(xb, xf + 8);
+#pragma unroll
+                        for (int i = 0; i < 16; ++i) acc[m] = fmaf(xf[i], w[i], acc[m]);
+                    }
                 }
             }
         }
