@@ -197,7 +197,7 @@ __global__ void __launch_bounds__(kThreads) w8_quantize_rows_kernel(
     }
 }
 
-// Code byte i of a word pair as a signed (SYM) or unsigned integer.
+// Code byte i of a 32-bit word as a signed (SYM) or unsigned integer.
 template <bool SYM>
 __device__ __forceinline__ int32_t code_of(uint32_t word, int i) {
     const uint32_t b = (word >> (8 * i)) & 0xFFu;
