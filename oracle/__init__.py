@@ -19,6 +19,9 @@ Parity status of each function (what pins it is in ``tests/test_oracle_pins.py``
       gemm_w8a16_sampled (W8A16: 8-bit codes, one per byte) — pinned
       (hand-computed 8-bit groups, brute force over all 256 codes, error
       bounds, on-grid recovery, invariants, one-hot activations)
+  scale_activations / gemm_w4a16_act_scaled (per-K activation scale) — pinned
+      (identity, exact power-of-two scaling, single rounding of the exact
+      product, one-hot activations, the equivalent-scaling identity)
 """
 from __future__ import annotations
 
@@ -88,6 +91,7 @@ def _load():
             lib.oracle_gemm_w8a16_sampled.argtypes = [vp, i64, i64, vp, vp, vp, i64, i64, i32,
                                                       vp, vp, i64, vp]
             lib.oracle_gemm_w8a16_sampled.restype = ctypes.c_int
+            lib.oracle_scale_activations.argtypes = [vp, i64, i64, vp, vp]
             lib.oracle_round_to_bf16.argtypes = [vp, i64, vp]
             lib.oracle_f32_array_to_bf16.argtypes = [vp, i64, vp]
             lib.oracle_num_threads.restype = ctypes.c_int
@@ -311,6 +315,24 @@ def gemm_w8a16_sampled(X_bits, codes, scales, zeros, g: int, sym: bool, ms, ns) 
     if rc != 0:
         raise ValueError("oracle_gemm_w8a16_sampled rejected its arguments")
     return out
+
+
+# ---------------------------------------------------------------- per-K activation scale
+def scale_activations(X_bits, a_bits) -> np.ndarray:
+    """X'[m, k] = bf16_rn(X[m, k]·a[k]) (bf16 bits in and out)."""
+    lib = _load()
+    X = _u16(X_bits)
+    a = _u16(a_bits)
+    M, K = X.shape
+    assert a.shape == (K,)
+    out = np.zeros((M, K), dtype=np.uint16)
+    lib.oracle_scale_activations(_ptr(X), M, K, _ptr(a), _ptr(out))
+    return out
+
+
+def gemm_w4a16_act_scaled(X_bits, a_bits, packed, scales, zeros, g: int, sym: bool) -> np.ndarray:
+    """Y64 = (X·diag(a))' · Ŵᵀ with the scaled activations rounded to bf16 first."""
+    return gemm_w4a16(scale_activations(X_bits, a_bits), packed, scales, zeros, g, sym)
 
 
 def num_threads() -> int:

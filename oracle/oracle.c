@@ -458,6 +458,24 @@ int oracle_gemm_w8a16_sampled(const uint16_t* X, int64_t M, int64_t K, const uin
     return 0;
 }
 
+/* ---------------------------------------------------------------------------
+ * Per-input-channel activation scale: the X/s half of the equivalent
+ * per-channel scaling [P2] §三 describes, (X/s)·(s·W) = X·W, with the vector
+ * a = 1/s supplied by the caller.  Reading R15: the scaled activation is
+ * x' = bf16_rn(x·a) — the product of two bf16 values has at most 16
+ * significant bits, so it is exact in binary32 and is rounded once, as if the
+ * caller had scaled X in bf16 before the GEMM.
+ * ------------------------------------------------------------------------- */
+void oracle_scale_activations(const uint16_t* X, int64_t M, int64_t K, const uint16_t* a,
+                              uint16_t* Xs) {
+    for (int64_t m = 0; m < M; ++m) {
+        for (int64_t k = 0; k < K; ++k) {
+            float prod = oracle_bf16_to_f32(X[m * K + k]) * oracle_bf16_to_f32(a[k]);
+            Xs[m * K + k] = oracle_f32_to_bf16_rn(prod);
+        }
+    }
+}
+
 /* Elementwise bf16_rn of a binary32 array. */
 void oracle_f32_array_to_bf16(const float* x, int64_t n, uint16_t* out) {
     for (int64_t i = 0; i < n; ++i) out[i] = oracle_f32_to_bf16_rn(x[i]);

@@ -36,6 +36,10 @@ MUTANTS = {
     "w8_zero_point_clamped_to_15": ("rintf(-mn / s), 0.0f, 255.0f", "rintf(-mn / s), 0.0f, 15.0f"),
     "w8_dequant_truncates": ("W_hat[n * K + k] = oracle_f32_to_bf16_rn(prod);",
                              "uint32_t u; memcpy(&u, &prod, 4); W_hat[n * K + k] = (uint16_t)(u >> 16);"),
+    # per-K activation scale
+    "act_scale_truncates": ("Xs[m * K + k] = oracle_f32_to_bf16_rn(prod);",
+                            "uint32_t u; memcpy(&u, &prod, 4); Xs[m * K + k] = (uint16_t)(u >> 16);"),
+    "act_scale_indexed_by_row": ("oracle_bf16_to_f32(a[k]);", "oracle_bf16_to_f32(a[m % K]);"),
 }
 
 

@@ -605,3 +605,66 @@ def test_w8_gemm_one_hot_and_sampled():
         Yf = oracle.gemm_w8a16(Xr, C, S, Z, 128, sym)
         ms, ns = np.array([0, 2, 1, 2]), np.array([0, 23, 7, 11])
         assert np.array_equal(oracle.gemm_w8a16_sampled(Xr, C, S, Z, 128, sym, ms, ns), Yf[ms, ns])
+
+
+# ------------------------------------------------------------------ per-K activation scale
+def _rand_bf16(shape, seed, scale=1.0):
+    x = np.random.default_rng(seed).standard_normal(shape).astype(np.float32) * np.float32(scale)
+    return oracle.bf16_from_f32(x)
+
+
+def test_activation_scale_by_one_is_identity():
+    X = _rand_bf16((5, 96), 1)
+    a = oracle.bf16_from_f32(np.ones(96, np.float32))
+    assert np.array_equal(oracle.scale_activations(X, a), X)
+
+
+def test_activation_scale_by_powers_of_two_is_exact():
+    X = _rand_bf16((7, 128), 2)
+    e = np.random.default_rng(3).integers(-20, 21, 128)
+    a = oracle.bf16_from_f32((2.0 ** e).astype(np.float32))
+    got = oracle.f32_from_bf16(oracle.scale_activations(X, a)).astype(np.float64)
+    exp = oracle.f32_from_bf16(X).astype(np.float64) * 2.0 ** e      # exact
+    assert np.array_equal(got, exp)
+
+
+def test_activation_scale_rounds_the_exact_product_once():
+    """x·a of two bf16 values is exact in binary64; the result must be that
+    product rounded once to bf16 (not a double rounding, not a truncation)."""
+    X = _rand_bf16((16, 512), 4)
+    a = _rand_bf16((512,), 5, 3.0)
+    exact = oracle.f32_from_bf16(X).astype(np.float64) * oracle.f32_from_bf16(a).astype(np.float64)
+    assert np.array_equal(oracle.scale_activations(X, a), oracle.bf16_from_f64(exact))
+
+
+def test_act_scaled_gemm_one_hot():
+    """One-hot rows of X select a[k]·x̂[n, k], exact in binary64."""
+    W = workloads.bits(workloads.make_weight(24, 256, 0.02, seed=21))
+    P, S, Z = oracle.quantize(W, 64, False)
+    Wh = oracle.f32_from_bf16(oracle.dequantize(P, S, Z, 256, 64, False)).astype(np.float64)
+    a = _rand_bf16((256,), 6, 2.0)
+    ks = np.array([0, 3, 63, 64, 200, 255])
+    X = np.zeros((ks.size, 256), np.float32)
+    X[np.arange(ks.size), ks] = 1.0
+    Y = oracle.gemm_w4a16_act_scaled(oracle.bf16_from_f32(X), a, P, S, Z, 64, False)
+    af = oracle.f32_from_bf16(a).astype(np.float64)
+    assert np.array_equal(Y, (Wh[:, ks] * af[ks]).T)
+
+
+@pytest.mark.parametrize("sym", [False, True])
+def test_equivalent_scaling_identity(sym):
+    """The identity the activation scale serves ((X/s)·(s·W) = X·W): with s a
+    power of two constant over each weight group, quantizing s·W gives the same
+    codes and scales multiplied by s, so X·diag(1/s) against them reproduces
+    the unscaled result exactly."""
+    N, K, g = 12, 256, 32
+    W = workloads.make_weight(N, K, 0.02, seed=22, outlier_frac=0.02, outlier_scale=20.0)
+    e = np.repeat(np.random.default_rng(7).integers(-6, 7, K // g), g)
+    Ws = (W.to(torch.float32) * torch.tensor(2.0 ** e, dtype=torch.float32)).to(torch.bfloat16)
+    X = workloads.bits(workloads.make_activation(3, K, 8))
+    a = oracle.bf16_from_f32((2.0 ** -e).astype(np.float32))
+    P, S, Z = oracle.quantize(workloads.bits(W), g, sym)
+    Ps, Ss, Zs = oracle.quantize(workloads.bits(Ws), g, sym)
+    Y = oracle.gemm_w4a16(X, P, S, Z, g, sym)
+    Ysc = oracle.gemm_w4a16_act_scaled(X, a, Ps, Ss, Zs, g, sym)
+    assert np.array_equal(Y, Ysc)
