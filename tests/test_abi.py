@@ -319,3 +319,16 @@ def test_w8a16_entry_points_reject_invalid(lib):
     assert ws(16, 4096, 4096, 128) == 0                     # the GEMV needs none
     assert ws(17, 8192, 8192, 32) == w4.workspace_size(17, 8192, 8192, 32) > 0
     assert ws(2048, 8192, 8192, 128) == w4.workspace_size(2048, 8192, 8192, 128)
+
+
+@pytest.mark.parametrize("compiler,std", [("gcc", "-std=c99"), ("g++", "-std=c++11")])
+def test_header_compiles_as_plain_c_and_cpp(tmp_path, compiler, std):
+    """The public header is a C ABI: it must compile as strict C99 (no C++
+    constructs leaking in) as well as C++, and every declared entry point must be
+    callable through it."""
+    calls = "\n".join(f"    (void){n};" for n in declared_functions())
+    src = tmp_path / ("use.c" if compiler == "gcc" else "use.cpp")
+    src.write_text('#include "w4a16.h"\nint main(void) {\n' + calls + "\n    return 0;\n}\n")
+    r = subprocess.run([compiler, std, "-Wall", "-Werror", "-pedantic", "-fsyntax-only",
+                        "-I", os.path.dirname(HEADER), str(src)], capture_output=True, text=True)
+    assert r.returncode == 0, r.stderr
