@@ -332,3 +332,37 @@ def test_header_compiles_as_plain_c_and_cpp(tmp_path, compiler, std):
     r = subprocess.run([compiler, std, "-Wall", "-Werror", "-pedantic", "-fsyntax-only",
                         "-I", os.path.dirname(HEADER), str(src)], capture_output=True, text=True)
     assert r.returncode == 0, r.stderr
+
+
+def test_plain_c_program_links_and_plans(tmp_path):
+    """A C program linked against the library (no Python, no torch) can call the
+    host-only entry points: version, status strings, plans and workspace sizes."""
+    src = tmp_path / "plan.c"
+    src.write_text(r'''
+#include <stdio.h>
+#include "w4a16.h"
+int main(void) {
+    w4a16_plan p;
+    if (w4a16_abi_version() != W4A16_ABI_VERSION) return 1;
+    if (w4a16_gemm_plan(1, 11008, 4096, 128, 0, W4A16_PATH_AUTO, 0, &p) != W4A16_OK) return 2;
+    printf("%d %lld %d %lld\n", p.path, (long long)p.grid, p.kernels, (long long)p.workspace_bytes);
+    if (w4a16_gemm_plan(17, 4096, 4096, 48, 0, W4A16_PATH_AUTO, 0, &p) != W4A16_EINVAL) return 3;
+    printf("%zu %zu\n", w4a16_gemm_workspace_size(2048, 8192, 8192, 128),
+           w8a16_gemm_workspace_size(2048, 8192, 8192, 128));
+    printf("%s\n", w4a16_status_string(W4A16_EWORKSPACE));
+    return 0;
+}
+''')
+    exe = tmp_path / "plan"
+    libdir = os.path.dirname(w4.LIB_PATH)
+    subprocess.run(["gcc", "-std=c99", "-I", os.path.dirname(HEADER), str(src), "-o", str(exe),
+                    "-L", libdir, "-lw4a16", f"-Wl,-rpath,{libdir}"], check=True)
+    out = subprocess.run([str(exe)], capture_output=True, text=True)
+    assert out.returncode == 0, (out.returncode, out.stderr)
+    lines = out.stdout.split("\n")
+    path, grid, kernels, ws = map(int, lines[0].split())
+    p = w4.plan(1, 11008, 4096, 128)
+    assert (path, grid, kernels, ws) == (1, p["grid"], p["kernels"], p["workspace_bytes"])
+    a, b = map(int, lines[1].split())
+    assert a == b == w4.workspace_size(2048, 8192, 8192, 128)
+    assert lines[2].startswith("W4A16_EWORKSPACE")
