@@ -4,7 +4,7 @@
  * W4A16: weights stored as 4-bit integer codes, activations kept in 16-bit
  * floating point (bf16 here).  The method, as the pages describe it:
  *
- *  - qwbw.cn, "推理优化中“用精度换性能“的核心技术：量化":
+ *  - "推理优化中“用精度换性能“的核心技术：量化":
  *      §2.2  INT4 holds [−8, 7] or [0, 15];
  *      §2.3  x_int = round(x_float / s) + z,  x̂_float = (x_int − z) × s;
  *      §3.3  symmetric:  s = max|x| / max_int, z = 0;
@@ -13,13 +13,13 @@
  *            16-bit scale and an optional 16-bit zero point (4.25 bits/weight);
  *      §3.2  weight-only inference: load INT4 from memory, dequantize to
  *            16-bit, multiply with 16-bit activations.
- *  - meko1.github.io, "量化实战深入（GPTQ / AWQ / SmoothQuant / KV 量化）",
+ *  - "量化实战深入（GPTQ / AWQ / SmoothQuant / KV 量化）",
  *      §二  q = round(x/s) + z, x ≈ s·(q − z); absmax s = max|x| / (2^(b−1) − 1);
  *           per-group = one scale per 128 elements.
- *  - offer.aigcbaba.com, "大模型推理中 Weight-only、W8A8 和 FP8 量化有什么区别？",
+ *  - "大模型推理中 Weight-only、W8A8 和 FP8 量化有什么区别？如何选型？",
  *      §二  a fused kernel reads INT4, unpacks and scales in registers or shared
  *           memory, and multiplies with the high-precision activations.
- *  - mianshidashi.cn, "LLM 量化中 W4A16 表示什么…", 显存收益主要来自权重 / 性能取决于 kernel:
+ *  - "LLM 量化中 W4A16 表示什么…｜蚂蚁集团 C/C++面经解析", 显存收益主要来自权重 / 性能取决于 kernel:
  *           0.5 byte per INT4 weight; dequantize inside the GEMM while reading
  *           INT4, rather than expanding the whole matrix first.
  *
@@ -43,8 +43,8 @@
  *
  * Supported: g ∈ {32, 64, 128} with K a positive multiple of g, or g = K with K
  * a positive multiple of 32 — per-channel granularity, one scale (and zero) per
- * output feature, scales/zeros [N, 1] (meko1 page, 量化粒度 table; qwbw.cn page
- * §3.4); N ≥ 0, M ≥ 0 (M = 0 or N = 0 is a no-op), N, K, M < 2^31.  Every pointer is a DEVICE
+ * output feature, scales/zeros [N, 1] ("量化实战深入（GPTQ / AWQ / SmoothQuant / KV 量化）",
+ * 量化粒度 table; "推理优化中“用精度换性能“的核心技术：量化", §3.4); N ≥ 0, M ≥ 0 (M = 0 or N = 0 is a no-op), N, K, M < 2^31.  Every pointer is a DEVICE
  * pointer owned by the caller; the library allocates no device memory and keeps
  * no state beyond per-device constants (device properties, tensor-map encoder)
  * and the fixed scratch array of w4a16_gemm_decode_noalloc.  Device scratch,
@@ -64,7 +64,7 @@
 extern "C" {
 #endif
 
-#define W4A16_ABI_VERSION 2   /* 2: the tensor-core path may need a workspace (split K) */
+#define W4A16_ABI_VERSION 3   /* 3: w4a16_plan.split_tiles; the decode path is one kernel */
 
 typedef enum w4a16_status {
     W4A16_OK = 0,
@@ -76,15 +76,15 @@ typedef enum w4a16_status {
 } w4a16_status;
 
 /* GEMM kernel choice (roofline-driven: decode is weight-bandwidth bound, prefill
- * is tensor-core bound — Quantization & Acceleration page, 关键判据; the
- * aigcbaba selection page, §二 and §五). */
+ * is tensor-core bound — "Quantization & Acceleration: 解释 W8A8 与 W4A16 的差异与取舍",
+ * 关键判据; "大模型推理中 Weight-only、W8A8 和 FP8 量化有什么区别？如何选型？", §二 and §五). */
 typedef enum w4a16_path {
     W4A16_PATH_AUTO = 0,       /* choose from M (roofline: M ≤ 16 is weight-bandwidth bound) */
     W4A16_PATH_DECODE = 1,     /* small-M kernel, M ≤ 16: persistent stream-K grid; TMA streams
                                   packed codes and X into a shared-memory ring; in-register
-                                  dequantization feeds bf16 MMAs with fp32 accumulation; row
-                                  blocks split across CTAs are added in a fixed order by a
-                                  second small kernel */
+                                  dequantization feeds bf16 MMAs with fp32 accumulation; a
+                                  row block split across CTAs is finished by its first
+                                  owner, which adds the other owners' parts in a fixed order */
     W4A16_PATH_TENSORCORE = 2  /* large-M kernel: TMA-fed INT4 tile dequantized into shared
                                   memory and fed to tcgen05 bf16 MMA with TMEM accumulators;
                                   when the output tiles are fewer than the SMs, or the last
@@ -102,11 +102,13 @@ typedef struct w4a16_plan {
     int64_t grid;            /* CTAs launched */
     int32_t smem_bytes;      /* dynamic shared memory per CTA */
     int32_t stages;          /* shared-memory pipeline depth */
-    int32_t kernels;         /* kernels the call launches: decode 2 when its stream-K
-                                partition splits a row block between CTAs, else 1;
-                                tensor core 1 unsplit, 2 when every tile splits K (+ the
-                                reduce), 3 with an unsplit head, a split tail and the reduce */
+    int32_t kernels;         /* kernels the call launches: decode 1; tensor core 1 unsplit,
+                                2 when every tile splits K (+ the reduce), 3 with an unsplit
+                                head, a split tail and the reduce */
     int64_t workspace_bytes; /* device workspace this launch needs */
+    int64_t split_tiles;     /* output tiles whose K range is split between CTAs, so that
+                                partial sums pass through the workspace: decode, the 256-row
+                                blocks its stream-K partition cuts; tensor core, the tail tiles */
 } w4a16_plan;
 
 /* Quantize W[N, K] group-wise by RTN (asymmetric when sym == 0, symmetric when
@@ -120,7 +122,7 @@ typedef struct w4a16_plan {
 w4a16_status w4a16_quantize(const void* W, int64_t N, int64_t K, int32_t g, int32_t sym,
                             void* packed, void* scales, void* zeros, void* stream);
 
-/* Expand packed codes to Ŵ[n, k] = bf16_rn((q − z)·s) (qwbw.cn page §2.3).
+/* Expand packed codes to Ŵ[n, k] = bf16_rn((q − z)·s) ("推理优化中“用精度换性能“的核心技术：量化", §2.3).
  * This is the unfused form the fused GEMM avoids; it is provided for checking
  * and for callers that need Ŵ.
  *   packed, scales in; zeros in (ignored, may be NULL, when sym == 1)
@@ -130,8 +132,8 @@ w4a16_status w4a16_dequantize(const void* packed, const void* scales, const void
                               void* stream);
 
 /* Bytes of device workspace w4a16_gemm needs for this shape.  The decode path
- * stores there the fp32 partial sums of the 32-row blocks that its stream-K
- * partition splits between CTAs.  The tensor-core path, for the output tiles
+ * stores there the fp32 partial sums of the 256-row blocks that its stream-K
+ * partition splits between CTAs, with a ready flag per part.  The tensor-core path, for the output tiles
  * whose K it splits into S parts (all tiles when they are fewer than the SMs,
  * else only a mostly-empty last wave), stores S fp32 partial tiles of
  * 128 weight rows x tile_m activation rows per split tile, and needs 0 bytes
@@ -156,9 +158,11 @@ w4a16_status w4a16_gemm(const void* X, int64_t M, int64_t K, const void* packed,
                         void* stream);
 
 /* w4a16_gemm with the dispatch decision overridden: `path` forces a kernel
- * (AUTO = same as w4a16_gemm) and `ctas` (decode only; 0 = automatic, one or
- * two CTAs per SM) sets the size of the persistent grid, hence where the
- * stream-K partition splits row blocks.  Used by tests, benchmarks and
+ * (AUTO = same as w4a16_gemm) and `ctas` (decode only; 0 = automatic) sets the
+ * size of the persistent grid, hence where the stream-K partition splits row
+ * blocks; it is capped at one resident wave (one or two CTAs per SM, as the
+ * plan reports), because the CTA finishing a split row block waits for parts
+ * from CTAs that run beside it.  Used by tests, benchmarks and
  * profiling to exercise both kernels and many partitions at the same shape.
  * Returns W4A16_EINVAL if the forced kernel cannot run the shape (DECODE with
  * M > 16, or `ctas` given for the tensor-core path), W4A16_EWORKSPACE if the
@@ -179,32 +183,32 @@ w4a16_status w4a16_gemm_plan(int64_t M, int64_t N, int64_t K, int32_t g, int32_t
 
 /* Decode-path GEMM (M ≤ 16) that allocates nothing and takes no workspace.
  * The pages have no counterpart: this exists for callers that cannot allocate
- * device memory — code running while a CUDA graph is being captured (where
- * cudaMalloc is not allowed), plug-ins whose host framework owns every device
- * allocation through its own pool, and hosts that forbid allocation after
- * start-up so that memory use stays fixed.
+ * device memory — plug-ins whose host framework owns every device allocation
+ * through its own pool, and hosts that forbid allocation after start-up so
+ * that memory use stays fixed.
  * Same arguments, result and determinism as w4a16_gemm_ex with
  * path = W4A16_PATH_DECODE and ctas = 0, minus the workspace: the split-K
  * partial sums live in a file-scope device array of
  * W4A16_NOALLOC_SCRATCH_BYTES that every GPU which loads the library keeps
  * until the process exits.  Returns W4A16_EWORKSPACE, launching nothing, when
- * the problem needs more scratch than that (its plan's workspace_bytes), and
- * W4A16_EINVAL for M > 16 or any argument w4a16_gemm_ex would reject.
+ * the problem needs more scratch than that (its plan's workspace_bytes: about
+ * 2000 row blocks plus CTAs at M ≤ 8, 1000 at M 9–16, i.e. N up to roughly
+ * 220 000 and 90 000 rows on 148 SMs), and W4A16_EINVAL for M > 16 or any
+ * argument w4a16_gemm_ex would reject.
  * The first call on a device looks up the array's device address for that
- * device (cudaGetSymbolAddress, with the device current); make that first
- * call before any stream capture.  All calls share the one array and it keeps
- * the last call's contents; nothing in it needs to start at zero.  Calls that
- * overlap on the GPU (other streams, other threads, other graph branches)
+ * device (cudaGetSymbolAddress, with the device current).  All calls share the
+ * one array and it keeps the last call's contents; nothing in it needs to
+ * start at zero.  Calls that overlap on the GPU (other streams, other threads)
  * race on it: serialize them. */
 w4a16_status w4a16_gemm_decode_noalloc(const void* X, int64_t M, int64_t K, const void* packed,
                                        const void* scales, const void* zeros, int64_t N,
                                        int32_t g, int32_t sym, void* Y, void* stream);
 
 /* ---------------------------------------------------------------------------
- * W8A16: the same method with 8-bit codes (the INT8 form the qwbw.cn page
- * states in §3.3: asymmetric s = (max − min)/255, z = round(−min/s); symmetric
- * s = max|x|/127, meko1 page §二 absmax with b = 8; W8A16 is listed beside
- * W4A16 on the aigcbaba page, 详细版).  Readings as above with the 8-bit
+ * W8A16: the same method with 8-bit codes (the INT8 form
+ * "推理优化中“用精度换性能“的核心技术：量化" states in §3.3: asymmetric s = (max − min)/255, z = round(−min/s); symmetric
+ * s = max|x|/127, "量化实战深入（GPTQ / AWQ / SmoothQuant / KV 量化）" §二 absmax with b = 8;
+ * W8A16 is listed beside W4A16 in "大模型推理中 Weight-only、W8A8 和 FP8 量化有什么区别？如何选型？", 详细版).  Readings as above with the 8-bit
  * ranges: codes clamped to [0, 255] (asym) or [−128, 127] (sym, stored as
  * int8 two's complement); zeros are integers 0..255 stored in bf16.
  * Layouts: codes uint8 [N, K] (element k of a row in byte k); scales and

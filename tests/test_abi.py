@@ -53,7 +53,7 @@ def test_library_is_sm100a_only_and_links_no_cudart_dso(lib):
 
 
 def test_status_strings_and_version(lib):
-    assert lib.w4a16_abi_version() == 2
+    assert lib.w4a16_abi_version() == 3
     for s in range(6):
         assert lib.w4a16_status_string(s).startswith(b"W4A16")
 
@@ -133,12 +133,14 @@ def test_workspace_sizes(lib):
     assert splits == 2 and p17["kernels"] == 2
     # tile-local parts: [split][tile][32 activation rows][128 weight rows] fp32
     assert w4.workspace_size(17, 8192, 8192, 32) == splits * 64 * 32 * 128 * 4
-    rb = 4096 // 32
-    p = w4.plan(1, 4096, 4096, 128)
-    assert p["workspace_bytes"] == (rb + p["grid"]) * 256 * 4
-    p16 = w4.plan(16, 4096, 4096, 128)
-    assert p16["workspace_bytes"] == (rb + p16["grid"]) * 512 * 4
-    assert w4.workspace_size(1, 4096, 4096, 128) == p["workspace_bytes"]
+    # decode: per slot (row blocks + CTAs) 16 ready flags (rounded to 256 bytes in
+    # all) and 16 warps x 32 lanes x 4·mb fp32 partial sums
+    rb = 4096 // 256
+    for M, mb in ((1, 1), (16, 2)):
+        p = w4.plan(M, 4096, 4096, 128)
+        slots = rb + p["grid"]
+        assert p["workspace_bytes"] == -(-slots * 16 * 4 // 256) * 256 + slots * 16 * 32 * 16 * mb
+    assert w4.workspace_size(1, 4096, 4096, 128) == w4.plan(1, 4096, 4096, 128)["workspace_bytes"]
 
 
 def test_decode_rejects_small_workspace(lib):
@@ -196,18 +198,35 @@ def test_decode_persistent_grid_and_smem():
     for M, N, K in ((1, 11008, 4096), (1, 4096, 11008), (1, 28672, 8192), (8, 8192, 28672),
                     (16, 8192, 8192), (1, 256, 256)):
         p = w4.plan(M, N, K)
-        units = -(-N // 32) * -(-K // 1024)
-        per_sm = 2 if (M <= 8 and p["smem_bytes"] * 2 + 2048 <= 233472) else 1
-        assert p["grid"] == min(units, 148 * per_sm)
-        assert p["smem_bytes"] <= 232448 and p["stages"] >= 2
-        assert p["threads"] == 288
-    # forced grid sizes (any positive count, capped at the number of units)
+        units = -(-N // 256) * -(-K // 256)
+        assert p["grid"] == min(units, 148)                    # one CTA per SM
+        assert p["smem_bytes"] <= 232448 and p["stages"] >= 2 and p["kernels"] == 1
+        assert p["threads"] == 576 and p["tile_n"] == 256
+    # the M=1 workloads keep at least five stages of 32 KB in flight per SM
+    assert w4.plan(1, 28672, 8192)["stages"] >= 5 and w4.plan(1, 28672, 8192)["grid"] == 148
+    # forced grid sizes: any positive count, capped at the units and at one resident wave
     assert w4.plan(1, 4096, 11008, ctas=7)["grid"] == 7
-    assert w4.plan(1, 64, 1024, ctas=50)["grid"] == 2          # 2 row blocks x 1 K block
+    assert w4.plan(1, 64, 1024, ctas=50)["grid"] == 4          # 1 row block x 4 K blocks
+    assert w4.plan(1, 28672, 8192, ctas=5000)["grid"] == 148
     with pytest.raises(w4.W4A16Error):
         w4.plan(17, 4096, 4096, path="decode")
     with pytest.raises(w4.W4A16Error):
         w4.plan(64, 4096, 4096, path="tensorcore", ctas=4)
+
+
+@pytest.mark.parametrize("M", list(range(1, 17)))
+def test_decode_stage_layout_is_valid_for_every_shape(M):
+    """The library refuses (W4A16_EUNSUPPORTED) a decode plan whose stage layout
+    breaks its invariants — TMA destinations 128-byte aligned, the codes tile
+    1024-byte aligned, the ring within one CTA's shared memory — so planning
+    every M, g and a spread of K and N here checks the layout arithmetic."""
+    for K in (32, 64, 96, 128, 160, 256, 384, 1024, 1056, 2304, 4096, 4352, 5376, 11008, 28672):
+        for g in (32, 64, 128, K):
+            if K % g:
+                continue
+            for N in (1, 128, 1000, 28672):
+                p = w4.plan(M, N, K, g, False, "decode")
+                assert p["stages"] >= 2 and p["smem_bytes"] <= 232448
 
 
 def _owner(u, U, C):
@@ -217,10 +236,8 @@ def _owner(u, U, C):
 @pytest.mark.parametrize("U,C", [(10, 3), (1376, 296), (1408, 296), (7, 7), (5, 1), (100, 99)])
 def test_stream_k_partition_arithmetic(U, C):
     """The kernel's split u_c = floor(c·U/C) and its inverse owner(u): every
-    unit has exactly one owner, owners are contiguous and non-decreasing, the
-    partial-sum slot rb + c of a split row block never collides, and the fixup
-    kernel's rule (boundary b handles the row block it falls in iff b is the
-    row block's first owner) finishes every split row block exactly once."""
+    unit has exactly one owner, owners are contiguous and non-decreasing, and
+    the partial-sum slot rb + c of a split row block never collides."""
     starts = [c * U // C for c in range(C + 1)]
     for c in range(C):
         for u in range(starts[c], starts[c + 1]):
@@ -236,17 +253,6 @@ def test_stream_k_partition_arithmetic(U, C):
                 slot = rb + c
                 assert slot not in used and slot < rbs + C
                 used.add(slot)
-        handled = []
-        for b in range(C - 1):
-            u_next = (b + 1) * U // C
-            if u_next % kbn == 0:
-                continue
-            rb = u_next // kbn
-            if _owner(rb * kbn, U, C) == b:
-                handled.append(rb)
-        split = [rb for rb in range(rbs)
-                 if _owner(rb * kbn, U, C) != _owner(rb * kbn + kbn - 1, U, C)]
-        assert sorted(handled) == split
 
 
 def _walk(u0, u1, kbn):
@@ -292,6 +298,60 @@ def test_stream_k_unit_walk(kbn):
                     idx = [i for i, (r, _, _) in enumerate(w) if r == rb]
                     assert idx == list(range(idx[0], idx[-1] + 1))
                     assert [i for i in idx if w[i][2]] == [idx[-1]]
+
+
+def _decode_events(U, C, kbn):
+    """Per CTA, in visiting order, what it does at each row-block end: 'store'
+    (whole row block), 'publish' (its part of a split row block, for the first
+    owner) or 'finish' (first owner: wait for the other parts, add, store)."""
+    ev = {}
+    for c in range(C):
+        u0, u1 = c * U // C, (c + 1) * U // C
+        out = []
+        for rb, kb, end in _walk(u0, u1, kbn):
+            if not end:
+                continue
+            first = rb * kbn
+            if first >= u0 and first + kbn <= u1:
+                out.append(("store", rb))
+            elif _owner(first, U, C) == c:
+                out.append(("finish", rb))
+            else:
+                out.append(("publish", rb))
+        ev[c] = out
+    return ev
+
+
+@pytest.mark.parametrize("kbn", [1, 2, 4, 11, 16, 32, 43])
+def test_decode_split_row_blocks_finish_once_and_never_deadlock(kbn):
+    """Every row block is stored exactly once; a split row block is finished by
+    its first owner after every other owner publishes a part; and every CTA
+    publishes all its parts before it waits for any, so with all CTAs resident
+    every wait ends (the waited-for CTAs never wait first)."""
+    for rbs in (1, 2, 3, 7, 20, 33):
+        U = rbs * kbn
+        for C in sorted({1, 2, 3, 5, 7, 13, 40, 97, 296, U} & set(range(1, U + 1))):
+            ev = _decode_events(U, C, kbn)
+            stored = [rb for c in range(C) for kind, rb in ev[c] if kind in ("store", "finish")]
+            assert sorted(stored) == list(range(rbs))
+            for rb in range(rbs):
+                cf, cl = _owner(rb * kbn, U, C), _owner(rb * kbn + kbn - 1, U, C)
+                pubs = sorted(c for c in range(C) for kind, r in ev[c] if kind == "publish" and r == rb)
+                assert pubs == list(range(cf + 1, cl + 1))
+            for c in range(C):
+                kinds = [k for k, _ in ev[c]]
+                if "finish" in kinds and "publish" in kinds:
+                    assert max(i for i, k in enumerate(kinds) if k == "publish") < kinds.index("finish")
+
+
+def test_decode_plan_reports_split_row_blocks():
+    U_rows, kbn = -(-4096 // 256), -(-4096 // 256)
+    p = w4.plan(1, 4096, 4096, 128)
+    U, C = U_rows * kbn, p["grid"]
+    cut = {(b * U // C) // kbn for b in range(1, C) if (b * U // C) % kbn}
+    assert p["split_tiles"] == len(cut) > 0
+    assert w4.plan(1, 4096, 4096, 128, ctas=U_rows)["split_tiles"] == 0   # one row block per CTA
+    assert w4.plan(2048, 8192, 8192)["split_tiles"] == 68                  # the tensor-core tail
 
 
 # ------------------------------------------------------------------ W8A16 entry points

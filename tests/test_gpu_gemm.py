@@ -66,7 +66,8 @@ def test_decode_path_small(M, N, K, g, sym):
 @pytest.mark.parametrize("M", [1, 12])
 def test_decode_stream_k_partitions(ctas, M):
     """Many persistent-grid sizes: row blocks split 0..n times between CTAs, their
-    parts added by the fixup kernel; two calls in a row reuse the workspace."""
+    parts added by each row block's first owner; two calls in a row reuse the
+    workspace (its flags must read as consumed again after every call)."""
     _check_full(M, 300, 1024 * 5 + 256, 128, False, "decode", seed=5, ctas=ctas)
     _check_full(M, 300, 1024 * 5 + 256, 128, False, "decode", seed=6, ctas=ctas)
 

@@ -288,8 +288,8 @@ def test_on_grid_matrix_is_recovered_exactly(g):
 # ------------------------------------------------------------------ per-channel (g = K)
 @pytest.mark.parametrize("sym", [False, True])
 def test_hand_computed_rows_per_channel(sym):
-    """Per-channel granularity (one scale per output row; meko1 page, 量化粒度
-    table; qwbw.cn page §3.4) is g = K: each row of a [rows, 4] matrix is one of
+    """Per-channel granularity (one scale per output row; "量化实战深入（GPTQ / AWQ / SmoothQuant / KV 量化）",
+    量化粒度 table; "推理优化中“用精度换性能“的核心技术：量化", §3.4) is g = K: each row of a [rows, 4] matrix is one of
     the hand-computed groups and must get that group's s, z, codes and x̂."""
     cases = [c for c in CASES if (c["mode"] == "sym") == sym]
     assert cases
@@ -432,7 +432,8 @@ CASES_W8 = json.load(open(GOLDEN_W8))["cases"]
 
 @pytest.mark.parametrize("case", CASES_W8, ids=[c["name"] for c in CASES_W8])
 def test_hand_computed_group_w8(case):
-    """8-bit groups worked by hand (INT8 form of qwbw.cn page §3.3; meko1 page
+    """8-bit groups worked by hand (INT8 form of "推理优化中“用精度换性能“的核心技术：量化", §3.3;
+    "量化实战深入（GPTQ / AWQ / SmoothQuant / KV 量化）",
     §二 absmax with b = 8): scale bits, zero point and codes."""
     x = _f32(case["x"])
     if case["mode"] == "sym":

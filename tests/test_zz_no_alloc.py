@@ -44,8 +44,9 @@ def _case(M, N, K, g, sym, seed):
     return X, P, S, Z
 
 
-# Both cases split rows across CTAs (non-zero workspace), so the scratch carries
-# partial sums; the second call finds the first call's values still there.
+# Every case splits row blocks between CTAs (the plan's split_tiles), so partial
+# sums and ready flags pass through the scratch; the second call finds the first
+# call's values still there.
 CASES = [(1, 4096, 4096, 128, False, 101), (12, 11008, 4096, 64, True, 103),
          (3, 1000, 2304, 32, False, 105)]
 
@@ -55,7 +56,7 @@ def test_noalloc_matches_decode_entry_point(lib):
     prepared = []
     for (M, N, K, g, sym, seed) in CASES:
         p = w4.plan(M, N, K, g, sym, "decode")
-        assert 0 < p["workspace_bytes"] <= SCRATCH_BYTES
+        assert 0 < p["workspace_bytes"] <= SCRATCH_BYTES and p["split_tiles"] > 0
         X, P, S, Z = _case(M, N, K, g, sym, seed)
         Y_ref = w4.gemm(X, P, S, Z, g, sym, path="decode")
         prepared.append((X, P, S, Z, g, sym, Y_ref))
@@ -100,3 +101,21 @@ def test_noalloc_rejects_without_launching(lib):
     assert lib.w4a16_gemm_decode_noalloc(f, 17, K, f, f, f, 256, g, 0, f, None) == EINVAL
     assert lib.w4a16_gemm_decode_noalloc(f, 1, K, f, f, None, 256, g, 0, f, None) == EINVAL
     assert lib.w4a16_gemm_decode_noalloc(f, 0, K, f, f, f, 256, g, 0, f, None) == 0
+
+
+@pytest.mark.gpu
+def test_noalloc_binding_rejects_mismatched_tensors(lib):
+    """The binding checks shapes, dtypes and devices before the C call, so a
+    mismatched tensor raises here and nothing is launched."""
+    X, P, S, Z = _case(2, 256, 512, 128, False, 109)
+    with pytest.raises(ValueError):
+        w4.gemm_decode_noalloc(X[:, :256].contiguous(), P, S, Z, 128, False)   # K differs
+    with pytest.raises(ValueError):
+        w4.gemm_decode_noalloc(X, P, S, Z, 128, False,
+                               out=torch.empty(2, 255, dtype=torch.bfloat16, device=X.device))
+    with pytest.raises(TypeError):
+        w4.gemm_decode_noalloc(X, P, S, Z, 128, False,
+                               out=torch.empty(2, 256, dtype=torch.float32, device=X.device))
+    with pytest.raises(ValueError):
+        w4.gemm_decode_noalloc(X, P, S, Z, 128, False,
+                               out=torch.empty(256, 2, dtype=torch.bfloat16, device=X.device).t())

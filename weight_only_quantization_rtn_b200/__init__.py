@@ -24,7 +24,7 @@ __all__ = ["lib", "quantize", "dequantize", "gemm", "gemm_decode_noalloc", "plan
 LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libw4a16.so")
 
 # W4A16_ABI_VERSION in include/w4a16.h that the argument lists below follow
-ABI_VERSION = 2
+ABI_VERSION = 3
 PATH_AUTO, PATH_DECODE, PATH_TENSORCORE = 0, 1, 2
 _PATHS = {"auto": PATH_AUTO, "decode": PATH_DECODE, "tensorcore": PATH_TENSORCORE}
 _STATUS = {0: "OK", 1: "EINVAL", 2: "EUNSUPPORTED", 3: "ECUDA", 4: "EWORKSPACE", 5: "EDEVICE"}
@@ -41,7 +41,7 @@ class Plan(ctypes.Structure):
                 ("tile_n", ctypes.c_int32), ("threads", ctypes.c_int32),
                 ("grid", ctypes.c_int64), ("smem_bytes", ctypes.c_int32),
                 ("stages", ctypes.c_int32), ("kernels", ctypes.c_int32),
-                ("workspace_bytes", ctypes.c_int64)]
+                ("workspace_bytes", ctypes.c_int64), ("split_tiles", ctypes.c_int64)]
 
 
 def _load() -> ctypes.CDLL:
@@ -116,6 +116,12 @@ def _need(t: torch.Tensor, dtype: torch.dtype, name: str, ndim: int = 2) -> None
         raise ValueError(f"{name} must be contiguous")
 
 
+def _same_device(dev: torch.device, **tensors) -> None:
+    for name, t in tensors.items():
+        if t is not None and t.device != dev:
+            raise ValueError(f"{name} is on {t.device}, the weights are on {dev}")
+
+
 def quantize(W: torch.Tensor, g: int = 128, sym: bool = False):
     """Group-wise RTN quantization of W[N, K] (bf16, cuda); g = K quantizes per
     channel (one scale and zero per row).
@@ -171,7 +177,7 @@ def plan(M: int, N: int, K: int, g: int = 128, sym: bool = False, path: str | in
     return {"path": {v: k for k, v in _PATHS.items()}[p.path], "tile_m": p.tile_m,
             "tile_n": p.tile_n, "grid": p.grid, "threads": p.threads,
             "smem_bytes": p.smem_bytes, "stages": p.stages, "kernels": p.kernels,
-            "workspace_bytes": p.workspace_bytes}
+            "workspace_bytes": p.workspace_bytes, "split_tiles": p.split_tiles}
 
 
 _workspaces: dict = {}
@@ -260,8 +266,16 @@ def gemm_decode_noalloc(X: torch.Tensor, packed: torch.Tensor, scales: torch.Ten
     M, K = X.shape
     N = packed.shape[0]
     dev = packed.device
+    if packed.shape[1] * 2 != K:
+        raise ValueError(f"packed has K={packed.shape[1] * 2}, X has K={K}")
+    _same_device(dev, X=X, scales=scales, zeros=None if sym else zeros)
     if out is None:
         out = torch.empty((M, N), dtype=torch.bfloat16, device=dev)
+    else:
+        _need(out, torch.bfloat16, "out")
+        if tuple(out.shape) != (M, N):
+            raise ValueError("out has the wrong shape")
+        _same_device(dev, out=out)
     with torch.cuda.device(dev):
         _check(lib().w4a16_gemm_decode_noalloc(_ptr(X), M, K, _ptr(packed), _ptr(scales),
                                                _ptr(zeros if not sym else None), N, g,

@@ -1,6 +1,6 @@
 // Device helpers shared by the W4A16 kernels (sm_100a only).
 //
-// Dequantization arithmetic (qwbw.cn, "推理优化中“用精度换性能“的核心技术：量化",
+// Dequantization arithmetic ("推理优化中“用精度换性能“的核心技术：量化",
 // §2.3: x̂ = (x_int − z) × s), done on bf16 pairs:
 //   a 4-bit code q placed in the low mantissa bits of the bf16 pattern 0x4300
 //   (the value 128) gives the bf16 value 128 + q exactly; subtracting the bf16
@@ -112,6 +112,20 @@ __device__ __forceinline__ uint32_t dq_pair(uint32_t a, uint32_t zz, uint32_t ss
     return bf16x2_mul(bf16x2_sub(isolate_magic<SYM>(a, 0x000F000Fu), zz), ss);
 }
 
+// A constant the compiler cannot see through: it is materialized once into a
+// register and kept there, rather than re-created next to every use.
+__device__ __forceinline__ uint32_t opaque_u32(uint32_t v) {
+    uint32_t r;
+    asm volatile("mov.b32 %0, %1;" : "=r"(r) : "r"(v));
+    return r;
+}
+
+// dq_pair with the nibble mask (0x000F000F) supplied by the caller in a register.
+template <bool SYM>
+__device__ __forceinline__ uint32_t dq_pair_m(uint32_t a, uint32_t mask, uint32_t zz, uint32_t ss) {
+    return bf16x2_mul(bf16x2_sub(isolate_magic<SYM>(a, mask), zz), ss);
+}
+
 // Eight codes of one 32-bit word (code i in nibble i) -> four bf16x2 values of
 // bf16_rn((q − z)·s), in INTERLEAVED order: (q0,q4) (q1,q5) (q2,q6) (q3,q7).
 template <bool SYM>
@@ -141,6 +155,17 @@ __device__ __forceinline__ void mma_bf16_16816(float c[4], uint32_t a0, uint32_t
                                                uint32_t a3, uint32_t b0, uint32_t b1) {
     asm volatile(
         "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 "
+        "{%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, {%0,%1,%2,%3};"
+        : "+f"(c[0]), "+f"(c[1]), "+f"(c[2]), "+f"(c[3])
+        : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
+}
+
+// The same MMA as a plain (non-volatile) asm statement: it only reads and writes
+// registers, so the compiler may schedule it freely among the shared-memory
+// loads that feed it.
+__device__ __forceinline__ void mma_bf16_16816_nv(float c[4], uint32_t a0, uint32_t a1, uint32_t a2,
+                                                  uint32_t a3, uint32_t b0, uint32_t b1) {
+    asm("mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 "
         "{%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, {%0,%1,%2,%3};"
         : "+f"(c[0]), "+f"(c[1]), "+f"(c[2]), "+f"(c[3])
         : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
@@ -229,6 +254,38 @@ __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity) {
     const uint64_t t0 = global_timer_ns();
     while (true) {
         if (mbar_try_wait_sleep(bar, parity, 20000u)) return true;
+        if (global_timer_ns() - t0 > kWaitTimeoutNs) {
+            report_error(kErrMbarTimeout);
+            return false;
+        }
+    }
+}
+
+// Non-blocking test of the phase with the given parity.
+__device__ __forceinline__ bool mbar_test_wait(uint32_t bar, uint32_t parity) {
+    uint32_t ok;
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "mbarrier.test_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t}"
+        : "=r"(ok)
+        : "r"(bar), "r"(parity)
+        : "memory");
+    return ok != 0;
+}
+
+// Wait for a phase, polling with exponentially growing sleeps (32 ns up to
+// max_sleep_ns) so that a warp that waits takes almost no issue slots from the
+// warps that compute.  For roles off the critical path (a producer refilling a
+// deep ring, a helper preparing data ahead).  Bounded like mbar_wait.
+__device__ __forceinline__ bool mbar_wait_backoff(uint32_t bar, uint32_t parity, uint32_t max_sleep_ns) {
+    if (mbar_test_wait(bar, parity)) return true;
+    const uint64_t t0 = global_timer_ns();
+    uint32_t ns = 32;
+    while (true) {
+        __nanosleep(ns);
+        if (mbar_test_wait(bar, parity)) return true;
+        ns = ns < max_sleep_ns ? 2 * ns : max_sleep_ns;
         if (global_timer_ns() - t0 > kWaitTimeoutNs) {
             report_error(kErrMbarTimeout);
             return false;

@@ -1,7 +1,8 @@
 // Prefill-path fused W4A16 GEMM (large M) on the 5th-generation tensor cores.
 //
 // Large-M work is compute bound, and there the per-use dequantization cost
-// shows (aigcbaba selection page §二: "每次都要反量化的开销会凸显"; qwbw.cn page
+// shows ("大模型推理中 Weight-only、W8A8 和 FP8 量化有什么区别？如何选型？", §二:
+// "每次都要反量化的开销会凸显"; "推理优化中“用精度换性能“的核心技术：量化",
 // §3.2).  So the dequantization runs in dedicated warps, overlapped with the
 // tensor core through a multi-stage shared-memory pipeline, and each
 // dequantized weight serves up to 256 activation rows:

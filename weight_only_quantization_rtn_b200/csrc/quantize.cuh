@@ -1,6 +1,6 @@
 // Quantize/pack and dequantize kernels (HBM-bound, one pass each).
 //
-// Quantization follows qwbw.cn, "推理优化中“用精度换性能“的核心技术：量化",
+// Quantization follows "推理优化中“用精度换性能“的核心技术：量化",
 // §2.3 (x_int = round(x/s) + z) and §3.3 (asymmetric s = (max − min)/(2^b − 1),
 // z = round(−min/s); symmetric s = max|x|/max_int, z = 0), with b = 4 and
 // groups of g elements along K (§3.4).  Arithmetic is binary32 with IEEE
@@ -131,7 +131,8 @@ __global__ void __launch_bounds__(256) quantize_pack_kernel(const uint16_t* __re
 }
 
 // Per-channel granularity (g = K: one scale, and one zero point, per output row;
-// meko1 page, 量化粒度 table; qwbw.cn page §3.4).  One CTA of 256 threads per row
+// "量化实战深入（GPTQ / AWQ / SmoothQuant / KV 量化）", 量化粒度 table;
+// "推理优化中“用精度换性能“的核心技术：量化", §3.4).  One CTA of 256 threads per row
 // and step: a first pass over the row finds its range (min/max are exact, so the
 // order of the reduction does not matter), a second pass forms the codes.  The
 // row (at most 64 KB at K = 32768) is still in L2 for the second read.

@@ -43,7 +43,8 @@ bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) ==
 bool grouped(int32_t g) { return g == 32 || g == 64 || g == 128; }
 
 // Per-channel granularity: one group spanning the whole row (g == K), one scale
-// and zero point per output feature (meko1 page, 量化粒度 table; qwbw.cn page §3.4).
+// and zero point per output feature ("量化实战深入（GPTQ / AWQ / SmoothQuant / KV 量化）", 量化粒度 table;
+// "推理优化中“用精度换性能“的核心技术：量化", §3.4).
 // Kernels take it as group size 0.
 bool per_channel(int32_t g, int64_t K) { return !grouped(g) && (int64_t)g == K; }
 
@@ -92,74 +93,121 @@ w4a16_status launch_status() {
 }
 
 // ---------------------------------------------------------------- plans
-constexpr int kSmemPerSm = 233472;        // shared memory per SM (228 KB)
 constexpr int kSmemPerBlockMax = 232448;  // opt-in maximum per CTA (227 KB)
-constexpr int kSmemReservedPerCta = 1024; // reserved by the system per resident CTA
 constexpr int kMaxCtas = 65535;
 
-// Decode kernel geometry for (M, N, K, g): 32-row x 1024-K units, a ring of
-// shared-memory stages sized to fit one or two CTAs per SM.
+// Decode kernel geometry for (M, N, K, g): 256-row x 256-K units, one CTA per
+// SM with a ring of shared-memory stages and scale slabs filling its shared
+// memory.
 struct DecodeGeometry {
     int mb;            // n8 MMA column blocks (1: M ≤ 8, 2: M ≤ 16)
-    int rb;            // row blocks of 32 rows
-    int kbn;           // K blocks of 1024
+    int rb;            // row blocks of 256 rows
+    int kbn;           // K blocks of 256
     int64_t units;     // rb · kbn
-    int stage_bytes;   // packed tile + X slice, multiple of 1024
+    int gu;            // scale groups per row per unit (1 for per-channel)
+    int sz_tma;        // scales staged by TMA in 8-group slabs (rows 16-byte aligned)
+    int slabs;         // slab ring slots (0 without TMA slabs)
+    int slab_off;      // slab ring inside the dynamic shared memory
+    int xf_off;        // fragment-ordered X inside a stage
+    int sz_off;        // scales and zeros inside a stage
+    int stage_bytes;   // multiple of 1024
     int stages;
     int ctas_per_sm;
     int smem_bytes;    // dynamic shared memory per CTA
 };
 
-int decode_fixed_smem(int mb) {
-    return kDecConsumers * 2 * mb * 128 * 4     // per-warp partial tiles
-           + 2 * kDecMaxStages * 8 + 16         // barriers and flags
-           + 1024;                              // alignment slack
-}
+// Outside the stages: zero fragments, barriers and flags (< 1024 bytes), plus
+// slack to align the dynamic shared memory base to 1024 bytes.
+constexpr int kDecFixedSmem = 1024 + 1024;
 
-// Stage: packed tile (16 KB) | X slice (M x 1024 bf16) | scales + zeros (2 x 32 x gb bf16).
-int decode_sz_offset(int64_t M) { return kDecPBytes + (int)M * 2048; }
-
-// Scale (and zero) groups of one row inside a 1024-wide K block.
+// Scale (and zero) groups of one row inside a 256-wide K block.
 int decode_unit_groups(int32_t g, int64_t K) { return per_channel(g, K) ? 1 : kDecBlockK / g; }
 
-int decode_stage_bytes(int64_t M, int gb) {
-    const int raw = decode_sz_offset(M) + 2 * kDecRows * gb * 2;
-    return (raw + 1023) / 1024 * 1024;
-}
-
+// Stage: codes tile (16 KB, TMA, 128-byte swizzle) | X slice, natural order
+// (M x 512 B, TMA) | X in fragment order (rows 576 B apart, the last one 512 B;
+// 128-byte aligned) | without TMA slabs, scales and zeros (2 x 256 rows x gu bf16).
 DecodeGeometry decode_geometry(int64_t M, int64_t N, int64_t K, int g) {
     DecodeGeometry d{};
     d.mb = M <= 8 ? 1 : 2;
     d.rb = (int)((N + kDecRows - 1) / kDecRows);
     d.kbn = (int)((K + kDecBlockK - 1) / kDecBlockK);
     d.units = (int64_t)d.rb * d.kbn;
-    d.stage_bytes = decode_stage_bytes(M, decode_unit_groups(g, K));
-    const int fixed = decode_fixed_smem(d.mb);
-    const int two = (kSmemPerSm / 2 - kSmemReservedPerCta - fixed) / d.stage_bytes;
-    if (d.mb == 1 && two >= 3) {
-        d.ctas_per_sm = 2;
-        d.stages = two < kDecMaxStages ? two : kDecMaxStages;
-    } else {
-        const int one = (kSmemPerBlockMax - fixed) / d.stage_bytes;
-        d.ctas_per_sm = 1;
-        d.stages = one < kDecMaxStages ? one : kDecMaxStages;
-    }
-    d.smem_bytes = d.stages * d.stage_bytes + fixed;
+    d.gu = decode_unit_groups(g, K);
+    d.sz_tma = (!per_channel(g, K) && (K / g) % 8 == 0) ? 1 : 0;
+    const int m = M < 1 ? 1 : (int)M;
+    const int xnat_end = kDecPBytes + m * kDecXRowBytes;
+    d.xf_off = (xnat_end + 127) / 128 * 128;
+    const int xf_end = d.xf_off + (m - 1) * kDecXfRowBytes + kDecXRowBytes;
+    d.sz_off = (xf_end + 127) / 128 * 128;      // TMA destinations are 128-byte aligned
+    // Scales in the stage only without TMA slabs; with them, a ring of slab slots.
+    const int stage_raw = d.sz_off + (d.sz_tma ? 0 : 2 * kDecRows * d.gu * 2);
+    d.stage_bytes = (stage_raw + 1023) / 1024 * 1024;
+    // Slab slots: one the consumers read, plus enough for the units the producer
+    // may run ahead (the ring depth) at 8/gu units per slab, plus one for a slab
+    // boundary in between; at least 2, at most one per stage plus one.
+    const int ups = d.sz_tma ? 8 / d.gu : 1;
+    auto slabs_for = [&](int stages) {
+        if (!d.sz_tma) return 0;
+        int sl = (stages + 1 + ups - 1) / ups + 1;
+        if (sl > stages + 1) sl = stages + 1;
+        if (sl < 2) sl = 2;
+        if (sl > kDecMaxSlabs) sl = kDecMaxSlabs;
+        return sl;
+    };
+    auto fits = [&](int stages, int budget) {
+        return stages * d.stage_bytes + slabs_for(stages) * kDecSlabBytes <= budget;
+    };
+    // One CTA per SM (16 consumer warps; two such CTAs would not fit the registers).
+    int one = 0;
+    while (one < kDecMaxStages && fits(one + 1, kSmemPerBlockMax - kDecFixedSmem)) ++one;
+    d.ctas_per_sm = 1;
+    d.stages = one;
+    d.slabs = slabs_for(d.stages);
+    d.slab_off = d.stages * d.stage_bytes;
+    d.smem_bytes = d.slab_off + d.slabs * kDecSlabBytes + kDecFixedSmem;
     return d;
 }
 
-// Workspace: (rb + ctas) fp32 partial row blocks of 256·MB values; slot rb + c
-// holds CTA c's part of a row block that the stream-K partition splits.  It is
-// scratch: no initialization is needed and nothing survives a call.
-int64_t decode_workspace_bytes(const DecodeGeometry& d, int64_t ctas) {
-    return (int64_t)(d.rb + ctas) * 256 * d.mb * 4;
+// The stage layout's invariants: every TMA destination (codes, X, scale and zero
+// slabs) 128-byte aligned, the codes tile 1024-byte aligned (128-byte swizzle),
+// the fragment-ordered X 128-byte aligned (bank spread of the consumers' loads),
+// and the ring within the shared memory of one CTA.
+bool decode_geometry_ok(const DecodeGeometry& d, int64_t M) {
+    const int m = M < 1 ? 1 : (int)M;
+    const int sw = d.sz_tma ? 0 : d.gu;        // scales in the stage only without slabs
+    return d.stage_bytes % 1024 == 0 && kDecPBytes % 128 == 0 && d.xf_off % 128 == 0 &&
+           d.xf_off >= kDecPBytes + m * kDecXRowBytes && d.sz_off % 128 == 0 &&
+           d.sz_off >= d.xf_off + (m - 1) * kDecXfRowBytes + kDecXRowBytes &&
+           (kDecRows * sw * 2) % 128 == 0 && d.sz_off + 2 * kDecRows * sw * 2 <= d.stage_bytes &&
+           d.stages >= 2 && d.stages <= kDecMaxStages && d.slab_off % 1024 == 0 &&
+           (d.sz_tma ? d.slabs >= 2 && d.slabs <= kDecMaxSlabs : d.slabs == 0) &&
+           kDecSlabBytes % 1024 == 0 && d.smem_bytes <= kSmemPerBlockMax;
 }
 
-// True if some boundary of the even unit split falls inside a row block.
-bool decode_has_split(const DecodeGeometry& d, int64_t ctas) {
-    for (int64_t b = 1; b < ctas; ++b)
-        if ((b * d.units / ctas) % d.kbn != 0) return true;
-    return false;
+// Workspace of a decode launch with `ctas` CTAs: (rb + ctas) slots, slot rb + c
+// holding CTA c's part of a row block that the stream-K partition splits —
+// per slot 16 ready flags, then 16 warps x 32 lanes x 4·mb fp32 partial sums.
+// Scratch: no initialization is needed (a flag counts only when it holds the
+// ready pattern, which the consuming CTA clears again).
+int64_t decode_flag_bytes(const DecodeGeometry& d, int64_t ctas) {
+    return ((int64_t)(d.rb + ctas) * kDecConsumers * 4 + 255) / 256 * 256;
+}
+
+int64_t decode_workspace_bytes(const DecodeGeometry& d, int64_t ctas) {
+    return decode_flag_bytes(d, ctas) + (int64_t)(d.rb + ctas) * kDecConsumers * 32 * 16 * d.mb;
+}
+
+// Row blocks the even unit split cuts between CTAs.
+int64_t decode_split_blocks(const DecodeGeometry& d, int64_t ctas) {
+    int64_t n = 0, last = -1;
+    for (int64_t b = 1; b < ctas; ++b) {
+        const int64_t u = b * d.units / ctas;
+        if (u % d.kbn != 0 && u / d.kbn != last) {
+            ++n;
+            last = u / d.kbn;
+        }
+    }
+    return n;
 }
 
 int tc_tile_m(int64_t M) {
@@ -262,7 +310,12 @@ w4a16_status make_plan(int64_t M, int64_t N, int64_t K, int32_t g, int32_t sym, 
     p->path = chosen;
     if (chosen == W4A16_PATH_DECODE) {
         const DecodeGeometry d = decode_geometry(M, N, K, g);
-        int64_t grid = ctas > 0 ? ctas : (int64_t)sm_count * d.ctas_per_sm;
+        if (!decode_geometry_ok(d, M)) return W4A16_EUNSUPPORTED;
+        // At most one resident wave: the CTA that finishes a split row block waits
+        // for parts from its neighbours, which must be running too.
+        const int64_t resident = (int64_t)sm_count * d.ctas_per_sm;
+        int64_t grid = ctas > 0 ? ctas : resident;
+        if (grid > resident) grid = resident;
         if (grid > d.units) grid = d.units;
         if (grid < 1) grid = 1;
         p->tile_m = 8 * d.mb;
@@ -271,7 +324,8 @@ w4a16_status make_plan(int64_t M, int64_t N, int64_t K, int32_t g, int32_t sym, 
         p->threads = kDecThreads;
         p->smem_bytes = d.smem_bytes;
         p->stages = d.stages;
-        p->kernels = decode_has_split(d, grid) ? 2 : 1;
+        p->kernels = 1;
+        p->split_tiles = decode_split_blocks(d, grid);
         p->workspace_bytes = decode_workspace_bytes(d, grid);
     } else {
         const int bm = tc_tile_m(M);
@@ -283,6 +337,7 @@ w4a16_status make_plan(int64_t M, int64_t N, int64_t K, int32_t g, int32_t sym, 
         if (bits == 8) tc_smem_and_stages<8>(bm, &p->smem_bytes, &p->stages);
         else tc_smem_and_stages<4>(bm, &p->smem_bytes, &p->stages);
         p->kernels = (ts.head > 0 ? 1 : 0) + (ts.tail > 0 ? 2 : 0);
+        p->split_tiles = ts.tail;
         p->workspace_bytes = ts.tail > 0 ? (int64_t)ts.splits * ts.tail * bm * kTcTileN * 4 : 0;
     }
     return W4A16_OK;
@@ -316,8 +371,8 @@ w4a16_status encode_2d(CUtensorMap* map, CUtensorMapDataType dtype, const void* 
 // ---------------------------------------------------------------- decode launch
 template <int MB, bool SYM, int G>
 w4a16_status launch_decode_t(const w4a16_plan& p, const CUtensorMap& tmP, const CUtensorMap& tmX,
-                             const CUtensorMap& tmS, const CUtensorMap& tmZ, const DecodeArgs& args,
-                             bool has_split, cudaStream_t stream) {
+                             const CUtensorMap& tmS, const CUtensorMap& tmZ,
+                             const DecodeArgs& args, cudaStream_t stream) {
     auto kern = gemv_decode_kernel<MB, SYM, G>;
     static bool attr_set[kMaxDevices] = {};
     int dev = 0;
@@ -342,15 +397,16 @@ w4a16_status launch_decode_t(const w4a16_plan& p, const CUtensorMap& tmP, const 
     cfg.attrs = attr;
     cfg.numAttrs = 1;
     if (cudaLaunchKernelEx(&cfg, kern, tmP, tmX, tmS, tmZ, args) != cudaSuccess) return W4A16_ECUDA;
-    if (has_split) {
-        cudaLaunchConfig_t fcfg = cfg;
-        fcfg.gridDim = dim3((unsigned)(p.grid - 1), 1, 1);
-        fcfg.blockDim = dim3(256, 1, 1);
-        fcfg.dynamicSmemBytes = 0;
-        if (cudaLaunchKernelEx(&fcfg, decode_fixup_kernel<MB>, args, (int64_t)p.grid) != cudaSuccess)
-            return W4A16_ECUDA;
-    }
     return W4A16_OK;
+}
+
+// Bytes per scale copy for grouped scales: the largest of 16, 8, 4 that divides
+// both a unit's scale bytes per row (gu·2) and the scale row stride (K/g·2), so
+// that copies are aligned and never cross the end of a row; 2 = plain loads.
+int decode_scale_copy(int gu, int64_t groups) {
+    for (int cs = 16; cs >= 4; cs /= 2)
+        if (cs <= gu * 2 && (gu * 2) % cs == 0 && (groups * 2) % cs == 0) return cs;
+    return 2;
 }
 
 w4a16_status launch_decode(const w4a16_plan& p, const void* X, int64_t M, int64_t K,
@@ -359,53 +415,56 @@ w4a16_status launch_decode(const w4a16_plan& p, const void* X, int64_t M, int64_
     const DecodeGeometry d = decode_geometry(M, N, K, g);
     CUtensorMap tmP, tmX;
     w4a16_status st = encode_2d(&tmP, CU_TENSOR_MAP_DATA_TYPE_UINT8, packed, (uint64_t)(K / 2),
-                                (uint64_t)N, (uint64_t)(K / 2), 128, kDecRows,
+                                (uint64_t)N, (uint64_t)(K / 2), kDecBlockK / 2, kDecRows,
                                 CU_TENSOR_MAP_SWIZZLE_128B);
     if (st != W4A16_OK) return st;
     st = encode_2d(&tmX, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, X, (uint64_t)K, (uint64_t)M,
-                   (uint64_t)K * 2, 256, (uint32_t)M, CU_TENSOR_MAP_SWIZZLE_NONE);
+                   (uint64_t)K * 2, kDecBlockK, (uint32_t)M, CU_TENSOR_MAP_SWIZZLE_NONE);
     if (st != W4A16_OK) return st;
+    const bool pc = per_channel(g, K);
     DecodeArgs args{};
     args.scales = static_cast<const uint16_t*>(scales);
     args.zeros = static_cast<const uint16_t*>(zeros);
     args.Y = static_cast<uint16_t*>(Y);
-    args.ws_part = static_cast<float*>(workspace);
+    args.ws_flag = static_cast<uint32_t*>(workspace);
+    args.ws_part = reinterpret_cast<float*>(static_cast<uint8_t*>(workspace) +
+                                            decode_flag_bytes(d, p.grid));
     args.M = (int)M;
     args.N = (int)N;
     args.K = (int)K;
     args.RB = d.rb;
     args.KBn = d.kbn;
+    args.Gtot = pc ? 1 : (int)(K / g);
     args.stages = d.stages;
     args.stage_bytes = d.stage_bytes;
-    args.sz_offset = decode_sz_offset(M);
-    const bool pc = per_channel(g, K);             // scales [N]: the kernel copies 16-byte runs
-    args.sz_async = (!pc && (K / g) % 2 == 0) ? 1 : 0;   // 4-byte aligned scale rows
-    args.sz_tma = (!pc && (K / g) % 8 == 0) ? 1 : 0;     // 16-byte aligned scale rows
-    args.U = d.units;
-    const bool split = p.kernels > 1;
-    // Scales and zeros [N][K/g]: boxes of 32 rows x (1024/g) groups, when their rows are
+    args.xf_off = d.xf_off;
+    args.sz_off = d.sz_off;
+    args.sz_tma = d.sz_tma;
+    args.slab_off = d.slab_off;
+    args.slabs = d.slabs;
+    args.sz_copy = pc ? 16 : decode_scale_copy(d.gu, K / g);
+    // Scales and zeros [N][K/g] in slabs of 8 groups x 256 rows, when their rows are
     // 16-byte aligned; otherwise the kernel copies them with cp.async and these are unused.
     CUtensorMap tmS = tmP, tmZ = tmP;
-    if (args.sz_tma) {
-        st = encode_2d(&tmS, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, scales, (uint64_t)(K / g),
-                       (uint64_t)N, (uint64_t)(K / g) * 2, (uint32_t)(kDecBlockK / g), kDecRows,
-                       CU_TENSOR_MAP_SWIZZLE_NONE);
+    if (d.sz_tma) {
+        st = encode_2d(&tmS, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, scales, (uint64_t)(K / g), (uint64_t)N,
+                       (uint64_t)(K / g) * 2, 8, kDecRows, CU_TENSOR_MAP_SWIZZLE_NONE);
         if (st != W4A16_OK) return st;
         if (!sym) {
-            st = encode_2d(&tmZ, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, zeros, (uint64_t)(K / g),
-                           (uint64_t)N, (uint64_t)(K / g) * 2, (uint32_t)(kDecBlockK / g), kDecRows,
-                           CU_TENSOR_MAP_SWIZZLE_NONE);
+            st = encode_2d(&tmZ, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, zeros, (uint64_t)(K / g), (uint64_t)N,
+                           (uint64_t)(K / g) * 2, 8, kDecRows, CU_TENSOR_MAP_SWIZZLE_NONE);
             if (st != W4A16_OK) return st;
         }
     }
+    args.U = d.units;
     const int gsel = pc ? 0 : g;                   // kernel group size, 0 = per-channel
-#define W4A16_DEC_G(MBV, SYMV)                                                                  \
-    switch (gsel) {                                                                             \
-        case 32: return launch_decode_t<MBV, SYMV, 32>(p, tmP, tmX, tmS, tmZ, args, split, stream); \
-        case 64: return launch_decode_t<MBV, SYMV, 64>(p, tmP, tmX, tmS, tmZ, args, split, stream); \
-        case 128: return launch_decode_t<MBV, SYMV, 128>(p, tmP, tmX, tmS, tmZ, args, split, stream); \
-        case 0: return launch_decode_t<MBV, SYMV, 0>(p, tmP, tmX, tmS, tmZ, args, split, stream);   \
-        default: return W4A16_EINVAL;                                                           \
+#define W4A16_DEC_G(MBV, SYMV)                                                          \
+    switch (gsel) {                                                                     \
+        case 32: return launch_decode_t<MBV, SYMV, 32>(p, tmP, tmX, tmS, tmZ, args, stream);     \
+        case 64: return launch_decode_t<MBV, SYMV, 64>(p, tmP, tmX, tmS, tmZ, args, stream);     \
+        case 128: return launch_decode_t<MBV, SYMV, 128>(p, tmP, tmX, tmS, tmZ, args, stream);   \
+        case 0: return launch_decode_t<MBV, SYMV, 0>(p, tmP, tmX, tmS, tmZ, args, stream);       \
+        default: return W4A16_EINVAL;                                                   \
     }
     if (d.mb == 1) {
         if (sym) W4A16_DEC_G(1, true)

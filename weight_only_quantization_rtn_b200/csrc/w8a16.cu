@@ -1,9 +1,9 @@
 // W8A16: the 8-bit form of weight-only RTN quantization, one code per byte.
 //
-// The quantization page (qwbw.cn, "推理优化中“用精度换性能“的核心技术：量化")
+// The page "推理优化中“用精度换性能“的核心技术：量化"
 // states the INT8 form directly in §3.3: asymmetric s = (max − min)/255,
-// z = round(−min/s); symmetric s = max|x|/max_int with max_int = 127 (meko1
-// page §二, absmax with b = 8).  The aigcbaba page (详细版) lists W8A16 beside
+// z = round(−min/s); symmetric s = max|x|/max_int with max_int = 127 ("量化实战深入（GPTQ / AWQ / SmoothQuant / KV 量化）"
+// §二, absmax with b = 8).  "大模型推理中 Weight-only、W8A8 和 FP8 量化有什么区别？如何选型？" (详细版) lists W8A16 beside
 // W4A16.  Readings as for INT4: round half to even in binary32, s rounded to
 // bf16 before z and q, the asymmetric range widened to contain 0, codes clamped
 // to [0, 255] or [−128, 127] (symmetric codes stored as int8), x̂ =

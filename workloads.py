@@ -11,8 +11,8 @@ layers; no model weights or datasets are used, these draws stand in for them):
     (columns of W) multiplied by a factor (weight outliers);
   * activations X[M, K] ~ N(0, 1), optionally with a fraction of channels either
     multiplied by a factor or set to sign(x)·value (activation outliers of
-    magnitude ≈100, the "|x|≈1 vs |x|≈100" example of the Weight-only/W8A8/FP8
-    selection page, §三).
+    magnitude ≈100, the "|x|≈1 vs |x|≈100" example of "大模型推理中 Weight-only、
+    W8A8 和 FP8 量化有什么区别？如何选型？", §三).
 Outlier channel sets are ``randperm(K)[:round(frac·K)]`` from the same stream.
 """
 from __future__ import annotations
