@@ -1,23 +1,26 @@
 """Benchmark of the W4A16 fused GEMM on B200.
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
-                    [--workload decode7b|decode70b|prefill|decode7b_pc|prefill_pc]
+                    [--workload decode70b|decode70b_sym|decode7b|prefill|decode7b_pc|prefill_pc]
                     [--no-extras] [--no-cpu-baseline] [--crossover]
 
 Metric: W4A16 GEMM HBM GB/s at M=1 and TFLOPS at M=2048, as % of the B200
 roofline.  The headline line (default workload) is the M=1 decode of the two
-Llama-2-7B-shaped layers (K=4096,N=11008 and K=11008,N=4096; g=128, asym):
-one step = both fused GEMMs, through the library's dispatch, on synthetic
-seeded weights/activations of that shape.  `value` is algorithmic bytes per
-step (packed weights + scales + zeros + X read once + Y written once) times
-steps, over the device time of the timed region, summed over ranks and
-divided by the max over ranks.  The same JSON line carries the M=2048 prefill
-TFLOPS (K=N=8192) with its tensor-core roofline, a dense bf16 cuBLAS GEMM and
-the unfused dequantize-then-GEMM at the same shapes, the end-to-end number
-through the public API with host buffers, and the host oracle on the CPU.
-Extras on the same line: standalone quantize/dequantize bandwidth, the
-per-channel (g = K) decode and prefill, and the W8A16 (8-bit code) quantize,
-dequantize and M=1 GEMV.
+Llama-2-70B-shaped layers (K=8192,N=28672 and K=28672,N=8192; g=128, asym),
+the largest single-GPU M=1 configuration: one step = both fused GEMMs,
+through the library's dispatch, on synthetic seeded weights/activations of
+that shape.  `value` is algorithmic bytes per step (packed weights + scales +
+zeros + X read once + Y written once) times steps, over the device time of the
+timed region, summed over ranks and divided by the max over ranks.  The same
+JSON line carries, each with its own roofline object, the other M=1 decode
+workloads (the 70B-shaped layers with symmetric codes, the 7B-shaped layers),
+the M=2048 prefill TFLOPS (K=N=8192) against the tensor-core roofline, dense
+bf16 cuBLAS and the unfused dequantize-then-GEMM at the same shapes, the
+crossover sweep (K=N=8192, every M, g and mode, each kernel the dispatch can
+choose), the end-to-end number through the public API with host buffers, and
+the host oracle on the CPU.  Further extras: standalone quantize/dequantize
+bandwidth, the per-channel (g = K) decode and prefill, and the W8A16 (8-bit
+code) quantize, dequantize, M=1 GEMV and M=2048 GEMM.
 
 Timing: W warm-up steps, then exactly K steps replayed from CUDA graphs (one
 graph holds a full rotation over the weight copies, so graph launches are
@@ -446,14 +449,15 @@ WORKLOAD_DEFS = {
     # name: (workload, M, g, sym, metric half); g = 0: per-channel (g = K)
     "decode7b": (workloads.DECODE_7B, 1, 128, False, "hbm"),
     "decode70b": (workloads.DECODE_70B, 1, 128, False, "hbm"),
+    "decode70b_sym": (workloads.DECODE_70B, 1, 128, True, "hbm"),
     "prefill": (workloads.PREFILL, 2048, 128, False, "tensor"),
     "decode7b_pc": (workloads.DECODE_7B, 1, 0, False, "hbm"),
     "prefill_pc": (workloads.PREFILL, 2048, 0, False, "tensor"),
 }
 
 
-def workload_name(wl, M, g) -> str:
-    return f"{wl.name}_M{M}" + ("_per_channel" if g == 0 else "")
+def workload_name(wl, M, g, sym=False) -> str:
+    return f"{wl.name}_M{M}" + ("_per_channel" if g == 0 else "") + ("_sym" if sym else "")
 
 
 def run_ours(args):
@@ -514,7 +518,7 @@ def run_ours(args):
         "warmup": args.warmup, "ms_per_step": ms_max / args.steps, "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
         "config": {
-            "workload": workload_name(wl, M, g), "M": M,
+            "workload": workload_name(wl, M, g, sym), "M": M,
             "layers_KxN": [[l.K, l.N] for l in wl.layers], "g": g if g else "K (per-channel)",
             "mode": "sym" if sym else "asym", "description": wl.description,
             "l2": f"{copies} rotating copies of weights+activations "
@@ -530,14 +534,17 @@ def run_ours(args):
 
     # ------------------------------------------------ end to end through the public API
     pinned = [c.X[0].cpu().pin_memory() for c in cases]
+    host_y = [torch.empty(c.M, c.N, dtype=torch.bfloat16, pin_memory=True) for c in cases]
     h2d = sum(x.numel() * 2 for x in pinned)
     d2h = sum(c.M * c.N * 2 for c in cases)
-    e2e_steps = min(args.steps, 200)
+    e2e_steps = min(args.steps, 2000)
 
     def e2e_step(i):
-        for c, xh in zip(cases, pinned):
+        # host X in, host Y out for every layer; the step waits once, for its last copy
+        for c, xh, yh in zip(cases, pinned, host_y):
             j = i % copies
-            w4.gemm(xh, c.P[j], c.S[j], c.Z[j], c.g, c.sym)   # host X in, host Y out
+            w4.gemm(xh, c.P[j], c.S[j], c.Z[j], c.g, c.sym, out=yh, sync=False)
+        torch.cuda.current_stream().synchronize()
 
     for i in range(args.warmup):
         e2e_step(i)
@@ -569,11 +576,15 @@ def run_ours(args):
         else:
             roof["frac_of_nominal"] = roof["achieved"] / NOMINAL_BF16_TFLOPS
         if args.workload != "prefill":
+            others = [n for n in ("decode70b", "decode70b_sym", "decode7b") if n != args.workload]
+            line["decode_workloads"] = workload_extras(w4, others, peaks, peak_src, l2, dev)
             line["prefill"] = prefill_extra(w4, peaks, peak_src, l2, dev)
             pr = line["prefill"]["roofline"]
             pr["frac_of_nominal"] = pr["achieved"] / NOMINAL_BF16_TFLOPS
+            line["crossover"] = crossover_rows(w4, dev, l2)
             line["quantize_dequantize"] = elementwise_extras(w4, peaks, l2, dev)
-            line["per_channel"] = per_channel_extras(w4, peaks, peak_src, l2, dev)
+            line["per_channel"] = workload_extras(w4, ["decode7b_pc", "prefill_pc"], peaks, peak_src,
+                                                  l2, dev)
             line["w8a16"] = w8a16_extras(w4, peaks, l2, dev)
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         cb = cpu_baseline(wl.layers, M, g, sym, unit_bytes=(half == "hbm")) \
@@ -640,19 +651,21 @@ def elementwise_extras(w4, peaks, l2, dev, iters=20):
             "dequantize": {"us": dms * 1e3, "GB/s": db / (dms / 1e3) / 1e9, "frac": db / (dms / 1e3) / 1e9 / pk}}
 
 
-def per_channel_extras(w4, peaks, peak_src, l2, dev, iters=200):
-    """Per-channel granularity (g = K: one scale and zero per output row) on the
-    7B-shaped decode layers at M=1 and on the prefill shape, timed like the
-    headline: rotation graphs over copies larger than L2, CUDA events on the
-    replay stream.  Bytes per GEMM count one scale (and zero) per row."""
+def workload_extras(w4, names, peaks, peak_src, l2, dev, decode_iters=400, tensor_iters=30):
+    """Other workloads of WORKLOAD_DEFS measured like the headline — rotation
+    graphs over copies larger than L2, CUDA events on the replay stream — each
+    with its own roofline object (achieved = the workload's algorithmic bytes or
+    FLOPs per step over the time per step; traffic from the committed ncu table
+    when it matches the kernel's current source).  Per-channel workloads count
+    one scale (and zero) per row."""
     out = {}
-    for name in ("decode7b_pc", "prefill_pc"):
+    for name in names:
         wl, M, g, sym, half = WORKLOAD_DEFS[name]
-        in_bytes = sum(input_bytes(M, l.N, l.K, l.K, sym) for l in wl.layers)
+        in_bytes = sum(input_bytes(M, l.N, l.K, group_of(g, l.K), sym) for l in wl.layers)
         copies = copies_for(in_bytes, l2)
-        cases = [GemmCase(w4, l, M, l.K, sym, copies, dev) for l in wl.layers]
+        cases = [GemmCase(w4, l, M, group_of(g, l.K), sym, copies, dev) for l in wl.layers]
         rot, singles = capture_rotation_graph(w4, cases, copies)
-        n = iters if half == "hbm" else 30
+        n = decode_iters if half == "hbm" else tensor_iters
         replay_steps(rot, singles, copies, 3)
         torch.cuda.synchronize()
         a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
@@ -661,6 +674,7 @@ def per_channel_extras(w4, peaks, peak_src, l2, dev, iters=200):
         b.record()
         b.synchronize()
         ms = a.elapsed_time(b) / n
+        kms = per_layer_ms(w4, cases, copies, reps=20 if half == "hbm" else 5)
         plans = [w4.plan(M, c.N, c.K, c.g, sym) for c in cases]
         kernel = "gemv_decode_kernel" if plans[0]["path"] == "decode" else "gemm_tc_kernel"
         if half == "hbm":
@@ -669,11 +683,15 @@ def per_channel_extras(w4, peaks, peak_src, l2, dev, iters=200):
         else:
             work = sum(c.flops for c in cases)
             ach, pk, unit = work / (ms / 1e3) / 1e12, peaks["bf16_tflops"], "TFLOP/s"
-        out[name] = {"workload": workload_name(wl, M, g), "ms_per_step": ms,
+        out[name] = {"workload": workload_name(wl, M, g, sym), "ms_per_step": ms, "value": ach,
+                     "unit": unit,
                      "roofline": {"bound": "hbm" if half == "hbm" else "tensor", "achieved": ach,
                                   "peak": pk, "unit": unit, "frac": ach / pk,
                                   "peak_source": peak_src + ("" if half == "hbm" else " (burst)"),
-                                  "traffic": ncu_traffic(f"{kernel}:{name}"), "kernel": kernel},
+                                  "traffic": ncu_traffic(f"{kernel}:{name}"), "kernel": kernel,
+                                  "avg_launch_us": ms / len(cases) * 1e3,
+                                  "per_layer_us_alone": [round(x * 1e3, 3) for x in kms],
+                                  "algorithmic_bytes_per_launch": [c.bytes for c in cases]},
                      "plan": plans}
         del rot, singles, cases
         torch.cuda.empty_cache()
@@ -830,35 +848,33 @@ def prefill_extra(w4, peaks, peak_src, l2, dev, iters=50):
     return res
 
 
-def crossover_sweep(args):
-    """M-dispatch evidence: at K=N=8192 time each kernel that can run each M
-    (decode for M <= 16, tensor-core for every M) and a dense bf16 cuBLAS GEMM
-    of the same shape, with inputs rotated over copies larger than L2.  Prints
-    one JSON object {"crossover": [...]}; not a benchmark line."""
-    import weight_only_quantization_rtn_b200 as w4
-    from weight_only_quantization_rtn_b200 import build as w4build
-    w4build.build()
-    w4.lib()
-    dev = torch.device("cuda", 0)
-    props = torch.cuda.get_device_properties(dev)
-    l2 = getattr(props, "L2_cache_size", 0) or L2_BYTES_FALLBACK
+CROSSOVER_MODES = ((128, False), (128, True), (64, False), (64, True), (32, False), (32, True))
+
+
+def crossover_rows(w4, dev, l2, iters=40, iters_large=12):
+    """M-dispatch evidence at K=N=8192 (the crossover workload): for every M, g
+    and mode, the time of each kernel that can run it (the decode kernel for
+    M <= 16, the tensor-core kernel for every M), which one the dispatch takes,
+    and — for g=128 asym — a dense bf16 cuBLAS GEMM of the same shape; inputs
+    rotate over copies larger than L2.  Rows: {g, mode, M, dispatch, decode_us,
+    tensorcore_us, dense_bf16_cublas_us, fastest, ...}."""
     layer = workloads.CROSSOVER.layers[0]
     N, K = layer.N, layer.K
     W = layer.weight().to(dev)
     rows = []
-    for g, sym in ((128, False), (128, True), (64, False), (32, False)):
+    for g, sym in CROSSOVER_MODES:
         P, S, Z = w4.quantize(W, g, sym)
         wbytes = N * K // 2 + 2 * N * (K // g) * (1 if sym else 2)
+        copies = copies_for(wbytes, l2)
+        Ps = [P] + [P.clone() for _ in range(copies - 1)]
+        Ss = [S] + [S.clone() for _ in range(copies - 1)]
+        Zs = [Z] + [Z.clone() for _ in range(copies - 1)]
         for M in workloads.CROSSOVER.Ms:
-            copies = copies_for(wbytes + 2 * M * K, l2)
-            Ps = [P] + [P.clone() for _ in range(copies - 1)]
-            Ss = [S] + [S.clone() for _ in range(copies - 1)]
-            Zs = [Z] + [Z.clone() for _ in range(copies - 1)]
             X = layer.activation(M).to(dev)
             Xs = [X] + [X.clone() for _ in range(copies - 1)]
             Y = torch.empty(M, N, dtype=torch.bfloat16, device=dev)
-            iters = 40 if M <= 1024 else 12
-            row = {"g": g, "mode": "sym" if sym else "asym", "M": M, "N": N, "K": K,
+            n = iters if M <= 1024 else iters_large
+            row = {"g": g, "mode": "sym" if sym else "asym", "M": M,
                    "dispatch": w4.plan(M, N, K, g, sym)["path"],
                    "algorithmic_bytes": algorithmic_bytes(M, N, K, g, sym), "flops": 2 * M * N * K}
             for path in ("decode", "tensorcore"):
@@ -867,7 +883,7 @@ def crossover_sweep(args):
                 gs = graph_of(lambda i, path=path: w4.gemm(Xs[i % copies], Ps[i % copies],
                                                            Ss[i % copies], Zs[i % copies], g, sym,
                                                            path=path, out=Y), copies)
-                row[path + "_us"] = time_graphs(gs, iters) * 1e3
+                row[path + "_us"] = round(time_graphs(gs, n) * 1e3, 3)
                 del gs
             if g == 128 and not sym:
                 dcopies = max(2, -(-2 * l2 // (N * K * 2 + 2 * M * K)) + 1)
@@ -875,15 +891,32 @@ def crossover_sweep(args):
                 Xd = Xs[:1] + [X.clone() for _ in range(dcopies - 1)]
                 gs = graph_of(lambda i: torch.matmul(Xd[i % dcopies], Wd[i % dcopies].t(), out=Y),
                               dcopies)
-                row["dense_bf16_cublas_us"] = time_graphs(gs, iters) * 1e3
+                row["dense_bf16_cublas_us"] = round(time_graphs(gs, n) * 1e3, 3)
                 del gs, Wd, Xd
             cand = {k[:-3]: v for k, v in row.items() if k in ("decode_us", "tensorcore_us")}
             row["fastest"] = min(cand, key=cand.get)
+            t = row[row["dispatch"] + "_us"] * 1e-6
+            row["dispatched_GBps"] = round(row["algorithmic_bytes"] / t / 1e9, 1)
+            row["dispatched_TFLOPs"] = round(row["flops"] / t / 1e12, 2)
             rows.append(row)
-            del Ps, Ss, Zs, Xs, X, Y
+            del Xs, X, Y
             torch.cuda.empty_cache()
-        del P, S, Z
-    print(json.dumps({"crossover": rows}))
+        del P, S, Z, Ps, Ss, Zs
+        torch.cuda.empty_cache()
+    return rows
+
+
+def crossover_sweep(args):
+    """Print the crossover rows as one JSON object {"crossover": [...]}; not a
+    benchmark line."""
+    import weight_only_quantization_rtn_b200 as w4
+    from weight_only_quantization_rtn_b200 import build as w4build
+    w4build.build()
+    w4.lib()
+    dev = torch.device("cuda", 0)
+    props = torch.cuda.get_device_properties(dev)
+    l2 = getattr(props, "L2_cache_size", 0) or L2_BYTES_FALLBACK
+    print(json.dumps({"crossover": crossover_rows(w4, dev, l2)}))
 
 
 def run_reference(args):
@@ -924,7 +957,7 @@ def run_reference(args):
             "steps": steps, "warmup": args.warmup, "ms_per_step": el / steps * 1e3,
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
             "data": "synthetic",
-            "config": {"workload": workload_name(wl, M, g), "M": M,
+            "config": {"workload": workload_name(wl, M, g, sym), "M": M,
                        "layers_KxN": [[l.K, l.N] for l in wl.layers],
                        "g": g if g else "K (per-channel)",
                        "mode": "sym" if sym else "asym"},
@@ -941,7 +974,7 @@ def main():
     ap.add_argument("--steps", type=int, default=50000)
     ap.add_argument("--warmup", type=int, default=50)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
-    ap.add_argument("--workload", choices=sorted(WORKLOAD_DEFS), default="decode7b")
+    ap.add_argument("--workload", choices=sorted(WORKLOAD_DEFS), default="decode70b")
     ap.add_argument("--no-extras", action="store_true",
                     help="skip comparisons and the prefill half (profiling runs)")
     ap.add_argument("--no-cpu-baseline", action="store_true")

@@ -209,14 +209,31 @@ def _workspace(dev: torch.device, nbytes: int):
     return ws
 
 
+_dev_bufs: dict = {}
+
+
+def _device_buffer(dev: torch.device, M: int, N: int) -> torch.Tensor:
+    """A device Y buffer per (device, stream, shape) for calls whose result goes
+    to host memory; calls on one stream are ordered, so they can share it."""
+    key = (dev, torch.cuda.current_stream(dev).cuda_stream, M, N)
+    buf = _dev_bufs.get(key)
+    if buf is None:
+        buf = torch.empty((M, N), dtype=torch.bfloat16, device=dev)
+        _dev_bufs[key] = buf
+    return buf
+
+
 def gemm(X: torch.Tensor, packed: torch.Tensor, scales: torch.Tensor,
          zeros: torch.Tensor | None, g: int = 128, sym: bool = False, path: str | int = "auto",
-         ctas: int = 0, out: torch.Tensor | None = None) -> torch.Tensor:
+         ctas: int = 0, out: torch.Tensor | None = None, sync: bool = True) -> torch.Tensor:
     """Fused W4A16 GEMM: Y[M, N] = X[M, K] · Ŵ[N, K]ᵀ (bf16 in/out, fp32 accumulation).
 
     If X lives in host memory (ideally pinned) it is copied to the weights'
-    device and Y is copied back into pinned host memory, waiting for the copy:
-    the end-to-end form of the call."""
+    device and Y is copied back into host memory — ``out`` when given (a pinned
+    bf16 [M, N] host tensor), else new pinned memory: the end-to-end form of the
+    call.  With ``sync`` (the default) the call waits for that copy; with
+    ``sync=False`` it returns at once and the caller synchronizes the current
+    stream before reading Y (e.g. once per step of several calls)."""
     host_in = not X.is_cuda
     dev = packed.device
     Xd = X.to(dev, non_blocking=True) if host_in else X
@@ -229,12 +246,22 @@ def gemm(X: torch.Tensor, packed: torch.Tensor, scales: torch.Tensor,
     N = packed.shape[0]
     if packed.shape[1] * 2 != K:
         raise ValueError(f"packed has K={packed.shape[1] * 2}, X has K={K}")
-    if out is None:
+    _same_device(dev, X=Xd, scales=scales, zeros=None if sym else zeros)
+    host_out = None
+    if host_in:
+        if out is not None:
+            if out.is_cuda or out.dtype != torch.bfloat16 or tuple(out.shape) != (M, N) \
+                    or not out.is_contiguous():
+                raise ValueError("out must be a contiguous bf16 [M, N] host tensor when X is on the host")
+            host_out = out
+        out = _device_buffer(dev, M, N)
+    elif out is None:
         out = torch.empty((M, N), dtype=torch.bfloat16, device=dev)
     else:
         _need(out, torch.bfloat16, "out")
         if tuple(out.shape) != (M, N):
             raise ValueError("out has the wrong shape")
+        _same_device(dev, out=out)
     pid = _PATHS[path] if isinstance(path, str) else int(path)
     with torch.cuda.device(dev):
         ws_bytes = _workspace_bytes(dev, M, N, K, g, sym, pid, ctas)
@@ -244,10 +271,12 @@ def gemm(X: torch.Tensor, packed: torch.Tensor, scales: torch.Tensor,
                                    _ptr(out), _ptr(ws), ws_bytes, pid, ctas, _stream(dev)),
                "w4a16_gemm")
     if host_in:
-        host = torch.empty((M, N), dtype=torch.bfloat16, pin_memory=True)
-        host.copy_(out, non_blocking=True)
-        torch.cuda.current_stream(dev).synchronize()
-        return host
+        if host_out is None:
+            host_out = torch.empty((M, N), dtype=torch.bfloat16, pin_memory=True)
+        host_out.copy_(out, non_blocking=True)
+        if sync:
+            torch.cuda.current_stream(dev).synchronize()
+        return host_out
     return out
 
 

@@ -4,6 +4,7 @@
 #include <cudaTypedefs.h>
 #include <cuda_runtime.h>
 
+#include <atomic>
 #include <mutex>
 
 #include "../../include/w4a16.h"
@@ -343,18 +344,66 @@ w4a16_status make_plan(int64_t M, int64_t N, int64_t K, int32_t g, int32_t sym, 
     return W4A16_OK;
 }
 
+// SM count of the current device, queried once per device (148 when no device
+// can be queried, e.g. for host-only planning on a machine without a GPU).
 int current_sm_count() {
-    int dev = 0, sms = 0;
-    if (cudaGetDevice(&dev) == cudaSuccess &&
-        cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) == cudaSuccess && sms > 0)
-        return sms;
-    cudaGetLastError();
-    return 148;
+    static std::atomic<int> cached[kMaxDevices] = {};
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) {
+        cudaGetLastError();
+        return 148;
+    }
+    int sms = cached[dev].load(std::memory_order_relaxed);
+    if (sms > 0) return sms;
+    if (cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || sms <= 0) {
+        cudaGetLastError();
+        return 148;
+    }
+    cached[dev].store(sms, std::memory_order_relaxed);
+    return sms;
+}
+
+// Tensor maps are encoded on the host for every launch; a call repeated with
+// the same buffers (the common case: fixed weights, reused activation and output
+// buffers) finds its maps in this per-thread cache instead of re-encoding them.
+struct TmKey {
+    const void* base;
+    uint64_t inner, outer, row_bytes;
+    uint32_t box_inner, box_outer;
+    int dtype, swizzle;
+    bool operator==(const TmKey& o) const {
+        return base == o.base && inner == o.inner && outer == o.outer && row_bytes == o.row_bytes &&
+               box_inner == o.box_inner && box_outer == o.box_outer && dtype == o.dtype &&
+               swizzle == o.swizzle;
+    }
+};
+
+struct TmEntry {
+    bool valid;
+    TmKey key;
+    CUtensorMap map;
+};
+
+constexpr int kTmCacheSize = 256;
+
+size_t tm_hash(const TmKey& k) {
+    uint64_t h = reinterpret_cast<uintptr_t>(k.base) * 0x9E3779B97F4A7C15ull;
+    for (uint64_t v : {k.inner, k.outer, k.row_bytes, (uint64_t)k.box_inner, (uint64_t)k.box_outer,
+                       (uint64_t)k.dtype, (uint64_t)k.swizzle})
+        h = (h ^ v) * 0x100000001B3ull;
+    return (size_t)(h >> 17) % kTmCacheSize;
 }
 
 w4a16_status encode_2d(CUtensorMap* map, CUtensorMapDataType dtype, const void* base,
                        uint64_t inner, uint64_t outer, uint64_t row_bytes, uint32_t box_inner,
                        uint32_t box_outer, CUtensorMapSwizzle swizzle) {
+    thread_local TmEntry cache[kTmCacheSize];
+    const TmKey key{base, inner, outer, row_bytes, box_inner, box_outer, (int)dtype, (int)swizzle};
+    TmEntry& e = cache[tm_hash(key)];
+    if (e.valid && e.key == key) {
+        *map = e.map;
+        return W4A16_OK;
+    }
     PFN_cuTensorMapEncodeTiled_v12000 fn;
     w4a16_status st = encoder(&fn);
     if (st != W4A16_OK) return st;
@@ -365,7 +414,11 @@ w4a16_status encode_2d(CUtensorMap* map, CUtensorMapDataType dtype, const void* 
     CUresult r = fn(map, dtype, 2, const_cast<void*>(base), dims, strides, box, estr,
                     CU_TENSOR_MAP_INTERLEAVE_NONE, swizzle, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
                     CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
-    return r == CUDA_SUCCESS ? W4A16_OK : W4A16_ECUDA;
+    if (r != CUDA_SUCCESS) return W4A16_ECUDA;
+    e.valid = true;
+    e.key = key;
+    e.map = *map;
+    return W4A16_OK;
 }
 
 // ---------------------------------------------------------------- decode launch
