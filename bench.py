@@ -19,8 +19,9 @@ bf16 cuBLAS and the unfused dequantize-then-GEMM at the same shapes, the
 crossover sweep (K=N=8192, every M, g and mode, each kernel the dispatch can
 choose), the end-to-end number through the public API with host buffers, and
 the host oracle on the CPU.  Further extras: standalone quantize/dequantize
-bandwidth, the per-channel (g = K) decode and prefill, and the W8A16 (8-bit
-code) quantize, dequantize, M=1 GEMV and M=2048 GEMM.
+bandwidth, the per-channel (g = K) decode and prefill, the W8A16 (8-bit
+code) quantize, dequantize, M=1 GEMV and M=2048 GEMM, and the cost of the fused
+per-input-channel activation scale.
 
 Timing: W warm-up steps, then exactly K steps replayed from CUDA graphs (one
 graph holds a full rotation over the weight copies, so graph launches are
@@ -586,6 +587,7 @@ def run_ours(args):
             line["per_channel"] = workload_extras(w4, ["decode7b_pc", "prefill_pc"], peaks, peak_src,
                                                   l2, dev)
             line["w8a16"] = w8a16_extras(w4, peaks, l2, dev)
+            line["act_scale"] = act_scale_extras(w4, l2, dev)
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         cb = cpu_baseline(wl.layers, M, g, sym, unit_bytes=(half == "hbm")) \
             if half == "hbm" else cpu_baseline_sampled(wl.layers[0], M, g, sym, rows=16)
@@ -771,6 +773,33 @@ def w8a16_extras(w4, peaks, l2, dev, iters=200):
             "prefill_2048x8192x8192": {"us": pms * 1e3, "TFLOP/s": ptf,
                                        "frac": ptf / peaks["bf16_tflops"],
                                        "kernel": "gemm_tc_kernel (8-bit codes)"}}
+
+
+def act_scale_extras(w4, l2, dev, iters=100):
+    """Cost of the fused per-input-channel activation scale (w4a16_gemm_act_scaled):
+    the same GEMM with and without a[K], graph-replayed over weight copies past
+    L2 — the first 70B-shaped layer at M=1 (decode kernel) and the M=2048,
+    K=N=8192 prefill (tensor-core kernel)."""
+    out = {}
+    for name, layer, M in (("decode70b_layer0_M1", workloads.DECODE_70B.layers[0], 1),
+                           ("prefill_2048x8192x8192", workloads.PREFILL.layers[0], 2048)):
+        g, sym = 128, False
+        copies = copies_for(input_bytes(M, layer.N, layer.K, g, sym), l2)
+        case = GemmCase(w4, layer, M, g, sym, copies, dev)
+        a = workloads.make_act_scale(layer.K, 77).to(dev)
+        times = {}
+        for label, act in (("plain_us", None), ("act_scaled_us", a)):
+            def call(i, act=act):
+                j = i % copies
+                w4.gemm(case.X[j], case.P[j], case.S[j], case.Z[j], g, sym, out=case.Y[j], act_scale=act)
+            gs = graph_of(call, copies)
+            times[label] = time_graphs(gs, iters if M == 1 else 20) * 1e3
+            del gs
+        times["overhead"] = times["act_scaled_us"] / times["plain_us"] - 1.0
+        out[name] = times
+        del case, a
+        torch.cuda.empty_cache()
+    return out
 
 
 def comparisons(w4, cases, copies, l2, half):

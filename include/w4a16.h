@@ -172,6 +172,35 @@ w4a16_status w4a16_gemm_ex(const void* X, int64_t M, int64_t K, const void* pack
                            int32_t sym, void* Y, void* workspace, size_t workspace_bytes,
                            int32_t path, int32_t ctas, void* stream);
 
+/* Bytes of device workspace w4a16_gemm_act_scaled needs for this shape: the
+ * plan's workspace for M ≤ 16; for the tensor-core path that, rounded up to 256
+ * bytes, plus M·K bf16 for the scaled activations.  0 for rejected shapes. */
+size_t w4a16_gemm_act_scaled_workspace_size(int64_t M, int64_t N, int64_t K, int32_t g);
+
+/* W4A16 GEMM with a per-input-channel activation scale:
+ *   Y[M, N] = X'[M, K] · Ŵ[N, K]ᵀ,  X'[m, k] = bf16_rn(X[m, k] · a[k]).
+ * This is the activation half of the equivalent scaling W·X = (W·diag(a)⁻¹)·
+ * (diag(a)·X) that activation-aware weight quantization and SmoothQuant use to
+ * move outlier magnitude between activations and weights ("推理优化中“用精度换
+ * 性能“的核心技术：量化", §5.2 and §6.2; "大模型推理中 Weight-only、W8A8 和 FP8
+ * 量化有什么区别？如何选型？", §三): the weights are quantized after being
+ * divided by a, and the GEMM multiplies each activation by a[k].  The product
+ * of two bf16 values is exact in binary32 and is rounded once, so the result
+ * equals a w4a16_gemm on activations the caller scaled in bf16 beforehand.
+ * M ≤ 16 (decode kernel): the scale is fused into the kernel's X path (one warp
+ * scales each staged X slice as it reorders it; no extra bytes, measured cost
+ * a few percent).  Larger M (tensor-core kernel): every X tile is read by the
+ * N/128 CTAs of its row of output tiles, so X' is formed once by an elementwise
+ * pass into the workspace before the GEMM, rather than once per tile.
+ *   act_scale  in  bf16 [K], 16-byte aligned (computing it needs calibration
+ *              data, so it is the caller's); other arguments as w4a16_gemm, same
+ *              dispatch; workspace at least w4a16_gemm_act_scaled_workspace_size().
+ * Returns W4A16_EINVAL for a null act_scale (when M, N > 0). */
+w4a16_status w4a16_gemm_act_scaled(const void* X, int64_t M, int64_t K, const void* act_scale,
+                                   const void* packed, const void* scales, const void* zeros,
+                                   int64_t N, int32_t g, int32_t sym, void* Y, void* workspace,
+                                   size_t workspace_bytes, void* stream);
+
 /* Host-only: report the launch w4a16_gemm_ex would make, including the
  * workspace it needs.  Returns W4A16_EINVAL for shapes or overrides it would
  * reject. */

@@ -143,6 +143,28 @@ def test_workspace_sizes(lib):
     assert w4.workspace_size(1, 4096, 4096, 128) == w4.plan(1, 4096, 4096, 128)["workspace_bytes"]
 
 
+def test_act_scaled_rejects_without_launching(lib):
+    f = ctypes.c_void_p(FAKE)
+    g = lib.w4a16_gemm_act_scaled
+    assert g(f, 1, 256, None, f, f, f, 256, 128, 0, f, f, 1 << 30, None) == EINVAL     # no scale
+    assert g(f, 1, 256, ctypes.c_void_p(FAKE + 2), f, f, f, 256, 128, 0, f, f, 1 << 30, None) == EINVAL
+    assert g(f, 1, 250, f, f, f, f, 256, 128, 0, f, f, 1 << 30, None) == EINVAL        # K % g
+    assert g(f, 0, 256, None, f, f, f, 256, 128, 0, f, f, 0, None) == 0                # M = 0
+
+
+def test_act_scaled_workspace_sizes(lib):
+    """Decode path: the plan's workspace (the kernel scales X itself); tensor-core
+    path: that rounded up to 256 bytes plus M·K bf16 for the scaled activations."""
+    f = lib.w4a16_gemm_act_scaled_workspace_size
+    f.argtypes = [ctypes.c_int64, ctypes.c_int64, ctypes.c_int64, ctypes.c_int32]
+    f.restype = ctypes.c_size_t
+    assert f(1, 28672, 8192, 128) == w4.workspace_size(1, 28672, 8192, 128)
+    for M, N, K in ((2048, 8192, 8192), (17, 300, 1024), (4096, 8192, 8192)):
+        base = w4.workspace_size(M, N, K, 128)
+        assert f(M, N, K, 128) == -(-base // 256) * 256 + M * K * 2
+    assert f(17, 300, 1000, 128) == 0                       # rejected shape
+
+
 def test_decode_rejects_small_workspace(lib):
     need = w4.plan(1, 64, 128, 128)["workspace_bytes"]
     assert need > 0

@@ -58,6 +58,10 @@ def _load() -> ctypes.CDLL:
     lib.w4a16_gemm_ex.argtypes = [vp, i64, i64, vp, vp, vp, i64, i32, i32, vp, vp, sz, i32, i32,
                                   vp]
     lib.w4a16_gemm_plan.argtypes = [i64, i64, i64, i32, i32, i32, i32, ctypes.POINTER(Plan)]
+    lib.w4a16_gemm_act_scaled.argtypes = [vp, i64, i64, vp, vp, vp, vp, i64, i32, i32, vp, vp, sz,
+                                          vp]
+    lib.w4a16_gemm_act_scaled_workspace_size.argtypes = [i64, i64, i64, i32]
+    lib.w4a16_gemm_act_scaled_workspace_size.restype = sz
     lib.w4a16_gemm_decode_noalloc.argtypes = [vp, i64, i64, vp, vp, vp, i64, i32, i32, vp, vp]
     lib.w4a16_gemm_decode_noalloc.restype = ctypes.c_int
     lib.w4a16_device_error.argtypes = [ctypes.POINTER(ctypes.c_int32)]
@@ -70,6 +74,7 @@ def _load() -> ctypes.CDLL:
     lib.w8a16_gemm_workspace_size.argtypes = [i64, i64, i64, i32]
     lib.w8a16_gemm_workspace_size.restype = sz
     for name in ("w4a16_quantize", "w4a16_dequantize", "w4a16_gemm", "w4a16_gemm_ex",
+                 "w4a16_gemm_act_scaled",
                  "w4a16_gemm_plan", "w4a16_device_error", "w8a16_quantize", "w8a16_dequantize",
                  "w8a16_gemm"):
         getattr(lib, name).restype = ctypes.c_int
@@ -225,8 +230,13 @@ def _device_buffer(dev: torch.device, M: int, N: int) -> torch.Tensor:
 
 def gemm(X: torch.Tensor, packed: torch.Tensor, scales: torch.Tensor,
          zeros: torch.Tensor | None, g: int = 128, sym: bool = False, path: str | int = "auto",
-         ctas: int = 0, out: torch.Tensor | None = None, sync: bool = True) -> torch.Tensor:
+         ctas: int = 0, out: torch.Tensor | None = None, sync: bool = True,
+         act_scale: torch.Tensor | None = None) -> torch.Tensor:
     """Fused W4A16 GEMM: Y[M, N] = X[M, K] · Ŵ[N, K]ᵀ (bf16 in/out, fp32 accumulation).
+
+    ``act_scale`` (bf16 [K] on the weights' device): multiply each activation
+    by its input channel's scale as it is loaded, X'[m, k] = bf16_rn(X[m, k]·a[k])
+    (w4a16_gemm_act_scaled; the automatic kernel choice only).
 
     If X lives in host memory (ideally pinned) it is copied to the weights'
     device and Y is copied back into host memory — ``out`` when given (a pinned
@@ -263,13 +273,34 @@ def gemm(X: torch.Tensor, packed: torch.Tensor, scales: torch.Tensor,
             raise ValueError("out has the wrong shape")
         _same_device(dev, out=out)
     pid = _PATHS[path] if isinstance(path, str) else int(path)
+    if act_scale is not None:
+        _need(act_scale, torch.bfloat16, "act_scale", ndim=1)
+        if act_scale.shape[0] != K:
+            raise ValueError(f"act_scale has {act_scale.shape[0]} entries, X has K={K}")
+        _same_device(dev, act_scale=act_scale)
+        if pid != PATH_AUTO or ctas:
+            raise ValueError("act_scale uses the automatic kernel choice")
     with torch.cuda.device(dev):
-        ws_bytes = _workspace_bytes(dev, M, N, K, g, sym, pid, ctas)
+        if act_scale is None:
+            ws_bytes = _workspace_bytes(dev, M, N, K, g, sym, pid, ctas)
+        else:
+            key = ("act", dev.index, M, N, K, g)
+            ws_bytes = _plan_bytes.get(key)
+            if ws_bytes is None:
+                ws_bytes = int(lib().w4a16_gemm_act_scaled_workspace_size(M, N, K, g)) if M and N else 0
+                _plan_bytes[key] = ws_bytes
         ws = _workspace(dev, ws_bytes)
-        _check(lib().w4a16_gemm_ex(_ptr(Xd), M, K, _ptr(packed), _ptr(scales),
-                                   _ptr(zeros if not sym else None), N, g, int(bool(sym)),
-                                   _ptr(out), _ptr(ws), ws_bytes, pid, ctas, _stream(dev)),
-               "w4a16_gemm")
+        if act_scale is None:
+            _check(lib().w4a16_gemm_ex(_ptr(Xd), M, K, _ptr(packed), _ptr(scales),
+                                       _ptr(zeros if not sym else None), N, g, int(bool(sym)),
+                                       _ptr(out), _ptr(ws), ws_bytes, pid, ctas, _stream(dev)),
+                   "w4a16_gemm")
+        else:
+            _check(lib().w4a16_gemm_act_scaled(_ptr(Xd), M, K, _ptr(act_scale), _ptr(packed),
+                                               _ptr(scales), _ptr(zeros if not sym else None), N, g,
+                                               int(bool(sym)), _ptr(out), _ptr(ws), ws_bytes,
+                                               _stream(dev)),
+                   "w4a16_gemm_act_scaled")
     if host_in:
         if host_out is None:
             host_out = torch.empty((M, N), dtype=torch.bfloat16, pin_memory=True)

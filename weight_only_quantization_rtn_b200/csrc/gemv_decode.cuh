@@ -29,7 +29,11 @@
 //  * Warp 17 (helper): once a stage has landed, rewrites its X slice into
 //    MMA-fragment order (the pairs (x_j, x_{j+4}) the nibble isolation below
 //    produces) in a separate area, and signals "xf".  One warp does this once
-//    per stage instead of every consumer thread permuting its own copy.
+//    per stage instead of every consumer thread permuting its own copy.  With a
+//    per-input-channel activation scale a[K] (the activation half of the
+//    equivalent scaling (X·diag(a))·(diag(a)⁻¹·W) of "推理优化中“用精度换性能“的
+//    核心技术：量化", §5.2 and §6.2), the helper also forms x' = bf16_rn(x·a[k])
+//    here, one rounding of the exact product, before permuting.
 //  * Warps 0..15 (consumers): warp w owns rows 16w .. 16w+15 of every unit, so
 //    its accumulators hold whole output rows across the K blocks of a row block
 //    and no warp ever waits for another.  Lane (g, q) — g = lane/4, q = lane%4 —
@@ -137,6 +141,7 @@ struct DecodeArgs {
     const uint16_t* scales;
     const uint16_t* zeros;
     uint16_t* Y;
+    const uint16_t* act_scale;   // bf16 [K] per-input-channel activation scale, or null
     uint32_t* ws_flag;    // [(RB + C) slots][16 warps] ready flags
     float* ws_part;       // [(RB + C) slots][16 warps][32 lanes][4·MB] fp32 parts
     int M;
@@ -464,8 +469,15 @@ __global__ void __launch_bounds__(kDecThreads, 1)
         // ((x0,x4),(x1,x5),(x2,x6),(x3,x7)) at row m, slot i, lane-group q.
         int s = 0;
         uint32_t ph = 0;
+        UnitWalk wk;
+        wk.init(u0, u1, a.KBn);
+        const uint16_t* act = a.act_scale;
+        if (act != nullptr) grid_dependency_wait();   // the scales may be the previous grid's output
         for (int i = 0; i < nunits; ++i) {
-            if (i > 0 && ++s == S) { s = 0; ph ^= 1u; }
+            if (i > 0) {
+                wk.advance();
+                if (++s == S) { s = 0; ph ^= 1u; }
+            }
             bool ok = mbar_test_wait(smem_u32(&full[s]), ph);
             if (!ok && *abort_flag == 0) ok = mbar_wait_backoff(smem_u32(&full[s]), ph, kDecHelperSleepNs);
             if (!ok) {
@@ -478,7 +490,17 @@ __global__ void __launch_bounds__(kDecThreads, 1)
 #pragma unroll 1
             for (int it = lane; it < M * 32; it += 32) {
                 const int m = it >> 5, c = it & 31;
-                const uint4 v = lds128_u32addr(xn + m * kDecXRowBytes + c * 16);
+                uint4 v = lds128_u32addr(xn + m * kDecXRowBytes + c * 16);
+                if (act != nullptr) {
+                    // x' = bf16_rn(x·a): the chunk's 8 scales (K is a multiple of 32, so a
+                    // chunk is wholly inside or wholly past the end of X, where x = 0)
+                    const int k0 = wk.kb * kDecBlockK + 8 * c;
+                    const uint4 av = k0 < a.K ? ldg_cached(act + k0) : make_uint4(0, 0, 0, 0);
+                    v.x = bf16x2_mul(v.x, av.x);
+                    v.y = bf16x2_mul(v.y, av.y);
+                    v.z = bf16x2_mul(v.z, av.z);
+                    v.w = bf16x2_mul(v.w, av.w);
+                }
                 uint4 o;
                 o.x = __byte_perm(v.x, v.z, 0x5410);   // (x0, x4)
                 o.y = __byte_perm(v.x, v.z, 0x7632);   // (x1, x5)

@@ -234,4 +234,23 @@ __global__ void __launch_bounds__(256) dequantize_rows_kernel(const uint32_t* __
     }
 }
 
+// X'[m, k] = bf16_rn(X[m, k]·a[k]): the per-input-channel activation scale for
+// the tensor-core GEMM, formed once per call ("推理优化中“用精度换性能“的核心技术：
+// 量化", §5.2 and §6.2, the activation half of the equivalent scaling).  The
+// product of two bf16 values is exact in binary32 and mul.rn.bf16x2 rounds it
+// once.  One 16-byte chunk (8 elements) per thread and step; K is a multiple of
+// 8, so a chunk never crosses a row.
+__global__ void __launch_bounds__(256) scale_activations_kernel(const uint4* __restrict__ X,
+                                                                const uint4* __restrict__ a,
+                                                                int64_t chunks, int64_t row_chunks,
+                                                                uint4* __restrict__ Xs) {
+    for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < chunks;
+         i += (int64_t)gridDim.x * blockDim.x) {
+        const uint4 v = X[i];
+        const uint4 s = a[i % row_chunks];
+        Xs[i] = make_uint4(bf16x2_mul(v.x, s.x), bf16x2_mul(v.y, s.y), bf16x2_mul(v.z, s.z),
+                           bf16x2_mul(v.w, s.w));
+    }
+}
+
 }  // namespace w4a16

@@ -464,7 +464,8 @@ int decode_scale_copy(int gu, int64_t groups) {
 
 w4a16_status launch_decode(const w4a16_plan& p, const void* X, int64_t M, int64_t K,
                            const void* packed, const void* scales, const void* zeros, int64_t N,
-                           int32_t g, int32_t sym, void* Y, void* workspace, cudaStream_t stream) {
+                           int32_t g, int32_t sym, void* Y, void* workspace, cudaStream_t stream,
+                           const void* act_scale = nullptr) {
     const DecodeGeometry d = decode_geometry(M, N, K, g);
     CUtensorMap tmP, tmX;
     w4a16_status st = encode_2d(&tmP, CU_TENSOR_MAP_DATA_TYPE_UINT8, packed, (uint64_t)(K / 2),
@@ -479,6 +480,7 @@ w4a16_status launch_decode(const w4a16_plan& p, const void* X, int64_t M, int64_
     args.scales = static_cast<const uint16_t*>(scales);
     args.zeros = static_cast<const uint16_t*>(zeros);
     args.Y = static_cast<uint16_t*>(Y);
+    args.act_scale = static_cast<const uint16_t*>(act_scale);
     args.ws_flag = static_cast<uint32_t*>(workspace);
     args.ws_part = reinterpret_cast<float*>(static_cast<uint8_t*>(workspace) +
                                             decode_flag_bytes(d, p.grid));
@@ -688,6 +690,49 @@ w4a16_status noalloc_scratch(void** out) {
     return W4A16_OK;
 }
 
+// Workspace of an activation-scaled GEMM: the tensor-core path forms X' once into
+// the workspace, after the GEMM's own scratch (rounded to 256 bytes); the decode
+// path scales X inside the kernel and needs nothing extra.
+int64_t act_scaled_workspace_bytes(const w4a16_plan& p, int64_t M, int64_t K) {
+    if (p.path == W4A16_PATH_DECODE) return p.workspace_bytes;
+    return (p.workspace_bytes + 255) / 256 * 256 + M * K * 2;
+}
+
+// The fused GEMM behind every W4A16 GEMM entry point; act_scale (bf16 [K]) or null.
+w4a16_status gemm_impl(const void* X, int64_t M, int64_t K, const void* packed, const void* scales,
+                       const void* zeros, int64_t N, int32_t g, int32_t sym, const void* act_scale,
+                       void* Y, void* workspace, size_t workspace_bytes, int32_t path, int32_t ctas,
+                       void* stream) {
+    w4a16_plan p;
+    w4a16_status st = make_plan(M, N, K, g, sym, path, ctas, current_sm_count(), &p);
+    if (st != W4A16_OK) return st;
+    if (M == 0 || N == 0) return W4A16_OK;
+    if (!X || !packed || !scales || !Y || (!sym && !zeros)) return W4A16_EINVAL;
+    if (!aligned16(X) || !aligned16(packed) || !aligned16(scales) || !aligned16(Y) ||
+        (!sym && !aligned16(zeros)) || (act_scale && !aligned16(act_scale)))
+        return W4A16_EINVAL;
+    const int64_t need = act_scale ? act_scaled_workspace_bytes(p, M, K) : p.workspace_bytes;
+    if (workspace_bytes < (size_t)need) return W4A16_EWORKSPACE;
+    if (need > 0 && (workspace == nullptr || !aligned16(workspace))) return W4A16_EINVAL;
+    DeviceInfo di;
+    if ((st = device_info(&di)) != W4A16_OK) return st;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    if (p.path == W4A16_PATH_DECODE)
+        return launch_decode(p, X, M, K, packed, scales, zeros, N, g, sym, Y, workspace, s, act_scale);
+    if (act_scale) {
+        // Large M: every X tile is read by all N/128 CTAs of its row of tiles, so X' is
+        // formed once, by an elementwise pass into the workspace, rather than per tile.
+        void* xs = static_cast<uint8_t*>(workspace) + (p.workspace_bytes + 255) / 256 * 256;
+        const int64_t chunks = M * K / 8;
+        scale_activations_kernel<<<grid_for(chunks, 256, di.sm_count), 256, 0, s>>>(
+            static_cast<const uint4*>(X), static_cast<const uint4*>(act_scale), chunks, K / 8,
+            static_cast<uint4*>(xs));
+        if ((st = launch_status()) != W4A16_OK) return st;
+        X = xs;
+    }
+    return launch_tc(p, X, M, K, packed, scales, zeros, N, g, sym, Y, workspace, s, 4);
+}
+
 }  // namespace
 
 // ==================================================================== ABI
@@ -801,22 +846,8 @@ w4a16_status w4a16_gemm_ex(const void* X, int64_t M, int64_t K, const void* pack
                            const void* scales, const void* zeros, int64_t N, int32_t g,
                            int32_t sym, void* Y, void* workspace, size_t workspace_bytes,
                            int32_t path, int32_t ctas, void* stream) {
-    w4a16_plan p;
-    w4a16_status st = make_plan(M, N, K, g, sym, path, ctas, current_sm_count(), &p);
-    if (st != W4A16_OK) return st;
-    if (M == 0 || N == 0) return W4A16_OK;
-    if (!X || !packed || !scales || !Y || (!sym && !zeros)) return W4A16_EINVAL;
-    if (!aligned16(X) || !aligned16(packed) || !aligned16(scales) || !aligned16(Y) ||
-        (!sym && !aligned16(zeros)))
-        return W4A16_EINVAL;
-    if (workspace_bytes < (size_t)p.workspace_bytes) return W4A16_EWORKSPACE;
-    if (p.workspace_bytes > 0 && (workspace == nullptr || !aligned16(workspace))) return W4A16_EINVAL;
-    DeviceInfo di;
-    if ((st = device_info(&di)) != W4A16_OK) return st;
-    cudaStream_t s = static_cast<cudaStream_t>(stream);
-    if (p.path == W4A16_PATH_DECODE)
-        return launch_decode(p, X, M, K, packed, scales, zeros, N, g, sym, Y, workspace, s);
-    return launch_tc(p, X, M, K, packed, scales, zeros, N, g, sym, Y, workspace, s);
+    return gemm_impl(X, M, K, packed, scales, zeros, N, g, sym, nullptr, Y, workspace,
+                     workspace_bytes, path, ctas, stream);
 }
 
 w4a16_status w4a16_gemm(const void* X, int64_t M, int64_t K, const void* packed,
@@ -825,6 +856,21 @@ w4a16_status w4a16_gemm(const void* X, int64_t M, int64_t K, const void* packed,
                         void* stream) {
     return w4a16_gemm_ex(X, M, K, packed, scales, zeros, N, g, sym, Y, workspace,
                          workspace_bytes, W4A16_PATH_AUTO, 0, stream);
+}
+
+size_t w4a16_gemm_act_scaled_workspace_size(int64_t M, int64_t N, int64_t K, int32_t g) {
+    w4a16_plan p;
+    if (make_plan(M, N, K, g, 0, W4A16_PATH_AUTO, 0, current_sm_count(), &p) != W4A16_OK) return 0;
+    return (size_t)act_scaled_workspace_bytes(p, M, K);
+}
+
+w4a16_status w4a16_gemm_act_scaled(const void* X, int64_t M, int64_t K, const void* act_scale,
+                                   const void* packed, const void* scales, const void* zeros,
+                                   int64_t N, int32_t g, int32_t sym, void* Y, void* workspace,
+                                   size_t workspace_bytes, void* stream) {
+    if (!act_scale && M > 0 && N > 0) return W4A16_EINVAL;
+    return gemm_impl(X, M, K, packed, scales, zeros, N, g, sym, act_scale, Y, workspace,
+                     workspace_bytes, W4A16_PATH_AUTO, 0, stream);
 }
 
 w4a16_status w4a16_gemm_decode_noalloc(const void* X, int64_t M, int64_t K, const void* packed,

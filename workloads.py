@@ -64,6 +64,15 @@ def make_activation(M: int, K: int, seed: int, outlier_frac: float = 0.0,
     return X.to(torch.bfloat16)
 
 
+def make_act_scale(K: int, seed: int, lo: float = -1.5, hi: float = 1.5) -> torch.Tensor:
+    """Per-input-channel activation scale a[K] (bf16), 2^u with u ~ U(lo, hi):
+    positive factors of the size activation-aware scaling uses, with arbitrary
+    bf16 mantissas (so x·a rounds).  Drawn on the CPU from its own seed."""
+    g = _gen(seed)
+    u = torch.rand(K, generator=g, dtype=torch.float32) * (hi - lo) + lo
+    return torch.exp2(u).to(torch.bfloat16)
+
+
 def bits(t: torch.Tensor) -> np.ndarray:
     """bf16 tensor -> numpy uint16 bit patterns (CPU copy)."""
     assert t.dtype == torch.bfloat16
