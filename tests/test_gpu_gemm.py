@@ -262,3 +262,29 @@ def test_tiny_config_full_compare():
         ref = oracle.gemm_w4a16(workloads.bits(X), P.cpu().numpy(), workloads.bits(S),
                                 workloads.bits(Z), 128, False)
         assert_y_close(workloads.bits(Y), ref, f"tiny {path}")
+
+
+def test_sharded_layer_on_one_rank_nccl():
+    """The N-sharded layer's GPU path (fused kernel + NCCL all-gather) on a
+    one-rank NCCL group: the rank owns every row and the result matches the
+    oracle like the plain GEMM."""
+    import os
+    import torch.distributed as dist
+    from weight_only_quantization_rtn_b200 import sharded
+    N, K, M, g = 1000, 2048, 3, 128
+    os.environ.setdefault("MASTER_ADDR", "127.0.0.1")
+    os.environ.setdefault("MASTER_PORT", str(29500 + os.getpid() % 1000))
+    dist.init_process_group("nccl", rank=0, world_size=1, device_id=torch.device("cuda", 0))
+    try:
+        W = workloads.make_weight(N, K, 0.02, 9, outlier_frac=0.01, outlier_scale=20.0)
+        X = workloads.make_activation(M, K, 10, outlier_frac=0.01, outlier_mode="set")
+        layer = sharded.ShardedW4A16Linear.from_weight(W.cuda(), g, False, world=1, rank=0)
+        Y = layer(X.cuda())
+        torch.cuda.synchronize()
+        Y64 = oracle.gemm_w4a16(workloads.bits(X), layer.packed.cpu().numpy(),
+                                workloads.bits(layer.scales), workloads.bits(layer.zeros), g, False)
+        assert_y_close(workloads.bits(Y), Y64, "sharded, one rank")
+        Yg = sharded.gather_columns(torch.zeros(M, N, dtype=torch.bfloat16, device="cuda"), N, 1)
+        assert tuple(Yg.shape) == (M, N)
+    finally:
+        dist.destroy_process_group()
