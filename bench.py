@@ -909,18 +909,24 @@ def crossover_rows(w4, dev, l2, iters=40, iters_large=12):
             for path in ("decode", "tensorcore"):
                 if path == "decode" and M > 16:
                     continue
+                # an NVTX range per measurement, so that a profiler's launch list can
+                # name each kernel launch by (g, mode, M, kernel)
+                torch.cuda.nvtx.range_push(f"xover_g{g}_{row['mode']}_M{M}_{path}")
                 gs = graph_of(lambda i, path=path: w4.gemm(Xs[i % copies], Ps[i % copies],
                                                            Ss[i % copies], Zs[i % copies], g, sym,
                                                            path=path, out=Y), copies)
                 row[path + "_us"] = round(time_graphs(gs, n) * 1e3, 3)
+                torch.cuda.nvtx.range_pop()
                 del gs
             if g == 128 and not sym:
                 dcopies = max(2, -(-2 * l2 // (N * K * 2 + 2 * M * K)) + 1)
                 Wd = [W] + [W.clone() for _ in range(dcopies - 1)]
                 Xd = Xs[:1] + [X.clone() for _ in range(dcopies - 1)]
+                torch.cuda.nvtx.range_push(f"xover_g{g}_{row['mode']}_M{M}_dense")
                 gs = graph_of(lambda i: torch.matmul(Xd[i % dcopies], Wd[i % dcopies].t(), out=Y),
                               dcopies)
                 row["dense_bf16_cublas_us"] = round(time_graphs(gs, n) * 1e3, 3)
+                torch.cuda.nvtx.range_pop()
                 del gs, Wd, Xd
             cand = {k[:-3]: v for k, v in row.items() if k in ("decode_us", "tensorcore_us")}
             row["fastest"] = min(cand, key=cand.get)
