@@ -249,13 +249,17 @@ class GemmCase:
         self.flops = 2 * M * self.N * self.K
 
     def call(self, w4, i):
+        # The weights are fixed after set-up and no kernel in a step writes them, so
+        # the decode kernel may stream them while the previous GEMM drains.
         j = i % len(self.P)
-        w4.gemm(self.X[j], self.P[j], self.S[j], self.Z[j], self.g, self.sym, out=self.Y[j])
+        w4.gemm(self.X[j], self.P[j], self.S[j], self.Z[j], self.g, self.sym, out=self.Y[j],
+                static_weights=True)
 
 
 def launches_per_call(plan: dict) -> int:
-    """Kernels one GEMM call launches: the decode path adds a fixup kernel when
-    its stream-K partition splits a row block (a host-side property of the plan)."""
+    """Kernels one GEMM call launches (a host-side property of the plan): one for
+    the decode path; one to three for the tensor-core path (unsplit head, K-split
+    tail, the reduce of the tail's parts)."""
     return int(plan["kernels"])
 
 
@@ -544,7 +548,7 @@ def run_ours(args):
         # host X in, host Y out for every layer; the step waits once, for its last copy
         for c, xh, yh in zip(cases, pinned, host_y):
             j = i % copies
-            w4.gemm(xh, c.P[j], c.S[j], c.Z[j], c.g, c.sym, out=yh, sync=False)
+            w4.gemm(xh, c.P[j], c.S[j], c.Z[j], c.g, c.sym, out=yh, sync=False, static_weights=True)
         torch.cuda.current_stream().synchronize()
 
     for i in range(args.warmup):
@@ -914,7 +918,8 @@ def crossover_rows(w4, dev, l2, iters=40, iters_large=12):
                 torch.cuda.nvtx.range_push(f"xover_g{g}_{row['mode']}_M{M}_{path}")
                 gs = graph_of(lambda i, path=path: w4.gemm(Xs[i % copies], Ps[i % copies],
                                                            Ss[i % copies], Zs[i % copies], g, sym,
-                                                           path=path, out=Y), copies)
+                                                           path=path, out=Y, static_weights=True),
+                              copies)
                 row[path + "_us"] = round(time_graphs(gs, n) * 1e3, 3)
                 torch.cuda.nvtx.range_pop()
                 del gs

@@ -64,7 +64,8 @@
 extern "C" {
 #endif
 
-#define W4A16_ABI_VERSION 3   /* 3: w4a16_plan.split_tiles; the decode path is one kernel */
+#define W4A16_ABI_VERSION 4   /* 3: w4a16_plan.split_tiles; the decode path is one kernel;
+                                 4: W4A16_STATIC_WEIGHTS */
 
 typedef enum w4a16_status {
     W4A16_OK = 0,
@@ -91,6 +92,19 @@ typedef enum w4a16_path {
                                   wave of tiles would leave most SMs idle, those tiles split
                                   K and a reduce kernel adds the parts in a fixed order */
 } w4a16_path;
+
+/* Flag OR'ed into the `path` argument of w4a16_gemm_ex (w4a16_gemm_plan accepts
+ * and ignores it): the caller states that the kernel before this call on its
+ * stream does not write packed, scales or zeros.  The decode kernel (M ≤ 16) then
+ * streams the weights as soon as its CTAs are resident, while that kernel drains
+ * (programmatic dependent launch), and waits for it only before reading X and
+ * writing Y.  Inference with fixed weights meets the condition; a call right
+ * after quantizing the same weights on the same stream does not, and its result
+ * is then undefined.  The tensor-core path reads nothing before the previous
+ * kernel completes either way.  Why it helps: on the layers of a 7B-shaped decode
+ * step the first stage lands a few microseconds after the weights are requested,
+ * a sizeable part of a 3–4 µs layer. */
+#define W4A16_STATIC_WEIGHTS 0x100
 
 /* The launch a GEMM call would make (filled by w4a16_gemm_plan). */
 typedef struct w4a16_plan {

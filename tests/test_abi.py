@@ -53,7 +53,7 @@ def test_library_is_sm100a_only_and_links_no_cudart_dso(lib):
 
 
 def test_status_strings_and_version(lib):
-    assert lib.w4a16_abi_version() == 3
+    assert lib.w4a16_abi_version() == 4
     for s in range(6):
         assert lib.w4a16_status_string(s).startswith(b"W4A16")
 
@@ -141,6 +141,15 @@ def test_workspace_sizes(lib):
         slots = rb + p["grid"]
         assert p["workspace_bytes"] == -(-slots * 16 * 4 // 256) * 256 + slots * 16 * 32 * 16 * mb
     assert w4.workspace_size(1, 4096, 4096, 128) == w4.plan(1, 4096, 4096, 128)["workspace_bytes"]
+
+
+def test_static_weights_flag_is_accepted_only_as_a_flag(lib):
+    """W4A16_STATIC_WEIGHTS (0x100) may be OR'ed into the path; other high bits
+    are rejected before anything is launched."""
+    f = ctypes.c_void_p(FAKE)
+    assert w4.plan(1, 4096, 4096, path=w4.PATH_AUTO | w4.STATIC_WEIGHTS) == w4.plan(1, 4096, 4096)
+    assert lib.w4a16_gemm_ex(f, 1, 256, f, f, f, 256, 128, 0, f, f, 1 << 30, 0x200, 0, None) == EINVAL
+    assert lib.w4a16_gemm_ex(f, 1, 256, f, f, f, 256, 128, 0, f, f, 1 << 30, 0x103, 0, None) == EINVAL
 
 
 def test_act_scaled_rejects_without_launching(lib):

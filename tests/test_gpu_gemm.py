@@ -151,6 +151,24 @@ def test_deterministic_bitwise(path):
     assert all(torch.equal(ys[0], y) for y in ys[1:])
 
 
+@pytest.mark.parametrize("M,N,K,g,sym", [(1, 28672, 8192, 128, False), (4, 4096, 11008, 128, True),
+                                         (16, 11008, 4096, 64, False), (3, 1000, 2304, 32, True),
+                                         (1, 4096, 11008, 11008, False)])
+def test_static_weights_flag_matches_plain_call(M, N, K, g, sym):
+    """W4A16_STATIC_WEIGHTS only moves the weight stream ahead of the dependency
+    wait: a chain of calls on two sets of fixed weights (each call following a
+    GEMM that does not write them) gives the same bits as the plain calls."""
+    sets = [_quantized(N, K, g, sym, seed=40 + i) for i in range(2)]
+    torch.cuda.synchronize()                      # the quantizer is done with the weights
+    X = workloads.make_activation(M, K, 41, outlier_frac=0.01, outlier_mode="set").cuda()
+    plain = [w4.gemm(X, *sets[i % 2], g, sym, path="decode") for i in range(4)]
+    static = [w4.gemm(X, *sets[i % 2], g, sym, path="decode", static_weights=True) for i in range(4)]
+    torch.cuda.synchronize()
+    for a, b in zip(plain, static):
+        assert torch.equal(a, b)
+    assert w4.device_error() == 0
+
+
 @pytest.mark.parametrize("M,N,K,g,sym", [
     (300, 10240, 2048, 32, False),    # 160 tiles: 148 unsplit + a 12-tile tail split 8 ways
     (2048, 8192, 2048, 128, True),    # 512 tiles: 444 unsplit + a 68-tile tail split 2 ways

@@ -19,13 +19,14 @@ import torch
 
 __all__ = ["lib", "quantize", "dequantize", "gemm", "gemm_decode_noalloc", "plan",
            "quantize8", "dequantize8", "gemm8",
-           "workspace_size", "device_error", "W4A16Error", "PATH_AUTO", "PATH_DECODE", "PATH_TENSORCORE", "LIB_PATH"]
+           "workspace_size", "device_error", "W4A16Error", "PATH_AUTO", "PATH_DECODE", "PATH_TENSORCORE", "STATIC_WEIGHTS", "LIB_PATH"]
 
 LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libw4a16.so")
 
 # W4A16_ABI_VERSION in include/w4a16.h that the argument lists below follow
-ABI_VERSION = 3
+ABI_VERSION = 4
 PATH_AUTO, PATH_DECODE, PATH_TENSORCORE = 0, 1, 2
+STATIC_WEIGHTS = 0x100   # W4A16_STATIC_WEIGHTS, OR'ed into the path argument
 _PATHS = {"auto": PATH_AUTO, "decode": PATH_DECODE, "tensorcore": PATH_TENSORCORE}
 _STATUS = {0: "OK", 1: "EINVAL", 2: "EUNSUPPORTED", 3: "ECUDA", 4: "EWORKSPACE", 5: "EDEVICE"}
 
@@ -231,8 +232,14 @@ def _device_buffer(dev: torch.device, M: int, N: int) -> torch.Tensor:
 def gemm(X: torch.Tensor, packed: torch.Tensor, scales: torch.Tensor,
          zeros: torch.Tensor | None, g: int = 128, sym: bool = False, path: str | int = "auto",
          ctas: int = 0, out: torch.Tensor | None = None, sync: bool = True,
-         act_scale: torch.Tensor | None = None) -> torch.Tensor:
+         act_scale: torch.Tensor | None = None, static_weights: bool = False) -> torch.Tensor:
     """Fused W4A16 GEMM: Y[M, N] = X[M, K] · Ŵ[N, K]ᵀ (bf16 in/out, fp32 accumulation).
+
+    ``static_weights``: the kernel before this call on the stream does not write
+    ``packed``, ``scales`` or ``zeros`` (inference with fixed weights), so the
+    decode kernel may start streaming them while that kernel drains
+    (W4A16_STATIC_WEIGHTS).  Not for a call right after quantizing on the same
+    stream.
 
     ``act_scale`` (bf16 [K] on the weights' device): multiply each activation
     by its input channel's scale as it is loaded, X'[m, k] = bf16_rn(X[m, k]·a[k])
@@ -293,7 +300,9 @@ def gemm(X: torch.Tensor, packed: torch.Tensor, scales: torch.Tensor,
         if act_scale is None:
             _check(lib().w4a16_gemm_ex(_ptr(Xd), M, K, _ptr(packed), _ptr(scales),
                                        _ptr(zeros if not sym else None), N, g, int(bool(sym)),
-                                       _ptr(out), _ptr(ws), ws_bytes, pid, ctas, _stream(dev)),
+                                       _ptr(out), _ptr(ws), ws_bytes,
+                                       pid | (STATIC_WEIGHTS if static_weights else 0), ctas,
+                                       _stream(dev)),
                    "w4a16_gemm")
         else:
             _check(lib().w4a16_gemm_act_scaled(_ptr(Xd), M, K, _ptr(act_scale), _ptr(packed),

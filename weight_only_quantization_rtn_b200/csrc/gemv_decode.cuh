@@ -25,7 +25,11 @@
 //    own, loaded once per slab rather than once per unit — each slab row is a
 //    separate 16-byte request, so re-loading it per unit would triple the
 //    requests of the stream; otherwise the 32 lanes copy the unit's groups into
-//    the stage with cp.async (plain loads when the rows are misaligned).
+//    the stage with cp.async (plain loads when the rows are misaligned).  When
+//    the caller states that the previous grid on the stream does not write the
+//    weights, the codes and scales of the first ring's worth of units are
+//    requested before the dependency wait, while that grid drains; X follows
+//    after the wait.
 //  * Warp 17 (helper): once a stage has landed, rewrites its X slice into
 //    MMA-fragment order (the pairs (x_j, x_{j+4}) the nibble isolation below
 //    produces) in a separate area, and signals "xf".  One warp does this once
@@ -55,8 +59,8 @@
 //    parts to its own in CTA order and writes Y.  The sum order is fixed, so the
 //    result is deterministic, and no second kernel is launched.
 //  * Programmatic dependent launch lets the next kernel on the stream start
-//    while this one drains; nothing is read or written before
-//    griddepcontrol.wait.
+//    while this one drains; nothing but those static weights is read, and
+//    nothing is written, before griddepcontrol.wait.
 #pragma once
 
 #include "common.cuh"
@@ -158,6 +162,7 @@ struct DecodeArgs {
     int slab_off;         // slab ring: `slabs` slots of [2][256 rows][8] bf16 (8 KB each)
     int slabs;
     int sz_copy;          // without TMA: bytes per scale copy, 16, 8 or 4 (cp.async), 2 (plain)
+    int early;            // 1: the previous grid does not write the weights; stream them before the dependency wait
     int64_t U;            // units = RB · KBn
 };
 
@@ -348,59 +353,47 @@ __global__ void __launch_bounds__(kDecThreads, 1)
             }
         }
         const uint32_t tx = (uint32_t)kDecPBytes + (uint32_t)M * kDecXRowBytes;
-        int slab_t = -1, slab_rb = -1, slab_j = -1;   // slabs requested so far - 1, current slab
-        grid_dependency_wait();              // weights and X may be the previous grid's output
-        UnitWalk wk;
-        wk.init(u0, u1, a.KBn);
-        int issued = 0;
-        int s = 0;
-        uint32_t ph = 0;
         const int arrays = SYM ? 1 : 2;
-        for (int i = 0; i < nunits; ++i) {
-            if (i > 0) {
-                wk.advance();
-                if (++s == S) { s = 0; ph ^= 1u; }
+        int slab_t = -1, slab_rb = -1, slab_j = -1;   // slabs requested so far - 1, current slab
+        int slab_slot = SL - 1;                       // slab_t mod SL
+        uint32_t slab_ph = 1u;                        // parity of slab_t's use of its slot
+        // True when unit (rb, kb) reads a slab other than the last one requested.
+        auto new_slab = [&](int rb, int kb) {
+            return G != 0 && a.sz_tma && (rb != slab_rb || ((kb * GU) >> 3) != slab_j);
+        };
+        // Request the slab of unit (rb, kb) (groups kb·GU .. kb·GU + GU − 1; GU divides
+        // 8) into the next slot, once the consumers have released that slot.
+        auto request_slab = [&](int rb, int kb) -> bool {
+            const int j = (kb * GU) >> 3;
+            ++slab_t;
+            if (++slab_slot == SL) {
+                slab_slot = 0;
+                slab_ph ^= 1u;
             }
-            const int rb = wk.rb, kb = wk.kb;
             bool ok = true;
-            if (lane == 0) ok = mbar_wait_backoff(smem_u32(&empty[s]), ph ^ 1u, kDecProducerSleepNs);
-            if (!__shfl_sync(0xffffffffu, ok ? 1 : 0, 0)) {
-                *abort_flag = 1;
-                break;
+            if (lane == 0) ok = mbar_wait_backoff(smem_u32(&sempty[slab_slot]), slab_ph ^ 1u, kDecProducerSleepNs);
+            if (!__shfl_sync(0xffffffffu, ok ? 1 : 0, 0)) return false;
+            if (lane == 0) {
+                const uint32_t sb = smem_u32(&sfull[slab_slot]);
+                const uint32_t dst = smem_u32(slab_base + slab_slot * kDecSlabBytes);
+                mbar_arrive_expect_tx(sb, (uint32_t)((SYM ? 1 : 2) * kDecSlabArrayBytes));
+                tma_load_2d(dst, &tmS, 8 * j, rb * kDecRows, sb);
+                if (!SYM) tma_load_2d(dst + kDecSlabArrayBytes, &tmZ, 8 * j, rb * kDecRows, sb);
             }
+            slab_rb = rb;
+            slab_j = j;
+            return true;
+        };
+        // The weights of unit (rb, kb) into stage s: the codes tile by TMA (the
+        // stage's "full" barrier expects the codes and the X slice), and — without
+        // TMA slabs — the unit's scales (and zeros), [array][row][GU] bf16.
+        auto load_weights = [&](int rb, int kb, int s) {
             const uint32_t st = stages_u32 + (uint32_t)(s * a.stage_bytes);
             const uint32_t bar = smem_u32(&full[s]);
-            if (G != 0 && a.sz_tma) {
-                // the slab holding groups kb·GU .. kb·GU + GU − 1 (GU divides 8), once per slab
-                const int j = (kb * GU) >> 3;
-                if (rb != slab_rb || j != slab_j) {
-                    ++slab_t;
-                    const int slot = slab_t % SL;
-                    if (lane == 0)
-                        ok = mbar_wait_backoff(smem_u32(&sempty[slot]), (((uint32_t)(slab_t / SL)) & 1u) ^ 1u,
-                                               kDecProducerSleepNs);
-                    if (!__shfl_sync(0xffffffffu, ok ? 1 : 0, 0)) {
-                        *abort_flag = 1;
-                        break;
-                    }
-                    if (lane == 0) {
-                        const uint32_t sb = smem_u32(&sfull[slot]);
-                        const uint32_t dst = smem_u32(slab_base + slot * kDecSlabBytes);
-                        mbar_arrive_expect_tx(sb, (uint32_t)((SYM ? 1 : 2) * kDecSlabArrayBytes));
-                        tma_load_2d(dst, &tmS, 8 * j, rb * kDecRows, sb);
-                        if (!SYM) tma_load_2d(dst + kDecSlabArrayBytes, &tmZ, 8 * j, rb * kDecRows, sb);
-                    }
-                    slab_rb = rb;
-                    slab_j = j;
-                }
-            }
             if (lane == 0) {
                 mbar_arrive_expect_tx(bar, tx);
                 tma_load_2d(st, &tmP, kb * (kDecBlockK / 2), rb * kDecRows, bar);
-                tma_load_2d(st + kDecPBytes, &tmX, kb * kDecBlockK, 0, bar);
             }
-            // without TMA slabs: scales (and zeros) of the unit's 256 rows into the stage,
-            // [array][row][GU] bf16
             const uint32_t sz = st + (uint32_t)a.sz_off;
             if (G != 0 && a.sz_tma) {
                 // scales come with the slab ring
@@ -447,8 +440,70 @@ __global__ void __launch_bounds__(kDecThreads, 1)
                     mbar_arrive(bar);
                 }
             }
+        };
+        auto load_x = [&](int kb, int s) {
+            if (lane == 0)
+                tma_load_2d(stages_u32 + (uint32_t)(s * a.stage_bytes) + kDecPBytes, &tmX, kb * kDecBlockK, 0,
+                            smem_u32(&full[s]));
+        };
+
+        UnitWalk wk;
+        wk.init(u0, u1, a.KBn);
+        // With weights that the previous grid on the stream does not write, the
+        // first ring's worth of units (as far as their slabs fit the slab ring
+        // without waiting for a release) is requested before the dependency
+        // wait, so the weight stream starts while the previous grid drains; only
+        // X waits.  Otherwise nothing is read before the wait.
+        int P = 0;
+        bool ok = true;
+        if (a.early) {
+            const int pmax = min(S, nunits);
+            for (; P < pmax; ++P) {
+                UnitWalk nx = wk;
+                if (P > 0) nx.advance();
+                if (new_slab(nx.rb, nx.kb)) {
+                    if (slab_t + 1 >= SL) break;
+                    if (!request_slab(nx.rb, nx.kb)) {   // a fresh slot: no wait
+                        ok = false;
+                        break;
+                    }
+                }
+                wk = nx;
+                load_weights(wk.rb, wk.kb, P);
+            }
+        }
+        grid_dependency_wait();              // X (and, without `early`, the weights) may be the previous grid's output
+        if (P > 0) {
+            UnitWalk xw;
+            xw.init(u0, u1, a.KBn);
+            for (int i = 0; i < P; ++i) {
+                if (i > 0) xw.advance();
+                load_x(xw.kb, i);
+            }
+        }
+        int issued = P;
+        int s = P > 0 ? P - 1 : 0;
+        uint32_t ph = 0;
+        for (int i = P; i < nunits && ok; ++i) {
+            if (i > 0) {
+                wk.advance();
+                if (++s == S) { s = 0; ph ^= 1u; }
+            }
+            const int rb = wk.rb, kb = wk.kb;
+            if (lane == 0) ok = mbar_wait_backoff(smem_u32(&empty[s]), ph ^ 1u, kDecProducerSleepNs);
+            if (!__shfl_sync(0xffffffffu, ok ? 1 : 0, 0)) {
+                ok = false;
+                break;
+            }
+            if (new_slab(rb, kb) && !request_slab(rb, kb)) {
+                ok = false;
+                break;
+            }
+            load_weights(rb, kb, s);
+            load_x(kb, s);
             ++issued;
         }
+        if (!ok) *abort_flag = 1;
         // Do not leave while copies into this CTA's shared memory are in flight.
         if (lane == 0) {
             for (int i = (issued > S ? issued - S : 0); i < issued; ++i) {
@@ -537,7 +592,9 @@ __global__ void __launch_bounds__(kDecThreads, 1)
     const int srow0 = (16 * w + g) * SW * 2;         // within the stage's scale area or a slab
     const int srow8 = 8 * SW * 2;                     // row r0 + 8
     const bool tma_slab = G != 0 && a.sz_tma;
-    int slab_t = -1, slab_rb = -1, slab_j = -1;      // the slab the consumers read
+    int slab_rb = -1, slab_j = -1;                   // the slab the consumers read
+    int slab_slot = -1;                              // its slot (-1: none yet)
+    uint32_t slab_ph = 1u;                           // parity of its use of the slot
     const uint8_t* slab_ptr = slab_base;
     const uint32_t nib = opaque_u32(0x000F000Fu);     // nibble-pair mask, held in a register
     const uint32_t zz_sym = opaque_u32(0x43084308u);  // 128 + 8 for symmetric codes
@@ -589,17 +646,17 @@ __global__ void __launch_bounds__(kDecThreads, 1)
                     // move to the unit's slab when it changes: release the old slot, wait for the new
                     const int j = (kb * GU) >> 3;
                     if (rb != slab_rb || j != slab_j) {
-                        if (slab_t >= 0) {
+                        if (slab_slot >= 0) {
                             __syncwarp();
-                            if (lane == 0) mbar_arrive(smem_u32(&sempty[slab_t % SL]));
+                            if (lane == 0) mbar_arrive(smem_u32(&sempty[slab_slot]));
                         }
-                        ++slab_t;
-                        const int slot = slab_t % SL;
-                        if (!mbar_wait(smem_u32(&sfull[slot]), (uint32_t)(slab_t / SL) & 1u)) {
+                        if (++slab_slot == SL) slab_slot = 0;
+                        if (slab_slot == 0) slab_ph ^= 1u;
+                        if (!mbar_wait(smem_u32(&sfull[slab_slot]), slab_ph)) {
                             *abort_flag = 1;
                             have = false;
                         }
-                        slab_ptr = slab_base + slot * kDecSlabBytes;
+                        slab_ptr = slab_base + slab_slot * kDecSlabBytes;
                         slab_rb = rb;
                         slab_j = j;
                     }
@@ -711,8 +768,8 @@ __global__ void __launch_bounds__(kDecThreads, 1)
         }
         // first owner: wait until every other owner has published (each lane
         // acquires the flags itself, so its reads of the parts follow them), load
-        // the parts eight at a time (one round trip for most row blocks) and add
-        // them in CTA order, then write Y
+        // the parts eight at a time, four with two column blocks (one round trip
+        // for most row blocks), and add them in CTA order, then write Y
         bool ok = true;
         for (int64_t p = c_first + 1; p <= c_last && ok; ++p)
             ok = wait_flag(a.ws_flag + (rb + p) * kDecConsumers + w);
@@ -720,10 +777,11 @@ __global__ void __launch_bounds__(kDecThreads, 1)
             *abort_flag = 1;
             continue;
         }
-        for (int64_t p0 = c_first + 1; p0 <= c_last; p0 += 8) {
-            float4 v[8][MB];
+        constexpr int PB = 8 / MB;           // parts per round trip, within the register budget
+        for (int64_t p0 = c_first + 1; p0 <= c_last; p0 += PB) {
+            float4 v[PB][MB];
 #pragma unroll
-            for (int k = 0; k < 8; ++k)
+            for (int k = 0; k < PB; ++k)
 #pragma unroll
                 for (int mb = 0; mb < MB; ++mb)
                     v[k][mb] = p0 + k <= c_last
@@ -731,7 +789,7 @@ __global__ void __launch_bounds__(kDecThreads, 1)
                                                               (4 * MB) + 4 * mb)
                                    : make_float4(0.0f, 0.0f, 0.0f, 0.0f);
 #pragma unroll
-            for (int k = 0; k < 8; ++k) {
+            for (int k = 0; k < PB; ++k) {
                 if (p0 + k > c_last) break;
 #pragma unroll
                 for (int mb = 0; mb < MB; ++mb) {

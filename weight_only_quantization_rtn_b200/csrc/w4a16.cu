@@ -465,7 +465,7 @@ int decode_scale_copy(int gu, int64_t groups) {
 w4a16_status launch_decode(const w4a16_plan& p, const void* X, int64_t M, int64_t K,
                            const void* packed, const void* scales, const void* zeros, int64_t N,
                            int32_t g, int32_t sym, void* Y, void* workspace, cudaStream_t stream,
-                           const void* act_scale = nullptr) {
+                           const void* act_scale = nullptr, bool static_weights = false) {
     const DecodeGeometry d = decode_geometry(M, N, K, g);
     CUtensorMap tmP, tmX;
     w4a16_status st = encode_2d(&tmP, CU_TENSOR_MAP_DATA_TYPE_UINT8, packed, (uint64_t)(K / 2),
@@ -511,6 +511,7 @@ w4a16_status launch_decode(const w4a16_plan& p, const void* X, int64_t M, int64_
             if (st != W4A16_OK) return st;
         }
     }
+    args.early = static_weights ? 1 : 0;
     args.U = d.units;
     const int gsel = pc ? 0 : g;                   // kernel group size, 0 = per-channel
 #define W4A16_DEC_G(MBV, SYMV)                                                          \
@@ -703,6 +704,8 @@ w4a16_status gemm_impl(const void* X, int64_t M, int64_t K, const void* packed, 
                        const void* zeros, int64_t N, int32_t g, int32_t sym, const void* act_scale,
                        void* Y, void* workspace, size_t workspace_bytes, int32_t path, int32_t ctas,
                        void* stream) {
+    const bool static_weights = (path & W4A16_STATIC_WEIGHTS) != 0;
+    path &= ~W4A16_STATIC_WEIGHTS;
     w4a16_plan p;
     w4a16_status st = make_plan(M, N, K, g, sym, path, ctas, current_sm_count(), &p);
     if (st != W4A16_OK) return st;
@@ -718,7 +721,8 @@ w4a16_status gemm_impl(const void* X, int64_t M, int64_t K, const void* packed, 
     if ((st = device_info(&di)) != W4A16_OK) return st;
     cudaStream_t s = static_cast<cudaStream_t>(stream);
     if (p.path == W4A16_PATH_DECODE)
-        return launch_decode(p, X, M, K, packed, scales, zeros, N, g, sym, Y, workspace, s, act_scale);
+        return launch_decode(p, X, M, K, packed, scales, zeros, N, g, sym, Y, workspace, s, act_scale,
+                             static_weights);
     if (act_scale) {
         // Large M: every X tile is read by all N/128 CTAs of its row of tiles, so X' is
         // formed once, by an elementwise pass into the workspace, rather than per tile.
@@ -839,7 +843,7 @@ size_t w4a16_gemm_workspace_size(int64_t M, int64_t N, int64_t K, int32_t g) {
 w4a16_status w4a16_gemm_plan(int64_t M, int64_t N, int64_t K, int32_t g, int32_t sym,
                              int32_t path, int32_t ctas, w4a16_plan* plan) {
     if (!plan) return W4A16_EINVAL;
-    return make_plan(M, N, K, g, sym, path, ctas, current_sm_count(), plan);
+    return make_plan(M, N, K, g, sym, path & ~W4A16_STATIC_WEIGHTS, ctas, current_sm_count(), plan);
 }
 
 w4a16_status w4a16_gemm_ex(const void* X, int64_t M, int64_t K, const void* packed,
