@@ -235,8 +235,8 @@ w4a16_status w4a16_gemm_plan(int64_t M, int64_t N, int64_t K, int32_t g, int32_t
  * W4A16_NOALLOC_SCRATCH_BYTES that every GPU which loads the library keeps
  * until the process exits.  Returns W4A16_EWORKSPACE, launching nothing, when
  * the problem needs more scratch than that (its plan's workspace_bytes: about
- * 2000 row blocks plus CTAs at M ≤ 8, 1000 at M 9–16, i.e. N up to roughly
- * 220 000 and 90 000 rows on 148 SMs), and W4A16_EINVAL for M > 16 or any
+ * 1000 row blocks plus CTAs at M ≤ 8, 500 at M 9–16, i.e. N up to roughly
+ * 218 000 and 90 000 rows on 148 SMs), and W4A16_EINVAL for M > 16 or any
  * argument w4a16_gemm_ex would reject.
  * The first call on a device looks up the array's device address for that
  * device (cudaGetSymbolAddress, with the device current).  All calls share the
