@@ -706,8 +706,9 @@ def workload_extras(w4, names, peaks, peak_src, l2, dev, decode_iters=400, tenso
 
 def w8a16_extras(w4, peaks, l2, dev, iters=200):
     """W8A16 (8-bit codes, one per byte) at g=128 asym: quantize/pack and
-    dequantize of a 7B-shaped weight (N=11008, K=4096), the fused M=1 GEMV over
-    both 7B-shaped layers, and the tensor-core kernel at M=2048, K=N=8192, with
+    dequantize of a 7B-shaped weight (N=11008, K=4096), the fused M=1 decode GEMM
+    over both 7B-shaped and both 70B-shaped layers, and the tensor-core kernel at
+    M=2048, K=N=8192, with
     inputs rotated past L2 and graph-replayed.
     Bytes: quantize reads W and writes codes + scales + zeros; dequantize the
     reverse; the GEMV reads codes + scales + zeros + X and writes Y."""
@@ -729,28 +730,34 @@ def w8a16_extras(w4, peaks, l2, dev, iters=200):
     dms = time_graphs(gs, 20)
     del gs, Ws, outs, Wh, W
     qb = db = N * K * 2 + N * K + meta
-    # fused GEMV, M=1, both layers per step
-    per_step = sum(l.N * l.K + 4 * l.N * (l.K // g) + 2 * l.K for l in layers)
-    gcopies = copies_for(per_step, l2)
-    sets = []
-    for l in layers:
-        C, S, Z = w4.quantize8(l.weight().to(dev), g, sym)
-        X = l.activation(1).to(dev)
-        Y = torch.empty(1, l.N, dtype=torch.bfloat16, device=dev)
-        sets.append([(C, S, Z, X, Y)] + [(C.clone(), S.clone(), Z.clone(), X.clone(), Y)
-                                         for _ in range(gcopies - 1)])
+    # fused decode GEMM, M=1, both layers per step: the 7B- and the 70B-shaped pair
+    def decode_step_ms(layers):
+        per_step = sum(l.N * l.K + 4 * l.N * (l.K // g) + 2 * l.K for l in layers)
+        gcopies = copies_for(per_step, l2)
+        sets = []
+        for l in layers:
+            C, S, Z = w4.quantize8(l.weight().to(dev), g, sym)
+            X = l.activation(1).to(dev)
+            Y = torch.empty(1, l.N, dtype=torch.bfloat16, device=dev)
+            sets.append([(C, S, Z, X, Y)] + [(C.clone(), S.clone(), Z.clone(), X.clone(), Y)
+                                             for _ in range(gcopies - 1)])
 
-    def step(i):
-        for cs in sets:
-            C, S, Z, X, Y = cs[i % gcopies]
-            w4.gemm8(X, C, S, Z, g, sym, out=Y)
+        def step(i):
+            for cs in sets:
+                C, S, Z, X, Y = cs[i % gcopies]
+                w4.gemm8(X, C, S, Z, g, sym, out=Y)
 
-    gs = graph_of(step, gcopies)
-    gms = time_graphs(gs, iters)
-    del gs, sets
-    torch.cuda.empty_cache()
-    gbytes = sum(algorithmic_bytes(1, l.N, l.K, g, sym) + l.N * l.K // 2 for l in layers)
+        gs = graph_of(step, gcopies)
+        ms = time_graphs(gs, iters)
+        del gs, sets
+        torch.cuda.empty_cache()
+        nbytes = sum(algorithmic_bytes(1, l.N, l.K, g, sym) + l.N * l.K // 2 for l in layers)
+        return ms, nbytes
+
+    gms, gbytes = decode_step_ms(layers)
     gbs = gbytes / (gms / 1e3) / 1e9
+    gms70, gbytes70 = decode_step_ms(workloads.DECODE_70B.layers)
+    gbs70 = gbytes70 / (gms70 / 1e3) / 1e9
     # tensor-core kernel with 8-bit codes: prefill M=2048, K=N=8192
     P = workloads.PREFILL.layers[0]
     M = 2048
@@ -773,7 +780,10 @@ def w8a16_extras(w4, peaks, l2, dev, iters=200):
             "quantize": {"us": qms * 1e3, "GB/s": qb / (qms / 1e3) / 1e9, "frac": qb / (qms / 1e3) / 1e9 / pk},
             "dequantize": {"us": dms * 1e3, "GB/s": db / (dms / 1e3) / 1e9, "frac": db / (dms / 1e3) / 1e9 / pk},
             "gemv_M1": {"us_per_step": gms * 1e3, "bytes_per_step": gbytes, "GB/s": gbs,
-                        "frac": gbs / pk, "kernel": "w8_gemv_kernel"},
+                        "frac": gbs / pk, "kernel": "gemv_decode_kernel (8-bit codes)"},
+            "gemv_M1_70b": {"us_per_step": gms70 * 1e3, "bytes_per_step": gbytes70, "GB/s": gbs70,
+                            "frac": gbs70 / pk, "kernel": "gemv_decode_kernel (8-bit codes)",
+                            "layers_KxN": [[l.K, l.N] for l in workloads.DECODE_70B.layers]},
             "prefill_2048x8192x8192": {"us": pms * 1e3, "TFLOP/s": ptf,
                                        "frac": ptf / peaks["bf16_tflops"],
                                        "kernel": "gemm_tc_kernel (8-bit codes)"}}

@@ -270,15 +270,26 @@ w4a16_status w8a16_dequantize(const void* codes, const void* scales, const void*
                               int64_t N, int64_t K, int32_t g, int32_t sym, void* W_hat,
                               void* stream);
 
-/* Bytes of device workspace w8a16_gemm needs: 0 for M ≤ 16; for larger M the
- * tensor-core kernel's split-K partial tiles, as w4a16_gemm_workspace_size
- * describes.  Uses the current device's SM count; 0 for rejected shapes. */
+/* Bytes of device workspace w8a16_gemm needs: for M ≤ 16 the decode kernel's
+ * split row blocks (the same layout and size rule as w4a16_gemm_workspace_size:
+ * it depends on the row blocks and the grid), for larger M the tensor-core
+ * kernel's split-K partial tiles.  Uses the current device's SM count; 0 for
+ * rejected shapes.  (Before ABI version 4 the M ≤ 16 path needed none.) */
 size_t w8a16_gemm_workspace_size(int64_t M, int64_t N, int64_t K, int32_t g);
+
+/* Host-only: the launch w8a16_gemm would make (decode kernel for M ≤ 16, else
+ * the tensor-core kernel, both with 8-bit codes), including its workspace.
+ * Returns W4A16_EINVAL for shapes w8a16_gemm would reject. */
+w4a16_status w8a16_gemm_plan(int64_t M, int64_t N, int64_t K, int32_t g, int32_t sym,
+                             w4a16_plan* plan);
 
 /* Fused W8A16 GEMM: Y[M, N] = X[M, K] · Ŵ[N, K]ᵀ with Ŵ = bf16_rn((q − z)·s)
  * formed on chip, binary32 accumulation, one rounding of each output to bf16;
- * deterministic.  M ≤ 16: one warp per weight row streams the row's codes with
- * 16-byte loads (no workspace).  M > 16: the tensor-core kernel with 8-bit
+ * deterministic.  M ≤ 16: the decode kernel with 8-bit codes (units of 256
+ * rows x 128 K, i.e. the same 32 KB TMA tiles; each word of 4 codes becomes two
+ * bf16 pairs — the byte in a binary32 mantissa, 2^23 + z subtracted, the exact
+ * product with s rounded once — and feeds one mma.sync; split row blocks are
+ * finished in the kernel, as for INT4).  M > 16: the tensor-core kernel with 8-bit
  * codes (64-byte code rows per K block, binary32-exact dequantization into the
  * shared-memory A tile, tcgen05 MMA), split-K as for INT4.  workspace: at least
  * w8a16_gemm_workspace_size() bytes, 16-byte aligned, when that is nonzero;

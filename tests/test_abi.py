@@ -34,7 +34,7 @@ def test_header_declares_the_abi():
     for n in ("w4a16_quantize", "w4a16_dequantize", "w4a16_gemm", "w4a16_gemm_ex",
               "w4a16_gemm_workspace_size", "w4a16_gemm_plan", "w4a16_status_string",
               "w4a16_device_error", "w4a16_abi_version", "w8a16_quantize", "w8a16_dequantize",
-              "w8a16_gemm"):
+              "w8a16_gemm", "w8a16_gemm_plan"):
         assert n in names
 
 
@@ -260,6 +260,22 @@ def test_decode_stage_layout_is_valid_for_every_shape(M):
                 assert p["stages"] >= 2 and p["smem_bytes"] <= 232448
 
 
+@pytest.mark.parametrize("M", list(range(1, 17)))
+def test_w8_decode_stage_layout_is_valid_for_every_shape(M):
+    """The same layout checks for the decode kernel with 8-bit codes (units of
+    256 rows x 128 K, X rows of 256 bytes, the pair-copy mode for one scale group
+    per unit): every M, g and a spread of K and N plans without EUNSUPPORTED."""
+    for K in (32, 64, 96, 128, 160, 256, 384, 1024, 1056, 2304, 4096, 4352, 5376, 11008, 28672):
+        for g in (32, 64, 128, K):
+            if K % g:
+                continue
+            for N in (1, 128, 1000, 28672):
+                p = w4.plan8(M, N, K, g, False)
+                assert p["path"] == "decode" and p["stages"] >= 2 and p["smem_bytes"] <= 232448
+                assert p["threads"] == 576 and p["grid"] == min(148, -(-N // 256) * -(-K // 128))
+    assert w4.plan8(17, 4096, 4096)["path"] == "tensorcore"
+
+
 def _owner(u, U, C):
     return ((u + 1) * C - 1) // U
 
@@ -407,7 +423,9 @@ def test_w8a16_entry_points_reject_invalid(lib):
     assert gm(X, 0, 128, FAKE, S, Z, 64, 128, 0, Y, FAKE, big, None) == 0         # empty: no launch
     assert gm(X, 4, 128, FAKE, S, Z, 0, 128, 0, Y, FAKE, big, None) == 0
     ws = lib.w8a16_gemm_workspace_size
-    assert ws(16, 4096, 4096, 128) == 0                     # the GEMV needs none
+    # M ≤ 16: the decode kernel with 8-bit codes; its workspace depends on the row
+    # blocks and the grid only, so it equals the INT4 one when both grids are full
+    assert ws(16, 4096, 4096, 128) == w4.workspace_size(16, 4096, 4096, 128) > 0
     assert ws(17, 8192, 8192, 32) == w4.workspace_size(17, 8192, 8192, 32) > 0
     assert ws(2048, 8192, 8192, 128) == w4.workspace_size(2048, 8192, 8192, 128)
 

@@ -129,6 +129,27 @@ def test_w8_gemm_deterministic_and_7b_full_size():
 
 
 @pytest.mark.parametrize("sym", [False, True])
+@pytest.mark.parametrize("li", [0, 1])
+def test_w8_decode_70b_full_size(li, sym):
+    """The decode kernel with 8-bit codes on a 70B-shaped layer (M=1; the stream-K
+    partition splits row blocks between CTAs), on sampled outputs including the
+    last row."""
+    layer = workloads.DECODE_70B.layers[li]
+    W, X = layer.weight(), layer.activation(1)
+    C, S, Z = w4.quantize8(W.cuda(), 128, sym)
+    Y = w4.gemm8(X.cuda(), C, S, Z, 128, sym)
+    torch.cuda.synchronize()
+    rng = np.random.default_rng(13 + li)
+    ns = rng.integers(0, layer.N, 1024)
+    ns[:2] = [0, layer.N - 1]
+    ms = np.zeros_like(ns)
+    ref = oracle.gemm_w8a16_sampled(workloads.bits(X), C.cpu().numpy(), workloads.bits(S),
+                                    workloads.bits(Z), 128, sym, ms, ns)
+    assert_y_close(workloads.bits(Y)[ms, ns], ref, f"W8 70B-shaped layer {li} sym={sym}")
+    assert w4.device_error() == 0
+
+
+@pytest.mark.parametrize("sym", [False, True])
 @pytest.mark.parametrize("g", [32, 64, 128, 0])
 @pytest.mark.parametrize("M,N,K", [(17, 128, 96), (33, 384, 512), (48, 1000, 4352),
                                    (129, 64, 4096), (300, 700, 1056), (600, 1000, 1024)])

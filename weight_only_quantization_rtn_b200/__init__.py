@@ -17,7 +17,7 @@ import os
 
 import torch
 
-__all__ = ["lib", "quantize", "dequantize", "gemm", "gemm_decode_noalloc", "plan",
+__all__ = ["lib", "quantize", "dequantize", "gemm", "gemm_decode_noalloc", "plan", "plan8",
            "quantize8", "dequantize8", "gemm8",
            "workspace_size", "device_error", "W4A16Error", "PATH_AUTO", "PATH_DECODE", "PATH_TENSORCORE", "STATIC_WEIGHTS", "LIB_PATH"]
 
@@ -73,11 +73,12 @@ def _load() -> ctypes.CDLL:
     lib.w8a16_dequantize.argtypes = [vp, vp, vp, i64, i64, i32, i32, vp, vp]
     lib.w8a16_gemm.argtypes = [vp, i64, i64, vp, vp, vp, i64, i32, i32, vp, vp, sz, vp]
     lib.w8a16_gemm_workspace_size.argtypes = [i64, i64, i64, i32]
+    lib.w8a16_gemm_plan.argtypes = [i64, i64, i64, i32, i32, ctypes.POINTER(Plan)]
     lib.w8a16_gemm_workspace_size.restype = sz
     for name in ("w4a16_quantize", "w4a16_dequantize", "w4a16_gemm", "w4a16_gemm_ex",
                  "w4a16_gemm_act_scaled",
                  "w4a16_gemm_plan", "w4a16_device_error", "w8a16_quantize", "w8a16_dequantize",
-                 "w8a16_gemm"):
+                 "w8a16_gemm", "w8a16_gemm_plan"):
         getattr(lib, name).restype = ctypes.c_int
     if lib.w4a16_abi_version() != ABI_VERSION:
         raise ImportError(f"{LIB_PATH} has ABI version {lib.w4a16_abi_version()}, this binding "
@@ -173,6 +174,13 @@ def workspace_size(M: int, N: int, K: int, g: int) -> int:
     return int(lib().w4a16_gemm_workspace_size(M, N, K, g))
 
 
+def _plan_dict(p) -> dict:
+    return {"path": {v: k for k, v in _PATHS.items()}[p.path], "tile_m": p.tile_m,
+            "tile_n": p.tile_n, "grid": p.grid, "threads": p.threads,
+            "smem_bytes": p.smem_bytes, "stages": p.stages, "kernels": p.kernels,
+            "workspace_bytes": p.workspace_bytes, "split_tiles": p.split_tiles}
+
+
 def plan(M: int, N: int, K: int, g: int = 128, sym: bool = False, path: str | int = "auto",
          ctas: int = 0) -> dict:
     """The launch w4a16_gemm would make for this shape (host only)."""
@@ -180,10 +188,14 @@ def plan(M: int, N: int, K: int, g: int = 128, sym: bool = False, path: str | in
     pid = _PATHS[path] if isinstance(path, str) else int(path)
     _check(lib().w4a16_gemm_plan(M, N, K, g, int(bool(sym)), pid, ctas, ctypes.byref(p)),
            "w4a16_gemm_plan")
-    return {"path": {v: k for k, v in _PATHS.items()}[p.path], "tile_m": p.tile_m,
-            "tile_n": p.tile_n, "grid": p.grid, "threads": p.threads,
-            "smem_bytes": p.smem_bytes, "stages": p.stages, "kernels": p.kernels,
-            "workspace_bytes": p.workspace_bytes, "split_tiles": p.split_tiles}
+    return _plan_dict(p)
+
+
+def plan8(M: int, N: int, K: int, g: int = 128, sym: bool = False) -> dict:
+    """The launch w8a16_gemm would make for this shape (host only)."""
+    p = Plan()
+    _check(lib().w8a16_gemm_plan(M, N, K, g, int(bool(sym)), ctypes.byref(p)), "w8a16_gemm_plan")
+    return _plan_dict(p)
 
 
 _workspaces: dict = {}
@@ -398,9 +410,9 @@ def gemm8(X: torch.Tensor, codes: torch.Tensor, scales: torch.Tensor,
           zeros: torch.Tensor | None, g: int = 128, sym: bool = False,
           out: torch.Tensor | None = None) -> torch.Tensor:
     """Fused W8A16 GEMM: Y[M, N] = X[M, K] · Ŵ[N, K]ᵀ (bf16 in/out, fp32
-    accumulation), device tensors.  M ≤ 16 runs the warp-per-row GEMV, larger M
-    the tensor-core kernel with 8-bit codes (with a split-K workspace when the
-    library asks for one)."""
+    accumulation), device tensors.  M ≤ 16 runs the decode kernel with 8-bit
+    codes, larger M the tensor-core kernel with 8-bit codes (each with the
+    workspace the library asks for)."""
     _need(X, torch.bfloat16, "X")
     _need(codes, torch.uint8, "codes")
     _need(scales, torch.bfloat16, "scales")

@@ -68,15 +68,19 @@
 namespace w4a16 {
 
 constexpr int kDecRows = 256;                   // weight rows per unit (16 warps x 16)
-constexpr int kDecBlockK = 256;                 // K per unit
-constexpr int kDecPBytes = kDecRows * kDecBlockK / 2;   // packed bytes per unit (32 KB)
+constexpr int kDecUnitRowBytes = 128;          // code bytes of one row per unit (one TMA box row)
+constexpr int kDecPBytes = kDecRows * kDecUnitRowBytes; // code bytes per unit (32 KB)
+// K per unit: 256 four-bit or 128 eight-bit codes per 128-byte row
+template <int BITS> __host__ __device__ constexpr int dec_block_k() { return kDecUnitRowBytes * 8 / BITS; }
 constexpr int kDecConsumers = 16;
 constexpr int kDecProducerWarp = kDecConsumers;
 constexpr int kDecHelperWarp = kDecConsumers + 1;
 constexpr int kDecThreads = (kDecConsumers + 2) * 32;
 constexpr int kDecMaxStages = 8;
-constexpr int kDecXRowBytes = kDecBlockK * 2;   // one X row of a unit, natural order (512 B)
-constexpr int kDecXfRowBytes = 576;             // fragment-ordered X row: 512 B + 64 B pad
+// X rows of a unit: natural order (BK bf16), and in fragment order padded to
+// 64 mod 128 bytes (576 B for 4-bit codes, 320 B for 8-bit codes)
+template <int BITS> __host__ __device__ constexpr int dec_x_row_bytes() { return dec_block_k<BITS>() * 2; }
+template <int BITS> __host__ __device__ constexpr int dec_xf_row_bytes() { return dec_block_k<BITS>() * 2 + 64; }
 constexpr int kDecZeroBytes = 512;              // zero B fragments for columns m >= M
 constexpr int kDecMaxSlabs = 8;
 constexpr int kDecSlabArrayBytes = kDecRows * 8 * 2;    // 8 groups x 256 rows of bf16
@@ -161,7 +165,8 @@ struct DecodeArgs {
     int sz_tma;           // 1: scales by TMA into the slab ring
     int slab_off;         // slab ring: `slabs` slots of [2][256 rows][8] bf16 (8 KB each)
     int slabs;
-    int sz_copy;          // without TMA: bytes per scale copy, 16, 8 or 4 (cp.async), 2 (plain)
+    int sz_copy;          // without TMA: bytes per scale copy, 16, 8 or 4 (cp.async), 2 (plain);
+                          // 3: one group per unit, copied as the 4-byte aligned pair holding it
     int early;            // 1: the previous grid does not write the weights; stream them before the dependency wait
     int64_t U;            // units = RB · KBn
 };
@@ -282,16 +287,34 @@ __device__ __forceinline__ void decode_store_y(const DecodeArgs& a, const float 
         }
 }
 
-template <int MB, bool SYM, int G>
+// Four 8-bit codes of a word -> (q0, q1) and (q2, q3) as bf16 pairs of
+// bf16_rn((q − z)·s).  The byte placed in a binary32 mantissa gives 2^23 + q
+// exactly; subtracting zoff = 2^23 + z leaves q − z (exact), the product with s
+// is exact (8-bit by 8-bit significands), and cvt.rn.bf16x2 rounds once.
+// Symmetric words are XORed with 0x80808080 by the caller (offset-128 codes,
+// zoff = 2^23 + 128).
+__device__ __forceinline__ void dq_word8(uint32_t w, float s, float zoff, uint32_t& lo, uint32_t& hi) {
+    float f[4];
+#pragma unroll
+    for (int i = 0; i < 4; ++i)
+        f[i] = (__uint_as_float(__byte_perm(w, 0x4B000000u, 0x7540u + (uint32_t)i)) - zoff) * s;
+    asm("cvt.rn.bf16x2.f32 %0, %1, %2;" : "=r"(lo) : "f"(f[1]), "f"(f[0]));
+    asm("cvt.rn.bf16x2.f32 %0, %1, %2;" : "=r"(hi) : "f"(f[3]), "f"(f[2]));
+}
+
+template <int MB, bool SYM, int G, int BITS>
 __global__ void __launch_bounds__(kDecThreads, 1)
     gemv_decode_kernel(const __grid_constant__ CUtensorMap tmP,
                        const __grid_constant__ CUtensorMap tmX,
                        const __grid_constant__ CUtensorMap tmS,
                        const __grid_constant__ CUtensorMap tmZ, const DecodeArgs a) {
     // G == 0: per-channel granularity, one scale (and zero) per row for all of K.
-    constexpr int GU = G == 0 ? 1 : kDecBlockK / G;    // scale groups per row per unit
+    constexpr int BK = dec_block_k<BITS>();            // K per unit
+    constexpr int XRB = dec_x_row_bytes<BITS>();
+    constexpr int XFRB = dec_xf_row_bytes<BITS>();
+    constexpr int GU = G == 0 ? 1 : BK / G;            // scale groups per row per unit
     // Groups per staged scale row: a TMA slab of 8 (16 bytes), else the unit's GU.
-    const int SW = a.sz_tma ? 8 : GU;
+    const int SW = a.sz_tma ? 8 : (a.sz_copy == 3 ? 2 : GU);
     const int kSzArray = kDecRows * SW * 2;            // bytes of one scale (or zero) array
 
     extern __shared__ uint8_t smem_raw[];
@@ -352,7 +375,7 @@ __global__ void __launch_bounds__(kDecThreads, 1)
                 if (!SYM) prefetch_tensormap(&tmZ);
             }
         }
-        const uint32_t tx = (uint32_t)kDecPBytes + (uint32_t)M * kDecXRowBytes;
+        const uint32_t tx = (uint32_t)kDecPBytes + (uint32_t)M * XRB;
         const int arrays = SYM ? 1 : 2;
         int slab_t = -1, slab_rb = -1, slab_j = -1;   // slabs requested so far - 1, current slab
         int slab_slot = SL - 1;                       // slab_t mod SL
@@ -392,7 +415,7 @@ __global__ void __launch_bounds__(kDecThreads, 1)
             const uint32_t bar = smem_u32(&full[s]);
             if (lane == 0) {
                 mbar_arrive_expect_tx(bar, tx);
-                tma_load_2d(st, &tmP, kb * (kDecBlockK / 2), rb * kDecRows, bar);
+                tma_load_2d(st, &tmP, kb * kDecUnitRowBytes, rb * kDecRows, bar);
             }
             const uint32_t sz = st + (uint32_t)a.sz_off;
             if (G != 0 && a.sz_tma) {
@@ -422,20 +445,55 @@ __global__ void __launch_bounds__(kDecThreads, 1)
                     }
                     if (cs == 4) copy_scale_rows<GU, 4>(a, sz, kSzArray, rb, g0, arrays, lane);
                     cp_async_arrive_noinc(bar);
+                } else if (cs == 3) {
+                    // one group per unit (8-bit codes at g = 128) and an even number of
+                    // groups per row: the 4-byte aligned pair of groups holding g0, per row
+                    // (the consumers read its half g0 mod 2)
+                    if constexpr (GU == 1) {
+                        const int gp = g0 & ~1;
+                        for (int arr = 0; arr < arrays; ++arr) {
+                            const uint16_t* base = arr == 0 ? a.scales : a.zeros;
+#pragma unroll 4
+                            for (int r = lane; r < kDecRows; r += 32) {
+                                const int n = rb * kDecRows + r;
+                                const bool in = n < a.N && gp < a.Gtot;
+                                cp_async_4(sz + arr * kSzArray + r * 4, base + (in ? (int64_t)n * a.Gtot + gp : 0),
+                                           in ? 4u : 0u);
+                            }
+                        }
+                    }
+                    cp_async_arrive_noinc(bar);
                 } else {
-                    // odd scale rows: two bytes at a time
+                    // odd scale rows: two bytes at a time, eight loads in flight per lane
+                    const int total = kDecRows * GU * arrays;
 #pragma unroll 1
-                    for (int e = lane; e < kDecRows * GU * arrays; e += 32) {
-                        const int arr = e / (kDecRows * GU);
-                        const int rem = e - arr * (kDecRows * GU);
-                        const int r = rem / GU, j = rem - r * GU;
-                        const int n = rb * kDecRows + r;
-                        const bool in = n < a.N && g0 + j < a.Gtot;
-                        const uint16_t* src = arr == 0 ? a.scales : a.zeros;
-                        const uint16_t v = in ? ldg_u16(src + (int64_t)n * a.Gtot + g0 + j) : (uint16_t)0;
-                        asm volatile("st.shared.u16 [%0], %1;" ::"r"(sz + arr * kSzArray + (r * SW + j) * 2),
-                                     "h"(v)
-                                     : "memory");
+                    for (int e0 = lane; e0 < total; e0 += 32 * 8) {
+                        uint16_t v[8];
+#pragma unroll
+                        for (int t = 0; t < 8; ++t) {
+                            const int e = e0 + 32 * t;
+                            v[t] = 0;
+                            if (e < total) {
+                                const int arr = e / (kDecRows * GU);
+                                const int rem = e - arr * (kDecRows * GU);
+                                const int r = rem / GU, j = rem - r * GU;
+                                const int n = rb * kDecRows + r;
+                                const uint16_t* src = arr == 0 ? a.scales : a.zeros;
+                                if (n < a.N && g0 + j < a.Gtot) v[t] = ldg_u16(src + (int64_t)n * a.Gtot + g0 + j);
+                            }
+                        }
+#pragma unroll
+                        for (int t = 0; t < 8; ++t) {
+                            const int e = e0 + 32 * t;
+                            if (e < total) {
+                                const int arr = e / (kDecRows * GU);
+                                const int rem = e - arr * (kDecRows * GU);
+                                const int r = rem / GU, j = rem - r * GU;
+                                asm volatile("st.shared.u16 [%0], %1;" ::"r"(sz + arr * kSzArray + (r * SW + j) * 2),
+                                             "h"(v[t])
+                                             : "memory");
+                            }
+                        }
                     }
                     mbar_arrive(bar);
                 }
@@ -443,7 +501,7 @@ __global__ void __launch_bounds__(kDecThreads, 1)
         };
         auto load_x = [&](int kb, int s) {
             if (lane == 0)
-                tma_load_2d(stages_u32 + (uint32_t)(s * a.stage_bytes) + kDecPBytes, &tmX, kb * kDecBlockK, 0,
+                tma_load_2d(stages_u32 + (uint32_t)(s * a.stage_bytes) + kDecPBytes, &tmX, kb * BK, 0,
                             smem_u32(&full[s]));
         };
 
@@ -519,9 +577,10 @@ __global__ void __launch_bounds__(kDecThreads, 1)
 
     if (warp == kDecHelperWarp) {
         // ---------------------------------------------------------------- helper
-        // X slice of each landed stage, natural order [m][256] -> fragment order:
-        // 16-byte chunk c = 8q + i of row m (elements x0..x7) becomes
+        // X slice of each landed stage, natural order [m][BK] -> fragment order.
+        // 4-bit codes: 16-byte chunk c = 8q + i of row m (elements x0..x7) becomes
         // ((x0,x4),(x1,x5),(x2,x6),(x3,x7)) at row m, slot i, lane-group q.
+        // 8-bit codes: chunk c = 4q + i moves unchanged to slot i, lane-group q.
         int s = 0;
         uint32_t ph = 0;
         UnitWalk wk;
@@ -543,25 +602,30 @@ __global__ void __launch_bounds__(kDecThreads, 1)
             const uint32_t xn = st + kDecPBytes;
             const uint32_t xf = st + (uint32_t)a.xf_off;
 #pragma unroll 1
-            for (int it = lane; it < M * 32; it += 32) {
-                const int m = it >> 5, c = it & 31;
-                uint4 v = lds128_u32addr(xn + m * kDecXRowBytes + c * 16);
+            for (int it = lane; it < M * (BK / 8); it += 32) {
+                constexpr int kShift = BITS == 4 ? 5 : 4;    // chunks of 8 per X row: 32 or 16
+                const int m = it >> kShift, c = it & ((1 << kShift) - 1);
+                uint4 v = lds128_u32addr(xn + m * XRB + c * 16);
                 if (act != nullptr) {
                     // x' = bf16_rn(x·a): the chunk's 8 scales (K is a multiple of 32, so a
                     // chunk is wholly inside or wholly past the end of X, where x = 0)
-                    const int k0 = wk.kb * kDecBlockK + 8 * c;
+                    const int k0 = wk.kb * BK + 8 * c;
                     const uint4 av = k0 < a.K ? ldg_cached(act + k0) : make_uint4(0, 0, 0, 0);
                     v.x = bf16x2_mul(v.x, av.x);
                     v.y = bf16x2_mul(v.y, av.y);
                     v.z = bf16x2_mul(v.z, av.z);
                     v.w = bf16x2_mul(v.w, av.w);
                 }
-                uint4 o;
-                o.x = __byte_perm(v.x, v.z, 0x5410);   // (x0, x4)
-                o.y = __byte_perm(v.x, v.z, 0x7632);   // (x1, x5)
-                o.z = __byte_perm(v.y, v.w, 0x5410);   // (x2, x6)
-                o.w = __byte_perm(v.y, v.w, 0x7632);   // (x3, x7)
-                sts128(xf + m * kDecXfRowBytes + (c & 7) * 64 + (c >> 3) * 16, o);
+                if constexpr (BITS == 4) {
+                    uint4 o;
+                    o.x = __byte_perm(v.x, v.z, 0x5410);   // (x0, x4)
+                    o.y = __byte_perm(v.x, v.z, 0x7632);   // (x1, x5)
+                    o.z = __byte_perm(v.y, v.w, 0x5410);   // (x2, x6)
+                    o.w = __byte_perm(v.y, v.w, 0x7632);   // (x3, x7)
+                    sts128(xf + m * XFRB + (c & 7) * 64 + (c >> 3) * 16, o);
+                } else {
+                    sts128(xf + m * XFRB + (c & 3) * 64 + (c >> 2) * 16, v);
+                }
             }
             __syncwarp();
             if (lane == 0) mbar_arrive(smem_u32(&xfb[s]));
@@ -581,14 +645,15 @@ __global__ void __launch_bounds__(kDecThreads, 1)
     // columns beyond M.
     const bool col0 = g < M;
     const bool col1 = MB > 1 && g + 8 < M;
-    const int xf0 = a.xf_off + g * kDecXfRowBytes + q * 16;
-    const int xf1 = a.xf_off + (g + 8) * kDecXfRowBytes + q * 16;
+    const int xf0 = a.xf_off + g * XFRB + q * 16;
+    const int xf1 = a.xf_off + (g + 8) * XFRB + q * 16;
     const uint4* zero_lane = reinterpret_cast<const uint4*>(zero_ptr) + q;
     // Scale (and zero) byte offsets of rows r0 and r0 + 8 for the groups of this
-    // lane's two chunks (K = 64q + 32h within the unit).
+    // lane's two chunks (4-bit: K = 64q + 32h within the unit; 8-bit: K = 32q +
+    // 16h, one group for both as g ≥ 32).
     constexpr int kG = G == 0 ? 1 : G;
-    const int sgrp0 = G == 0 ? 0 : (64 * q) / kG;
-    const int sgrp1 = G == 0 ? 0 : (64 * q + 32) / kG;
+    const int sgrp0 = G == 0 ? 0 : ((BITS == 4 ? 64 : 32) * q) / kG;
+    const int sgrp1 = G == 0 ? 0 : ((BITS == 4 ? 64 : 32) * q + (BITS == 4 ? 32 : 16)) / kG;
     const int srow0 = (16 * w + g) * SW * 2;         // within the stage's scale area or a slab
     const int srow8 = 8 * SW * 2;                     // row r0 + 8
     const bool tma_slab = G != 0 && a.sz_tma;
@@ -663,9 +728,11 @@ __global__ void __launch_bounds__(kDecThreads, 1)
                     // the unit's groups start at (kb·GU) mod 8 within a slab row
                     sb = slab_ptr + srow0 + ((kb * GU) & 7) * 2;
                 } else {
-                    sb = stp + a.sz_off + srow0;
+                    // (pair copies: the unit's group is the half g0 mod 2 of its 4 bytes)
+                    sb = stp + a.sz_off + srow0 + (a.sz_copy == 3 ? ((kb * GU) & 1) * 2 : 0);
                 }
                 if (have) {
+                if constexpr (BITS == 4) {
                 // scale and zero pairs of rows r0, r0 + 8 for chunk h = 0 (and h = 1 when
                 // the two chunks lie in different groups)
                 uint32_t ss[2][2], zz[2][2];
@@ -717,6 +784,49 @@ __global__ void __launch_bounds__(kDecThreads, 1)
                                 const uint32_t c0 = hh == 0 ? xv1[ii].x : xv1[ii].z;
                                 const uint32_t c1 = hh == 0 ? xv1[ii].y : xv1[ii].w;
                                 mma_bf16_16816_nv(acc[hh][MB - 1], f0, f1, f2, f3, c0, c1);
+                            }
+                        }
+                    }
+                }
+                } else {
+                    // 8-bit codes: one scale group per lane and unit; s and 2^23 + z in binary32
+                    float sf[2], zf[2];
+#pragma unroll
+                    for (int hr = 0; hr < 2; ++hr) {
+                        const uint8_t* sr = sb + sgrp0 * 2 + hr * srow8;
+                        sf[hr] = bf16_bits_to_f32(*reinterpret_cast<const uint16_t*>(sr));
+                        zf[hr] = SYM ? 8388736.0f
+                                     : 8388608.0f + bf16_bits_to_f32(*reinterpret_cast<const uint16_t*>(
+                                                        sr + (tma_slab ? kDecSlabArrayBytes : kSzArray)));
+                    }
+                    const uint32_t flip = SYM ? 0x80808080u : 0u;
+#pragma unroll
+                    for (int h = 0; h < 2; ++h) {
+                        const uint8_t* ap = stp + (h == 0 ? a_off0 : a_off1);
+                        const uint4 va = *reinterpret_cast<const uint4*>(ap);
+                        const uint4 vb = *reinterpret_cast<const uint4*>(ap + 1024);
+                        const uint32_t w0[4] = {va.x ^ flip, va.y ^ flip, va.z ^ flip, va.w ^ flip};
+                        const uint32_t w1[4] = {vb.x ^ flip, vb.y ^ flip, vb.z ^ flip, vb.w ^ flip};
+                        // X of this lane's chunk: 16 values at slots 2h, 2h + 1
+                        uint4 xv0[2], xv1[2];
+#pragma unroll
+                        for (int j = 0; j < 2; ++j) {
+                            xv0[j] = xp0[(2 * h + j) * 4];
+                            xv1[j] = MB > 1 ? xp1[(2 * h + j) * 4] : make_uint4(0, 0, 0, 0);
+                        }
+#pragma unroll
+                        for (int ii = 0; ii < 4; ++ii) {
+                            // word ii = codes K .. K+3: (q0,q1) as the low k pair, (q2,q3) high
+                            uint32_t f0, f1, f2, f3;
+                            dq_word8(w0[ii], sf[0], zf[0], f0, f2);
+                            dq_word8(w1[ii], sf[1], zf[1], f1, f3);
+                            const uint4 xa = xv0[ii >> 1];
+                            mma_bf16_16816_nv(acc[ii & 1][0], f0, f1, f2, f3, (ii & 1) ? xa.z : xa.x,
+                                              (ii & 1) ? xa.w : xa.y);
+                            if (MB > 1) {
+                                const uint4 xb = xv1[ii >> 1];
+                                mma_bf16_16816_nv(acc[ii & 1][MB - 1], f0, f1, f2, f3, (ii & 1) ? xb.z : xb.x,
+                                                  (ii & 1) ? xb.w : xb.y);
                             }
                         }
                     }

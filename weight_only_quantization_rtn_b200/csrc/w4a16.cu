@@ -15,13 +15,6 @@
 
 using namespace w4a16;
 
-namespace w8 {
-// The 8-bit-code GEMV for M ≤ 16 (csrc/w8a16.cu).
-w4a16_status w8_gemv_launch(const void* X, int64_t M, int64_t K, const void* codes,
-                            const void* scales, const void* zeros, int64_t N, int32_t g,
-                            int32_t sym, void* Y, int sm_count, cudaStream_t stream);
-}
-
 namespace {
 
 constexpr int kMaxDevices = 64;
@@ -101,11 +94,13 @@ constexpr int kMaxCtas = 65535;
 // SM with a ring of shared-memory stages and scale slabs filling its shared
 // memory.
 struct DecodeGeometry {
+    int bits;          // code width, 4 or 8
     int mb;            // n8 MMA column blocks (1: M ≤ 8, 2: M ≤ 16)
     int rb;            // row blocks of 256 rows
     int kbn;           // K blocks of 256
     int64_t units;     // rb · kbn
     int gu;            // scale groups per row per unit (1 for per-channel)
+    int sw;            // groups per staged scale row without TMA slabs (0 with them)
     int sz_tma;        // scales staged by TMA in 8-group slabs (rows 16-byte aligned)
     int slabs;         // slab ring slots (0 without TMA slabs)
     int slab_off;      // slab ring inside the dynamic shared memory
@@ -122,26 +117,36 @@ struct DecodeGeometry {
 constexpr int kDecFixedSmem = 1024 + 1024;
 
 // Scale (and zero) groups of one row inside a 256-wide K block.
-int decode_unit_groups(int32_t g, int64_t K) { return per_channel(g, K) ? 1 : kDecBlockK / g; }
+int decode_block_k(int bits) { return bits == 8 ? dec_block_k<8>() : dec_block_k<4>(); }
+int decode_unit_groups(int32_t g, int64_t K, int bits) {
+    return per_channel(g, K) ? 1 : decode_block_k(bits) / g;
+}
 
 // Stage: codes tile (16 KB, TMA, 128-byte swizzle) | X slice, natural order
 // (M x 512 B, TMA) | X in fragment order (rows 576 B apart, the last one 512 B;
 // 128-byte aligned) | without TMA slabs, scales and zeros (2 x 256 rows x gu bf16).
-DecodeGeometry decode_geometry(int64_t M, int64_t N, int64_t K, int g) {
+DecodeGeometry decode_geometry(int64_t M, int64_t N, int64_t K, int g, int bits = 4) {
     DecodeGeometry d{};
+    d.bits = bits;
     d.mb = M <= 8 ? 1 : 2;
     d.rb = (int)((N + kDecRows - 1) / kDecRows);
-    d.kbn = (int)((K + kDecBlockK - 1) / kDecBlockK);
+    const int bk = decode_block_k(bits);
+    const int xrb = bk * 2, xfrb = bk * 2 + 64;   // X rows: natural, fragment order (padded)
+    d.kbn = (int)((K + bk - 1) / bk);
     d.units = (int64_t)d.rb * d.kbn;
-    d.gu = decode_unit_groups(g, K);
+    d.gu = decode_unit_groups(g, K, bits);
     d.sz_tma = (!per_channel(g, K) && (K / g) % 8 == 0) ? 1 : 0;
     const int m = M < 1 ? 1 : (int)M;
-    const int xnat_end = kDecPBytes + m * kDecXRowBytes;
+    const int xnat_end = kDecPBytes + m * xrb;
     d.xf_off = (xnat_end + 127) / 128 * 128;
-    const int xf_end = d.xf_off + (m - 1) * kDecXfRowBytes + kDecXRowBytes;
+    const int xf_end = d.xf_off + (m - 1) * xfrb + xrb;
     d.sz_off = (xf_end + 127) / 128 * 128;      // TMA destinations are 128-byte aligned
     // Scales in the stage only without TMA slabs; with them, a ring of slab slots.
-    const int stage_raw = d.sz_off + (d.sz_tma ? 0 : 2 * kDecRows * d.gu * 2);
+    // A unit with a single group whose rows hold an even number of groups stages
+    // the 4-byte aligned pair around it (the copy mode decode_scale_copy picks).
+    const bool pairs = !d.sz_tma && !per_channel(g, K) && d.gu == 1 && (K / g) % 2 == 0;
+    d.sw = d.sz_tma ? 0 : (pairs ? 2 : d.gu);
+    const int stage_raw = d.sz_off + 2 * kDecRows * d.sw * 2;
     d.stage_bytes = (stage_raw + 1023) / 1024 * 1024;
     // Slab slots: one the consumers read, plus enough for the units the producer
     // may run ahead (the ring depth) at 8/gu units per slab, plus one for a slab
@@ -175,10 +180,11 @@ DecodeGeometry decode_geometry(int64_t M, int64_t N, int64_t K, int g) {
 // and the ring within the shared memory of one CTA.
 bool decode_geometry_ok(const DecodeGeometry& d, int64_t M) {
     const int m = M < 1 ? 1 : (int)M;
-    const int sw = d.sz_tma ? 0 : d.gu;        // scales in the stage only without slabs
-    return d.stage_bytes % 1024 == 0 && kDecPBytes % 128 == 0 && d.xf_off % 128 == 0 &&
-           d.xf_off >= kDecPBytes + m * kDecXRowBytes && d.sz_off % 128 == 0 &&
-           d.sz_off >= d.xf_off + (m - 1) * kDecXfRowBytes + kDecXRowBytes &&
+    const int sw = d.sw;                       // scales in the stage only without slabs
+    const int xrb = decode_block_k(d.bits) * 2, xfrb = xrb + 64;
+    return (d.bits == 4 || d.bits == 8) && d.stage_bytes % 1024 == 0 && kDecPBytes % 128 == 0 &&
+           d.xf_off % 128 == 0 && d.xf_off >= kDecPBytes + m * xrb && d.sz_off % 128 == 0 &&
+           d.sz_off >= d.xf_off + (m - 1) * xfrb + xrb &&
            (kDecRows * sw * 2) % 128 == 0 && d.sz_off + 2 * kDecRows * sw * 2 <= d.stage_bytes &&
            d.stages >= 2 && d.stages <= kDecMaxStages && d.slab_off % 1024 == 0 &&
            (d.sz_tma ? d.slabs >= 2 && d.slabs <= kDecMaxSlabs : d.slabs == 0) &&
@@ -310,7 +316,7 @@ w4a16_status make_plan(int64_t M, int64_t N, int64_t K, int32_t g, int32_t sym, 
     *p = w4a16_plan{};
     p->path = chosen;
     if (chosen == W4A16_PATH_DECODE) {
-        const DecodeGeometry d = decode_geometry(M, N, K, g);
+        const DecodeGeometry d = decode_geometry(M, N, K, g, bits);
         if (!decode_geometry_ok(d, M)) return W4A16_EUNSUPPORTED;
         // At most one resident wave: the CTA that finishes a split row block waits
         // for parts from its neighbours, which must be running too.
@@ -422,11 +428,11 @@ w4a16_status encode_2d(CUtensorMap* map, CUtensorMapDataType dtype, const void* 
 }
 
 // ---------------------------------------------------------------- decode launch
-template <int MB, bool SYM, int G>
+template <int MB, bool SYM, int G, int BITS>
 w4a16_status launch_decode_t(const w4a16_plan& p, const CUtensorMap& tmP, const CUtensorMap& tmX,
                              const CUtensorMap& tmS, const CUtensorMap& tmZ,
                              const DecodeArgs& args, cudaStream_t stream) {
-    auto kern = gemv_decode_kernel<MB, SYM, G>;
+    auto kern = gemv_decode_kernel<MB, SYM, G, BITS>;
     static bool attr_set[kMaxDevices] = {};
     int dev = 0;
     cudaGetDevice(&dev);
@@ -459,21 +465,24 @@ w4a16_status launch_decode_t(const w4a16_plan& p, const CUtensorMap& tmP, const 
 int decode_scale_copy(int gu, int64_t groups) {
     for (int cs = 16; cs >= 4; cs /= 2)
         if (cs <= gu * 2 && (gu * 2) % cs == 0 && (groups * 2) % cs == 0) return cs;
+    // one group per unit (8-bit codes at g = 128): the aligned pair holding it
+    if (gu == 1 && groups % 2 == 0) return 3;
     return 2;
 }
 
 w4a16_status launch_decode(const w4a16_plan& p, const void* X, int64_t M, int64_t K,
                            const void* packed, const void* scales, const void* zeros, int64_t N,
                            int32_t g, int32_t sym, void* Y, void* workspace, cudaStream_t stream,
-                           const void* act_scale = nullptr, bool static_weights = false) {
-    const DecodeGeometry d = decode_geometry(M, N, K, g);
+                           const void* act_scale = nullptr, bool static_weights = false, int bits = 4) {
+    const DecodeGeometry d = decode_geometry(M, N, K, g, bits);
+    const int bk = decode_block_k(bits);
+    const uint64_t row_bytes = (uint64_t)K * (uint64_t)bits / 8;   // code bytes per weight row
     CUtensorMap tmP, tmX;
-    w4a16_status st = encode_2d(&tmP, CU_TENSOR_MAP_DATA_TYPE_UINT8, packed, (uint64_t)(K / 2),
-                                (uint64_t)N, (uint64_t)(K / 2), kDecBlockK / 2, kDecRows,
-                                CU_TENSOR_MAP_SWIZZLE_128B);
+    w4a16_status st = encode_2d(&tmP, CU_TENSOR_MAP_DATA_TYPE_UINT8, packed, row_bytes, (uint64_t)N,
+                                row_bytes, kDecUnitRowBytes, kDecRows, CU_TENSOR_MAP_SWIZZLE_128B);
     if (st != W4A16_OK) return st;
     st = encode_2d(&tmX, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, X, (uint64_t)K, (uint64_t)M,
-                   (uint64_t)K * 2, kDecBlockK, (uint32_t)M, CU_TENSOR_MAP_SWIZZLE_NONE);
+                   (uint64_t)K * 2, (uint32_t)bk, (uint32_t)M, CU_TENSOR_MAP_SWIZZLE_NONE);
     if (st != W4A16_OK) return st;
     const bool pc = per_channel(g, K);
     DecodeArgs args{};
@@ -514,20 +523,26 @@ w4a16_status launch_decode(const w4a16_plan& p, const void* X, int64_t M, int64_
     args.early = static_weights ? 1 : 0;
     args.U = d.units;
     const int gsel = pc ? 0 : g;                   // kernel group size, 0 = per-channel
-#define W4A16_DEC_G(MBV, SYMV)                                                          \
-    switch (gsel) {                                                                     \
-        case 32: return launch_decode_t<MBV, SYMV, 32>(p, tmP, tmX, tmS, tmZ, args, stream);     \
-        case 64: return launch_decode_t<MBV, SYMV, 64>(p, tmP, tmX, tmS, tmZ, args, stream);     \
-        case 128: return launch_decode_t<MBV, SYMV, 128>(p, tmP, tmX, tmS, tmZ, args, stream);   \
-        case 0: return launch_decode_t<MBV, SYMV, 0>(p, tmP, tmX, tmS, tmZ, args, stream);       \
-        default: return W4A16_EINVAL;                                                   \
+#define W4A16_DEC_G(MBV, SYMV, BV)                                                              \
+    switch (gsel) {                                                                             \
+        case 32: return launch_decode_t<MBV, SYMV, 32, BV>(p, tmP, tmX, tmS, tmZ, args, stream);   \
+        case 64: return launch_decode_t<MBV, SYMV, 64, BV>(p, tmP, tmX, tmS, tmZ, args, stream);   \
+        case 128: return launch_decode_t<MBV, SYMV, 128, BV>(p, tmP, tmX, tmS, tmZ, args, stream); \
+        case 0: return launch_decode_t<MBV, SYMV, 0, BV>(p, tmP, tmX, tmS, tmZ, args, stream);     \
+        default: return W4A16_EINVAL;                                                           \
     }
-    if (d.mb == 1) {
-        if (sym) W4A16_DEC_G(1, true)
-        W4A16_DEC_G(1, false)
+#define W4A16_DEC_MS(BV)                      \
+    if (d.mb == 1) {                          \
+        if (sym) W4A16_DEC_G(1, true, BV)     \
+        W4A16_DEC_G(1, false, BV)             \
+    }                                         \
+    if (sym) W4A16_DEC_G(2, true, BV)         \
+    W4A16_DEC_G(2, false, BV)
+    if (bits == 8) {
+        W4A16_DEC_MS(8)
     }
-    if (sym) W4A16_DEC_G(2, true)
-    W4A16_DEC_G(2, false)
+    W4A16_DEC_MS(4)
+#undef W4A16_DEC_MS
 #undef W4A16_DEC_G
 }
 
@@ -846,6 +861,13 @@ w4a16_status w4a16_gemm_plan(int64_t M, int64_t N, int64_t K, int32_t g, int32_t
     return make_plan(M, N, K, g, sym, path & ~W4A16_STATIC_WEIGHTS, ctas, current_sm_count(), plan);
 }
 
+w4a16_status w8a16_gemm_plan(int64_t M, int64_t N, int64_t K, int32_t g, int32_t sym,
+                             w4a16_plan* plan) {
+    if (!plan) return W4A16_EINVAL;
+    const int path = M <= 16 ? W4A16_PATH_DECODE : W4A16_PATH_TENSORCORE;
+    return make_plan(M, N, K, g, sym, path, 0, current_sm_count(), plan, 8);
+}
+
 w4a16_status w4a16_gemm_ex(const void* X, int64_t M, int64_t K, const void* packed,
                            const void* scales, const void* zeros, int64_t N, int32_t g,
                            int32_t sym, void* Y, void* workspace, size_t workspace_bytes,
@@ -899,9 +921,8 @@ w4a16_status w4a16_gemm_decode_noalloc(const void* X, int64_t M, int64_t K, cons
 
 size_t w8a16_gemm_workspace_size(int64_t M, int64_t N, int64_t K, int32_t g) {
     w4a16_plan p;
-    if (M <= 16) return 0;                                  // the GEMV needs no workspace
-    if (make_plan(M, N, K, g, 0, W4A16_PATH_TENSORCORE, 0, current_sm_count(), &p, 8) != W4A16_OK)
-        return 0;
+    const int path = M <= 16 ? W4A16_PATH_DECODE : W4A16_PATH_TENSORCORE;
+    if (make_plan(M, N, K, g, 0, path, 0, current_sm_count(), &p, 8) != W4A16_OK) return 0;
     return (size_t)p.workspace_bytes;
 }
 
@@ -918,13 +939,15 @@ w4a16_status w8a16_gemm(const void* X, int64_t M, int64_t K, const void* codes, 
     DeviceInfo di;
     if ((st = device_info(&di)) != W4A16_OK) return st;
     cudaStream_t s = static_cast<cudaStream_t>(stream);
-    if (M <= 16)
-        return w8::w8_gemv_launch(X, M, K, codes, scales, zeros, N, g, sym, Y, di.sm_count, s);
     w4a16_plan p;
-    st = make_plan(M, N, K, g, sym, W4A16_PATH_TENSORCORE, 0, current_sm_count(), &p, 8);
+    const int path = M <= 16 ? W4A16_PATH_DECODE : W4A16_PATH_TENSORCORE;
+    st = make_plan(M, N, K, g, sym, path, 0, current_sm_count(), &p, 8);
     if (st != W4A16_OK) return st;
     if (workspace_bytes < (size_t)p.workspace_bytes) return W4A16_EWORKSPACE;
     if (p.workspace_bytes > 0 && (workspace == nullptr || !aligned16(workspace))) return W4A16_EINVAL;
+    if (p.path == W4A16_PATH_DECODE)
+        return launch_decode(p, X, M, K, codes, scales, zeros, N, g, sym, Y, workspace, s, nullptr,
+                             false, 8);
     return launch_tc(p, X, M, K, codes, scales, zeros, N, g, sym, Y, workspace, s, 8);
 }
 

@@ -14,14 +14,9 @@
 //  * w8_quantize_kernel / w8_quantize_rows_kernel: one pass over W, grouped
 //    (G/8 lanes per group, butterfly shuffles) or per-channel (g = K, one CTA
 //    per row, block-wide range reduction and a second pass from L2);
-//  * w8_dequantize_kernel: 8 codes (one 8-byte load) per thread and step;
-//  * w8_gemv_kernel (M ≤ 16; w8a16_gemm launches it through w8_gemv_launch and
-//    runs larger M on the tensor-core kernel with 8-bit codes): one warp per
-//    weight row; each lane streams 16-byte chunks of the row's codes
-//    (coalesced 128-bit loads, four chunks in flight per lane), forms
-//    x̂ = bf16_rn((q − z)·s) exactly in binary32, and accumulates Σ x·x̂ in
-//    binary32 for every activation row; the lanes' sums are combined by a
-//    fixed butterfly of warp shuffles, so results are deterministic.
+//  * w8_dequantize_kernel: 8 codes (one 8-byte load) per thread and step.
+// The fused GEMMs for 8-bit codes are instances of the INT4 translation unit's
+// kernels: gemv_decode_kernel for M ≤ 16 and gemm_tc_kernel for larger M.
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
 
@@ -238,95 +233,6 @@ __global__ void __launch_bounds__(kThreads) w8_dequantize_kernel(const uint2* __
     }
 }
 
-// Four 8-bit codes of a word -> their bf16_rn((q − z)·s) values widened to
-// binary32.  The byte placed in a binary32 mantissa gives 2^23 + q exactly;
-// subtracting zoff = 2^23 + z (exact: < 2^24) leaves q − z, the product with s
-// is exact, and cvt.rn.bf16x2 rounds once.  Symmetric words are XORed with
-// 0x80808080 by the caller (offset-128 codes, zoff = 2^23 + 128).
-__device__ __forceinline__ void dequant_word(uint32_t w, float s, float zoff, float out[4]) {
-    float f[4];
-#pragma unroll
-    for (int i = 0; i < 4; ++i)
-        f[i] = (__uint_as_float(__byte_perm(w, 0x4B000000u, 0x7540u + (uint32_t)i)) - zoff) * s;
-#pragma unroll
-    for (int i = 0; i < 4; i += 2) {
-        uint32_t p;
-        asm("cvt.rn.bf16x2.f32 %0, %1, %2;" : "=r"(p) : "f"(f[i + 1]), "f"(f[i]));
-        out[i] = __uint_as_float(p << 16);
-        out[i + 1] = __uint_as_float(p & 0xFFFF0000u);
-    }
-}
-
-// Fused GEMV for M ≤ MM (MM ∈ {1, 2, 4, 8, 16}): warp = weight row n.  Each lane
-// issues the loads of kUnroll 16-code chunks (32 chunks apart) before using
-// any, so a warp keeps 2 KB of codes in flight.
-constexpr int kUnroll = 4;
-
-template <int MM, bool SYM>
-__global__ void __launch_bounds__(kThreads) w8_gemv_kernel(const uint16_t* __restrict__ X, int M,
-                                                          int64_t K, const uint8_t* __restrict__ codes,
-                                                          const uint16_t* __restrict__ scales,
-                                                          const uint16_t* __restrict__ zeros,
-                                                          int64_t N, int64_t g,
-                                                          uint16_t* __restrict__ Y) {
-    const int lane = threadIdx.x & 31;
-    const int64_t warp0 = ((int64_t)blockIdx.x * blockDim.x + threadIdx.x) >> 5;
-    const int64_t nwarps = ((int64_t)gridDim.x * blockDim.x) >> 5;
-    const int64_t Gn = K / g;                      // groups per row
-    const int64_t chunks = K / 16;                 // 16-code chunks per row
-    const uint32_t flip = SYM ? 0x80808080u : 0u;
-    for (int64_t n = warp0; n < N; n += nwarps) {
-        float acc[MM];
-#pragma unroll
-        for (int m = 0; m < MM; ++m) acc[m] = 0.0f;
-        const uint8_t* row = codes + n * K;
-        for (int64_t c0 = lane; c0 < chunks; c0 += 32 * kUnroll) {
-            uint4 v[kUnroll];
-#pragma unroll
-            for (int u = 0; u < kUnroll; ++u) {
-                const int64_t c = c0 + 32 * u;
-                v[u] = c < chunks ? ldg16(row + c * 16) : make_uint4(0, 0, 0, 0);
-            }
-#pragma unroll
-            for (int u = 0; u < kUnroll; ++u) {
-                const int64_t c = c0 + 32 * u;
-                if (c >= chunks) break;
-                const int64_t grp = (c * 16) / g;
-                const float s = bf16_to_f32(__ldg(scales + n * Gn + grp));
-                const float zoff = SYM ? 8388736.0f
-                                       : 8388608.0f + bf16_to_f32(__ldg(zeros + n * Gn + grp));
-                const uint32_t wv[4] = {v[u].x, v[u].y, v[u].z, v[u].w};
-                float w[16];
-#pragma unroll
-                for (int j = 0; j < 4; ++j) dequant_word(wv[j] ^ flip, s, zoff, w + 4 * j);
-#pragma unroll
-                for (int m = 0; m < MM; ++m) {
-                    if (m < M) {
-                        const uint16_t* xr = X + (int64_t)m * K + c * 16;
-                        const uint4 xa = __ldg(reinterpret_cast<const uint4*>(xr));
-                        const uint4 xb = __ldg(reinterpret_cast<const uint4*>(xr + 8));
-                        float xf[16];
-                        unpack8(xa, xf);
-                        unpack8(xb, xf + 8);
-#pragma unroll
-                        for (int i = 0; i < 16; ++i) acc[m] = fmaf(xf[i], w[i], acc[m]);
-                    }
-                }
-            }
-        }
-#pragma unroll
-        for (int m = 0; m < MM; ++m) {
-#pragma unroll
-            for (int o = 16; o > 0; o >>= 1) acc[m] += __shfl_xor_sync(0xffffffffu, acc[m], o);
-        }
-        if (lane == 0) {
-#pragma unroll
-            for (int m = 0; m < MM; ++m)
-                if (m < M) Y[(int64_t)m * N + n] = (uint16_t)f32_to_bf16_rn(acc[m]);
-        }
-    }
-}
-
 // ---------------------------------------------------------------- host side
 struct DeviceInfo {
     bool ready = false;
@@ -376,33 +282,6 @@ int grid_for(int64_t items, int sm_count) {
 
 w4a16_status launch_status() { return cudaGetLastError() == cudaSuccess ? W4A16_OK : W4A16_ECUDA; }
 
-// Fused GEMV launch for M ≤ 16 (arguments already checked by the caller).
-w4a16_status w8_gemv_launch(const void* X, int64_t M, int64_t K, const void* codes,
-                            const void* scales, const void* zeros, int64_t N, int32_t g,
-                            int32_t sym, void* Y, int sm_count, cudaStream_t s) {
-    const int64_t gl = per_channel(g, K) ? K : (int64_t)g;
-    int64_t grid = (N + kThreads / 32 - 1) / (kThreads / 32);      // one warp per row
-    const int64_t cap = (int64_t)sm_count * 16;
-    if (grid > cap) grid = cap;
-    auto* Xp = static_cast<const uint16_t*>(X);
-    auto* Cp = static_cast<const uint8_t*>(codes);
-    auto* Sp = static_cast<const uint16_t*>(scales);
-    auto* Zp = static_cast<const uint16_t*>(zeros);
-    auto* Yp = static_cast<uint16_t*>(Y);
-    const int m = (int)M;
-#define W8_GEMV(MMV)                                                                           \
-    do {                                                                                       \
-        if (sym) w8_gemv_kernel<MMV, true><<<(unsigned)grid, kThreads, 0, s>>>(Xp, m, K, Cp, Sp, Zp, N, gl, Yp); \
-        else w8_gemv_kernel<MMV, false><<<(unsigned)grid, kThreads, 0, s>>>(Xp, m, K, Cp, Sp, Zp, N, gl, Yp); \
-    } while (0)
-    if (M <= 1) W8_GEMV(1);
-    else if (M <= 2) W8_GEMV(2);
-    else if (M <= 4) W8_GEMV(4);
-    else if (M <= 8) W8_GEMV(8);
-    else W8_GEMV(16);
-#undef W8_GEMV
-    return launch_status();
-}
 
 }  // namespace w8
 
