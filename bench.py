@@ -72,14 +72,14 @@ def group_of(g: int, K: int) -> int:
     return K if g == 0 else g
 
 
-def input_bytes(M: int, N: int, K: int, g: int, sym: bool) -> int:
-    """Packed codes + scales (+ zeros if asymmetric) + X."""
-    return N * K // 2 + 2 * N * (K // g) * (1 if sym else 2) + 2 * M * K
+def input_bytes(M: int, N: int, K: int, g: int, sym: bool, bits: int = 4) -> int:
+    """Packed codes (bits per weight) + scales (+ zeros if asymmetric) + X."""
+    return N * K * bits // 8 + 2 * N * (K // g) * (1 if sym else 2) + 2 * M * K
 
 
-def algorithmic_bytes(M: int, N: int, K: int, g: int, sym: bool) -> int:
+def algorithmic_bytes(M: int, N: int, K: int, g: int, sym: bool, bits: int = 4) -> int:
     """Packed codes + scales (+ zeros if asymmetric) + X read once + Y written once."""
-    return input_bytes(M, N, K, g, sym) + 2 * M * N
+    return input_bytes(M, N, K, g, sym, bits) + 2 * M * N
 
 
 # Sources each timed kernel is built from (its device code, the shared device
@@ -233,11 +233,11 @@ class GemmCase:
     """One layer of a workload, resident on the device, with `copies` rotating
     copies of the quantized weights (and activations)."""
 
-    def __init__(self, w4, layer, M, g, sym, copies, dev):
-        self.layer, self.M, self.g, self.sym = layer, M, g, sym
+    def __init__(self, w4, layer, M, g, sym, copies, dev, bits=4):
+        self.layer, self.M, self.g, self.sym, self.bits = layer, M, g, sym, bits
         self.N, self.K = layer.N, layer.K
         W = layer.weight().to(dev)
-        P, S, Z = w4.quantize(W, g, sym)
+        P, S, Z = (w4.quantize8 if bits == 8 else w4.quantize)(W, g, sym)
         self.W_dense = W
         self.P = [P] + [P.clone() for _ in range(copies - 1)]
         self.S = [S] + [S.clone() for _ in range(copies - 1)]
@@ -245,15 +245,16 @@ class GemmCase:
         X = layer.activation(M).to(dev)
         self.X = [X] + [X.clone() for _ in range(copies - 1)]
         self.Y = [torch.empty(M, self.N, dtype=torch.bfloat16, device=dev) for _ in range(copies)]
-        self.bytes = algorithmic_bytes(M, self.N, self.K, g, sym)
+        self.bytes = algorithmic_bytes(M, self.N, self.K, g, sym, bits)
         self.flops = 2 * M * self.N * self.K
 
     def call(self, w4, i):
         # The weights are fixed after set-up and no kernel in a step writes them, so
         # the decode kernel may stream them while the previous GEMM drains.
         j = i % len(self.P)
-        w4.gemm(self.X[j], self.P[j], self.S[j], self.Z[j], self.g, self.sym, out=self.Y[j],
-                static_weights=True)
+        gemm = w4.gemm8 if self.bits == 8 else w4.gemm
+        gemm(self.X[j], self.P[j], self.S[j], self.Z[j], self.g, self.sym, out=self.Y[j],
+             static_weights=True)
 
 
 def launches_per_call(plan: dict) -> int:
@@ -451,18 +452,22 @@ def cpu_baseline_sampled(layer, M, g, sym, rows: int):
 
 # ---------------------------------------------------------------------------- main arms
 WORKLOAD_DEFS = {
-    # name: (workload, M, g, sym, metric half); g = 0: per-channel (g = K)
-    "decode7b": (workloads.DECODE_7B, 1, 128, False, "hbm"),
-    "decode70b": (workloads.DECODE_70B, 1, 128, False, "hbm"),
-    "decode70b_sym": (workloads.DECODE_70B, 1, 128, True, "hbm"),
-    "prefill": (workloads.PREFILL, 2048, 128, False, "tensor"),
-    "decode7b_pc": (workloads.DECODE_7B, 1, 0, False, "hbm"),
-    "prefill_pc": (workloads.PREFILL, 2048, 0, False, "tensor"),
+    # name: (workload, M, g, sym, metric half, code bits); g = 0: per-channel (g = K)
+    "decode7b": (workloads.DECODE_7B, 1, 128, False, "hbm", 4),
+    "decode70b": (workloads.DECODE_70B, 1, 128, False, "hbm", 4),
+    "decode70b_sym": (workloads.DECODE_70B, 1, 128, True, "hbm", 4),
+    "prefill": (workloads.PREFILL, 2048, 128, False, "tensor", 4),
+    "decode7b_pc": (workloads.DECODE_7B, 1, 0, False, "hbm", 4),
+    "prefill_pc": (workloads.PREFILL, 2048, 0, False, "tensor", 4),
+    # W8A16 (8-bit codes): for profiling the 8-bit kernels; no end-to-end leg
+    "w8_decode70b": (workloads.DECODE_70B, 1, 128, False, "hbm", 8),
+    "w8_prefill": (workloads.PREFILL, 2048, 128, False, "tensor", 8),
 }
 
 
-def workload_name(wl, M, g, sym=False) -> str:
-    return f"{wl.name}_M{M}" + ("_per_channel" if g == 0 else "") + ("_sym" if sym else "")
+def workload_name(wl, M, g, sym=False, bits=4) -> str:
+    return (("w8a16_" if bits == 8 else "") + f"{wl.name}_M{M}" + ("_per_channel" if g == 0 else "")
+            + ("_sym" if sym else ""))
 
 
 def run_ours(args):
@@ -478,12 +483,12 @@ def run_ours(args):
     props = torch.cuda.get_device_properties(dev)
     l2 = getattr(props, "L2_cache_size", 0) or L2_BYTES_FALLBACK
 
-    wl, M, g, sym, half = WORKLOAD_DEFS[args.workload]
-    bytes_step = sum(algorithmic_bytes(M, l.N, l.K, group_of(g, l.K), sym) for l in wl.layers)
+    wl, M, g, sym, half, bits = WORKLOAD_DEFS[args.workload]
+    bytes_step = sum(algorithmic_bytes(M, l.N, l.K, group_of(g, l.K), sym, bits) for l in wl.layers)
     flops_step = sum(2 * M * l.N * l.K for l in wl.layers)
-    in_bytes_step = sum(input_bytes(M, l.N, l.K, group_of(g, l.K), sym) for l in wl.layers)
+    in_bytes_step = sum(input_bytes(M, l.N, l.K, group_of(g, l.K), sym, bits) for l in wl.layers)
     copies = copies_for(in_bytes_step, l2)
-    cases = [GemmCase(w4, l, M, group_of(g, l.K), sym, copies, dev) for l in wl.layers]
+    cases = [GemmCase(w4, l, M, group_of(g, l.K), sym, copies, dev, bits) for l in wl.layers]
     rot, singles = capture_rotation_graph(w4, cases, copies)
     ms, clocks = run_timed(world, rot, singles, copies, args.steps, args.warmup, sampler_index=local)
     ms_max = max_over_ranks(world, ms)
@@ -496,7 +501,7 @@ def run_ours(args):
         value, unit = total_flops / sec / 1e12, "TFLOP/s"
     kms = per_layer_ms(w4, cases, copies)
 
-    plans = [w4.plan(M, c.N, c.K, c.g, sym) for c in cases]
+    plans = [(w4.plan8 if bits == 8 else w4.plan)(M, c.N, c.K, c.g, sym) for c in cases]
     kernel_name = "gemv_decode_kernel" if plans[0]["path"] == "decode" else "gemm_tc_kernel"
     # The timed region holds only this workload's GEMM launches, so the kernel's
     # average launch duration is the region's time over its launches.
@@ -523,7 +528,7 @@ def run_ours(args):
         "warmup": args.warmup, "ms_per_step": ms_max / args.steps, "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
         "config": {
-            "workload": workload_name(wl, M, g, sym), "M": M,
+            "workload": workload_name(wl, M, g, sym, bits), "M": M,
             "layers_KxN": [[l.K, l.N] for l in wl.layers], "g": g if g else "K (per-channel)",
             "mode": "sym" if sym else "asym", "description": wl.description,
             "l2": f"{copies} rotating copies of weights+activations "
@@ -538,40 +543,42 @@ def run_ours(args):
     }
 
     # ------------------------------------------------ end to end through the public API
-    pinned = [c.X[0].cpu().pin_memory() for c in cases]
-    host_y = [torch.empty(c.M, c.N, dtype=torch.bfloat16, pin_memory=True) for c in cases]
-    h2d = sum(x.numel() * 2 for x in pinned)
-    d2h = sum(c.M * c.N * 2 for c in cases)
-    e2e_steps = min(args.steps, 2000)
+    # (4-bit workloads; the 8-bit ones exist to profile the 8-bit kernels)
+    if bits == 4:
+        pinned = [c.X[0].cpu().pin_memory() for c in cases]
+        host_y = [torch.empty(c.M, c.N, dtype=torch.bfloat16, pin_memory=True) for c in cases]
+        h2d = sum(x.numel() * 2 for x in pinned)
+        d2h = sum(c.M * c.N * 2 for c in cases)
+        e2e_steps = min(args.steps, 2000)
 
-    def e2e_step(i):
-        # host X in, host Y out for every layer; the step waits once, for its last copy
-        for c, xh, yh in zip(cases, pinned, host_y):
-            j = i % copies
-            w4.gemm(xh, c.P[j], c.S[j], c.Z[j], c.g, c.sym, out=yh, sync=False, static_weights=True)
-        torch.cuda.current_stream().synchronize()
+        def e2e_step(i):
+            # host X in, host Y out for every layer; the step waits once, for its last copy
+            for c, xh, yh in zip(cases, pinned, host_y):
+                j = i % copies
+                w4.gemm(xh, c.P[j], c.S[j], c.Z[j], c.g, c.sym, out=yh, sync=False, static_weights=True)
+            torch.cuda.current_stream().synchronize()
 
-    for i in range(args.warmup):
-        e2e_step(i)
-    torch.cuda.synchronize()
-    barrier(world)
-    torch.cuda.synchronize()
-    a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    a.record()
-    for i in range(e2e_steps):
-        e2e_step(i)
-    b.record()
-    b.synchronize()
-    barrier(world)
-    e2e_ms = max_over_ranks(world, a.elapsed_time(b))
-    e2e_total = sum_over_ranks(world, (bytes_step if half == "hbm" else flops_step) * e2e_steps)
-    e2e_val = e2e_total / (e2e_ms / 1e3) / (1e9 if half == "hbm" else 1e12)
-    line["e2e"] = {"value": e2e_val, "unit": unit, "h2d_bytes_per_step": h2d,
-                   "d2h_bytes_per_step": d2h, "steps": e2e_steps,
-                   "ms_per_step": e2e_ms / e2e_steps}
+        for i in range(args.warmup):
+            e2e_step(i)
+        torch.cuda.synchronize()
+        barrier(world)
+        torch.cuda.synchronize()
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record()
+        for i in range(e2e_steps):
+            e2e_step(i)
+        b.record()
+        b.synchronize()
+        barrier(world)
+        e2e_ms = max_over_ranks(world, a.elapsed_time(b))
+        e2e_total = sum_over_ranks(world, (bytes_step if half == "hbm" else flops_step) * e2e_steps)
+        e2e_val = e2e_total / (e2e_ms / 1e3) / (1e9 if half == "hbm" else 1e12)
+        line["e2e"] = {"value": e2e_val, "unit": unit, "h2d_bytes_per_step": h2d,
+                       "d2h_bytes_per_step": d2h, "steps": e2e_steps,
+                       "ms_per_step": e2e_ms / e2e_steps}
 
     # ------------------------------------------------ comparisons and the other metric half
-    if not args.no_extras:
+    if not args.no_extras and bits == 4:
         line["comparisons"] = comparisons(w4, cases, copies, l2, half)
         if half == "hbm":
             ro = read_only_stream_gbs(dev)
@@ -592,7 +599,7 @@ def run_ours(args):
                                                   l2, dev)
             line["w8a16"] = w8a16_extras(w4, peaks, l2, dev)
             line["act_scale"] = act_scale_extras(w4, l2, dev)
-    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+    if rank == 0 and world == 1 and not args.no_cpu_baseline and bits == 4:
         cb = cpu_baseline(wl.layers, M, g, sym, unit_bytes=(half == "hbm")) \
             if half == "hbm" else cpu_baseline_sampled(wl.layers[0], M, g, sym, rows=16)
         line["cpu_baseline"] = cb
@@ -666,10 +673,10 @@ def workload_extras(w4, names, peaks, peak_src, l2, dev, decode_iters=400, tenso
     one scale (and zero) per row."""
     out = {}
     for name in names:
-        wl, M, g, sym, half = WORKLOAD_DEFS[name]
-        in_bytes = sum(input_bytes(M, l.N, l.K, group_of(g, l.K), sym) for l in wl.layers)
+        wl, M, g, sym, half, bits = WORKLOAD_DEFS[name]
+        in_bytes = sum(input_bytes(M, l.N, l.K, group_of(g, l.K), sym, bits) for l in wl.layers)
         copies = copies_for(in_bytes, l2)
-        cases = [GemmCase(w4, l, M, group_of(g, l.K), sym, copies, dev) for l in wl.layers]
+        cases = [GemmCase(w4, l, M, group_of(g, l.K), sym, copies, dev, bits) for l in wl.layers]
         rot, singles = capture_rotation_graph(w4, cases, copies)
         n = decode_iters if half == "hbm" else tensor_iters
         replay_steps(rot, singles, copies, 3)
@@ -681,7 +688,7 @@ def workload_extras(w4, names, peaks, peak_src, l2, dev, decode_iters=400, tenso
         b.synchronize()
         ms = a.elapsed_time(b) / n
         kms = per_layer_ms(w4, cases, copies, reps=20 if half == "hbm" else 5)
-        plans = [w4.plan(M, c.N, c.K, c.g, sym) for c in cases]
+        plans = [(w4.plan8 if bits == 8 else w4.plan)(M, c.N, c.K, c.g, sym) for c in cases]
         kernel = "gemv_decode_kernel" if plans[0]["path"] == "decode" else "gemm_tc_kernel"
         if half == "hbm":
             work = sum(c.bytes for c in cases)
@@ -689,7 +696,7 @@ def workload_extras(w4, names, peaks, peak_src, l2, dev, decode_iters=400, tenso
         else:
             work = sum(c.flops for c in cases)
             ach, pk, unit = work / (ms / 1e3) / 1e12, peaks["bf16_tflops"], "TFLOP/s"
-        out[name] = {"workload": workload_name(wl, M, g, sym), "ms_per_step": ms, "value": ach,
+        out[name] = {"workload": workload_name(wl, M, g, sym, bits), "ms_per_step": ms, "value": ach,
                      "unit": unit,
                      "roofline": {"bound": "hbm" if half == "hbm" else "tensor", "achieved": ach,
                                   "peak": pk, "unit": unit, "frac": ach / pk,
@@ -956,6 +963,46 @@ def crossover_rows(w4, dev, l2, iters=40, iters_large=12):
     return rows
 
 
+CROSSOVER8_MS = (1, 2, 4, 8, 12, 16, 24, 32, 64)
+
+
+def crossover8_rows(w4, dev, l2, iters=40):
+    """The same evidence for 8-bit codes (W8A16, g=128 asym, K=N=8192): the decode
+    kernel (M <= 16) and the tensor-core kernel at each M, forced through
+    w8a16_gemm_ex, and which one the dispatch takes."""
+    layer = workloads.CROSSOVER.layers[0]
+    N, K = layer.N, layer.K
+    g, sym = 128, False
+    C, S, Z = w4.quantize8(layer.weight().to(dev), g, sym)
+    copies = copies_for(N * K + 4 * N * (K // g), l2)
+    Cs = [C] + [C.clone() for _ in range(copies - 1)]
+    Ss = [S] + [S.clone() for _ in range(copies - 1)]
+    Zs = [Z] + [Z.clone() for _ in range(copies - 1)]
+    rows = []
+    for M in CROSSOVER8_MS:
+        X = layer.activation(M).to(dev)
+        Xs = [X] + [X.clone() for _ in range(copies - 1)]
+        Y = torch.empty(M, N, dtype=torch.bfloat16, device=dev)
+        row = {"g": g, "mode": "asym", "M": M, "dispatch": w4.plan8(M, N, K, g, sym)["path"],
+               "algorithmic_bytes": algorithmic_bytes(M, N, K, g, sym) + N * K // 2}
+        for path in ("decode", "tensorcore"):
+            if path == "decode" and M > 16:
+                continue
+            torch.cuda.nvtx.range_push(f"xover8_M{M}_{path}")
+            gs = graph_of(lambda i, path=path: w4.gemm8(Xs[i % copies], Cs[i % copies], Ss[i % copies],
+                                                        Zs[i % copies], g, sym, out=Y, path=path,
+                                                        static_weights=True), copies)
+            row[path + "_us"] = round(time_graphs(gs, iters) * 1e3, 3)
+            torch.cuda.nvtx.range_pop()
+            del gs
+        cand = {k[:-3]: v for k, v in row.items() if k in ("decode_us", "tensorcore_us")}
+        row["fastest"] = min(cand, key=cand.get)
+        rows.append(row)
+        del Xs, X, Y
+        torch.cuda.empty_cache()
+    return rows
+
+
 def crossover_sweep(args):
     """Print the crossover rows as one JSON object {"crossover": [...]}; not a
     benchmark line."""
@@ -966,7 +1013,10 @@ def crossover_sweep(args):
     dev = torch.device("cuda", 0)
     props = torch.cuda.get_device_properties(dev)
     l2 = getattr(props, "L2_cache_size", 0) or L2_BYTES_FALLBACK
-    print(json.dumps({"crossover": crossover_rows(w4, dev, l2)}))
+    if args.crossover8:
+        print(json.dumps({"crossover_w8a16": crossover8_rows(w4, dev, l2)}))
+    else:
+        print(json.dumps({"crossover": crossover_rows(w4, dev, l2)}))
 
 
 def run_reference(args):
@@ -976,7 +1026,9 @@ def run_reference(args):
     rank = int(os.environ.get("RANK", "0"))
     if rank != 0:
         return
-    wl, M, g, sym, half = WORKLOAD_DEFS[args.workload]
+    wl, M, g, sym, half, bits = WORKLOAD_DEFS[args.workload]
+    if bits != 4:
+        raise SystemExit("the reference arm times the 4-bit workloads")
     if half == "hbm":
         import oracle
         oracle.build()
@@ -1030,10 +1082,12 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--crossover", action="store_true",
                     help="print the M-dispatch sweep at K=N=8192 instead of a benchmark line")
+    ap.add_argument("--crossover8", action="store_true",
+                    help="the same sweep for 8-bit codes (W8A16)")
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be at least 3")
-    if args.crossover:
+    if args.crossover or args.crossover8:
         crossover_sweep(args)
     elif args.impl == "reference":
         run_reference(args)

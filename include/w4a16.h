@@ -277,11 +277,12 @@ w4a16_status w8a16_dequantize(const void* codes, const void* scales, const void*
  * rejected shapes.  (Before ABI version 4 the M ≤ 16 path needed none.) */
 size_t w8a16_gemm_workspace_size(int64_t M, int64_t N, int64_t K, int32_t g);
 
-/* Host-only: the launch w8a16_gemm would make (decode kernel for M ≤ 16, else
- * the tensor-core kernel, both with 8-bit codes), including its workspace.
- * Returns W4A16_EINVAL for shapes w8a16_gemm would reject. */
+/* Host-only: the launch w8a16_gemm_ex would make with this `path` (AUTO: the
+ * decode kernel for M ≤ 16, else the tensor-core kernel, both with 8-bit codes),
+ * including its workspace.  Returns W4A16_EINVAL for shapes or paths
+ * w8a16_gemm_ex would reject. */
 w4a16_status w8a16_gemm_plan(int64_t M, int64_t N, int64_t K, int32_t g, int32_t sym,
-                             w4a16_plan* plan);
+                             int32_t path, w4a16_plan* plan);
 
 /* Fused W8A16 GEMM: Y[M, N] = X[M, K] · Ŵ[N, K]ᵀ with Ŵ = bf16_rn((q − z)·s)
  * formed on chip, binary32 accumulation, one rounding of each output to bf16;
@@ -298,6 +299,15 @@ w4a16_status w8a16_gemm(const void* X, int64_t M, int64_t K, const void* codes,
                         const void* scales, const void* zeros, int64_t N, int32_t g,
                         int32_t sym, void* Y, void* workspace, size_t workspace_bytes,
                         void* stream);
+
+/* w8a16_gemm with the kernel choice overridden, as w4a16_gemm_ex does for 4-bit
+ * codes (`path` AUTO, DECODE (M ≤ 16) or TENSORCORE, optionally OR'ed with
+ * W4A16_STATIC_WEIGHTS); the workspace is that of w8a16_gemm_plan for the same
+ * path.  Used by tests and benchmarks to measure both kernels at one shape. */
+w4a16_status w8a16_gemm_ex(const void* X, int64_t M, int64_t K, const void* codes,
+                           const void* scales, const void* zeros, int64_t N, int32_t g,
+                           int32_t sym, void* Y, void* workspace, size_t workspace_bytes,
+                           int32_t path, void* stream);
 
 /* Read and clear the current device's error word, written by a kernel that gave
  * up a bounded wait (a pipeline barrier that did not complete within about one

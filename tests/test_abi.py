@@ -34,7 +34,7 @@ def test_header_declares_the_abi():
     for n in ("w4a16_quantize", "w4a16_dequantize", "w4a16_gemm", "w4a16_gemm_ex",
               "w4a16_gemm_workspace_size", "w4a16_gemm_plan", "w4a16_status_string",
               "w4a16_device_error", "w4a16_abi_version", "w8a16_quantize", "w8a16_dequantize",
-              "w8a16_gemm", "w8a16_gemm_plan"):
+              "w8a16_gemm", "w8a16_gemm_plan", "w8a16_gemm_ex"):
         assert n in names
 
 
@@ -271,6 +271,7 @@ def test_w8_decode_stage_layout_is_valid_for_every_shape(M):
                 continue
             for N in (1, 128, 1000, 28672):
                 p = w4.plan8(M, N, K, g, False)
+                assert p == w4.plan8(M, N, K, g, False, path="decode")
                 assert p["path"] == "decode" and p["stages"] >= 2 and p["smem_bytes"] <= 232448
                 assert p["threads"] == 576 and p["grid"] == min(148, -(-N // 256) * -(-K // 128))
     assert w4.plan8(17, 4096, 4096)["path"] == "tensorcore"

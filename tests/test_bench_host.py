@@ -28,12 +28,16 @@ def test_group_sizes_and_byte_models():
 
 
 def test_workload_table():
-    for name, (wl, M, g, sym, half) in bench.WORKLOAD_DEFS.items():
-        assert half in ("hbm", "tensor")
+    for name, (wl, M, g, sym, half, bits) in bench.WORKLOAD_DEFS.items():
+        assert half in ("hbm", "tensor") and bits in (4, 8)
         assert (half == "hbm") == (M <= 16)
         for layer in wl.layers:
             assert layer.K % bench.group_of(g, layer.K) == 0
         assert bench.workload_name(wl, M, g).endswith("_per_channel") == (g == 0)
+        assert bench.workload_name(wl, M, g, sym, bits).startswith("w8a16_") == (bits == 8)
+    # 8-bit codes: one byte per weight
+    assert bench.algorithmic_bytes(1, 28672, 8192, 128, False, 8) == \
+        28672 * 8192 + 4 * 28672 * 64 + 2 * 8192 + 2 * 28672
     assert bench.WORKLOAD_DEFS["decode7b"][0] is workloads.DECODE_7B
     assert bench.WORKLOAD_DEFS["prefill"][1] == 2048
 

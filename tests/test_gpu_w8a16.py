@@ -129,6 +129,26 @@ def test_w8_gemm_deterministic_and_7b_full_size():
 
 
 @pytest.mark.parametrize("sym", [False, True])
+@pytest.mark.parametrize("M", [1, 9, 16])
+def test_w8_forced_paths_agree_with_the_oracle(M, sym):
+    """w8a16_gemm_ex: the decode and tensor-core kernels both run M <= 16 and both
+    match the oracle; the static-weights flag changes no bit."""
+    N, K, g = 700, 2304, 64
+    W = workloads.make_weight(N, K, 0.02, 31, outlier_frac=0.01, outlier_scale=20.0)
+    C, S, Z = w4.quantize8(W.cuda(), g, sym)
+    X = workloads.make_activation(M, K, 32, outlier_frac=0.01, outlier_mode="set")
+    ref = oracle.gemm_w8a16(workloads.bits(X), C.cpu().numpy(), workloads.bits(S),
+                            workloads.bits(Z), g, sym)
+    ys = {}
+    for path in ("decode", "tensorcore"):
+        ys[path] = w4.gemm8(X.cuda(), C, S, Z, g, sym, path=path)
+        torch.cuda.synchronize()
+        assert_y_close(workloads.bits(ys[path]), ref, f"W8 {path} M={M} sym={sym}")
+    Yst = w4.gemm8(X.cuda(), C, S, Z, g, sym, path="decode", static_weights=True)
+    assert torch.equal(Yst, ys["decode"])
+
+
+@pytest.mark.parametrize("sym", [False, True])
 @pytest.mark.parametrize("li", [0, 1])
 def test_w8_decode_70b_full_size(li, sym):
     """The decode kernel with 8-bit codes on a 70B-shaped layer (M=1; the stream-K

@@ -73,12 +73,13 @@ def _load() -> ctypes.CDLL:
     lib.w8a16_dequantize.argtypes = [vp, vp, vp, i64, i64, i32, i32, vp, vp]
     lib.w8a16_gemm.argtypes = [vp, i64, i64, vp, vp, vp, i64, i32, i32, vp, vp, sz, vp]
     lib.w8a16_gemm_workspace_size.argtypes = [i64, i64, i64, i32]
-    lib.w8a16_gemm_plan.argtypes = [i64, i64, i64, i32, i32, ctypes.POINTER(Plan)]
+    lib.w8a16_gemm_plan.argtypes = [i64, i64, i64, i32, i32, i32, ctypes.POINTER(Plan)]
+    lib.w8a16_gemm_ex.argtypes = [vp, i64, i64, vp, vp, vp, i64, i32, i32, vp, vp, sz, i32, vp]
     lib.w8a16_gemm_workspace_size.restype = sz
     for name in ("w4a16_quantize", "w4a16_dequantize", "w4a16_gemm", "w4a16_gemm_ex",
                  "w4a16_gemm_act_scaled",
                  "w4a16_gemm_plan", "w4a16_device_error", "w8a16_quantize", "w8a16_dequantize",
-                 "w8a16_gemm", "w8a16_gemm_plan"):
+                 "w8a16_gemm", "w8a16_gemm_plan", "w8a16_gemm_ex"):
         getattr(lib, name).restype = ctypes.c_int
     if lib.w4a16_abi_version() != ABI_VERSION:
         raise ImportError(f"{LIB_PATH} has ABI version {lib.w4a16_abi_version()}, this binding "
@@ -191,10 +192,13 @@ def plan(M: int, N: int, K: int, g: int = 128, sym: bool = False, path: str | in
     return _plan_dict(p)
 
 
-def plan8(M: int, N: int, K: int, g: int = 128, sym: bool = False) -> dict:
-    """The launch w8a16_gemm would make for this shape (host only)."""
+def plan8(M: int, N: int, K: int, g: int = 128, sym: bool = False,
+          path: str | int = "auto") -> dict:
+    """The launch w8a16_gemm_ex would make for this shape and path (host only)."""
     p = Plan()
-    _check(lib().w8a16_gemm_plan(M, N, K, g, int(bool(sym)), ctypes.byref(p)), "w8a16_gemm_plan")
+    pid = _PATHS[path] if isinstance(path, str) else int(path)
+    _check(lib().w8a16_gemm_plan(M, N, K, g, int(bool(sym)), pid, ctypes.byref(p)),
+           "w8a16_gemm_plan")
     return _plan_dict(p)
 
 
@@ -408,7 +412,8 @@ def dequantize8(codes: torch.Tensor, scales: torch.Tensor, zeros: torch.Tensor |
 
 def gemm8(X: torch.Tensor, codes: torch.Tensor, scales: torch.Tensor,
           zeros: torch.Tensor | None, g: int = 128, sym: bool = False,
-          out: torch.Tensor | None = None) -> torch.Tensor:
+          out: torch.Tensor | None = None, path: str | int = "auto",
+          static_weights: bool = False) -> torch.Tensor:
     """Fused W8A16 GEMM: Y[M, N] = X[M, K] · Ŵ[N, K]ᵀ (bf16 in/out, fp32
     accumulation), device tensors.  M ≤ 16 runs the decode kernel with 8-bit
     codes, larger M the tensor-core kernel with 8-bit codes (each with the
@@ -426,15 +431,18 @@ def gemm8(X: torch.Tensor, codes: torch.Tensor, scales: torch.Tensor,
         out = torch.empty((M, N), dtype=torch.bfloat16, device=codes.device)
     dev = codes.device
     with torch.cuda.device(dev):
-        key = ("w8", dev.index, M, N, K, g)
+        pid = _PATHS[path] if isinstance(path, str) else int(path)
+        key = ("w8", dev.index, M, N, K, g, pid)
         ws_bytes = _plan_bytes.get(key)
         if ws_bytes is None:
-            ws_bytes = int(lib().w8a16_gemm_workspace_size(M, N, K, g)) if M and N else 0
+            ws_bytes = plan8(M, N, K, g, sym, pid)["workspace_bytes"] if M and N else 0
             _plan_bytes[key] = ws_bytes
         ws = _workspace(dev, ws_bytes)
-        _check(lib().w8a16_gemm(_ptr(X), M, K, _ptr(codes), _ptr(scales),
-                                _ptr(zeros if not sym else None), N, g, int(bool(sym)), _ptr(out),
-                                _ptr(ws), ws_bytes, _stream(dev)), "w8a16_gemm")
+        _check(lib().w8a16_gemm_ex(_ptr(X), M, K, _ptr(codes), _ptr(scales),
+                                   _ptr(zeros if not sym else None), N, g, int(bool(sym)),
+                                   _ptr(out), _ptr(ws), ws_bytes,
+                                   pid | (STATIC_WEIGHTS if static_weights else 0), _stream(dev)),
+               "w8a16_gemm")
     return out
 
 

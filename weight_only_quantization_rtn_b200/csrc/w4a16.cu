@@ -862,10 +862,9 @@ w4a16_status w4a16_gemm_plan(int64_t M, int64_t N, int64_t K, int32_t g, int32_t
 }
 
 w4a16_status w8a16_gemm_plan(int64_t M, int64_t N, int64_t K, int32_t g, int32_t sym,
-                             w4a16_plan* plan) {
+                             int32_t path, w4a16_plan* plan) {
     if (!plan) return W4A16_EINVAL;
-    const int path = M <= 16 ? W4A16_PATH_DECODE : W4A16_PATH_TENSORCORE;
-    return make_plan(M, N, K, g, sym, path, 0, current_sm_count(), plan, 8);
+    return make_plan(M, N, K, g, sym, path & ~W4A16_STATIC_WEIGHTS, 0, current_sm_count(), plan, 8);
 }
 
 w4a16_status w4a16_gemm_ex(const void* X, int64_t M, int64_t K, const void* packed,
@@ -921,14 +920,16 @@ w4a16_status w4a16_gemm_decode_noalloc(const void* X, int64_t M, int64_t K, cons
 
 size_t w8a16_gemm_workspace_size(int64_t M, int64_t N, int64_t K, int32_t g) {
     w4a16_plan p;
-    const int path = M <= 16 ? W4A16_PATH_DECODE : W4A16_PATH_TENSORCORE;
-    if (make_plan(M, N, K, g, 0, path, 0, current_sm_count(), &p, 8) != W4A16_OK) return 0;
+    if (make_plan(M, N, K, g, 0, W4A16_PATH_AUTO, 0, current_sm_count(), &p, 8) != W4A16_OK) return 0;
     return (size_t)p.workspace_bytes;
 }
 
-w4a16_status w8a16_gemm(const void* X, int64_t M, int64_t K, const void* codes, const void* scales,
-                        const void* zeros, int64_t N, int32_t g, int32_t sym, void* Y,
-                        void* workspace, size_t workspace_bytes, void* stream) {
+w4a16_status w8a16_gemm_ex(const void* X, int64_t M, int64_t K, const void* codes,
+                           const void* scales, const void* zeros, int64_t N, int32_t g,
+                           int32_t sym, void* Y, void* workspace, size_t workspace_bytes,
+                           int32_t path, void* stream) {
+    const bool static_weights = (path & W4A16_STATIC_WEIGHTS) != 0;
+    path &= ~W4A16_STATIC_WEIGHTS;
     w4a16_status st = check_shape(M, N, K, g, sym);
     if (st != W4A16_OK) return st;
     if (M == 0 || N == 0) return W4A16_OK;
@@ -940,15 +941,21 @@ w4a16_status w8a16_gemm(const void* X, int64_t M, int64_t K, const void* codes, 
     if ((st = device_info(&di)) != W4A16_OK) return st;
     cudaStream_t s = static_cast<cudaStream_t>(stream);
     w4a16_plan p;
-    const int path = M <= 16 ? W4A16_PATH_DECODE : W4A16_PATH_TENSORCORE;
     st = make_plan(M, N, K, g, sym, path, 0, current_sm_count(), &p, 8);
     if (st != W4A16_OK) return st;
     if (workspace_bytes < (size_t)p.workspace_bytes) return W4A16_EWORKSPACE;
     if (p.workspace_bytes > 0 && (workspace == nullptr || !aligned16(workspace))) return W4A16_EINVAL;
     if (p.path == W4A16_PATH_DECODE)
         return launch_decode(p, X, M, K, codes, scales, zeros, N, g, sym, Y, workspace, s, nullptr,
-                             false, 8);
+                             static_weights, 8);
     return launch_tc(p, X, M, K, codes, scales, zeros, N, g, sym, Y, workspace, s, 8);
+}
+
+w4a16_status w8a16_gemm(const void* X, int64_t M, int64_t K, const void* codes, const void* scales,
+                        const void* zeros, int64_t N, int32_t g, int32_t sym, void* Y,
+                        void* workspace, size_t workspace_bytes, void* stream) {
+    return w8a16_gemm_ex(X, M, K, codes, scales, zeros, N, g, sym, Y, workspace, workspace_bytes,
+                         W4A16_PATH_AUTO, stream);
 }
 
 w4a16_status w4a16_device_error(int32_t* code) {
