@@ -22,6 +22,12 @@ Parity status of each function (what pins it is in ``tests/test_oracle_pins.py``
   scale_activations / gemm_w4a16_act_scaled (per-K activation scale) — pinned
       (identity, exact power-of-two scaling, single rounding of the exact
       product, one-hot activations, the equivalent-scaling identity)
+  quantize_act8 / gemm_w8a8 / gemm_w8a8_from_bf16 (W8A8: per-token INT8
+      activations × per-channel INT8 weights) — pinned (hand-computed rows with
+      half-to-even ties, nearest-grid-point brute force, absmax to ±127,
+      power-of-two scaling, sign symmetry, zero rows, exact rational brute
+      force of the GEMM, numpy's float64 matmul of the dequantized operands,
+      one-hot activations, the all-127 case)
 """
 from __future__ import annotations
 
@@ -92,6 +98,8 @@ def _load():
                                                       vp, vp, i64, vp]
             lib.oracle_gemm_w8a16_sampled.restype = ctypes.c_int
             lib.oracle_scale_activations.argtypes = [vp, i64, i64, vp, vp]
+            lib.oracle_quantize_act8.argtypes = [vp, i64, i64, vp, vp]
+            lib.oracle_gemm_w8a8.argtypes = [vp, vp, vp, vp, i64, i64, i64, vp]
             lib.oracle_round_to_bf16.argtypes = [vp, i64, vp]
             lib.oracle_f32_array_to_bf16.argtypes = [vp, i64, vp]
             lib.oracle_num_threads.restype = ctypes.c_int
@@ -333,6 +341,41 @@ def scale_activations(X_bits, a_bits) -> np.ndarray:
 def gemm_w4a16_act_scaled(X_bits, a_bits, packed, scales, zeros, g: int, sym: bool) -> np.ndarray:
     """Y64 = (X·diag(a))' · Ŵᵀ with the scaled activations rounded to bf16 first."""
     return gemm_w4a16(scale_activations(X_bits, a_bits), packed, scales, zeros, g, sym)
+
+
+def quantize_act8(X_bits):
+    """W8A8 activations: per-token (row) symmetric INT8, s_x = max|x|/127 in binary32.
+    Returns (q int8 [M, K], s_x float32 [M])."""
+    lib = _load()
+    X = _u16(X_bits)
+    M, K = X.shape
+    q = np.zeros((M, K), dtype=np.int8)
+    s = np.zeros(M, dtype=np.float32)
+    lib.oracle_quantize_act8(_ptr(X), M, K, _ptr(q), _ptr(s))
+    return q, s
+
+
+def gemm_w8a8(qx, sx, qw, sw_bits) -> np.ndarray:
+    """Y64[m, n] = s_x[m]·s_w[n]·Σ_k q_x[m, k]·q_w[n, k] (exact integer sum).
+    qx int8 [M, K], sx float32 [M], qw int8 (or its uint8 bytes) [N, K], sw bf16 bits [N] or [N, 1]."""
+    lib = _load()
+    qx = np.ascontiguousarray(qx, dtype=np.int8)
+    sx = np.ascontiguousarray(sx, dtype=np.float32)
+    qw = np.ascontiguousarray(qw).view(np.int8)
+    sw = _u16(np.ascontiguousarray(sw_bits).reshape(-1))
+    M, K = qx.shape
+    N, K2 = qw.shape
+    assert K == K2 and sx.shape == (M,) and sw.shape == (N,)
+    Y = np.zeros((M, N), dtype=np.float64)
+    lib.oracle_gemm_w8a8(_ptr(qx), _ptr(sx), _ptr(qw), _ptr(sw), M, N, K, _ptr(Y))
+    return Y
+
+
+def gemm_w8a8_from_bf16(X_bits, qw, sw_bits) -> np.ndarray:
+    """The whole W8A8 product for bf16 activations: quantize X per token, then
+    the integer GEMM with both scales."""
+    qx, sx = quantize_act8(X_bits)
+    return gemm_w8a8(qx, sx, qw, sw_bits)
 
 
 def num_threads() -> int:

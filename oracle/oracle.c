@@ -476,6 +476,58 @@ void oracle_scale_activations(const uint16_t* X, int64_t M, int64_t K, const uin
     }
 }
 
+/* ---------------------------------------------------------------------------
+ * W8A8: weights and activations both INT8, for the INT8 tensor cores
+ * ("Quantization & Acceleration: 解释 W8A8 与 W4A16 的差异与取舍", 数学机理 (1):
+ * both quantized to INT8, activations dynamic and quantized per token;
+ * "大模型推理中 Weight-only、W8A8 和 FP8 量化有什么区别？如何选型？", §三: an integer
+ * matrix multiply on both 8-bit sides).  Weights: the symmetric 8-bit quantizer
+ * above with one group per row (g = K, per output channel).  Activations:
+ * symmetric absmax per token (row of X), [P3] §二 with b = 8.
+ * Readings: R16 the activation scale s_x = max|x| / 127 stays in binary32
+ * (computed per call, never stored in a 16-bit format), q = round(x / s_x) with
+ * the binary32 quotient, half to even, clamped to [−128, 127] like the weight
+ * codes (never binding: |x| / s_x ≤ 127 up to one rounding); an all-zero row has
+ * s_x = 0 and q = 0.  R17 the product is Y = s_x[m]·s_w[n]·Σ_k q_x[m,k]·q_w[n,k]
+ * with the integer sum exact (as the INT8 tensor cores accumulate in int32).
+ * ------------------------------------------------------------------------- */
+void oracle_quantize_act8(const uint16_t* X, int64_t M, int64_t K, int8_t* q, float* s) {
+    for (int64_t m = 0; m < M; ++m) {
+        float amax = 0.0f;
+        for (int64_t k = 0; k < K; ++k) {
+            float a = fabsf(oracle_bf16_to_f32(X[m * K + k]));
+            if (a > amax) amax = a;
+        }
+        float sc = amax / 127.0f;
+        s[m] = sc;
+        for (int64_t k = 0; k < K; ++k) {
+            int32_t c = 0;
+            if (sc != 0.0f) {
+                float r = rintf(oracle_bf16_to_f32(X[m * K + k]) / sc);
+                if (r < -128.0f) r = -128.0f;
+                if (r > 127.0f) r = 127.0f;
+                c = (int32_t)r;
+            }
+            q[m * K + k] = (int8_t)c;
+        }
+    }
+}
+
+/* Y64[m, n] = s_x[m] · s_w[n] · Σ_k q_x[m, k]·q_w[n, k]: the integer sum exactly
+ * (int64), then the two scales and the sum multiplied in binary64.  Weight codes
+ * are int8 bytes [N, K] and their scales bf16 [N] (one per output channel). */
+void oracle_gemm_w8a8(const int8_t* qx, const float* sx, const int8_t* qw, const uint16_t* sw,
+                      int64_t M, int64_t N, int64_t K, double* Y) {
+#pragma omp parallel for collapse(2) schedule(static)
+    for (int64_t m = 0; m < M; ++m) {
+        for (int64_t n = 0; n < N; ++n) {
+            int64_t acc = 0;
+            for (int64_t k = 0; k < K; ++k) acc += (int64_t)qx[m * K + k] * (int64_t)qw[n * K + k];
+            Y[m * N + n] = (double)sx[m] * (double)oracle_bf16_to_f32(sw[n]) * (double)acc;
+        }
+    }
+}
+
 /* Elementwise bf16_rn of a binary32 array. */
 void oracle_f32_array_to_bf16(const float* x, int64_t n, uint16_t* out) {
     for (int64_t i = 0; i < n; ++i) out[i] = oracle_f32_to_bf16_rn(x[i]);

@@ -40,6 +40,16 @@ MUTANTS = {
     "act_scale_truncates": ("Xs[m * K + k] = oracle_f32_to_bf16_rn(prod);",
                             "uint32_t u; memcpy(&u, &prod, 4); Xs[m * K + k] = (uint16_t)(u >> 16);"),
     "act_scale_indexed_by_row": ("oracle_bf16_to_f32(a[k]);", "oracle_bf16_to_f32(a[m % K]);"),
+    # W8A8 (per-token INT8 activations x per-channel INT8 weights)
+    "w8a8_act_divides_by_128": ("float sc = amax / 127.0f;", "float sc = amax / 128.0f;"),
+    "w8a8_act_truncates": ("float r = rintf(oracle_bf16_to_f32(X[m * K + k]) / sc);",
+                           "float r = truncf(oracle_bf16_to_f32(X[m * K + k]) / sc);"),
+    "w8a8_scale_of_first_token": ("float a = fabsf(oracle_bf16_to_f32(X[m * K + k]));",
+                                  "float a = fabsf(oracle_bf16_to_f32(X[k]));"),
+    "w8a8_gemm_drops_weight_scale": ("(double)sx[m] * (double)oracle_bf16_to_f32(sw[n]) * (double)acc;",
+                                     "(double)sx[m] * (double)acc;"),
+    "w8a8_gemm_weight_transposed": ("(int64_t)qx[m * K + k] * (int64_t)qw[n * K + k];",
+                                    "(int64_t)qx[m * K + k] * (int64_t)qw[(k * N + n) % (N * K)];"),
 }
 
 

@@ -669,3 +669,145 @@ def test_equivalent_scaling_identity(sym):
     Y = oracle.gemm_w4a16(X, P, S, Z, g, sym)
     Ysc = oracle.gemm_w4a16_act_scaled(X, a, Ps, Ss, Zs, g, sym)
     assert np.array_equal(Y, Ysc)
+
+
+# ---------------------------------------------------------------------------- W8A8
+# Per-token INT8 activations × per-channel INT8 weights (oracle.quantize_act8,
+# oracle.gemm_w8a8): pinned to hand-computed rows, nearest-grid-point brute
+# force, invariants, and exact rational / independent library evaluations of
+# the integer GEMM.
+
+W8A8_ROWS = json.load(open(os.path.join(os.path.dirname(os.path.abspath(__file__)), "golden",
+                                        "hand_rows_w8a8.json")))["rows"]
+
+
+def _bf16_bits_of(values):
+    return torch.tensor([float(v) for v in values], dtype=torch.float32).to(
+        torch.bfloat16).view(torch.int16).numpy().view(np.uint16)
+
+
+@pytest.mark.parametrize("row", W8A8_ROWS, ids=[r["name"] for r in W8A8_ROWS])
+def test_w8a8_hand_computed_rows(row):
+    X = _bf16_bits_of(row["x"]).reshape(1, -1)
+    q, s = oracle.quantize_act8(X)
+    assert float(s[0]) == float(row["s"])
+    assert q[0].tolist() == row["q"]
+
+
+def test_w8a8_rows_are_independent():
+    """Each token gets its own scale: the hand rows quantized together, zero-padded
+    to one width, give each row's own hand result."""
+    width = max(len(r["x"]) for r in W8A8_ROWS)
+    X = np.stack([np.pad(_bf16_bits_of(r["x"]), (0, width - len(r["x"]))) for r in W8A8_ROWS])
+    q, s = oracle.quantize_act8(X)
+    for i, r in enumerate(W8A8_ROWS):
+        assert float(s[i]) == float(r["s"])
+        assert q[i, :len(r["q"])].tolist() == r["q"] and not q[i, len(r["q"]):].any()
+
+
+def _act_rows(seed, M=6, K=97):
+    rng = np.random.default_rng(seed)
+    x = rng.standard_normal((M, K)) * np.exp(rng.uniform(-6, 6, (M, 1)))
+    x[1, 7] *= 300.0                                   # an outlier channel in one token
+    x[2] = 0.0                                         # an all-zero token
+    return torch.tensor(x, dtype=torch.float32).to(torch.bfloat16).view(torch.int16).numpy().view(np.uint16)
+
+
+@pytest.mark.parametrize("seed", [1, 2, 3])
+def test_w8a8_codes_are_the_nearest_grid_point(seed):
+    """Brute force over all 256 codes with exact rationals: q minimizes |x − s·q|
+    (ties to the even code); the binary32 quotient may decide a near-tie either
+    way, so within 2^-18 of a tie both neighbours are accepted."""
+    X = _act_rows(seed)
+    q, s = oracle.quantize_act8(X)
+    xs = oracle.f32_from_bf16(X)
+    for m in range(X.shape[0]):
+        S = Fraction(float(s[m]))
+        if S == 0:
+            assert not q[m].any()
+            continue
+        for k in range(X.shape[1]):
+            x = Fraction(float(xs[m, k]))
+            best = min(range(-128, 128), key=lambda c: (abs(x - S * c), c % 2))
+            r = x / S
+            near_tie = abs(r - (r.numerator // r.denominator) - Fraction(1, 2)) < Fraction(1, 2 ** 18)
+            assert q[m, k] == best or (near_tie and abs(int(q[m, k]) - best) == 1), (m, k)
+
+
+def test_w8a8_absmax_maps_to_127_and_errors_are_bounded():
+    X = _act_rows(4)
+    q, s = oracle.quantize_act8(X)
+    xs = oracle.f32_from_bf16(X).astype(np.float64)
+    for m in range(X.shape[0]):
+        if s[m] == 0:
+            continue
+        k = int(np.argmax(np.abs(xs[m])))
+        assert abs(int(q[m, k])) == 127 and np.sign(q[m, k]) == np.sign(xs[m, k])
+        err = np.abs(xs[m] - float(s[m]) * q[m].astype(np.float64))
+        assert np.all(err <= 0.5 * float(s[m]) * (1 + 2 ** -20))
+
+
+def test_w8a8_power_of_two_scaling_and_sign_symmetry():
+    X = _act_rows(5)
+    q, s = oracle.quantize_act8(X)
+    xs = oracle.f32_from_bf16(X)
+    for k in (-3, 5):
+        X2 = torch.tensor(xs * 2.0 ** k).to(torch.bfloat16).view(torch.int16).numpy().view(np.uint16)
+        q2, s2 = oracle.quantize_act8(X2)
+        assert np.array_equal(q2, q) and np.array_equal(s2, s * np.float32(2.0 ** k))
+    Xn = torch.tensor(-xs).to(torch.bfloat16).view(torch.int16).numpy().view(np.uint16)
+    qn, sn = oracle.quantize_act8(Xn)
+    assert np.array_equal(qn, -q) and np.array_equal(sn, s)
+
+
+def test_w8a8_gemm_exact_rational_bruteforce():
+    rng = np.random.default_rng(6)
+    M, N, K = 3, 5, 9
+    qx = rng.integers(-128, 128, (M, K)).astype(np.int8)
+    qw = rng.integers(-128, 128, (N, K)).astype(np.int8)
+    sx = (rng.standard_normal(M) * 0.01).astype(np.float32)
+    sw = _bf16_bits_of(rng.standard_normal(N) * 0.003)
+    Y = oracle.gemm_w8a8(qx, sx, qw, sw)
+    swv = oracle.f32_from_bf16(sw)
+    for m in range(M):
+        for n in range(N):
+            exact = Fraction(float(sx[m])) * Fraction(float(swv[n])) * sum(
+                int(qx[m, k]) * int(qw[n, k]) for k in range(K))
+            assert abs(Fraction(Y[m, n]) - exact) <= abs(exact) * Fraction(1, 2 ** 50)
+
+
+def test_w8a8_gemm_matches_numpy_on_dequantized_operands():
+    """numpy's float64 matmul of (s_x·q_x) and (s_w·q_w) — every product exact in
+    binary64 — against the oracle's exact integer sum times the scales."""
+    rng = np.random.default_rng(7)
+    M, N, K = 7, 33, 256
+    X = torch.tensor(rng.standard_normal((M, K)), dtype=torch.float32).to(torch.bfloat16)
+    W = torch.tensor(rng.standard_normal((N, K)) * 0.02, dtype=torch.float32).to(torch.bfloat16)
+    Xb = X.view(torch.int16).numpy().view(np.uint16)
+    Wb = W.view(torch.int16).numpy().view(np.uint16)
+    qw, sw, _ = oracle.quantize8(Wb, K, True)
+    qw = qw.view(np.int8)
+    qx, sx = oracle.quantize_act8(Xb)
+    Y = oracle.gemm_w8a8(qx, sx, qw, sw)
+    ref = (sx[:, None].astype(np.float64) * qx) @ (oracle.f32_from_bf16(sw).reshape(-1, 1).astype(np.float64) * qw).T
+    assert np.allclose(Y, ref, rtol=1e-12, atol=1e-12 * np.max(np.abs(ref)))
+    assert np.allclose(oracle.gemm_w8a8_from_bf16(Xb, qw, sw), Y, rtol=0, atol=0)
+
+
+def test_w8a8_gemm_one_hot_and_saturated_cases():
+    K, N = 64, 4
+    rng = np.random.default_rng(8)
+    qw = rng.integers(-128, 128, (N, K)).astype(np.int8)
+    sw = _bf16_bits_of([0.5, 0.25, 2.0, 1.0])
+    # one-hot token: x = c at k0 -> s_x = |c|/127, q = ±127 there
+    X = np.zeros((1, K), dtype=np.float32)
+    X[0, 11] = -3.0
+    Xb = torch.tensor(X).to(torch.bfloat16).view(torch.int16).numpy().view(np.uint16)
+    Y = oracle.gemm_w8a8_from_bf16(Xb, qw, sw)
+    sx = np.float32(3.0) / np.float32(127.0)
+    want = [float(sx) * w * (-127) * int(qw[n, 11]) for n, w in enumerate([0.5, 0.25, 2.0, 1.0])]
+    assert np.allclose(Y[0], want, rtol=1e-15, atol=0)
+    # every code 127: the integer sum is 127²·K exactly
+    big = np.full((1, 4096), 127, dtype=np.int8)
+    Y2 = oracle.gemm_w8a8(big, np.ones(1, np.float32), big, _bf16_bits_of([1.0]))
+    assert Y2[0, 0] == 127 * 127 * 4096
