@@ -599,6 +599,7 @@ def run_ours(args):
                                                   l2, dev)
             line["w8a16"] = w8a16_extras(w4, peaks, l2, dev)
             line["act_scale"] = act_scale_extras(w4, l2, dev)
+            line["w8a8"] = w8a8_extras(w4, peaks, l2, dev)
     if rank == 0 and world == 1 and not args.no_cpu_baseline and bits == 4:
         cb = cpu_baseline(wl.layers, M, g, sym, unit_bytes=(half == "hbm")) \
             if half == "hbm" else cpu_baseline_sampled(wl.layers[0], M, g, sym, rows=16)
@@ -794,6 +795,51 @@ def w8a16_extras(w4, peaks, l2, dev, iters=200):
             "prefill_2048x8192x8192": {"us": pms * 1e3, "TFLOP/s": ptf,
                                        "frac": ptf / peaks["bf16_tflops"],
                                        "kernel": "gemm_tc_kernel (8-bit codes)"}}
+
+
+# Dense INT8 tensor-core rate relative to bf16 (nominal 4.5 vs 2.25 PFLOP/s per
+# B200): the INT8 roofline is the measured bf16 peak times this ratio.
+INT8_OVER_BF16 = 2.0
+
+
+def w8a8_extras(w4, peaks, l2, dev, iters=30):
+    """W8A8 at the prefill shape (M=2048, K=N=8192): per-token activation
+    quantization, the INT8 tensor-core GEMM, and both together, graph-replayed
+    over copies past L2; TOPS against the INT8 roofline (measured bf16 burst
+    peak x 2, the nominal INT8/bf16 ratio)."""
+    layer = workloads.PREFILL.layers[0]
+    M, N, K = 2048, layer.N, layer.K
+    C, S = w4.quantize8(layer.weight().to(dev), K, True)[:2]
+    X = layer.activation(M).to(dev)
+    copies = copies_for(N * K + 2 * M * K, l2)
+    Cs = [C] + [C.clone() for _ in range(copies - 1)]
+    Xs = [X] + [X.clone() for _ in range(copies - 1)]
+    qs = [w4.quantize_act8(x) for x in Xs]
+    Y = torch.empty(M, N, dtype=torch.bfloat16, device=dev)
+    gs = graph_of(lambda i: w4.quantize_act8(Xs[i % copies], out=qs[i % copies]), copies)
+    qms = time_graphs(gs, iters)
+    del gs
+    gs = graph_of(lambda i: w4.gemm_w8a8(*qs[i % copies], Cs[i % copies], S, out=Y), copies)
+    gms = time_graphs(gs, iters)
+    del gs
+    gs = graph_of(lambda i: (w4.quantize_act8(Xs[i % copies], out=qs[i % copies]),
+                             w4.gemm_w8a8(*qs[i % copies], Cs[i % copies], S, out=Y)), copies)
+    bms = time_graphs(gs, iters)
+    del gs, Cs, Xs, qs, Y
+    torch.cuda.empty_cache()
+    ops = 2 * M * N * K
+    pk = peaks["bf16_tflops"] * INT8_OVER_BF16
+    tops = ops / (gms / 1e3) / 1e12
+    qbytes = 2 * M * K + M * K + 4 * M
+    return {"shape": f"M={M},K={K},N={N}; weights per-channel int8, activations per-token int8",
+            "quantize_activations": {"us": qms * 1e3, "GB/s": qbytes / (qms / 1e3) / 1e9,
+                                     "frac": qbytes / (qms / 1e3) / 1e9 / peaks["hbm_gbs"]},
+            "gemm": {"us": gms * 1e3, "TOPS": tops,
+                     "roofline": {"bound": "tensor", "achieved": tops, "peak": pk, "unit": "TOPS",
+                                  "frac": tops / pk,
+                                  "peak_source": "measured bf16 burst x 2 (nominal INT8/bf16 ratio)"},
+                     "kernel": "gemm_w8a8_kernel"},
+            "quantize_and_gemm": {"us": bms * 1e3, "TOPS": ops / (bms / 1e3) / 1e12}}
 
 
 def act_scale_extras(w4, l2, dev, iters=100):

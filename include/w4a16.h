@@ -65,7 +65,7 @@ extern "C" {
 #endif
 
 #define W4A16_ABI_VERSION 4   /* 3: w4a16_plan.split_tiles; the decode path is one kernel;
-                                 4: W4A16_STATIC_WEIGHTS */
+                                 4: W4A16_STATIC_WEIGHTS, w8a16_gemm_ex/_plan, W8A8 */
 
 typedef enum w4a16_status {
     W4A16_OK = 0,
@@ -308,6 +308,33 @@ w4a16_status w8a16_gemm_ex(const void* X, int64_t M, int64_t K, const void* code
                            const void* scales, const void* zeros, int64_t N, int32_t g,
                            int32_t sym, void* Y, void* workspace, size_t workspace_bytes,
                            int32_t path, void* stream);
+
+/* ---------------------------------------------------------------------------
+ * W8A8: weights and activations both INT8 on the INT8 tensor cores
+ * ("Quantization & Acceleration: 解释 W8A8 与 W4A16 的差异与取舍", 数学机理 (1): both
+ * sides quantized to INT8; activations are dynamic and quantized per token;
+ * "大模型推理中 Weight-only、W8A8 和 FP8 量化有什么区别？如何选型？", §三: integer
+ * matrix multiply on both 8-bit sides, for compute-bound work).  Weights are
+ * quantized once with w8a16_quantize(sym = 1, g = K): int8 codes [N, K] and one
+ * bf16 scale per output channel [N].  Activations are quantized per call.
+ * K must be a multiple of 32; every pointer 16-byte aligned. */
+
+/* Per-token INT8 activations: for each row m of X (bf16 [M, K]),
+ * s[m] = max_k |X[m, k]| / 127 (binary32, IEEE division) and
+ * q[m, k] = round_half_even(X[m, k] / s[m]) clamped to [−128, 127] (0 for a
+ * row of zeros, whose s is 0).  q: int8 [M, K]; s: fp32 [M].  The codes and
+ * scales are bit-identical to the host reference's.  X must be finite. */
+w4a16_status w8a8_quantize_activations(const void* X, int64_t M, int64_t K, void* q, void* s,
+                                        void* stream);
+
+/* W8A8 GEMM: Y[m, n] = bf16_rn(s_x[m] · s_w[n] · Σ_k q_x[m, k]·q_w[n, k]) with the
+ * integer sum accumulated exactly in int32 on the tensor cores (tcgen05.mma
+ * kind::i8), converted to binary32 and multiplied by the two scales.
+ *   qx int8 [M, K], sx fp32 [M] (from w8a8_quantize_activations);
+ *   qw int8 [N, K], sw bf16 [N] (w8a16_quantize, sym = 1, g = K); Y bf16 [M, N].
+ * CTA tile 128 weight rows x 64/128/256 tokens, one CTA per tile; no workspace. */
+w4a16_status w8a8_gemm(const void* qx, const void* sx, int64_t M, int64_t K, const void* qw,
+                       const void* sw, int64_t N, void* Y, void* stream);
 
 /* Read and clear the current device's error word, written by a kernel that gave
  * up a bounded wait (a pipeline barrier that did not complete within about one

@@ -22,7 +22,7 @@ Parity status of each function (what pins it is in ``tests/test_oracle_pins.py``
   scale_activations / gemm_w4a16_act_scaled (per-K activation scale) — pinned
       (identity, exact power-of-two scaling, single rounding of the exact
       product, one-hot activations, the equivalent-scaling identity)
-  quantize_act8 / gemm_w8a8 / gemm_w8a8_from_bf16 (W8A8: per-token INT8
+  quantize_act8 / gemm_w8a8 / gemm_w8a8_sampled / gemm_w8a8_from_bf16 (W8A8: per-token INT8
       activations × per-channel INT8 weights) — pinned (hand-computed rows with
       half-to-even ties, nearest-grid-point brute force, absmax to ±127,
       power-of-two scaling, sign symmetry, zero rows, exact rational brute
@@ -100,6 +100,7 @@ def _load():
             lib.oracle_scale_activations.argtypes = [vp, i64, i64, vp, vp]
             lib.oracle_quantize_act8.argtypes = [vp, i64, i64, vp, vp]
             lib.oracle_gemm_w8a8.argtypes = [vp, vp, vp, vp, i64, i64, i64, vp]
+            lib.oracle_gemm_w8a8_sampled.argtypes = [vp, vp, vp, vp, i64, vp, vp, i64, vp]
             lib.oracle_round_to_bf16.argtypes = [vp, i64, vp]
             lib.oracle_f32_array_to_bf16.argtypes = [vp, i64, vp]
             lib.oracle_num_threads.restype = ctypes.c_int
@@ -369,6 +370,22 @@ def gemm_w8a8(qx, sx, qw, sw_bits) -> np.ndarray:
     Y = np.zeros((M, N), dtype=np.float64)
     lib.oracle_gemm_w8a8(_ptr(qx), _ptr(sx), _ptr(qw), _ptr(sw), M, N, K, _ptr(Y))
     return Y
+
+
+def gemm_w8a8_sampled(qx, sx, qw, sw_bits, ms, ns) -> np.ndarray:
+    """gemm_w8a8 at the listed (m, n) positions only (for full-size checks)."""
+    lib = _load()
+    qx = np.ascontiguousarray(qx, dtype=np.int8)
+    sx = np.ascontiguousarray(sx, dtype=np.float32)
+    qw = np.ascontiguousarray(qw).view(np.int8)
+    sw = _u16(np.ascontiguousarray(sw_bits).reshape(-1))
+    ms = np.ascontiguousarray(ms, dtype=np.int64)
+    ns = np.ascontiguousarray(ns, dtype=np.int64)
+    assert qx.shape[1] == qw.shape[1] and ms.shape == ns.shape
+    out = np.zeros(ms.shape[0], dtype=np.float64)
+    lib.oracle_gemm_w8a8_sampled(_ptr(qx), _ptr(sx), _ptr(qw), _ptr(sw), qx.shape[1], _ptr(ms), _ptr(ns),
+                                 ms.shape[0], _ptr(out))
+    return out
 
 
 def gemm_w8a8_from_bf16(X_bits, qw, sw_bits) -> np.ndarray:

@@ -528,6 +528,18 @@ void oracle_gemm_w8a8(const int8_t* qx, const float* sx, const int8_t* qw, const
     }
 }
 
+/* The same value at the listed (m, n) positions only. */
+void oracle_gemm_w8a8_sampled(const int8_t* qx, const float* sx, const int8_t* qw, const uint16_t* sw,
+                              int64_t K, const int64_t* ms, const int64_t* ns, int64_t count, double* out) {
+#pragma omp parallel for schedule(static)
+    for (int64_t i = 0; i < count; ++i) {
+        const int64_t m = ms[i], n = ns[i];
+        int64_t acc = 0;
+        for (int64_t k = 0; k < K; ++k) acc += (int64_t)qx[m * K + k] * (int64_t)qw[n * K + k];
+        out[i] = (double)sx[m] * (double)oracle_bf16_to_f32(sw[n]) * (double)acc;
+    }
+}
+
 /* Elementwise bf16_rn of a binary32 array. */
 void oracle_f32_array_to_bf16(const float* x, int64_t n, uint16_t* out) {
     for (int64_t i = 0; i < n; ++i) out[i] = oracle_f32_to_bf16_rn(x[i]);

@@ -26,7 +26,7 @@ def lib():
 def declared_functions():
     text = open(HEADER).read()
     text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
-    return sorted(set(re.findall(r"\b(w[48]a16_[a-z0-9_]+)\s*\(", text)))
+    return sorted(set(re.findall(r"\b(w(?:[48]a16|8a8)_[a-z0-9_]+)\s*\(", text)))
 
 
 def test_header_declares_the_abi():
@@ -34,14 +34,15 @@ def test_header_declares_the_abi():
     for n in ("w4a16_quantize", "w4a16_dequantize", "w4a16_gemm", "w4a16_gemm_ex",
               "w4a16_gemm_workspace_size", "w4a16_gemm_plan", "w4a16_status_string",
               "w4a16_device_error", "w4a16_abi_version", "w8a16_quantize", "w8a16_dequantize",
-              "w8a16_gemm", "w8a16_gemm_plan", "w8a16_gemm_ex"):
+              "w8a16_gemm", "w8a16_gemm_plan", "w8a16_gemm_ex", "w8a8_quantize_activations",
+              "w8a8_gemm"):
         assert n in names
 
 
 def test_library_exports_every_declared_symbol(lib):
     out = subprocess.run(["nm", "-D", "--defined-only", w4.LIB_PATH], capture_output=True,
                          text=True, check=True).stdout
-    exported = set(re.findall(r"\sT\s(w[48]a16_\w+)", out))
+    exported = set(re.findall(r"\sT\s(w(?:[48]a16|8a8)_\w+)", out))
     for name in declared_functions():
         assert name in exported, f"{name} declared in w4a16.h but not exported"
         assert hasattr(lib, name)
@@ -150,6 +151,21 @@ def test_static_weights_flag_is_accepted_only_as_a_flag(lib):
     assert w4.plan(1, 4096, 4096, path=w4.PATH_AUTO | w4.STATIC_WEIGHTS) == w4.plan(1, 4096, 4096)
     assert lib.w4a16_gemm_ex(f, 1, 256, f, f, f, 256, 128, 0, f, f, 1 << 30, 0x200, 0, None) == EINVAL
     assert lib.w4a16_gemm_ex(f, 1, 256, f, f, f, 256, 128, 0, f, f, 1 << 30, 0x103, 0, None) == EINVAL
+
+
+def test_w8a8_rejects_without_launching(lib):
+    f = ctypes.c_void_p(FAKE)
+    q = lib.w8a8_quantize_activations
+    assert q(f, 4, 48, f, f, None) == EINVAL                  # K not a multiple of 32
+    assert q(f, -1, 64, f, f, None) == EINVAL
+    assert q(ctypes.c_void_p(FAKE + 2), 4, 64, f, f, None) == EINVAL
+    assert q(f, 0, 64, f, f, None) == 0                       # empty: nothing launched
+    gm = lib.w8a8_gemm
+    assert gm(f, f, 4, 48, f, f, 16, f, None) == EINVAL
+    assert gm(f, f, 4, 64, f, None, 16, f, None) == EINVAL     # missing weight scales
+    assert gm(f, f, 4, 64, f, f, 16, ctypes.c_void_p(FAKE + 8), None) == EINVAL
+    assert gm(f, f, 0, 64, f, f, 16, f, None) == 0
+    assert gm(f, f, 4, 64, f, f, 0, f, None) == 0
 
 
 def test_act_scaled_rejects_without_launching(lib):

@@ -811,3 +811,16 @@ def test_w8a8_gemm_one_hot_and_saturated_cases():
     big = np.full((1, 4096), 127, dtype=np.int8)
     Y2 = oracle.gemm_w8a8(big, np.ones(1, np.float32), big, _bf16_bits_of([1.0]))
     assert Y2[0, 0] == 127 * 127 * 4096
+
+
+def test_w8a8_sampled_equals_full_product():
+    rng = np.random.default_rng(9)
+    M, N, K = 5, 7, 160
+    qx = rng.integers(-128, 128, (M, K)).astype(np.int8)
+    qw = rng.integers(-128, 128, (N, K)).astype(np.int8)
+    sx = (rng.standard_normal(M) * 0.01).astype(np.float32)
+    sw = _bf16_bits_of(rng.standard_normal(N) * 0.003)
+    Y = oracle.gemm_w8a8(qx, sx, qw, sw)
+    ms, ns = np.meshgrid(np.arange(M), np.arange(N), indexing="ij")
+    Ys = oracle.gemm_w8a8_sampled(qx, sx, qw, sw, ms.ravel(), ns.ravel())
+    assert np.array_equal(Ys, Y.ravel())

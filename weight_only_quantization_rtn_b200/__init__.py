@@ -18,7 +18,7 @@ import os
 import torch
 
 __all__ = ["lib", "quantize", "dequantize", "gemm", "gemm_decode_noalloc", "plan", "plan8",
-           "quantize8", "dequantize8", "gemm8",
+           "quantize8", "dequantize8", "gemm8", "quantize_act8", "gemm_w8a8", "linear_w8a8",
            "workspace_size", "device_error", "W4A16Error", "PATH_AUTO", "PATH_DECODE", "PATH_TENSORCORE", "STATIC_WEIGHTS", "LIB_PATH"]
 
 LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libw4a16.so")
@@ -75,11 +75,14 @@ def _load() -> ctypes.CDLL:
     lib.w8a16_gemm_workspace_size.argtypes = [i64, i64, i64, i32]
     lib.w8a16_gemm_plan.argtypes = [i64, i64, i64, i32, i32, i32, ctypes.POINTER(Plan)]
     lib.w8a16_gemm_ex.argtypes = [vp, i64, i64, vp, vp, vp, i64, i32, i32, vp, vp, sz, i32, vp]
+    lib.w8a8_quantize_activations.argtypes = [vp, i64, i64, vp, vp, vp]
+    lib.w8a8_gemm.argtypes = [vp, vp, i64, i64, vp, vp, i64, vp, vp]
     lib.w8a16_gemm_workspace_size.restype = sz
     for name in ("w4a16_quantize", "w4a16_dequantize", "w4a16_gemm", "w4a16_gemm_ex",
                  "w4a16_gemm_act_scaled",
                  "w4a16_gemm_plan", "w4a16_device_error", "w8a16_quantize", "w8a16_dequantize",
-                 "w8a16_gemm", "w8a16_gemm_plan", "w8a16_gemm_ex"):
+                 "w8a16_gemm", "w8a16_gemm_plan", "w8a16_gemm_ex",
+                 "w8a8_quantize_activations", "w8a8_gemm"):
         getattr(lib, name).restype = ctypes.c_int
     if lib.w4a16_abi_version() != ABI_VERSION:
         raise ImportError(f"{LIB_PATH} has ABI version {lib.w4a16_abi_version()}, this binding "
@@ -444,6 +447,53 @@ def gemm8(X: torch.Tensor, codes: torch.Tensor, scales: torch.Tensor,
                                    pid | (STATIC_WEIGHTS if static_weights else 0), _stream(dev)),
                "w8a16_gemm")
     return out
+
+
+def quantize_act8(X: torch.Tensor, out: tuple | None = None):
+    """W8A8 activations: per-token INT8 (w8a8_quantize_activations).  X bf16 [M, K]
+    on a device -> (q int8 [M, K], s float32 [M])."""
+    _need(X, torch.bfloat16, "X")
+    M, K = X.shape
+    if out is None:
+        q = torch.empty((M, K), dtype=torch.int8, device=X.device)
+        s = torch.empty((M,), dtype=torch.float32, device=X.device)
+    else:
+        q, s = out
+    with torch.cuda.device(X.device):
+        _check(lib().w8a8_quantize_activations(_ptr(X), M, K, _ptr(q), _ptr(s), _stream(X.device)),
+               "w8a8_quantize_activations")
+    return q, s
+
+
+def gemm_w8a8(qx: torch.Tensor, sx: torch.Tensor, qw: torch.Tensor, sw: torch.Tensor,
+              out: torch.Tensor | None = None) -> torch.Tensor:
+    """W8A8 GEMM on the INT8 tensor cores: Y = s_x·s_w·(q_x·q_wᵀ) (w8a8_gemm).
+    qx int8 [M, K], sx float32 [M]; qw int8 (or uint8 bytes) [N, K] and sw bf16 [N]
+    or [N, 1] from quantize8(W, g=K, sym=True); Y bf16 [M, N]."""
+    if qx.dtype != torch.int8 or sx.dtype != torch.float32:
+        raise TypeError("qx must be int8 and sx float32")
+    if qw.dtype not in (torch.int8, torch.uint8) or sw.dtype != torch.bfloat16:
+        raise TypeError("qw must be int8/uint8 codes and sw bf16 scales")
+    M, K = qx.shape
+    N = qw.shape[0]
+    if qw.shape[1] != K or sx.numel() != M or sw.numel() != N:
+        raise ValueError("W8A8 operand shapes disagree")
+    for t in (qx, sx, qw, sw):
+        if not t.is_contiguous() or t.device != qx.device:
+            raise ValueError("W8A8 operands must be contiguous and on one device")
+    if out is None:
+        out = torch.empty((M, N), dtype=torch.bfloat16, device=qx.device)
+    with torch.cuda.device(qx.device):
+        _check(lib().w8a8_gemm(_ptr(qx), _ptr(sx), M, K, _ptr(qw), _ptr(sw), N, _ptr(out),
+                               _stream(qx.device)), "w8a8_gemm")
+    return out
+
+
+def linear_w8a8(X: torch.Tensor, qw: torch.Tensor, sw: torch.Tensor,
+                out: torch.Tensor | None = None) -> torch.Tensor:
+    """Quantize X per token, then the W8A8 GEMM (two kernels)."""
+    qx, sx = quantize_act8(X)
+    return gemm_w8a8(qx, sx, qw, sw, out=out)
 
 
 def device_error() -> int:

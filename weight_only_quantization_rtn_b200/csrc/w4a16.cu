@@ -10,6 +10,7 @@
 #include "../../include/w4a16.h"
 #include "common.cuh"
 #include "gemm_tcgen05.cuh"
+#include "gemm_w8a8.cuh"
 #include "gemv_decode.cuh"
 #include "quantize.cuh"
 
@@ -755,6 +756,50 @@ w4a16_status gemm_impl(const void* X, int64_t M, int64_t K, const void* packed, 
 }  // namespace
 
 // ==================================================================== ABI
+// ---------------------------------------------------------------- W8A8 launch
+bool w8a8_shape_ok(int64_t M, int64_t N, int64_t K) {
+    return M >= 0 && N >= 0 && K > 0 && K % 32 == 0 && M <= kMaxDim && N <= kMaxDim && K <= kMaxDim;
+}
+
+template <int BM>
+w4a16_status launch_w8a8_t(const void* qx, const void* sx, int64_t M, int64_t K, const void* qw,
+                           const void* sw, int64_t N, void* Y, cudaStream_t stream) {
+    using Cfg = W8a8Config<BM>;
+    CUtensorMap tmW, tmX;
+    w4a16_status st = encode_2d(&tmW, CU_TENSOR_MAP_DATA_TYPE_UINT8, qw, (uint64_t)K, (uint64_t)N,
+                                (uint64_t)K, kW8a8BlockK, kW8a8TileN, CU_TENSOR_MAP_SWIZZLE_128B);
+    if (st != W4A16_OK) return st;
+    st = encode_2d(&tmX, CU_TENSOR_MAP_DATA_TYPE_UINT8, qx, (uint64_t)K, (uint64_t)M, (uint64_t)K,
+                   kW8a8BlockK, (uint32_t)BM, CU_TENSOR_MAP_SWIZZLE_128B);
+    if (st != W4A16_OK) return st;
+    auto kern = gemm_w8a8_kernel<BM>;
+    static bool attr_set[kMaxDevices] = {};
+    int dev = 0;
+    cudaGetDevice(&dev);
+    if (!attr_set[dev]) {
+        if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, Cfg::kSmemBytes) !=
+            cudaSuccess)
+            return W4A16_ECUDA;
+        attr_set[dev] = true;
+    }
+    const int64_t tiles = ((N + kW8a8TileN - 1) / kW8a8TileN) * ((M + BM - 1) / BM);
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3((unsigned)tiles, 1, 1);
+    cfg.blockDim = dim3(kW8a8Threads, 1, 1);
+    cfg.dynamicSmemBytes = (size_t)Cfg::kSmemBytes;
+    cfg.stream = stream;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    if (cudaLaunchKernelEx(&cfg, kern, tmW, tmX, static_cast<const uint16_t*>(sw),
+                           static_cast<const float*>(sx), static_cast<uint16_t*>(Y), (int)M, (int)N,
+                           (int)K) != cudaSuccess)
+        return W4A16_ECUDA;
+    return W4A16_OK;
+}
+
 extern "C" {
 
 int32_t w4a16_abi_version(void) { return W4A16_ABI_VERSION; }
@@ -956,6 +1001,36 @@ w4a16_status w8a16_gemm(const void* X, int64_t M, int64_t K, const void* codes, 
                         void* workspace, size_t workspace_bytes, void* stream) {
     return w8a16_gemm_ex(X, M, K, codes, scales, zeros, N, g, sym, Y, workspace, workspace_bytes,
                          W4A16_PATH_AUTO, stream);
+}
+
+w4a16_status w8a8_quantize_activations(const void* X, int64_t M, int64_t K, void* q, void* s,
+                                        void* stream) {
+    if (!w8a8_shape_ok(M, 0, K)) return W4A16_EINVAL;
+    if (M == 0) return W4A16_OK;
+    if (!X || !q || !s || !aligned16(X) || !aligned16(q) || !aligned16(s)) return W4A16_EINVAL;
+    DeviceInfo di;
+    w4a16_status st = device_info(&di);
+    if (st != W4A16_OK) return st;
+    const int grid = (int)(M < (int64_t)di.sm_count * 8 ? M : (int64_t)di.sm_count * 8);
+    w8a8_quantize_act_kernel<<<grid, kW8a8ActThreads, 0, static_cast<cudaStream_t>(stream)>>>(
+        static_cast<const uint16_t*>(X), M, K, static_cast<int8_t*>(q), static_cast<float*>(s));
+    return launch_status();
+}
+
+w4a16_status w8a8_gemm(const void* qx, const void* sx, int64_t M, int64_t K, const void* qw,
+                       const void* sw, int64_t N, void* Y, void* stream) {
+    if (!w8a8_shape_ok(M, N, K)) return W4A16_EINVAL;
+    if (M == 0 || N == 0) return W4A16_OK;
+    if (!qx || !sx || !qw || !sw || !Y) return W4A16_EINVAL;
+    if (!aligned16(qx) || !aligned16(sx) || !aligned16(qw) || !aligned16(sw) || !aligned16(Y))
+        return W4A16_EINVAL;
+    DeviceInfo di;
+    w4a16_status st = device_info(&di);
+    if (st != W4A16_OK) return st;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    if (M <= 64) return launch_w8a8_t<64>(qx, sx, M, K, qw, sw, N, Y, s);
+    if (M <= 128) return launch_w8a8_t<128>(qx, sx, M, K, qw, sw, N, Y, s);
+    return launch_w8a8_t<256>(qx, sx, M, K, qw, sw, N, Y, s);
 }
 
 w4a16_status w4a16_device_error(int32_t* code) {
