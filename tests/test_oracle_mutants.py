@@ -48,8 +48,8 @@ MUTANTS = {
                                   "float a = fabsf(oracle_bf16_to_f32(X[k]));"),
     "w8a8_gemm_drops_weight_scale": ("(double)sx[m] * (double)oracle_bf16_to_f32(sw[n]) * (double)acc;",
                                      "(double)sx[m] * (double)acc;"),
-    "w8a8_gemm_weight_transposed": ("(int64_t)qx[m * K + k] * (int64_t)qw[n * K + k];",
-                                    "(int64_t)qx[m * K + k] * (int64_t)qw[(k * N + n) % (N * K)];"),
+    "w8a8_gemm_weight_transposed": ("(int64_t)qw[n * K + k];\n            Y[m * N + n]",
+                                    "(int64_t)qw[(k * N + n) % (N * K)];\n            Y[m * N + n]"),
 }
 
 
