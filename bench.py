@@ -87,6 +87,7 @@ def algorithmic_bytes(M: int, N: int, K: int, g: int, sym: bool, bits: int = 4) 
 KERNEL_SOURCES = {
     "gemv_decode_kernel": ("common.cuh", "gemv_decode.cuh", "w4a16.cu"),
     "gemm_tc_kernel": ("common.cuh", "gemm_tcgen05.cuh", "w4a16.cu"),
+    "gemm_w8a8_kernel": ("common.cuh", "gemm_w8a8.cuh", "w4a16.cu"),
 }
 
 
@@ -837,7 +838,8 @@ def w8a8_extras(w4, peaks, l2, dev, iters=30):
             "gemm": {"us": gms * 1e3, "TOPS": tops,
                      "roofline": {"bound": "tensor", "achieved": tops, "peak": pk, "unit": "TOPS",
                                   "frac": tops / pk,
-                                  "peak_source": "measured bf16 burst x 2 (nominal INT8/bf16 ratio)"},
+                                  "peak_source": "measured bf16 burst x 2 (nominal INT8/bf16 ratio)",
+                                  "traffic": ncu_traffic("gemm_w8a8_kernel:w8a8")},
                      "kernel": "gemm_w8a8_kernel"},
             "quantize_and_gemm": {"us": bms * 1e3, "TOPS": ops / (bms / 1e3) / 1e12}}
 
@@ -1065,6 +1067,20 @@ def crossover_sweep(args):
         print(json.dumps({"crossover": crossover_rows(w4, dev, l2)}))
 
 
+def run_extra(args):
+    """One extra of the benchmark line, printed alone ({"<name>": {...}})."""
+    import weight_only_quantization_rtn_b200 as w4
+    from weight_only_quantization_rtn_b200 import build as w4build
+    w4build.build()
+    w4.lib()
+    dev = torch.device("cuda", 0)
+    props = torch.cuda.get_device_properties(dev)
+    l2 = getattr(props, "L2_cache_size", 0) or L2_BYTES_FALLBACK
+    peaks, _ = load_peaks()
+    if args.extra == "w8a8":
+        print(json.dumps({"w8a8": w8a8_extras(w4, peaks, l2, dev)}))
+
+
 def run_reference(args):
     """The reference arm: the host oracle as it stands, timed on this machine's
     cores, on the same workload and metric; each step a bounded sample."""
@@ -1130,10 +1146,14 @@ def main():
                     help="print the M-dispatch sweep at K=N=8192 instead of a benchmark line")
     ap.add_argument("--crossover8", action="store_true",
                     help="the same sweep for 8-bit codes (W8A16)")
+    ap.add_argument("--extra", choices=["w8a8"],
+                    help="print one extra measurement of the benchmark line by itself (profiling)")
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be at least 3")
-    if args.crossover or args.crossover8:
+    if args.extra:
+        run_extra(args)
+    elif args.crossover or args.crossover8:
         crossover_sweep(args)
     elif args.impl == "reference":
         run_reference(args)

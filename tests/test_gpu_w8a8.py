@@ -30,7 +30,11 @@ def _acts(M, K, seed):
     return X
 
 
-@pytest.mark.parametrize("M,K", [(1, 32), (5, 96), (7, 4096), (300, 1056), (2, 11008), (64, 256)])
+# K = 8192 fills the four register chunks per thread exactly; 8224, 11008 and
+# 28672 run the sixteen-chunk kernel with a ragged last chunk set; 32800 is
+# past the register cache (the row is read twice).
+@pytest.mark.parametrize("M,K", [(1, 32), (5, 96), (7, 4096), (300, 1056), (2, 11008), (64, 256),
+                                 (3, 8192), (4, 8224), (3, 28672), (3, 32768), (3, 32800)])
 def test_quantize_act8_bit_exact(M, K):
     X = _acts(M, K, seed=M + K)
     q, s = w4.quantize_act8(X.cuda())

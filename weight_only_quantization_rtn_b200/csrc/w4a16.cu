@@ -1008,12 +1008,18 @@ w4a16_status w8a8_quantize_activations(const void* X, int64_t M, int64_t K, void
     if (!w8a8_shape_ok(M, 0, K)) return W4A16_EINVAL;
     if (M == 0) return W4A16_OK;
     if (!X || !q || !s || !aligned16(X) || !aligned16(q) || !aligned16(s)) return W4A16_EINVAL;
-    DeviceInfo di;
-    w4a16_status st = device_info(&di);
-    if (st != W4A16_OK) return st;
-    const int grid = (int)(M < (int64_t)di.sm_count * 8 ? M : (int64_t)di.sm_count * 8);
-    w8a8_quantize_act_kernel<<<grid, kW8a8ActThreads, 0, static_cast<cudaStream_t>(stream)>>>(
-        static_cast<const uint16_t*>(X), M, K, static_cast<int8_t*>(q), static_cast<float*>(s));
+    const int grid = (int)(M < (int64_t(1) << 30) ? M : (int64_t(1) << 30));   // one CTA per token
+    const int64_t chunks = K / 8;
+    const uint16_t* x = static_cast<const uint16_t*>(X);
+    int8_t* qq = static_cast<int8_t*>(q);
+    float* ss = static_cast<float*>(s);
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    if (chunks <= 4 * kW8a8ActThreads)
+        w8a8_quantize_act_kernel<4><<<grid, kW8a8ActThreads, 0, st>>>(x, M, K, qq, ss);
+    else if (chunks <= 16 * kW8a8ActThreads)
+        w8a8_quantize_act_kernel<16><<<grid, kW8a8ActThreads, 0, st>>>(x, M, K, qq, ss);
+    else
+        w8a8_quantize_act_kernel<0><<<grid, kW8a8ActThreads, 0, st>>>(x, M, K, qq, ss);
     return launch_status();
 }
 
