@@ -1067,6 +1067,10 @@ def crossover_sweep(args):
         print(json.dumps({"crossover": crossover_rows(w4, dev, l2)}))
 
 
+# Extras that bench.py --extra NAME runs alone (their ncu captures use that command).
+EXTRAS = ("w8a8",)
+
+
 def run_extra(args):
     """One extra of the benchmark line, printed alone ({"<name>": {...}})."""
     import weight_only_quantization_rtn_b200 as w4
@@ -1146,7 +1150,7 @@ def main():
                     help="print the M-dispatch sweep at K=N=8192 instead of a benchmark line")
     ap.add_argument("--crossover8", action="store_true",
                     help="the same sweep for 8-bit codes (W8A16)")
-    ap.add_argument("--extra", choices=["w8a8"],
+    ap.add_argument("--extra", choices=list(EXTRAS),
                     help="print one extra measurement of the benchmark line by itself (profiling)")
     args = ap.parse_args()
     if args.warmup < 3:

@@ -46,7 +46,7 @@ def test_traffic_table_points_at_committed_profiles():
     table = json.load(open(os.path.join(ROOT, "profiles", "ncu_traffic.json")))
     for key, entry in table.items():
         kernel, workload = key.split(":")
-        assert kernel in bench.KERNEL_SOURCES and workload in bench.WORKLOAD_DEFS
+        assert kernel in bench.KERNEL_SOURCES and (workload in bench.WORKLOAD_DEFS or workload in bench.EXTRAS)
         src = entry["source"].split(" ")[0]
         assert os.path.exists(os.path.join(ROOT, src)), src
         assert entry["dram_bytes_per_launch"] > 0
