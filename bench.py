@@ -1068,7 +1068,7 @@ def crossover_sweep(args):
 
 
 # Extras that bench.py --extra NAME runs alone (their ncu captures use that command).
-EXTRAS = ("w8a8",)
+EXTRAS = ("w8a8", "quantize", "w8a16")
 
 
 def run_extra(args):
@@ -1083,6 +1083,10 @@ def run_extra(args):
     peaks, _ = load_peaks()
     if args.extra == "w8a8":
         print(json.dumps({"w8a8": w8a8_extras(w4, peaks, l2, dev)}))
+    elif args.extra == "quantize":
+        print(json.dumps({"quantize_dequantize": elementwise_extras(w4, peaks, l2, dev)}))
+    elif args.extra == "w8a16":
+        print(json.dumps({"w8a16": w8a16_extras(w4, peaks, l2, dev)}))
 
 
 def run_reference(args):

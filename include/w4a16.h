@@ -88,8 +88,10 @@ typedef enum w4a16_path {
                                   owner, which adds the other owners' parts in a fixed order */
     W4A16_PATH_TENSORCORE = 2  /* large-M kernel: TMA-fed INT4 tile dequantized into shared
                                   memory and fed to tcgen05 bf16 MMA with TMEM accumulators;
-                                  when the output tiles are fewer than the SMs, or the last
-                                  wave of tiles would leave most SMs idle, those tiles split
+                                  when the output tiles are fewer than the resident CTA
+                                  slots (two per SM for tiles of at most 64 activation rows,
+                                  else one), or the last wave of tiles would leave most
+                                  slots idle, those tiles split
                                   K and a reduce kernel adds the parts in a fixed order */
 } w4a16_path;
 
@@ -148,8 +150,8 @@ w4a16_status w4a16_dequantize(const void* packed, const void* scales, const void
 /* Bytes of device workspace w4a16_gemm needs for this shape.  The decode path
  * stores there the fp32 partial sums of the 256-row blocks that its stream-K
  * partition splits between CTAs, with a ready flag per part.  The tensor-core path, for the output tiles
- * whose K it splits into S parts (all tiles when they are fewer than the SMs,
- * else only a mostly-empty last wave), stores S fp32 partial tiles of
+ * whose K it splits into S parts (all tiles when they are fewer than the
+ * resident CTA slots, else only a mostly-empty last wave), stores S fp32 partial tiles of
  * 128 weight rows x tile_m activation rows per split tile, and needs 0 bytes
  * when it splits nothing.  In both cases a second, small kernel adds the parts
  * in a fixed order.  The contents are scratch: no

@@ -131,7 +131,8 @@ def test_workspace_sizes(lib):
     assert w4.workspace_size(4096, 8192, 8192, 32) == 0          # 1024 tiles: last wave 92% full
     p17 = w4.plan(17, 8192, 8192, 32)
     splits = p17["grid"] // ((8192 // 128) * 1)
-    assert splits == 2 and p17["kernels"] == 2
+    # 64 tiles, 2 x 148 resident slots (two CTAs per SM at 32 activation rows): 4 splits
+    assert splits == 4 and p17["kernels"] == 2
     # tile-local parts: [split][tile][32 activation rows][128 weight rows] fp32
     assert w4.workspace_size(17, 8192, 8192, 32) == splits * 64 * 32 * 128 * 4
     # decode: per slot (row blocks + CTAs) 16 ready flags (rounded to 256 bytes in
@@ -214,9 +215,10 @@ def test_dispatch_plans():
     assert w4.plan(9, 4096, 4096)["tile_m"] == 16
 
 
-def _tc_schedule(M, N, K, g, sms=148):
+def _tc_schedule(M, N, K, g, sm_count=148):
     """Mirror of the tensor-core launch schedule: (head tiles, tail tiles, splits)."""
     bm = 32 if M <= 32 else 64 if M <= 64 else 128 if M <= 128 else 256
+    sms = sm_count * (2 if bm <= 64 else 1)            # resident CTA slots
     tiles = -(-N // 128) * -(-M // bm)
     num_kb = -(-K // 64)
     tail = tiles if tiles < sms else (tiles % sms if 0 < tiles % sms <= sms // 2 else 0)

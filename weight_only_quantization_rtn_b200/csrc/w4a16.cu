@@ -225,8 +225,8 @@ int tc_tile_m(int64_t M) {
     return 256;
 }
 
-// Split-K for the tensor-core path: when the (n, m) tiles are fewer than the SMs,
-// split each tile's K blocks over up to sm_count / tiles CTAs (at most 8, at
+// Split-K for the tensor-core path: when the (n, m) tiles are fewer than the
+// resident CTA slots, split each tile's K blocks over up to slots / tiles CTAs (at most 8, at
 // least 4 K blocks each); split boundaries are multiples of the scale slab
 // (g/8 blocks) when scales come by TMA.  Returns K blocks per split.
 int tc_kb_split(int num_kb, int splits, int g, bool sz_tma) {
@@ -237,10 +237,11 @@ int tc_kb_split(int num_kb, int splits, int g, bool sz_tma) {
 
 // Tensor-core launch schedule.  Output tiles (128 weight rows x bm activation
 // rows) run unsplit in a "head" launch; K is split over `splits` CTAs per tile for
-// the "tail" tiles, whose partials a reduce kernel adds.  All tiles are tail when
-// they are fewer than the SMs; otherwise only a last partial wave that would leave
-// more than half of the SMs idle becomes the tail.  Splits: up to sm_count / tail
-// tiles, at most 8, at least 4 K blocks each.
+// the "tail" tiles, whose partials a reduce kernel adds.  A wave is one CTA per
+// resident slot (SMs x tc_ctas_per_sm(bm)).  All tiles are tail when they are
+// fewer than the slots; otherwise only a last partial wave that would leave more
+// than half of the slots idle becomes the tail.  Splits: up to slots / tail tiles,
+// at most 8, at least 4 K blocks each.
 struct TcSchedule {
     int tiles_n;      // n-tiles (128 weight rows each)
     int64_t head;     // unsplit tiles [0, head)
@@ -251,6 +252,7 @@ struct TcSchedule {
 
 TcSchedule tc_schedule(int64_t M, int64_t N, int64_t K, int g, int bm, int sm_count) {
     TcSchedule t{};
+    sm_count *= tc_ctas_per_sm(bm);           // resident CTA slots
     t.tiles_n = (int)((N + kTcTileN - 1) / kTcTileN);
     const int64_t tiles = (int64_t)t.tiles_n * ((M + bm - 1) / bm);
     const int num_kb = (int)((K + kTcBlockK - 1) / kTcBlockK);
@@ -561,6 +563,10 @@ w4a16_status launch_tc_t(const w4a16_plan& p, const CUtensorMap& tmX, const CUte
     if (!attr_set[dev]) {
         if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                  Cfg::kSmemBytes) != cudaSuccess)
+            return W4A16_ECUDA;
+        // all of the SM's unified L1 / shared storage as shared memory, so that
+        // tc_ctas_per_sm(BM) CTAs are resident at once
+        if (cudaFuncSetAttribute(kern, cudaFuncAttributePreferredSharedMemoryCarveout, 100) != cudaSuccess)
             return W4A16_ECUDA;
         attr_set[dev] = true;
     }
