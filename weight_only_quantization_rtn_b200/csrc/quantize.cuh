@@ -47,15 +47,18 @@ __device__ __forceinline__ uint32_t sym_params(float amax, float* s) {
 
 // Codes of eight elements, element i in nibble i: q = clamp(rint(x/s) + z, 0, 15)
 // (asymmetric) or clamp(rint(x/s), −8, 7) as 4-bit two's complement (symmetric).
-// All codes are 0 when s is 0.
+// All codes are 0 when s is 0.  rint is the binary32 addition of 1.5·2^23 to the
+// quotient (clamped to ±32 first, which changes no code): the sum rounds to the
+// nearest integer, ties to even, and its bit pattern minus that of 1.5·2^23 is
+// the integer itself, so no float-to-integer conversion is needed.
 template <bool SYM>
 __device__ __forceinline__ uint32_t codes8(const float x[8], float s, int32_t z) {
     uint32_t word = 0;
     if (s == 0.0f) return word;
 #pragma unroll
     for (int i = 0; i < 8; ++i) {
-        const float r = clampf(rintf(__fdiv_rn(x[i], s)), -32.0f, 32.0f);
-        int32_t q = (int32_t)r;
+        const float r = clampf(__fdiv_rn(x[i], s), -32.0f, 32.0f);
+        int32_t q = __float_as_int(r + 12582912.0f) - 0x4B400000;
         if (SYM) {
             q = q < -8 ? -8 : (q > 7 ? 7 : q);
             word |= ((uint32_t)q & 0xFu) << (4 * i);

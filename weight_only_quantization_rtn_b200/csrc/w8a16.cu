@@ -83,14 +83,18 @@ __device__ __forceinline__ uint32_t params(float mn, float mx, float* s, int32_t
     return s_bits;
 }
 
-// Codes of eight elements as eight bytes (element i in byte i).
+// Codes of eight elements as eight bytes (element i in byte i).  rint is the
+// binary32 addition of 1.5·2^23 to the quotient (clamped to ±512 first, which
+// changes no code): the sum rounds to the nearest integer, ties to even, and its
+// bit pattern minus that of 1.5·2^23 is the integer.
 template <bool SYM>
 __device__ __forceinline__ uint2 codes8(const float x[8], float s, int32_t z) {
     uint32_t b[2] = {0u, 0u};
     if (s != 0.0f) {
 #pragma unroll
         for (int i = 0; i < 8; ++i) {
-            int32_t q = (int32_t)clampf(rintf(__fdiv_rn(x[i], s)), -512.0f, 512.0f);
+            const float r = clampf(__fdiv_rn(x[i], s), -512.0f, 512.0f);
+            int32_t q = __float_as_int(r + 12582912.0f) - 0x4B400000;
             if (SYM) {
                 q = q < -128 ? -128 : (q > 127 ? 127 : q);
             } else {
