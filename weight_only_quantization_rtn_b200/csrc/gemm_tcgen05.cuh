@@ -76,14 +76,26 @@ struct TcConfig {
     static constexpr int kABytes = kTcTileN * kTcBlockK * 2;    // dequantized weight tile
     static constexpr int kPBytes = kTcTileN * kRowBytes;        // codes tile
     static constexpr int kSZBytes = 2 * kTcTileN * 4;              // scale and zero pairs per row
-    static constexpr int kStageBytes = kXBytes + kABytes + kPBytes + kSZBytes;
     static constexpr int kSlabBytes = 2 * 2 * kTcTileN * 8 * 2;  // two slots of scale + zero slabs
-    static constexpr int kBudget = 220 * 1024 / tc_ctas_per_sm(BM) - kSlabBytes;
-    static constexpr int kStagesRaw = kBudget / kStageBytes;
-    static constexpr int kStages = kStagesRaw > 8 ? 8 : kStagesRaw;
+    // What TMA (and the scale copies) bring per K block: one slot of the load ring.
+    static constexpr int kLoadBytes = kXBytes + kPBytes + kSZBytes;
+    // 8-bit codes double the load per K block; their loads get a ring of their own,
+    // deeper than the ring of dequantized A tiles (2 or 3), which needs only to
+    // cover the MMA (M=2048, K=N=8192: 318 -> 275 us; M=32: 34.8 -> 31.7 us).  With
+    // 4-bit codes, and 8-bit codes at BM = 128, each load slot carries its own A
+    // tile (one ring): there the extra barrier traffic of two rings cost 2–9%.
+    static constexpr bool kSplitRing = BITS == 8 && BM != 128;
+    static constexpr int kSplitABufs = BM >= 128 ? 3 : 2;
+    static constexpr int kBudget = 220 * 1024 / tc_ctas_per_sm(BM) - kSlabBytes -
+                                   (kSplitRing ? kSplitABufs * kABytes : 0);
+    static constexpr int kSlotBytes = kLoadBytes + (kSplitRing ? 0 : kABytes);
+    static constexpr int kStagesRaw = kBudget / kSlotBytes;
+    static constexpr int kStagesMax = kSplitRing ? 12 : 8;
+    static constexpr int kStages = kStagesRaw > kStagesMax ? kStagesMax : kStagesRaw;
+    static constexpr int kABufs = kSplitRing ? kSplitABufs : kStages;
     static constexpr int kBarrierBytes = 1024;
-    static constexpr int kSmemBytes =
-        kStages * kStageBytes + kSlabBytes + kBarrierBytes + 1024;   // + align slack
+    static constexpr int kSmemBytes = kStages * kLoadBytes + kABufs * kABytes + kSlabBytes +
+                                      kBarrierBytes + 1024;   // + align slack
     static constexpr int kTmemCols = BM < 32 ? 32 : BM;
 };
 
@@ -114,26 +126,31 @@ __global__ void __launch_bounds__(kTcThreads, tc_ctas_per_sm(BM))
     (void)tiles_n;                        // the order is m-tile fastest (below)
     static_assert(BITS == 4 || BITS == 8, "4- or 8-bit codes");
     using Cfg = TcConfig<BM, BITS>;
-    constexpr int S = Cfg::kStages;
-    static_assert(S >= 2, "pipeline needs at least two stages");
+    constexpr int S = Cfg::kStages;                 // load ring (X, codes, scale pairs)
+    constexpr int NA = Cfg::kABufs;                 // dequantized A ring
+    constexpr bool kSplit = Cfg::kSplitRing;        // else A tile i lives in load slot i % S
+    static_assert(S >= 2 && NA >= 2, "pipeline needs at least two slots per ring");
+    static_assert((2 * S + 2 * NA + 5) * 8 + 8 <= Cfg::kBarrierBytes, "barrier area");
     static_assert(BM % 16 == 0 && BM >= 16 && BM <= 256, "UMMA N must be 16..256, step 16");
 
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>(
         (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
     uint8_t* xs = smem;                                   // S x kXBytes
-    uint8_t* as = xs + S * Cfg::kXBytes;                  // S x kABytes
-    uint8_t* ps = as + S * Cfg::kABytes;                  // S x kPBytes
+    uint8_t* as = xs + S * Cfg::kXBytes;                  // NA x kABytes
+    uint8_t* ps = as + NA * Cfg::kABytes;                 // S x kPBytes
     uint32_t* szs = reinterpret_cast<uint32_t*>(ps + S * Cfg::kPBytes);   // S x [2][128] u32 pairs
     uint16_t* slab = reinterpret_cast<uint16_t*>(szs + S * 2 * kTcTileN); // 2 x [2][128][8] u16
     uint64_t* bars = reinterpret_cast<uint64_t*>(slab + 2 * 2 * kTcTileN * 8);
-    uint64_t* full = bars;             // TMA bytes landed
-    uint64_t* afull = bars + S;        // dequantized A tile written
-    uint64_t* empty = bars + 2 * S;    // MMAs reading the stage retired
-    uint64_t* accf = bars + 3 * S;     // all MMAs retired
-    uint64_t* slab_full = bars + 3 * S + 1;    // [2] slab of scales/zeros landed
-    uint64_t* slab_empty = bars + 3 * S + 3;   // [2] dequantizers done with the slab
-    uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(bars + 3 * S + 5);
+    uint64_t* full = bars;             // [S] load slot landed
+    uint64_t* empty = bars + S;        // [S] load slot free: its MMAs retired (and, with
+                                       //     two rings, the dequantizers read its codes)
+    uint64_t* afull = bars + 2 * S;    // [NA] dequantized A tile written
+    uint64_t* aempty = afull + NA;     // [NA] MMAs reading the A tile retired
+    uint64_t* accf = aempty + NA;      // all MMAs retired
+    uint64_t* slab_full = accf + 1;    // [2] slab of scales/zeros landed
+    uint64_t* slab_empty = accf + 3;   // [2] dequantizers done with the slab
+    uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(accf + 5);
     // G == 0: per-channel granularity, one scale (and zero) per row for all of K;
     // each dequantizing thread reads its row's pair once, nothing is staged.
     constexpr int kG = G == 0 ? 1 : G;                            // divisor for the grouped forms
@@ -159,8 +176,11 @@ __global__ void __launch_bounds__(kTcThreads, tc_ctas_per_sm(BM))
         for (int s = 0; s < S; ++s) {
             // TMA arrive (+ 32 scale-copying lanes)
             mbar_init(smem_u32(&full[s]), (sz_tma || G == 0) ? 1 : 1 + 32);
-            mbar_init(smem_u32(&afull[s]), kTcDequantWarps);
-            mbar_init(smem_u32(&empty[s]), 1);
+            mbar_init(smem_u32(&empty[s]), kSplit ? 1 + kTcDequantWarps : 1);
+        }
+        for (int a = 0; a < NA; ++a) {
+            mbar_init(smem_u32(&afull[a]), kTcDequantWarps);
+            mbar_init(smem_u32(&aempty[a]), 1);
         }
         mbar_init(smem_u32(accf), 1);
         grid_launch_dependents();          // the split-K reduction may start as this grid drains
@@ -269,10 +289,11 @@ __global__ void __launch_bounds__(kTcThreads, tc_ctas_per_sm(BM))
             for (int i = 0; i < nkb; ++i) {
                 const int s = i % S;
                 const uint32_t ph = (uint32_t)(i / S) & 1u;
+                const int ab = kSplit ? i % NA : s;
                 if (!mbar_wait(smem_u32(&full[s]), ph)) break;
-                if (!mbar_wait(smem_u32(&afull[s]), ph)) break;
+                if (!mbar_wait(smem_u32(&afull[ab]), (uint32_t)(i / NA) & 1u)) break;
                 tc_fence_after();
-                const uint32_t a_base = smem_u32(as + s * Cfg::kABytes);
+                const uint32_t a_base = smem_u32(as + ab * Cfg::kABytes);
                 const uint32_t x_base = smem_u32(xs + s * Cfg::kXBytes);
 #pragma unroll
                 for (int kk = 0; kk < kTcBlockK / 16; ++kk) {
@@ -280,7 +301,8 @@ __global__ void __launch_bounds__(kTcThreads, tc_ctas_per_sm(BM))
                                 sw128_kmajor_desc(x_base + kk * 32), idesc,
                                 (i | kk) != 0 ? 1u : 0u);
                 }
-                tc_commit(smem_u32(&empty[s]));
+                tc_commit(smem_u32(&empty[s]));       // X (and a one-ring A tile) read
+                if (kSplit) tc_commit(smem_u32(&aempty[ab]));   // the A tile may be rewritten
             }
             // Signals the epilogue; also taken on the error path so that every
             // issued MMA has retired before TMEM is released.
@@ -339,8 +361,9 @@ __global__ void __launch_bounds__(kTcThreads, tc_ctas_per_sm(BM))
                 spair = lds_u32(szs + s * 2 * kTcTileN + r);
                 zpair = SYM ? 0u : lds_u32(szs + s * 2 * kTcTileN + kTcTileN + r);
             }
+            const int ab = kSplit ? i % NA : s;
             const uint8_t* prow = ps + s * Cfg::kPBytes + r * Cfg::kRowBytes;
-            const uint32_t arow = smem_u32(as + s * Cfg::kABytes + r * 128);
+            const uint32_t arow = smem_u32(as + ab * Cfg::kABytes + r * 128);
             {
                 uint4 v, v8 = make_uint4(0, 0, 0, 0);
                 if constexpr (BITS == 4) {
@@ -373,6 +396,12 @@ __global__ void __launch_bounds__(kTcThreads, tc_ctas_per_sm(BM))
                 // offset-128 form by XOR with 0x80 and take z = 128)
                 const float s8 = __uint_as_float(ss << 16);
                 const float zoff = SYM ? 8388736.0f : 8388608.0f + __uint_as_float(zz << 16);
+                // two rings: the A tile is free once the MMAs of K block i − NA retired
+                // (one ring: the load slot's "full" wait already implied it)
+                if (kSplit && !mbar_wait(smem_u32(&aempty[ab]), ((uint32_t)(i / NA) & 1u) ^ 1u)) {
+                    ok = false;
+                    break;
+                }
 #pragma unroll
                 for (int i = 0; i < 4; ++i) {
                     uint32_t d[4];
@@ -392,7 +421,10 @@ __global__ void __launch_bounds__(kTcThreads, tc_ctas_per_sm(BM))
             }
             fence_proxy_async_smem();
             __syncwarp();
-            if (lane == 0) mbar_arrive(smem_u32(&afull[s]));
+            if (lane == 0) {
+                mbar_arrive(smem_u32(&afull[ab]));
+                if (kSplit) mbar_arrive(smem_u32(&empty[s]));   // its codes and scale pairs were read
+            }
         }
         // ------------------------------------------------------------ epilogue
         if (ok && mbar_wait(smem_u32(accf), 0)) {
