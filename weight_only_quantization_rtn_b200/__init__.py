@@ -12,6 +12,7 @@ the first call raises ImportError if the library is missing.
 """
 from __future__ import annotations
 
+import contextlib
 import ctypes
 import os
 
@@ -99,6 +100,9 @@ def lib() -> ctypes.CDLL:
     if _lib is None:
         _lib = _load()
     return _lib
+
+
+_NO_CONTEXT = contextlib.nullcontext()     # reusable: holds no state
 
 
 def _check(status: int, what: str) -> None:
@@ -221,12 +225,13 @@ def _workspace_bytes(dev: torch.device, M, N, K, g, sym, pid, ctas) -> int:
     return nbytes
 
 
-def _workspace(dev: torch.device, nbytes: int):
+def _workspace(dev: torch.device, nbytes: int, sid: int | None = None):
     """A scratch buffer per (device, stream), grown on demand; calls on one
-    stream never overlap, so they can share it."""
+    stream never overlap, so they can share it.  ``sid``: the current stream's
+    handle when the caller has it already."""
     if nbytes == 0:
         return None
-    key = (dev, torch.cuda.current_stream(dev).cuda_stream)
+    key = (dev, torch.cuda.current_stream(dev).cuda_stream if sid is None else sid)
     ws = _workspaces.get(key)
     if ws is None or ws.numel() < nbytes:
         ws = torch.empty(nbytes, dtype=torch.uint8, device=dev)
@@ -237,10 +242,10 @@ def _workspace(dev: torch.device, nbytes: int):
 _dev_bufs: dict = {}
 
 
-def _device_buffer(dev: torch.device, M: int, N: int) -> torch.Tensor:
+def _device_buffer(dev: torch.device, M: int, N: int, sid: int) -> torch.Tensor:
     """A device Y buffer per (device, stream, shape) for calls whose result goes
     to host memory; calls on one stream are ordered, so they can share it."""
-    key = (dev, torch.cuda.current_stream(dev).cuda_stream, M, N)
+    key = (dev, sid, M, N)
     buf = _dev_bufs.get(key)
     if buf is None:
         buf = torch.empty((M, N), dtype=torch.bfloat16, device=dev)
@@ -283,6 +288,8 @@ def gemm(X: torch.Tensor, packed: torch.Tensor, scales: torch.Tensor,
     if packed.shape[1] * 2 != K:
         raise ValueError(f"packed has K={packed.shape[1] * 2}, X has K={K}")
     _same_device(dev, X=Xd, scales=scales, zeros=None if sym else zeros)
+    stream = torch.cuda.current_stream(dev)      # looked up once per call: host overhead
+    sid = stream.cuda_stream
     host_out = None
     if host_in:
         if out is not None:
@@ -290,7 +297,7 @@ def gemm(X: torch.Tensor, packed: torch.Tensor, scales: torch.Tensor,
                     or not out.is_contiguous():
                 raise ValueError("out must be a contiguous bf16 [M, N] host tensor when X is on the host")
             host_out = out
-        out = _device_buffer(dev, M, N)
+        out = _device_buffer(dev, M, N, sid)
     elif out is None:
         out = torch.empty((M, N), dtype=torch.bfloat16, device=dev)
     else:
@@ -306,7 +313,7 @@ def gemm(X: torch.Tensor, packed: torch.Tensor, scales: torch.Tensor,
         _same_device(dev, act_scale=act_scale)
         if pid != PATH_AUTO or ctas:
             raise ValueError("act_scale uses the automatic kernel choice")
-    with torch.cuda.device(dev):
+    with (torch.cuda.device(dev) if dev.index != torch.cuda.current_device() else _NO_CONTEXT):
         if act_scale is None:
             ws_bytes = _workspace_bytes(dev, M, N, K, g, sym, pid, ctas)
         else:
@@ -315,26 +322,26 @@ def gemm(X: torch.Tensor, packed: torch.Tensor, scales: torch.Tensor,
             if ws_bytes is None:
                 ws_bytes = int(lib().w4a16_gemm_act_scaled_workspace_size(M, N, K, g)) if M and N else 0
                 _plan_bytes[key] = ws_bytes
-        ws = _workspace(dev, ws_bytes)
+        ws = _workspace(dev, ws_bytes, sid)
         if act_scale is None:
             _check(lib().w4a16_gemm_ex(_ptr(Xd), M, K, _ptr(packed), _ptr(scales),
                                        _ptr(zeros if not sym else None), N, g, int(bool(sym)),
                                        _ptr(out), _ptr(ws), ws_bytes,
                                        pid | (STATIC_WEIGHTS if static_weights else 0), ctas,
-                                       _stream(dev)),
+                                       ctypes.c_void_p(sid)),
                    "w4a16_gemm")
         else:
             _check(lib().w4a16_gemm_act_scaled(_ptr(Xd), M, K, _ptr(act_scale), _ptr(packed),
                                                _ptr(scales), _ptr(zeros if not sym else None), N, g,
                                                int(bool(sym)), _ptr(out), _ptr(ws), ws_bytes,
-                                               _stream(dev)),
+                                               ctypes.c_void_p(sid)),
                    "w4a16_gemm_act_scaled")
     if host_in:
         if host_out is None:
             host_out = torch.empty((M, N), dtype=torch.bfloat16, pin_memory=True)
         host_out.copy_(out, non_blocking=True)
         if sync:
-            torch.cuda.current_stream(dev).synchronize()
+            stream.synchronize()
         return host_out
     return out
 
