@@ -460,6 +460,9 @@ WORKLOAD_DEFS = {
     "prefill": (workloads.PREFILL, 2048, 128, False, "tensor", 4),
     "decode7b_pc": (workloads.DECODE_7B, 1, 0, False, "hbm", 4),
     "prefill_pc": (workloads.PREFILL, 2048, 0, False, "tensor", 4),
+    # mid-M: the tensor-core kernel at 32 activation rows on the prefill matrix
+    # (2 CTAs per SM, all tiles split over K); HBM-bound at this M (≈128 flop/B)
+    "mid32": (workloads.PREFILL, 32, 128, False, "hbm", 4),
     # W8A16 (8-bit codes): for profiling the 8-bit kernels; no end-to-end leg
     "w8_decode70b": (workloads.DECODE_70B, 1, 128, False, "hbm", 8),
     "w8_prefill": (workloads.PREFILL, 2048, 128, False, "tensor", 8),
