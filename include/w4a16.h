@@ -64,8 +64,9 @@
 extern "C" {
 #endif
 
-#define W4A16_ABI_VERSION 4   /* 3: w4a16_plan.split_tiles; the decode path is one kernel;
-                                 4: W4A16_STATIC_WEIGHTS, w8a16_gemm_ex/_plan, W8A8 */
+#define W4A16_ABI_VERSION 5   /* 3: w4a16_plan.split_tiles; the decode path is one kernel;
+                                 4: W4A16_STATIC_WEIGHTS, w8a16_gemm_ex/_plan, W8A8;
+                                 5: w4a16_gemm_host */
 
 typedef enum w4a16_status {
     W4A16_OK = 0,
@@ -187,6 +188,22 @@ w4a16_status w4a16_gemm_ex(const void* X, int64_t M, int64_t K, const void* pack
                            const void* scales, const void* zeros, int64_t N, int32_t g,
                            int32_t sym, void* Y, void* workspace, size_t workspace_bytes,
                            int32_t path, int32_t ctas, void* stream);
+
+/* w4a16_gemm_ex with the activations and the result in HOST memory: copies
+ * X_host (bf16 [M, K]) into X_dev, runs the GEMM into Y_dev, and copies Y_dev into
+ * Y_host (bf16 [M, N]), all three in order on `stream`; one call per layer of a
+ * host-driven step.  X_dev (M·K·2 bytes) and Y_dev (M·N·2 bytes) are device
+ * scratch owned by the caller, 16-byte aligned; nothing is allocated.  With
+ * page-locked host buffers the call returns before the copies complete: the
+ * caller synchronizes the stream before reading Y_host or reusing X_host.
+ * `flags` is w4a16_gemm_ex's `path` (kernel choice, W4A16_STATIC_WEIGHTS).
+ * Errors as w4a16_gemm_ex (checked before the first copy), plus W4A16_EINVAL for
+ * a null host or scratch pointer and W4A16_ECUDA when a copy cannot be queued. */
+w4a16_status w4a16_gemm_host(const void* X_host, int64_t M, int64_t K, const void* packed,
+                             const void* scales, const void* zeros, int64_t N, int32_t g,
+                             int32_t sym, void* Y_host, void* X_dev, void* Y_dev,
+                             void* workspace, size_t workspace_bytes, int32_t flags,
+                             void* stream);
 
 /* Bytes of device workspace w4a16_gemm_act_scaled needs for this shape: the
  * plan's workspace for M ≤ 16; for the tensor-core path that, rounded up to 256

@@ -54,7 +54,7 @@ def test_library_is_sm100a_only_and_links_no_cudart_dso(lib):
 
 
 def test_status_strings_and_version(lib):
-    assert lib.w4a16_abi_version() == 4
+    assert lib.w4a16_abi_version() == 5
     for s in range(6):
         assert lib.w4a16_status_string(s).startswith(b"W4A16")
 
@@ -76,6 +76,27 @@ def _gemm(lib, M=1, K=128, N=64, g=128, sym=0, X=FAKE, P=FAKE, S=FAKE, Z=FAKE, Y
 ])
 def test_gemm_rejects_invalid_arguments(lib, kw):
     assert _gemm(lib, **kw) == EINVAL
+
+
+def _gemm_host(lib, M=1, K=128, N=64, g=128, sym=0, Xh=FAKE, P=FAKE, S=FAKE, Z=FAKE, Yh=FAKE,
+               Xd=FAKE, Yd=FAKE, ws=FAKE, ws_bytes=1 << 30, flags=0):
+    return lib.w4a16_gemm_host(Xh, M, K, P, S, Z, N, g, sym, Yh, Xd, Yd, ws, ws_bytes, flags, None)
+
+
+@pytest.mark.parametrize("kw", [
+    dict(g=48), dict(K=96), dict(M=-1), dict(sym=2), dict(Xh=None), dict(Yh=None), dict(Xd=None),
+    dict(Yd=None), dict(Xd=FAKE + 8), dict(Yd=FAKE + 2), dict(P=None), dict(S=None), dict(Z=None),
+    dict(P=FAKE + 4), dict(M=17, flags=1), dict(flags=3),
+])
+def test_gemm_host_rejects_invalid_arguments(lib, kw):
+    """The host-buffer GEMM checks everything before it queues its first copy."""
+    assert _gemm_host(lib, **kw) == EINVAL
+
+
+def test_gemm_host_empty_and_workspace(lib):
+    assert _gemm_host(lib, M=0) == 0 and _gemm_host(lib, N=0) == 0
+    # a split shape needs its workspace: too small is reported before any copy
+    assert _gemm_host(lib, M=17, K=8192, N=8192, g=32, ws_bytes=16) == EWORKSPACE
 
 
 @pytest.mark.parametrize("K,g,ok", [

@@ -214,10 +214,30 @@ def test_empty_problems_are_noops():
 def test_host_buffers_end_to_end():
     P, S, Z = _quantized(256, 512, 128, False, seed=12)
     X = workloads.make_activation(2, 512, 13).pin_memory()
-    Y = w4.gemm(X, P, S, Z, 128, False)
+    Y = w4.gemm(X, P, S, Z, 128, False)                 # page-locked: w4a16_gemm_host
     assert not Y.is_cuda
     Yd = w4.gemm(X.cuda(), P, S, Z, 128, False)
     assert torch.equal(Y, Yd.cpu())
+    Yp = w4.gemm(X.clone(), P, S, Z, 128, False)        # pageable X: the torch copy path
+    assert not Yp.is_cuda and torch.equal(Yp, Y)
+
+
+@pytest.mark.parametrize("M,g,sym", [(1, 128, False), (16, 64, True), (40, 32, False), (300, 128, True)])
+def test_host_buffer_chain_matches_device(M, g, sym):
+    """Several host-buffer calls queued on one stream (both kernels, one sync at
+    the end, reused device scratch) give the device path's bits, each into its
+    own page-locked output."""
+    layers = [(1152, 768), (768, 1000), (1152, 640)]      # (K, N); K a multiple of every g
+    weights = [_quantized(N, K, g, sym, seed=70 + i) for i, (K, N) in enumerate(layers)]
+    xs = [workloads.make_activation(M, K, 80 + i).pin_memory() for i, (K, N) in enumerate(layers)]
+    torch.cuda.synchronize()          # the weights are written before the chain starts
+    outs = []
+    for (K, N), (P, S, Z), X in zip(layers, weights, xs):
+        Yh = torch.empty(M, N, dtype=torch.bfloat16, pin_memory=True)
+        outs.append(w4.gemm(X, P, S, Z, g, sym, out=Yh, sync=False, static_weights=True))
+    torch.cuda.synchronize()
+    for Yh, (P, S, Z), X in zip(outs, weights, xs):
+        assert torch.equal(Yh, w4.gemm(X.cuda(), P, S, Z, g, sym).cpu())
 
 
 # ------------------------------------------------------------------ full-size workloads

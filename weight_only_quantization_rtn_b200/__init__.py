@@ -25,7 +25,7 @@ __all__ = ["lib", "quantize", "dequantize", "gemm", "gemm_decode_noalloc", "plan
 LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libw4a16.so")
 
 # W4A16_ABI_VERSION in include/w4a16.h that the argument lists below follow
-ABI_VERSION = 4
+ABI_VERSION = 5
 PATH_AUTO, PATH_DECODE, PATH_TENSORCORE = 0, 1, 2
 STATIC_WEIGHTS = 0x100   # W4A16_STATIC_WEIGHTS, OR'ed into the path argument
 _PATHS = {"auto": PATH_AUTO, "decode": PATH_DECODE, "tensorcore": PATH_TENSORCORE}
@@ -64,6 +64,9 @@ def _load() -> ctypes.CDLL:
                                           vp]
     lib.w4a16_gemm_act_scaled_workspace_size.argtypes = [i64, i64, i64, i32]
     lib.w4a16_gemm_act_scaled_workspace_size.restype = sz
+    lib.w4a16_gemm_host.argtypes = [vp, i64, i64, vp, vp, vp, i64, i32, i32, vp, vp, vp, vp, sz,
+                                    i32, vp]
+    lib.w4a16_gemm_host.restype = ctypes.c_int
     lib.w4a16_gemm_decode_noalloc.argtypes = [vp, i64, i64, vp, vp, vp, i64, i32, i32, vp, vp]
     lib.w4a16_gemm_decode_noalloc.restype = ctypes.c_int
     lib.w4a16_device_error.argtypes = [ctypes.POINTER(ctypes.c_int32)]
@@ -242,10 +245,11 @@ def _workspace(dev: torch.device, nbytes: int, sid: int | None = None):
 _dev_bufs: dict = {}
 
 
-def _device_buffer(dev: torch.device, M: int, N: int, sid: int) -> torch.Tensor:
-    """A device Y buffer per (device, stream, shape) for calls whose result goes
-    to host memory; calls on one stream are ordered, so they can share it."""
-    key = (dev, sid, M, N)
+def _device_buffer(dev: torch.device, M: int, N: int, sid: int, tag: str = "y") -> torch.Tensor:
+    """A device bf16 [M, N] buffer per (device, stream, shape, role) for calls
+    whose operands live in host memory (``tag`` "x": the copied activations, "y":
+    the result); calls on one stream are ordered, so they can share it."""
+    key = (dev, sid, M, N, tag)
     buf = _dev_bufs.get(key)
     if buf is None:
         buf = torch.empty((M, N), dtype=torch.bfloat16, device=dev)
@@ -277,6 +281,9 @@ def gemm(X: torch.Tensor, packed: torch.Tensor, scales: torch.Tensor,
     stream before reading Y (e.g. once per step of several calls)."""
     host_in = not X.is_cuda
     dev = packed.device
+    if (host_in and act_scale is None and not ctas and X.is_pinned()
+            and (out is None or out.is_pinned())):
+        return _gemm_host(X, packed, scales, zeros, g, sym, path, out, sync, static_weights)
     Xd = X.to(dev, non_blocking=True) if host_in else X
     _need(Xd, torch.bfloat16, "X")
     _need(packed, torch.uint8, "packed")
@@ -343,6 +350,44 @@ def gemm(X: torch.Tensor, packed: torch.Tensor, scales: torch.Tensor,
         if sync:
             stream.synchronize()
         return host_out
+    return out
+
+
+def _gemm_host(X, packed, scales, zeros, g, sym, path, out, sync, static_weights):
+    """gemm() with X (and Y) in page-locked host memory: one w4a16_gemm_host call
+    copies X in, multiplies and copies Y out on the current stream."""
+    dev = packed.device
+    if X.dtype != torch.bfloat16 or X.dim() != 2 or not X.is_contiguous():
+        raise ValueError("X must be a contiguous bf16 [M, K] tensor")
+    _need(packed, torch.uint8, "packed")
+    _need(scales, torch.bfloat16, "scales")
+    if not sym:
+        _need(zeros, torch.bfloat16, "zeros")
+    M, K = X.shape
+    N = packed.shape[0]
+    if packed.shape[1] * 2 != K:
+        raise ValueError(f"packed has K={packed.shape[1] * 2}, X has K={K}")
+    _same_device(dev, scales=scales, zeros=None if sym else zeros)
+    if out is None:
+        out = torch.empty((M, N), dtype=torch.bfloat16, pin_memory=True)
+    elif out.dtype != torch.bfloat16 or tuple(out.shape) != (M, N) or not out.is_contiguous():
+        raise ValueError("out must be a contiguous bf16 [M, N] host tensor when X is on the host")
+    stream = torch.cuda.current_stream(dev)
+    sid = stream.cuda_stream
+    pid = _PATHS[path] if isinstance(path, str) else int(path)
+    with (torch.cuda.device(dev) if dev.index != torch.cuda.current_device() else _NO_CONTEXT):
+        ws_bytes = _workspace_bytes(dev, M, N, K, g, sym, pid, 0)
+        ws = _workspace(dev, ws_bytes, sid)
+        xd = _device_buffer(dev, M, K, sid, "x")
+        yd = _device_buffer(dev, M, N, sid, "y")
+        _check(lib().w4a16_gemm_host(X.data_ptr(), M, K, packed.data_ptr(), scales.data_ptr(),
+                                     None if sym else zeros.data_ptr(), N, g, int(bool(sym)),
+                                     out.data_ptr(), xd.data_ptr(), yd.data_ptr(),
+                                     None if ws is None else ws.data_ptr(), ws_bytes,
+                                     pid | (STATIC_WEIGHTS if static_weights else 0), sid),
+               "w4a16_gemm_host")
+    if sync:
+        stream.synchronize()
     return out
 
 

@@ -926,6 +926,35 @@ w4a16_status w4a16_gemm_ex(const void* X, int64_t M, int64_t K, const void* pack
                      workspace_bytes, path, ctas, stream);
 }
 
+w4a16_status w4a16_gemm_host(const void* X_host, int64_t M, int64_t K, const void* packed,
+                             const void* scales, const void* zeros, int64_t N, int32_t g,
+                             int32_t sym, void* Y_host, void* X_dev, void* Y_dev,
+                             void* workspace, size_t workspace_bytes, int32_t flags,
+                             void* stream) {
+    // every argument check of the GEMM first, on its plan, so that an invalid call
+    // queues no copy
+    w4a16_plan p;
+    w4a16_status st = make_plan(M, N, K, g, sym, flags & ~W4A16_STATIC_WEIGHTS, 0, current_sm_count(), &p);
+    if (st != W4A16_OK) return st;
+    if (M == 0 || N == 0) return W4A16_OK;
+    if (!X_host || !Y_host || !X_dev || !Y_dev || !aligned16(X_dev) || !aligned16(Y_dev))
+        return W4A16_EINVAL;
+    if (!packed || !scales || (!sym && !zeros) || !aligned16(packed) || !aligned16(scales) ||
+        (!sym && !aligned16(zeros)))
+        return W4A16_EINVAL;
+    if (workspace_bytes < (size_t)p.workspace_bytes) return W4A16_EWORKSPACE;
+    if (p.workspace_bytes > 0 && (workspace == nullptr || !aligned16(workspace))) return W4A16_EINVAL;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    if (cudaMemcpyAsync(X_dev, X_host, (size_t)(M * K * 2), cudaMemcpyHostToDevice, s) != cudaSuccess)
+        return W4A16_ECUDA;
+    st = w4a16_gemm_ex(X_dev, M, K, packed, scales, zeros, N, g, sym, Y_dev, workspace,
+                       workspace_bytes, flags, 0, stream);
+    if (st != W4A16_OK) return st;
+    if (cudaMemcpyAsync(Y_host, Y_dev, (size_t)(M * N * 2), cudaMemcpyDeviceToHost, s) != cudaSuccess)
+        return W4A16_ECUDA;
+    return W4A16_OK;
+}
+
 w4a16_status w4a16_gemm(const void* X, int64_t M, int64_t K, const void* packed,
                         const void* scales, const void* zeros, int64_t N, int32_t g,
                         int32_t sym, void* Y, void* workspace, size_t workspace_bytes,
